@@ -1,0 +1,131 @@
+"""fp64 CPU oracle for the S6 selective-scan forward (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg may import this package.  The product path (the CUDA library and
+its binding) never imports, links or runs anything here, and this package
+imports nothing from the product.
+
+The arithmetic lives in ``ss_oracle.c`` (plain serial recurrence in double,
+threads over channels); this module only compiles it with gcc and marshals
+numpy arrays.  See the C file's header for the passages it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ss_oracle.c")
+_LIB = os.path.join(_HERE, "libssoracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F32, BF16 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile ss_oracle.c into libssoracle.so (gcc, -O2, no fast-math)."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            vp, i64 = ctypes.c_void_p, ctypes.c_int64
+            lib.oracle_scan_fwd.argtypes = [
+                vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
+                i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, ctypes.c_int]
+            lib.oracle_scan_fwd.restype = ctypes.c_int
+            lib.oracle_softplus.argtypes = [ctypes.c_double]
+            lib.oracle_softplus.restype = ctypes.c_double
+            lib.oracle_silu.argtypes = [ctypes.c_double]
+            lib.oracle_silu.restype = ctypes.c_double
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _stored(a, name):
+    """Return (contiguous array, dtype code).  bf16 travels as uint16 bits."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, F32
+    if a.dtype == np.uint16:
+        return a, BF16
+    raise TypeError(f"{name}: expected float32 or uint16 (bf16 bits), got {a.dtype}")
+
+
+def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+             softplus=True, channels=None, nthreads=None):
+    """Serial fp64 selective scan.
+
+    u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; all float32 or all
+    bf16 bits (uint16).  A: [dim, N] float32; D, delta_bias: [dim] float32.
+    channels: optional 1-D int array of flat channel ids (b*dim + d); then
+    only those rows are computed.  Returns (y, last_state) as float64 with
+    shapes [batch, dim, L] / [batch, dim, N], or [len(channels), L] /
+    [len(channels), N] when channels is given.
+    """
+    u, dt = _stored(u, "u")
+    delta, dt2 = _stored(delta, "delta")
+    B, dt3 = _stored(B, "B")
+    C, dt4 = _stored(C, "C")
+    if len({dt, dt2, dt3, dt4}) != 1:
+        raise TypeError("u, delta, B, C must share one stored dtype")
+    if z is not None:
+        z, dt5 = _stored(z, "z")
+        if dt5 != dt:
+            raise TypeError("z must share the stored dtype of u")
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    if delta.shape != u.shape or B.shape != (batch, N, L) or C.shape != B.shape:
+        raise ValueError("shape mismatch")
+    if z is not None and z.shape != u.shape:
+        raise ValueError("z shape mismatch")
+    A = np.ascontiguousarray(A, dtype=np.float32)
+    if A.shape != (dim, N):
+        raise ValueError("A must be [dim, N]")
+    D = None if D is None else np.ascontiguousarray(D, dtype=np.float32)
+    delta_bias = None if delta_bias is None else np.ascontiguousarray(delta_bias, dtype=np.float32)
+    if channels is not None:
+        channels = np.ascontiguousarray(channels, dtype=np.int64)
+        nch = channels.size
+        y = np.empty((nch, L), np.float64)
+        h = np.empty((nch, N), np.float64)
+    else:
+        nch = batch * dim
+        y = np.empty((batch, dim, L), np.float64)
+        h = np.empty((batch, dim, N), np.float64)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().oracle_scan_fwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(softplus)), dt, batch, dim, L, N,
+        _ptr(channels), nch, _ptr(y), _ptr(h), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_scan_fwd rejected its arguments")
+    return y, h
+
+
+def softplus(x: float) -> float:
+    return _load().oracle_softplus(float(x))
+
+
+def silu(z: float) -> float:
+    return _load().oracle_silu(float(z))

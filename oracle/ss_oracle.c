@@ -1,0 +1,181 @@
+/*
+ * ss_oracle.c -- fp64 CPU oracle for the S6 selective-scan forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header or constant with the
+ * CUDA library; the two meet only through the seeded inputs handed to both.
+ *
+ * What it computes is the plain serial recurrence of the selective SSM,
+ * widened exactly from the stored input dtype to double:
+ *
+ *   for every (b, d):  h[n] = 0
+ *     for t = 0 .. L-1:
+ *       Delta  = softplus(delta[b,d,t] + delta_bias[d])   (or without softplus)
+ *       h[n]   = exp(Delta * A[d,n]) * h[n] + Delta * B[b,n,t] * u[b,d,t]
+ *       y      = sum_n C[b,n,t] * h[n] + D[d] * u[b,d,t]
+ *       y      = y * z * sigmoid(z)                       (when z is given)
+ *     last_state[b,d,n] = h[n]
+ *
+ * Passages followed (page title, section):
+ *  - "从Transformer的痛点说起 ... Mamba" (pwwt.cn), sec. 2.2: ZOH gives
+ *    A_bar = exp(Delta A); implementations simplify B_bar to Delta * B;
+ *    recurrence h_t = A_bar h_{t-1} + B_bar x_t, y_t = C h_t.
+ *  - same page, sec. 3.1: B_t, C_t, Delta_t are functions of x_t, with
+ *    Delta_t = softplus(Linear(x_t)); A stays input independent.
+ *  - same page, sec. 4.2 (pure-PyTorch SelectiveSSM): the bias of the Delta
+ *    projection sits inside the softplus; A = -exp(A_log) is diagonal [D,N];
+ *    the state starts at zero; the readout uses the state after the update
+ *    that includes token t; the skip term x*D is added before the gate
+ *    y * SiLU(z).
+ *  - "Mamba 选择性机制" (discosf.com), sec. 1.1 and 3.1: the discrete
+ *    recurrence and the associative operator it folds with.
+ *  - "Mamba 深度解读报告" (zako-mio.github.io), sec. 2.4: the state is never
+ *    materialised over (B,L,D,N); only y (B,L,D) is the output.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - softplus(x) = log(1 + e^x), evaluated as log1p(exp(x)) for x <= 30 and
+ *    x + log1p(exp(-x)) above, both exact to double rounding.
+ *  - softplus_flag == 0 means Delta = delta + delta_bias.
+ *  - SiLU(z) = z / (1 + exp(-z)).
+ *  - a null D, delta_bias or z means zero skip, zero bias and no gate.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Stored input dtypes: 0 = IEEE binary32, 1 = bfloat16 (upper half of a
+ * binary32).  Both widen to double without rounding. */
+static double widen(const void* p, int dtype, int64_t i) {
+  if (dtype == 1) {
+    uint32_t bits = (uint32_t)((const uint16_t*)p)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+  }
+  return (double)((const float*)p)[i];
+}
+
+static double softplus64(double x) {
+  if (x <= 30.0) return log1p(exp(x));
+  return x + log1p(exp(-x));
+}
+
+static double silu64(double z) { return z / (1.0 + exp(-z)); }
+
+typedef struct {
+  const void *u, *delta, *B, *C, *z;
+  const float *A, *D, *delta_bias;
+  int softplus_flag, dtype;
+  int64_t batch, dim, seqlen;
+  int dstate;
+  const int64_t* channels; /* optional list of flat channel ids b*dim+d */
+  int64_t n_channels;
+  double* y;          /* [n_channels, seqlen] */
+  double* last_state; /* [n_channels, dstate] or NULL */
+  int64_t next;       /* work counter (guarded by mu) */
+  pthread_mutex_t mu;
+} job_t;
+
+/* One (b, d) channel: the serial recurrence, nothing reordered. */
+static void run_channel(const job_t* J, int64_t slot, double* h) {
+  const int64_t flat = J->channels ? J->channels[slot] : slot;
+  const int64_t b = flat / J->dim, d = flat % J->dim;
+  const int64_t L = J->seqlen;
+  const int N = J->dstate;
+  const int64_t row = (b * J->dim + d) * L;    /* u, delta, z: [B,D,L] */
+  const int64_t bc_base = b * (int64_t)N * L;  /* B, C: [B,N,L] */
+  const double bias = J->delta_bias ? (double)J->delta_bias[d] : 0.0;
+  const double Dd = J->D ? (double)J->D[d] : 0.0;
+  double* yrow = J->y + slot * L;
+
+  for (int n = 0; n < N; ++n) h[n] = 0.0;
+  for (int64_t t = 0; t < L; ++t) {
+    const double x = widen(J->delta, J->dtype, row + t) + bias;
+    const double dt = J->softplus_flag ? softplus64(x) : x;
+    const double ut = widen(J->u, J->dtype, row + t);
+    double s = 0.0;
+    for (int n = 0; n < N; ++n) {
+      const double a_bar = exp(dt * (double)J->A[d * N + n]);
+      const double b_t = widen(J->B, J->dtype, bc_base + (int64_t)n * L + t);
+      const double c_t = widen(J->C, J->dtype, bc_base + (int64_t)n * L + t);
+      h[n] = a_bar * h[n] + dt * b_t * ut;
+      s += c_t * h[n];
+    }
+    s += Dd * ut;
+    if (J->z) s *= silu64(widen(J->z, J->dtype, row + t));
+    yrow[t] = s;
+  }
+  if (J->last_state)
+    for (int n = 0; n < N; ++n) J->last_state[slot * N + n] = h[n];
+}
+
+static void* worker(void* arg) {
+  job_t* J = (job_t*)arg;
+  double* h = (double*)malloc(sizeof(double) * (size_t)J->dstate);
+  if (!h) return NULL;
+  for (;;) {
+    pthread_mutex_lock(&J->mu);
+    const int64_t slot = J->next++;
+    pthread_mutex_unlock(&J->mu);
+    if (slot >= J->n_channels) break;
+    run_channel(J, slot, h);
+  }
+  free(h);
+  return NULL;
+}
+
+/*
+ * oracle_scan_fwd: returns 0 on success, -1 on a bad argument.
+ *
+ * u, delta, z : [batch, dim, seqlen] in `dtype` (0 f32, 1 bf16), L fastest
+ * B, C        : [batch, dstate, seqlen] in `dtype`
+ * A           : [dim, dstate] f32;  D, delta_bias: [dim] f32 (nullable)
+ * channels    : NULL for every channel (b*dim+d order), else n_channels flat
+ *               channel ids; y and last_state then hold only those rows.
+ * y           : [n_channels, seqlen] double
+ * last_state  : [n_channels, dstate] double (nullable)
+ * nthreads    : worker threads (>= 1)
+ */
+int oracle_scan_fwd(const void* u, const void* delta, const float* A,
+                    const void* B, const void* C, const float* D,
+                    const void* z, const float* delta_bias, int softplus_flag,
+                    int dtype, int64_t batch, int64_t dim, int64_t seqlen,
+                    int dstate, const int64_t* channels, int64_t n_channels,
+                    double* y, double* last_state, int nthreads) {
+  if (!u || !delta || !A || !B || !C || !y) return -1;
+  if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0) return -1;
+  if (dtype != 0 && dtype != 1) return -1;
+  if (!channels) n_channels = batch * dim;
+  if (n_channels <= 0) return -1;
+  if (channels)
+    for (int64_t i = 0; i < n_channels; ++i)
+      if (channels[i] < 0 || channels[i] >= batch * dim) return -1;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 512) nthreads = 512;
+
+  job_t J;
+  memset(&J, 0, sizeof J);
+  J.u = u; J.delta = delta; J.B = B; J.C = C; J.z = z;
+  J.A = A; J.D = D; J.delta_bias = delta_bias;
+  J.softplus_flag = softplus_flag; J.dtype = dtype;
+  J.batch = batch; J.dim = dim; J.seqlen = seqlen; J.dstate = dstate;
+  J.channels = channels; J.n_channels = n_channels;
+  J.y = y; J.last_state = last_state; J.next = 0;
+  pthread_mutex_init(&J.mu, NULL);
+
+  pthread_t tids[512];
+  int started = 0;
+  for (int i = 1; i < nthreads; ++i)
+    if (pthread_create(&tids[started], NULL, worker, &J) == 0) ++started;
+  worker(&J);
+  for (int i = 0; i < started; ++i) pthread_join(tids[i], NULL);
+  pthread_mutex_destroy(&J.mu);
+  return 0;
+}
+
+/* The scalar pieces, exported so that tests can pin them one by one. */
+double oracle_softplus(double x) { return softplus64(x); }
+double oracle_silu(double z) { return silu64(z); }

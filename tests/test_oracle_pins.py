@@ -1,0 +1,370 @@
+"""Pins for the fp64 oracle: facts the pages and the mathematics fix.
+
+None of these re-type the oracle's loop.  Each checks it against something
+else: a closed form, a limit, an identity, a brute-force evaluation in a
+different order, or a correctly rounded sum.  Together they are chosen so that
+a plausible slip in the oracle (a dropped term, a wrong sign or index, B and C
+swapped, the bias outside the softplus, the readout before the update, the
+gate missing the skip term) fails at least one of them.
+"""
+import math
+import random
+
+import numpy as np
+import pytest
+
+import oracle
+from selective_state_space_ss_b200 import inputs as I
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300))
+
+
+# ---------------------------------------------------------------- scalars --
+
+def test_softplus_identities():
+    # softplus(0) = ln 2; softplus(x) - softplus(-x) = x for every x;
+    # softplus(x) -> x for large x and -> e^x for very negative x.
+    assert oracle.softplus(0.0) == pytest.approx(math.log(2.0), rel=1e-16, abs=0)
+    for x in (-35.0, -7.25, -1e-3, 0.3, 2.0, 19.5, 29.9, 30.1, 55.0):
+        assert oracle.softplus(x) - oracle.softplus(-x) == pytest.approx(x, rel=1e-15, abs=1e-15)
+    assert oracle.softplus(60.0) == 60.0
+    assert oracle.softplus(-40.0) == pytest.approx(math.exp(-40.0), rel=1e-15)
+    # monotone and positive
+    xs = np.linspace(-50, 50, 1001)
+    v = np.array([oracle.softplus(x) for x in xs])
+    assert np.all(v > 0) and np.all(np.diff(v) > 0)
+
+
+def test_silu_identities():
+    # SiLU(z) = z * sigmoid(z): SiLU(0) = 0, SiLU(z) - SiLU(-z) = z,
+    # SiLU(z) -> z for large z and -> 0 for very negative z.
+    assert oracle.silu(0.0) == 0.0
+    for z in (-20.0, -3.0, -0.5, 0.25, 1.0, 4.0, 30.0):
+        assert oracle.silu(z) - oracle.silu(-z) == pytest.approx(z, rel=1e-15, abs=1e-15)
+    assert oracle.silu(50.0) == pytest.approx(50.0, rel=1e-20)
+    assert abs(oracle.silu(-50.0)) < 1e-19
+    assert oracle.silu(1.0) == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
+
+
+# ------------------------------------------------------ LTI closed form ----
+
+@pytest.mark.parametrize("softplus_on", [False, True])
+def test_lti_closed_form(softplus_on):
+    """Constant Delta, B, C: y = u * K_bar with K_k = sum_n C_n e^{k Delta A_n} Delta B_n.
+
+    The recurrence-equals-convolution identity of a time-invariant SSM
+    ("从Transformer的痛点 ... Mamba", sec. 2.3; "Mamba 深度解读报告", sec. 2.2).
+    With the softplus on, delta = -bias exactly, so Delta = softplus(0) = ln 2.
+    """
+    rng = np.random.default_rng(7)
+    batch, dim, L, N = 2, 3, 200, 5
+    A = -rng.uniform(0.05, 3.0, size=(dim, N))
+    Bc = rng.normal(size=(batch, N))
+    Cc = rng.normal(size=(batch, N))
+    u = rng.normal(size=(batch, dim, L))
+    if softplus_on:
+        bias = rng.uniform(-3, 3, size=dim).astype(np.float32)
+        delta = np.broadcast_to(-bias[None, :, None], (batch, dim, L))
+        dvals = np.full(dim, math.log(2.0))
+    else:
+        bias = None
+        dvals = rng.uniform(0.01, 0.2, size=dim).astype(np.float32).astype(np.float64)
+        delta = np.broadcast_to(dvals[None, :, None], (batch, dim, L))
+    Bt = np.broadcast_to(Bc[:, :, None], (batch, N, L))
+    Ct = np.broadcast_to(Cc[:, :, None], (batch, N, L))
+    y, h = oracle.scan_fwd(_f32(u), _f32(delta), _f32(A), _f32(Bt), _f32(Ct),
+                           delta_bias=bias, softplus=softplus_on)
+    # closed form from the fp32-rounded parameters, direct causal convolution
+    A32 = _f32(A).astype(np.float64)
+    B32, C32, u32 = (_f32(v).astype(np.float64) for v in (Bc, Cc, u))
+    k = np.arange(L, dtype=np.float64)
+    for b in range(batch):
+        for d in range(dim):
+            dl = dvals[d]
+            K = np.zeros(L)
+            for n in range(N):
+                K += C32[b, n] * np.exp(k * dl * A32[d, n]) * dl * B32[b, n]
+            ref = np.convolve(u32[b, d], K)[:L]
+            assert _rel(y[b, d], ref) < 1e-12
+            # final state: h_L[n] = sum_s e^{(L-1-s) Delta A_n} Delta B_n u_s
+            for n in range(N):
+                hs = np.sum(np.exp((L - 1 - k) * dl * A32[d, n]) * dl * B32[b, n] * u32[b, d])
+                assert h[b, d, n] == pytest.approx(hs, rel=1e-12, abs=1e-14)
+
+
+# ------------------------------------------- the associative operator ------
+
+def _combine(earlier, later):
+    """(a1,b1) then (a2,b2): the pages' (a,b)∘(c,d) = (ac, ad+b), later on the left."""
+    a1, b1 = earlier
+    a2, b2 = later
+    return (a2 * a1, a2 * b1 + b2)
+
+
+def test_operator_associative():
+    rng = np.random.default_rng(11)
+    n = 1_000_000
+    x = (rng.uniform(0.0, 1.0, n), rng.normal(size=n))
+    y = (rng.uniform(0.0, 1.0, n), rng.normal(size=n))
+    z = (rng.uniform(0.0, 1.0, n), rng.normal(size=n))
+    left = _combine(_combine(x, y), z)
+    right = _combine(x, _combine(y, z))
+    scale = np.abs(x[1]) + np.abs(y[1]) + np.abs(z[1])
+    assert np.max(np.abs(left[0] - right[0])) <= 1e-15
+    assert np.max(np.abs(left[1] - right[1]) / scale) <= 1e-14
+
+
+def _tree_prefix(pairs):
+    """Inclusive prefix of a list of (a, b) pairs by a Blelloch up/down sweep."""
+    n = len(pairs)
+    size = 1
+    while size < n:
+        size *= 2
+    ident = (np.ones_like(pairs[0][0]), np.zeros_like(pairs[0][1]))
+    t = list(pairs) + [ident] * (size - n)
+    step = 1
+    while step < size:  # up-sweep
+        for i in range(2 * step - 1, size, 2 * step):
+            t[i] = _combine(t[i - step], t[i])
+        step *= 2
+    t[size - 1] = ident
+    step = size // 2
+    while step >= 1:  # down-sweep (exclusive)
+        for i in range(2 * step - 1, size, 2 * step):
+            left = t[i - step]
+            t[i - step] = t[i]
+            t[i] = _combine(t[i], left)
+        step //= 2
+    return [_combine(t[i], pairs[i]) for i in range(n)]
+
+
+def test_tree_fold_equals_serial_oracle():
+    """A work-efficient tree scan over (A_bar_t, Delta_t B_t u_t) gives the oracle's states."""
+    rng = np.random.default_rng(5)
+    batch, dim, L, N = 1, 2, 37, 4
+    u = _f32(rng.normal(size=(batch, dim, L)))
+    delta = _f32(rng.uniform(0.01, 0.5, size=(batch, dim, L)))
+    A = _f32(-rng.uniform(0.1, 4.0, size=(dim, N)))
+    B = _f32(rng.normal(size=(batch, N, L)))
+    C = _f32(rng.normal(size=(batch, N, L)))
+    y, h = oracle.scan_fwd(u, delta, A, B, C, softplus=False)
+    for d in range(dim):
+        pairs = []
+        for t in range(L):
+            dl = float(delta[0, d, t])
+            a = np.exp(dl * A[d].astype(np.float64))
+            bb = dl * B[0, :, t].astype(np.float64) * float(u[0, d, t])
+            pairs.append((a, bb))
+        pref = _tree_prefix(pairs)
+        for t in range(L):
+            ht = pref[t][1]
+            yt = float(np.dot(C[0, :, t].astype(np.float64), ht))
+            assert yt == pytest.approx(y[0, d, t], rel=1e-12, abs=1e-13)
+        assert np.allclose(pref[-1][1], h[0, d], rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------- the Delta limits -----
+
+def _rand_case(rng, batch, dim, L, N):
+    return dict(u=_f32(rng.normal(size=(batch, dim, L))),
+                B=_f32(rng.normal(size=(batch, N, L))),
+                C=_f32(rng.normal(size=(batch, N, L))),
+                z=_f32(rng.normal(size=(batch, dim, L))),
+                D=_f32(rng.normal(size=dim)),
+                A=_f32(-rng.uniform(1.0, 8.0, size=(dim, N))))
+
+
+def test_hold_limit_exact_zero_delta():
+    """Delta = 0 exactly: A_bar = 1 and B_bar u = 0, so the state is held bitwise
+    ("Mamba 选择性机制", sec. 2.1: small Delta keeps the state)."""
+    rng = np.random.default_rng(3)
+    batch, dim, L, N, P = 2, 3, 50, 6, 20
+    c = _rand_case(rng, batch, dim, L, N)
+    delta = np.zeros((batch, dim, L), np.float32)
+    delta[:, :, :P] = rng.uniform(0.05, 0.5, size=(batch, dim, P))
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], softplus=False)
+    yp, hp = oracle.scan_fwd(c["u"][:, :, :P].copy(), delta[:, :, :P].copy(), c["A"],
+                             c["B"][:, :, :P].copy(), c["C"][:, :, :P].copy(), D=c["D"], softplus=False)
+    assert np.array_equal(h, hp)  # held bitwise from the end of the prefix
+    assert np.array_equal(y[:, :, :P], yp)
+    Cw, uw = c["C"].astype(np.float64), c["u"].astype(np.float64)
+    for t in range(P, L):
+        ref = np.einsum("bn,bdn->bd", Cw[:, :, t], hp) + c["D"].astype(np.float64)[None] * uw[:, :, t]
+        assert _rel(y[:, :, t], ref) < 1e-14
+
+
+def test_hold_limit_softplus_with_bias():
+    """delta + bias = -60 under the softplus: Delta ~ 9e-27, the state is held.
+
+    The bias is nonzero, so a bias added outside the softplus would give
+    Delta ~ 3 and fail here."""
+    rng = np.random.default_rng(4)
+    batch, dim, L, N, P = 1, 4, 40, 5, 15
+    c = _rand_case(rng, batch, dim, L, N)
+    bias = np.full(dim, 3.0, np.float32)
+    delta = np.full((batch, dim, L), -63.0, np.float32)
+    delta[:, :, :P] = _f32(rng.normal(scale=0.5, size=(batch, dim, P)))
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                           delta_bias=bias, softplus=True)
+    _, hp = oracle.scan_fwd(*(np.ascontiguousarray(v[:, :, :P]) for v in (c["u"], delta)), c["A"],
+                            *(np.ascontiguousarray(v[:, :, :P]) for v in (c["B"], c["C"])),
+                            D=c["D"], z=np.ascontiguousarray(c["z"][:, :, :P]),
+                            delta_bias=bias, softplus=True)
+    assert _rel(h, hp) < 1e-22
+    gate = np.vectorize(oracle.silu)(c["z"].astype(np.float64))
+    for t in range(P, L):
+        ref = (np.einsum("bn,bdn->bd", c["C"][:, :, t].astype(np.float64), hp)
+               + c["D"].astype(np.float64)[None] * c["u"][:, :, t]) * gate[:, :, t]
+        assert _rel(y[:, :, t], ref) < 1e-14
+
+
+def test_reset_limit():
+    """delta + bias = 60 under the softplus and A <= -1: A_bar <= e^-60, the state
+    resets every step to Delta B_t u_t, with Delta = 60
+    ("Mamba 选择性机制", sec. 2.1: large Delta forgets the past)."""
+    rng = np.random.default_rng(6)
+    batch, dim, L, N = 2, 3, 30, 7
+    c = _rand_case(rng, batch, dim, L, N)
+    bias = _f32(rng.uniform(-2, 2, size=dim))
+    delta = np.broadcast_to((60.0 - bias.astype(np.float64))[None, :, None], (batch, dim, L))
+    delta = _f32(delta)
+    x = delta.astype(np.float64) + bias.astype(np.float64)[None, :, None]  # ~60
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                           delta_bias=bias, softplus=True)
+    gate = np.vectorize(oracle.silu)(c["z"].astype(np.float64))
+    for t in range(L):
+        dl = x[:, :, t]  # softplus(x) = x to double precision at x ~ 60
+        cb = np.sum(c["C"][:, :, t].astype(np.float64) * c["B"][:, :, t].astype(np.float64), axis=1)
+        ut = c["u"][:, :, t].astype(np.float64)
+        ref = (dl * ut * cb[:, None] + c["D"].astype(np.float64)[None] * ut) * gate[:, :, t]
+        assert _rel(y[:, :, t], ref) < 1e-14
+    href = x[:, :, -1][:, :, None] * c["B"][:, None, :, -1].astype(np.float64) * c["u"][:, :, -1:].astype(np.float64)
+    assert _rel(h, href) < 1e-14
+
+
+# --------------------------------------------- brute-force unrolled sums ---
+
+@pytest.mark.parametrize("L", [1, 2, 5, 8])
+def test_bruteforce_unrolled(L):
+    """h_t = sum_{s<=t} (prod_{s<k<=t} A_bar_k) Delta_s B_s u_s with explicit products
+    ("从Transformer的痛点 ... Mamba", sec. 4.3), then y_t = (C_t.h_t + D u_t) SiLU(z_t)."""
+    rng = np.random.default_rng(100 + L)
+    batch, dim, N = 2, 3, 4
+    c = _rand_case(rng, batch, dim, L, N)
+    c["A"] = _f32(-rng.uniform(0.1, 3.0, size=(dim, N)))
+    delta = _f32(rng.normal(scale=0.5, size=(batch, dim, L)))
+    bias = _f32(rng.uniform(-4, 0, size=dim))
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                           delta_bias=bias, softplus=True)
+    for b in range(batch):
+        for d in range(dim):
+            dl = [oracle.softplus(float(delta[b, d, t]) + float(bias[d])) for t in range(L)]
+            for t in range(L):
+                acc = 0.0
+                hts = []
+                for n in range(N):
+                    a = float(c["A"][d, n])
+                    hn = 0.0
+                    for s in range(t + 1):
+                        prod = 1.0
+                        for k in range(s + 1, t + 1):
+                            prod *= math.exp(dl[k] * a)
+                        hn += prod * dl[s] * float(c["B"][b, n, s]) * float(c["u"][b, d, s])
+                    hts.append(hn)
+                    acc += float(c["C"][b, n, t]) * hn
+                ref = (acc + float(c["D"][d]) * float(c["u"][b, d, t])) * oracle.silu(float(c["z"][b, d, t]))
+                assert y[b, d, t] == pytest.approx(ref, rel=1e-13, abs=1e-15)
+            assert np.allclose(h[b, d], hts, rtol=1e-13, atol=1e-15)
+
+
+def test_prefix_sum_special_case():
+    """N = 1, A = 0, no softplus, C = 1, D = 0, no gate: h_t is the running sum of
+    Delta_s B_s u_s; compared with a correctly rounded sum (math.fsum)."""
+    rng = np.random.default_rng(9)
+    L = 3000
+    u = _f32(rng.normal(size=(1, 1, L)))
+    delta = _f32(rng.uniform(0.0, 1.0, size=(1, 1, L)))
+    B = _f32(rng.normal(size=(1, 1, L)))
+    C = np.ones((1, 1, L), np.float32)
+    A = np.zeros((1, 1), np.float32)
+    y, h = oracle.scan_fwd(u, delta, A, B, C, softplus=False)
+    terms = [float(delta[0, 0, s]) * float(B[0, 0, s]) * float(u[0, 0, s]) for s in range(L)]
+    running = [math.fsum(terms[: t + 1]) for t in range(0, L, 97)] + [math.fsum(terms)]
+    idx = list(range(0, L, 97)) + [L - 1]
+    bound = L * 2.0 ** -52 * math.fsum(abs(v) for v in terms)
+    for i, t in enumerate(idx):
+        assert abs(y[0, 0, t] - running[i]) <= bound
+    assert abs(h[0, 0, 0] - running[-1]) <= bound
+
+
+# ------------------------------------------------------ index plumbing -----
+
+def test_index_plumbing_single_impulse():
+    """One input at t = 0, then u = 0: h_L[b,d,n] = e^{(L-1) Delta A[d,n]} Delta B[b,n,0] u[b,d,0].
+
+    A[d,n], B[b,n,0], u[b,d,0], D[d] and the bias are distinct per index, so a
+    transposed or shifted index lands on a wrong value."""
+    batch, dim, L, N = 3, 5, 9, 4
+    d_idx = np.arange(dim)[:, None]
+    n_idx = np.arange(N)[None, :]
+    A = _f32(-(1 + d_idx + 100 * n_idx) * 1e-3)
+    u = np.zeros((batch, dim, L), np.float32)
+    u[:, :, 0] = _f32(1.0 + np.arange(batch)[:, None] * 0.5 + np.arange(dim)[None, :] * 0.125)
+    B = np.zeros((batch, N, L), np.float32)
+    B[:, :, 0] = _f32(1.0 + np.arange(batch)[:, None] * 0.25 + np.arange(N)[None, :] * 2.0)
+    C = np.zeros((batch, N, L), np.float32)
+    C[:, :, L - 1] = _f32(0.5 + np.arange(batch)[:, None] + 0.1 * np.arange(N)[None, :])
+    bias = _f32(0.1 + 0.01 * np.arange(dim))
+    Dv = _f32(10.0 + np.arange(dim))
+    delta = np.zeros((batch, dim, L), np.float32)
+    y, h = oracle.scan_fwd(u, delta, A, B, C, D=Dv, delta_bias=bias, softplus=False)
+    for b in range(batch):
+        for d in range(dim):
+            dl = float(bias[d])
+            for n in range(N):
+                ref = math.exp((L - 1) * dl * float(A[d, n])) * dl * float(B[b, n, 0]) * float(u[b, d, 0])
+                assert h[b, d, n] == pytest.approx(ref, rel=1e-14)
+            # y_0 = D u_0 + C_0.h_0 (C_0 = 0); y_{L-1} = C_{L-1}.h_{L-1}
+            assert y[b, d, 0] == pytest.approx(float(Dv[d]) * float(u[b, d, 0]), rel=1e-15)
+            assert y[b, d, L - 1] == pytest.approx(float(np.dot(C[b, :, L - 1].astype(np.float64), h[b, d])), rel=1e-14)
+            assert np.all(y[b, d, 1:L - 1] == 0.0)
+
+
+# ------------------------------------------------------- host plumbing -----
+
+def test_channel_subset_matches_full():
+    w = I.Workload("t", 2, 6, 33, 8, "bf16")
+    x = I.make_inputs(w, seed=3)
+    y, h = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"])
+    ch = np.array([11, 0, 7, 5])
+    ys, hs = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
+                             channels=ch)
+    assert np.array_equal(ys, y.reshape(-1, 33)[ch])
+    assert np.array_equal(hs, h.reshape(-1, 8)[ch])
+
+
+def test_bf16_widening_is_exact():
+    w = I.Workload("t", 1, 4, 17, 4, "bf16")
+    x = I.make_inputs(w, seed=8)
+    y1, h1 = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"])
+    wd = {k: I.bf16_to_f32(x[k]) for k in ("u", "delta", "B", "C", "z")}
+    y2, h2 = oracle.scan_fwd(wd["u"], wd["delta"], x["A"], wd["B"], wd["C"], x["D"], wd["z"], x["delta_bias"])
+    assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
+
+
+def test_oracle_rejects_bad_arguments():
+    u = np.zeros((1, 2, 3), np.float32)
+    with pytest.raises(ValueError):
+        oracle.scan_fwd(u, u, np.zeros((2, 4), np.float32), np.zeros((1, 4, 3), np.float32),
+                        np.zeros((1, 4, 2), np.float32))
+    with pytest.raises(TypeError):
+        oracle.scan_fwd(u, u.astype(np.float64), np.zeros((2, 4), np.float32),
+                        np.zeros((1, 4, 3), np.float32), np.zeros((1, 4, 3), np.float32))
