@@ -1,0 +1,383 @@
+"""Benchmark of the fused selective-scan forward (one B200 per rank).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path (ss_scan_fwd: discretise, scan,
+read out, gate, store y and the final state) over one batch of the workload.
+Rank 0 prints one JSON line.  Multi-GPU runs (torchrun, one rank per GPU)
+shard nothing: every rank scans its own full batch of the workload, with no
+data-path collective (weak scaling); the only collectives are the timing
+barrier and the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (the
+reference arm): each step is a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_ss_b200 import inputs as I  # noqa: E402
+
+DEFAULT_WORKLOAD = "b8_l2048_d1536_n16_bf16"
+METRIC = "selective-scan fwd (B·L·D) elements/s and % of HBM/SFU roofline"
+UNIT = "elements/s"
+L2_BYTES = 126 * 1024 * 1024
+NUM_SMS = 148
+MUFU_EX2_PER_CLK_PER_SM = 16  # ex2 results per clock per SM (special-function unit)
+KERNEL_SOURCES = ("selective_state_space_ss_b200/csrc/ss_scan.cu",
+                  "selective_state_space_ss_b200/csrc/scan_fwd_chunked.cuh",
+                  "selective_state_space_ss_b200/csrc/scan_common.cuh")
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        p.update(hbm_gbs=float(m["hbm_gbs"]), sm_max_mhz=float(m.get("sm_max_mhz", 1965.0)),
+                 source="measured")
+    return p
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(workload)
+    if not rec or rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------- clocks ------
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: report no clocks rather than fail the bench
+            self.nv = None
+
+    def _sample(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.nv or not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": sorted(self.reasons)}
+
+
+# ---------------------------------------------------------- GPU arm --------
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_gpu_arm(args, w: I.Workload):
+    import torch
+    import torch.distributed as dist
+
+    from selective_state_space_ss_b200 import ss_scan_fwd, load_library
+
+    world, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    load_library()
+    stream = torch.cuda.current_stream(dev)
+
+    # inputs: rotate over enough sets that each step reads data last touched
+    # more than one L2 capacity ago (flushing is not needed then)
+    per_set = w.algorithmic_bytes()
+    nsets = max(1, -(-4 * L2_BYTES // per_set))
+    host = [I.make_inputs(w, seed=1000 + 17 * rank + s) for s in range(nsets)]
+
+    def to_dev(x):
+        out = {}
+        for k, v in x.items():
+            if v is None:
+                out[k] = None
+            elif v.dtype == np.uint16:
+                out[k] = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev)
+            else:
+                out[k] = torch.from_numpy(v).to(dev)
+        return out
+
+    sets = [to_dev(x) for x in host]
+    ys = [torch.empty((w.batch, w.dim, w.seqlen), dtype=torch.float32, device=dev) for _ in sets]
+    hs = [torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev) for _ in sets]
+
+    def step(i):
+        s = i % nsets
+        x = sets[s]
+        ss_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+                    delta_bias=x["delta_bias"], softplus=w.softplus, y_out=ys[s], last_state_out=hs[s],
+                    stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = w.elements * world * args.steps / (ms_max * 1e-3)
+
+    # end to end through the public call: pinned host inputs -> device -> scan -> y back to host
+    ex = host[0]
+    pinned = {}
+    for k, v in ex.items():
+        if v is None:
+            pinned[k] = None
+        else:
+            src = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16 \
+                else torch.from_numpy(v)
+            pinned[k] = src.pin_memory()
+    y_host = torch.empty((w.batch, w.dim, w.seqlen), dtype=torch.float32).pin_memory()
+    h_host = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32).pin_memory()
+    dbuf = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in pinned.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values() if v is not None)
+    d2h = y_host.numel() * 4 + h_host.numel() * 4
+
+    def e2e_step():
+        for k, v in pinned.items():
+            if v is not None:
+                dbuf[k].copy_(v, non_blocking=True)
+        y, h = ss_scan_fwd(dbuf["u"], dbuf["delta"], dbuf["A"], dbuf["B"], dbuf["C"], D=dbuf["D"],
+                           z=dbuf["z"], delta_bias=dbuf["delta_bias"], softplus=w.softplus,
+                           y_out=ys[0], last_state_out=hs[0], stream=stream)
+        y_host.copy_(y, non_blocking=True)
+        h_host.copy_(h, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = w.elements * world * e2e_steps / (float(te.item()) * 1e-3)
+
+    if world > 1:
+        dist.destroy_process_group()
+    return dict(ms_per_step=ms_per_step, value=value, world=world, rank=rank,
+                clocks=clk.summary(), e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=h2d,
+                                                d2h_bytes_per_step=d2h, steps=e2e_steps),
+                nsets=nsets, host=host[0])
+
+
+def roofline(w: I.Workload, kernel_ms: float):
+    p = peaks()
+    t_hbm = w.algorithmic_bytes() / (p["hbm_gbs"] * 1e9)
+    sfu_rate = NUM_SMS * MUFU_EX2_PER_CLK_PER_SM * p["sm_max_mhz"] * 1e6  # ex2 per second
+    t_sfu = w.exps() / sfu_rate
+    s = kernel_ms * 1e-3
+    if t_sfu >= t_hbm:
+        achieved = w.exps() / s / 1e9
+        peak = sfu_rate / 1e9
+        r = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gexp2/s"}
+    else:
+        achieved = w.algorithmic_bytes() / s / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": p["hbm_gbs"], "unit": "GB/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["traffic"] = profiled_traffic(w.name)
+    r["peak_source"] = (f"SFU: {NUM_SMS} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
+                        f"{p['sm_max_mhz']:.0f} MHz" if r["bound"] == "alu"
+                        else f"HBM copy, {p['source']}")
+    r["hbm_bound_us"] = t_hbm * 1e6
+    r["sfu_bound_us"] = t_sfu * 1e6
+    r["hbm_frac"] = (w.algorithmic_bytes() / s / 1e9) / p["hbm_gbs"]
+    return r
+
+
+# ---------------------------------------------------------- CPU oracle -----
+
+def oracle_sample(w: I.Workload, x: dict, target_s: float):
+    """Time the fp64 oracle on a bounded sample of channels (full sequence each)."""
+    import oracle
+
+    cores = os.cpu_count() or 1
+    nch = w.batch * w.dim
+    rng = np.random.default_rng(0)
+    take = min(nch, max(cores, 64))
+    while True:
+        ch = np.sort(rng.choice(nch, take, replace=False))
+        t0 = time.perf_counter()
+        oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
+                        softplus=w.softplus, channels=ch, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or take == nch:
+            return take, dt, cores
+        take = min(nch, int(take * max(2.0, 1.2 * target_s / max(dt, 1e-3))))
+
+
+def run_reference_arm(args, w: I.Workload):
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return None
+    x = I.make_inputs(w, seed=1000)
+    import oracle
+
+    cores = os.cpu_count() or 1
+    # size one step to ~2 s of oracle work so that warmup + steps stay within minutes
+    take, dt, _ = oracle_sample(w, x, target_s=2.0)
+    nch = w.batch * w.dim
+    rng = np.random.default_rng(1)
+    times = []
+    for i in range(args.warmup + args.steps):
+        ch = np.sort(rng.choice(nch, take, replace=False))
+        t0 = time.perf_counter()
+        oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
+                        softplus=w.softplus, channels=ch, nthreads=cores)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = take * w.seqlen * len(times) / tot
+    sample = f"{take} of {nch} channels x full L={w.seqlen} per step, fp64, {cores} threads"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def config_of(w: I.Workload, world: int):
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate,
+            "in_dtype": w.dtype, "state_dtype": "f32", "y_dtype": "f32",
+            "parallelism": f"replicas x{world} (independent batch per GPU, no collective)",
+            "l2": "inputs rotated over sets totalling >= 4x L2 (126 MB); no flush"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = I.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        line = run_reference_arm(args, w)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    r = run_gpu_arm(args, w)
+    if r["rank"] != 0:
+        return
+    roof = roofline(w, r["ms_per_step"])
+    line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": r["world"],
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config_of(w, r["world"]), "roofline": roof,
+            "e2e": r["e2e"], "gpu_launches": args.steps, "clocks": r["clocks"]}
+    if r["world"] == 1 and not args.no_cpu_baseline:
+        take, dt, cores = oracle_sample(w, r["host"], target_s=10.0)
+        line["cpu_baseline"] = {"value": take * w.seqlen / dt, "unit": UNIT, "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{take} of {w.batch * w.dim} channels x full L={w.seqlen}, "
+                                          f"fp64, {cores} threads, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

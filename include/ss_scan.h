@@ -1,0 +1,105 @@
+/*
+ * ss_scan.h -- C ABI of libssscan.so: the S6 selective-scan forward on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (pages: "从Transformer的痛点说起 ... Mamba", sec. 2.2, 3.1 and
+ * the SelectiveSSM of sec. 4.2; "Mamba 选择性机制", sec. 1.1, 2.2 and 3.1;
+ * "Mamba 深度解读报告", sec. 2.3-2.4).  For every batch row b and channel d,
+ * with t = 0..L-1 and n = 0..N-1, starting from h = 0:
+ *
+ *   Delta_t = softplus(delta[b,d,t] + delta_bias[d])   (softplus_flag != 0)
+ *           = delta[b,d,t] + delta_bias[d]             (softplus_flag == 0)
+ *   h[n]    = exp(Delta_t * A[d,n]) * h[n] + Delta_t * B[b,n,t] * u[b,d,t]
+ *   y[b,d,t]= (sum_n C[b,n,t] * h[n] + D[d] * u[b,d,t]) * SiLU(z[b,d,t])
+ *   last_state[b,d,n] = h[n] after t = L-1
+ *
+ * B_bar is the simplified Delta*B of the first page's sec. 2.2; the readout
+ * uses the state after the update that includes token t; the gate multiplies
+ * the skip term too (sec. 4.2 order: add x*D, then multiply by SiLU(z)).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers, caller-owned, contiguous, with
+ *    the fastest axis last as written ([B,D,L] means L fastest).
+ *  - The library never allocates device memory, never synchronises the
+ *    stream (except ss_last_device_error) and keeps no state beyond one
+ *    device-side error word per device.
+ *  - Calls are asynchronous on `stream` (0 = the legacy default stream).
+ *  - Arguments are checked on the host before any launch; a rejected call
+ *    launches nothing and touches no buffer.
+ */
+#ifndef SS_SCAN_H_
+#define SS_SCAN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SS_OK = 0,
+  SS_ERR_INVALID_ARG = 1, /* null required pointer, bad size, bad alignment, workspace too small */
+  SS_ERR_UNSUPPORTED = 2, /* dstate not in {16, 32, 64, 128}, or unknown dtype */
+  SS_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+  SS_ERR_TIMEOUT = 4      /* a bounded inter-block wait gave up (see ss_last_device_error) */
+} ss_status;
+
+typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
+
+/*
+ * ss_scan_fwd -- the fused forward: discretise, scan, read out, gate, store.
+ *
+ *  u, delta, z   [batch, dim, seqlen]   in_dtype            (z nullable: no gate)
+ *  A             [dim, dstate]          float32             (real diagonal, normally < 0)
+ *  B, C          [batch, dstate, seqlen] in_dtype           (shared by all channels)
+ *  D, delta_bias [dim]                  float32             (nullable: treated as 0)
+ *  softplus_flag nonzero: Delta = softplus(delta + delta_bias)
+ *  y_out         [batch, dim, seqlen]   float32 (written)
+ *  last_state_out[batch, dim, dstate]   float32 (nullable: not written)
+ *  batch, dim, seqlen >= 1; batch*dim*seqlen < 2^62
+ *  dstate        16, 32, 64 or 128
+ *  workspace     device scratch of at least ss_scan_workspace_bytes(...) bytes,
+ *                caller-owned, 256-byte aligned (nullable when that is 0).
+ *                Its contents on entry do not matter; the call may overwrite it.
+ *                Two calls in flight at once must not share one workspace.
+ *
+ * Alignment: every tensor pointer must be aligned to its element size.  When
+ * seqlen*sizeof(in_dtype) is a multiple of 16 and u, delta, z, B, C, y_out are
+ * 16-byte aligned the kernel moves 16-byte vectors; otherwise it falls back to
+ * element-wise loads (correct, slower).
+ *
+ * Returns SS_OK after a successful launch (errors raised later inside the
+ * kernel are reported by ss_last_device_error), or an error code with nothing
+ * launched.
+ */
+ss_status ss_scan_fwd(const void* u, const void* delta, const float* A,
+                      const void* B, const void* C, const float* D,
+                      const void* z, const float* delta_bias,
+                      int softplus_flag, float* y_out, float* last_state_out,
+                      int64_t batch, int64_t dim, int64_t seqlen, int dstate,
+                      ss_dtype in_dtype, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of workspace ss_scan_fwd needs for these sizes on the current device
+ * (0 when the chosen kernel needs none).  Returns (size_t)-1 for sizes that
+ * ss_scan_fwd would reject. */
+size_t ss_scan_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen,
+                               int dstate);
+
+/* Static, NUL-terminated description of a status code. */
+const char* ss_status_string(ss_status status);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: SS_OK, or SS_ERR_TIMEOUT when a bounded wait inside a
+ * kernel gave up since the last query.  SS_ERR_CUDA if the synchronisation
+ * itself failed. */
+ss_status ss_last_device_error(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS_SCAN_H_ */

@@ -1,0 +1,24 @@
+"""B200-native S6 selective-scan forward.
+
+The compute lives in libssscan.so (hand-written sm_100a CUDA, C ABI in
+include/ss_scan.h); this package is its Python binding plus the seeded input
+generator (``selective_state_space_ss_b200.inputs``).  The library is loaded
+lazily on the first call, and a missing library raises: there is no CPU path.
+"""
+from ._native import (  # noqa: F401
+    EXPORTED,
+    SS_BF16,
+    SS_ERR_CUDA,
+    SS_ERR_INVALID_ARG,
+    SS_ERR_TIMEOUT,
+    SS_ERR_UNSUPPORTED,
+    SS_F32,
+    SS_OK,
+    SSError,
+    library_path,
+    load_library,
+    ss_last_device_error,
+    ss_scan_fwd,
+    ss_scan_workspace_bytes,
+    ss_status_string,
+)

@@ -1,0 +1,146 @@
+"""ctypes binding of libssscan.so (the C ABI in include/ss_scan.h).
+
+Argument marshalling only: every step of the scan runs in the CUDA library.
+PyTorch provides device memory and the stream.  There is no CPU fallback; if
+the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssscan.so")
+_lock = threading.Lock()
+_lib = None
+
+SS_OK, SS_ERR_INVALID_ARG, SS_ERR_UNSUPPORTED, SS_ERR_CUDA, SS_ERR_TIMEOUT = range(5)
+SS_F32, SS_BF16 = 0, 1
+
+EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
+            "ss_last_device_error")
+
+
+class SSError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {ss_status_string(status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libssscan.so once; raise if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m selective_state_space_ss_b200.build` "
+                "(nvcc, sm_100a).  There is no CPU fallback.")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        lib.ss_scan_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp,
+                                    i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
+        lib.ss_scan_fwd.restype = ci
+        lib.ss_scan_workspace_bytes.argtypes = [i64, i64, i64, ci]
+        lib.ss_scan_workspace_bytes.restype = ctypes.c_size_t
+        lib.ss_status_string.argtypes = [ci]
+        lib.ss_status_string.restype = ctypes.c_char_p
+        lib.ss_last_device_error.argtypes = [vp]
+        lib.ss_last_device_error.restype = ci
+        _lib = lib
+        return lib
+
+
+def ss_status_string(status: int) -> str:
+    return load_library().ss_status_string(int(status)).decode()
+
+
+def ss_scan_workspace_bytes(batch: int, dim: int, seqlen: int, dstate: int) -> int:
+    n = load_library().ss_scan_workspace_bytes(batch, dim, seqlen, dstate)
+    if n == ctypes.c_size_t(-1).value:
+        raise SSError(SS_ERR_INVALID_ARG, "ss_scan_workspace_bytes")
+    return n
+
+
+def _stream_handle(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def ss_last_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return load_library().ss_last_device_error(_stream_handle(stream, None))
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_dev(name, t, device, dtypes, shape=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.device != device:
+        raise ValueError(f"{name} must be a tensor on {device}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+
+
+def ss_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                y_out=None, last_state_out=None, return_last_state=True,
+                workspace=None, stream=None):
+    """Fused selective-scan forward on the GPU.
+
+    u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; one dtype, float32 or
+    bfloat16.  A: [dim, N] float32; D, delta_bias: [dim] float32 (optional).
+    Returns (y [batch, dim, L] float32, last_state [batch, dim, N] float32 or
+    None).  Output and workspace tensors are allocated with torch when not
+    given; the library itself allocates nothing.
+    """
+    lib = load_library()
+    device = u.device
+    if device.type != "cuda":
+        raise ValueError("ss_scan_fwd runs on CUDA tensors only (no CPU fallback)")
+    if u.dim() != 3 or B.dim() != 3:
+        raise ValueError("u must be [batch, dim, L] and B [batch, N, L]")
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    in_types = (torch.float32, torch.bfloat16)
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _check_dev(name, t, device, in_types, (batch, dim, L))
+    for name, t in (("B", B), ("C", C)):
+        _check_dev(name, t, device, in_types, (batch, N, L))
+    if len({t.dtype for t in (u, delta, B, C, z) if t is not None}) != 1:
+        raise ValueError("u, delta, B, C and z must share one dtype")
+    _check_dev("A", A, device, (torch.float32,), (dim, N))
+    _check_dev("D", D, device, (torch.float32,), (dim,))
+    _check_dev("delta_bias", delta_bias, device, (torch.float32,), (dim,))
+    if y_out is None:
+        y_out = torch.empty((batch, dim, L), dtype=torch.float32, device=device)
+    _check_dev("y_out", y_out, device, (torch.float32,), (batch, dim, L))
+    if last_state_out is None and return_last_state:
+        last_state_out = torch.empty((batch, dim, N), dtype=torch.float32, device=device)
+    _check_dev("last_state_out", last_state_out, device, (torch.float32,), (batch, dim, N))
+    need = ss_scan_workspace_bytes(batch, dim, L, N)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    dt = SS_F32 if u.dtype == torch.float32 else SS_BF16
+    st = lib.ss_scan_fwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                         _ptr(delta_bias), int(bool(softplus)), _ptr(y_out), _ptr(last_state_out),
+                         batch, dim, L, N, dt, _ptr(workspace), ws_bytes,
+                         _stream_handle(stream, device))
+    if st != SS_OK:
+        raise SSError(st, "ss_scan_fwd")
+    return y_out, last_state_out

@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any launch.
+
+Every call below fails host-side validation, so no CUDA call is made; the
+pointers are fake addresses that are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_ss_b200 import build as B
+from selective_state_space_ss_b200 import _native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return N.load_library()
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(ss_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert {"ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string", "ss_last_device_error"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(N.EXPORTED) <= declared
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert N.ss_status_string(s).startswith("SS_")
+    assert "unknown" in N.ss_status_string(99)
+
+
+def _call(lib, **over):
+    a = dict(u=0x10000, delta=0x20000, A=0x30000, B=0x40000, C=0x50000, D=None, z=None,
+             bias=None, sp=1, y=0x60000, h=None, batch=1, dim=1, L=8, N=16, dt=N.SS_F32,
+             ws=None, wsb=0)
+    a.update(over)
+    return lib.ss_scan_fwd(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
+                           a["sp"], a["y"], a["h"], a["batch"], a["dim"], a["L"], a["N"], a["dt"],
+                           a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("field", ["u", "delta", "A", "B", "C", "y"])
+def test_null_required_pointer(lib, field):
+    assert _call(lib, **{field: None}) == N.SS_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over", [dict(batch=0), dict(dim=0), dict(L=0), dict(batch=-1),
+                                  dict(L=1 << 62, dim=1 << 10)])
+def test_bad_sizes(lib, over):
+    assert _call(lib, **over) == N.SS_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("n", [0, 1, 8, 17, 24, 256])
+def test_unsupported_dstate(lib, n):
+    assert _call(lib, N=n) == N.SS_ERR_UNSUPPORTED
+
+
+def test_unsupported_dtype(lib):
+    assert _call(lib, dt=7) == N.SS_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("field,addr,dt", [("u", 0x10002, N.SS_F32), ("B", 0x40001, N.SS_BF16),
+                                           ("A", 0x30002, N.SS_F32), ("y", 0x60002, N.SS_BF16)])
+def test_misaligned(lib, field, addr, dt):
+    assert _call(lib, **{field: addr, "dt": dt}) == N.SS_ERR_INVALID_ARG
+
+
+def test_workspace_query(lib):
+    assert N.ss_scan_workspace_bytes(8, 1536, 2048, 16) >= 0
+    with pytest.raises(N.SSError):
+        N.ss_scan_workspace_bytes(8, 1536, 2048, 17)
+    assert lib.ss_scan_workspace_bytes(0, 1, 1, 16) == ctypes.c_size_t(-1).value
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    x = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError):
+        N.ss_scan_fwd(x, x, torch.zeros(2, 16), torch.zeros(1, 16, 8), torch.zeros(1, 16, 8))
