@@ -12,7 +12,9 @@ import threading
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssscan.so")
+# SSSCAN_LIBRARY may point at another build of the same library (tuning runs).
+_LIB_PATH = os.environ.get("SSSCAN_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libssscan.so")
 _lock = threading.Lock()
 _lib = None
 

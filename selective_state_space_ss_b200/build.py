@@ -33,17 +33,21 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps())
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not stale():
+def build(force: bool = False, ptxas_verbose: bool = False, out: str | None = None,
+          defines=()) -> str:
+    """Compile libssscan.so (or `out`, with extra -D `defines`, for tuning builds)."""
+    target = out or LIB
+    if out is None and not force and not stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = target + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
-           "-shared", "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-o", tmp, *sources()]
+           "-shared", "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-o", tmp,
+           *[f"-D{d}" for d in defines], *sources()]
     if ptxas_verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

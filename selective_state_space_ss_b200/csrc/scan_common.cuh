@@ -38,11 +38,74 @@ template <typename T> __device__ __forceinline__ T zero_elem();
 template <> __device__ __forceinline__ float zero_elem<float>() { return 0.f; }
 template <> __device__ __forceinline__ __nv_bfloat16 zero_elem<__nv_bfloat16>() { return __float2bfloat16_rn(0.f); }
 
-// softplus(x) = log(1 + e^x); above 20 the correction e^-x is below half an
-// fp32 ulp of x, so x itself is returned.
-__device__ __forceinline__ float softplus_f32(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+}  // namespace ssscan
 
-// SiLU(z) = z * sigmoid(z) = z / (1 + e^-z).
-__device__ __forceinline__ float silu_f32(float z) { return z / (1.f + expf(-z)); }
+namespace ssscan {
+
+// ------------------------------------------------------------ mbarrier/TMA ---
+
+// Device error word: a kernel that gives up a bounded wait sets a bit here
+// instead of trapping; ss_last_device_error reads and clears it.  (The library
+// is a single translation unit, so the definition lives in this header.)
+__device__ unsigned int g_error_word = 0;
+constexpr unsigned kErrTmaWait = 1u;     // a TMA completion wait timed out
+constexpr unsigned kErrLookback = 2u;    // an inter-CTA carry wait timed out
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after `limit` polls (each
+// poll may itself suspend for a hardware-chosen time).  Returns false and
+// records kErrTmaWait on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicOr(&g_error_word, kErrTmaWait);
+  return false;
+}
+
+// One 3-D tiled TMA load (no multicast) into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 }  // namespace ssscan

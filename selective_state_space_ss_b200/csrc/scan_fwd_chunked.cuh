@@ -7,23 +7,32 @@
 // memory (the SRAM-resident scan of "Mamba 深度解读报告", sec. 2.4, and the
 // fused discretise/scan/readout kernel of "Mamba 选择性机制", sec. 3.2).
 //
-// Per chunk, with the inputs staged in shared memory by cp.async (double
-// buffered, the next chunk's copy overlaps this chunk's math):
-//   phase 1  per element: Delta = softplus(delta + bias), w = Delta * u,
-//            and B, C widened to fp32 in a [t][state-group] layout;
+// Per chunk, with the inputs staged in shared memory (TMA tiles, double
+// buffered on mbarriers, so the next chunk's copy overlaps this chunk's math):
+//   phase 1  per element: Delta = softplus(delta + bias), w = Delta * u, kept
+//            as float4 of four timesteps; B_t and C_t transposed from their
+//            [n][t] rows into [t][4-state block][B0..B3, C0..C3] in the input
+//            dtype, so one 16-byte load gives a lane four states' B and C;
 //   phase 2  per (channel, state): A_bar = 2^(Delta * A * log2 e),
-//            h = A_bar * h + w * B_t[n], partial readout sum_n C_t[n] h[n],
-//            then a K-lane butterfly that leaves one timestep's full sum per
-//            lane (B_t and C_t are read once per CTA and broadcast to every
-//            channel, the per-token sharing of "从Transformer的痛点 ... Mamba",
-//            sec. 4.2);
-//   phase 3  per element: y = (s + D u) * SiLU(z), coalesced fp32 stores.
+//            h = A_bar * h + w * B_t[n], and the lane's partial readout
+//            sum_n C_t[n] h[n], in packed fp32x2 arithmetic; B_t and C_t are
+//            staged once per CTA and read by every channel (the per-token
+//            sharing of "从Transformer的痛点 ... Mamba", sec. 4.2);
+//   phase 3  per element: s = sum of the K lane partials,
+//            y = (s + D u) * SiLU(z), coalesced fp32 stores.
 // The serial time loop inside a thread is the recurrence itself; the
 // associative operator of "Mamba 选择性机制", sec. 3.1, is not needed here
 // because no thread ever holds a time range whose carry-in is unknown.
+//
+// Shared-memory layouts are chosen so that each quarter-warp (the unit a
+// 16-byte access is serviced in) touches distinct banks.  Rows whose start
+// is not 16-byte aligned (odd L, offset views) take an element-wise load
+// path instead of TMA.
 #pragma once
 
-#include "scan_common.cuh"
+#include <cuda.h>
+
+#include "pointwise.cuh"
 
 namespace ssscan {
 
@@ -40,8 +49,16 @@ struct FwdArgs {
   float* last_state;  // nullable
   int64_t batch, dim, seqlen;
   int softplus;
-  int vec;  // 1: every row starts on a 16-byte boundary and 16-byte copies are used
+  int vec;  // 1: TMA path (16-byte aligned rows); 0: element-wise loads
 };
+
+// TMA descriptors for the five input tiles ([B][D][L] activations with a
+// [1][CH][T] box, [B][N][L] selection parameters with a [1][N][T] box).
+struct FwdMaps {
+  CUtensorMap u, delta, z, B, C;
+};
+
+constexpr uint32_t kTmaSpinLimit = 1u << 24;
 
 template <typename Tin, int N_, int K_, int NWARPS_, int T_>
 struct ChunkedCfg {
@@ -54,227 +71,258 @@ struct ChunkedCfg {
   static constexpr int CPW = 32 / K;      // channels per warp
   static constexpr int CH = NWARPS * CPW; // channels per CTA
   static constexpr int NT = NWARPS * 32;
-  static constexpr int VE = 16 / (int)sizeof(Tin);  // elements per 16-byte vector
-  static constexpr int RS = T + VE;                  // staged row stride (elements)
+  static constexpr int ES = (int)sizeof(Tin);
+  static constexpr int QPR = T / 4;                  // 4-step quads per row
   static constexpr int RAW_ROWS = 3 * CH + 2 * N;    // u, delta, z rows then B, C rows
-  static constexpr int RAW_BYTES = RAW_ROWS * RS * (int)sizeof(Tin);
-  static constexpr int DW_STRIDE = CH + 1;           // float4 per half-row (pads banks)
-  static constexpr int DW_BYTES = (T / 2) * DW_STRIDE * 16;
-  static constexpr int BC_STRIDE = 2 * N + 4;        // floats per timestep
-  static constexpr int BC_BYTES = T * BC_STRIDE * 4;
-  static constexpr int SY_STRIDE = T + 4;            // floats per channel row
-  static constexpr int SY_BYTES = CH * SY_STRIDE * 4;
-  static constexpr int SMEM_BYTES = 2 * RAW_BYTES + DW_BYTES + BC_BYTES + SY_BYTES;
+  static constexpr int ACT_TILE = CH * T * ES;       // one activation tile (bytes)
+  static constexpr int SEL_TILE = N * T * ES;        // one B or C tile (bytes)
+  static constexpr int RAW_BYTES = RAW_ROWS * T * ES;
+  static constexpr int DW_STRIDE = CH + 1;           // float4 per quad row (odd: conflict-free)
+  static constexpr int DW_BYTES = QPR * DW_STRIDE * 16;
+  static constexpr int BC_BLOCK = 8 * ES;            // B0..B3, C0..C3
+  static constexpr int BC_ROW = (N / 4) * BC_BLOCK;  // bytes per timestep
+  static constexpr int BC_BYTES = T * BC_ROW;
+  static constexpr int SY_STRIDE = T + 4;            // floats per (channel, lane) row
+  static constexpr int SY_BYTES = CH * K * SY_STRIDE * 4;
+  static constexpr int OFF_RAW1 = RAW_BYTES;
+  static constexpr int OFF_DWD = 2 * RAW_BYTES;
+  static constexpr int OFF_DWW = OFF_DWD + DW_BYTES;
+  static constexpr int OFF_BC = OFF_DWW + DW_BYTES;
+  static constexpr int OFF_SY = OFF_BC + BC_BYTES;
+  static constexpr int SMEM_USED = OFF_SY + SY_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_USED + 128;  // slack to align the base to 128 bytes
+  static constexpr int ITEMS = CH * QPR;             // (channel, quad) items per chunk
+  static constexpr int ITEMS_PER_THREAD = (ITEMS + NT - 1) / NT;
 
   static_assert(N % K == 0 && 32 % K == 0, "lane split");
-  static_assert(T % 32 == 0, "chunk length");
-  static_assert(G == 1 || G % 2 == 0, "state group");
+  static_assert(G % 4 == 0, "a lane holds whole 4-state blocks");
+  static_assert(T % 8 == 0 && (T * ES) % 16 == 0 && T <= 256 && CH <= 256, "TMA box");
+  static_assert(ACT_TILE % 128 == 0 && SEL_TILE % 128 == 0, "TMA destinations 128-byte aligned");
+  static_assert(DW_BYTES % 16 == 0 && BC_BYTES % 16 == 0, "alignment");
+  static_assert(ITEMS % NT == 0, "whole items per thread");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
+
+// Both halves of a packed bf16 pair as fp32 (exact).
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
 
 // ---------------------------------------------------------------- loads ---
 
 template <class CF>
-__device__ __forceinline__ void load_chunk(const FwdArgs& a, typename CF::Elem* raw,
-                                           int64_t b, int64_t d0, int64_t t0) {
+__device__ __forceinline__ uint32_t chunk_tx_bytes(bool has_z) {
+  return (has_z ? 3 : 2) * CF::ACT_TILE + 2 * CF::SEL_TILE;
+}
+
+// Issue the TMA loads of chunk t0 into one raw stage (one thread).
+template <class CF>
+__device__ __forceinline__ void tma_chunk(const FwdMaps& m, unsigned char* raw, uint64_t* bar,
+                                          int32_t b, int32_t d0, int32_t t0, bool has_z) {
+  fence_proxy_async_smem();
+  mbar_arrive_expect_tx(bar, chunk_tx_bytes<CF>(has_z));
+  tma_load_3d(raw, &m.u, bar, t0, d0, b);
+  tma_load_3d(raw + CF::ACT_TILE, &m.delta, bar, t0, d0, b);
+  if (has_z) tma_load_3d(raw + 2 * CF::ACT_TILE, &m.z, bar, t0, d0, b);
+  tma_load_3d(raw + 3 * CF::ACT_TILE, &m.B, bar, t0, 0, b);
+  tma_load_3d(raw + 3 * CF::ACT_TILE + CF::SEL_TILE, &m.C, bar, t0, 0, b);
+}
+
+// Element-wise fallback for rows that TMA cannot address (all threads).
+template <class CF>
+__device__ __forceinline__ void load_chunk_scalar(const FwdArgs& a, typename CF::Elem* raw,
+                                                  int64_t b, int64_t d0, int64_t t0) {
   using E = typename CF::Elem;
-  const int tid = threadIdx.x;
-  const int64_t L = a.seqlen, D = a.dim;
-  const E* srcs[5] = {static_cast<const E*>(a.u), static_cast<const E*>(a.delta),
-                      static_cast<const E*>(a.z), static_cast<const E*>(a.B),
-                      static_cast<const E*>(a.C)};
-  if (a.vec) {
-    constexpr int VPR = CF::T / CF::VE;
-    for (int i = tid; i < CF::RAW_ROWS * VPR; i += CF::NT) {
-      const int r = i / VPR, v = i - r * VPR;
-      const int64_t t = t0 + (int64_t)v * CF::VE;
-      E* dst = raw + r * CF::RS + v * CF::VE;
-      const E* src = nullptr;
-      if (t < L) {
-        if (r < 3 * CF::CH) {
-          const int which = r / CF::CH, c = r - which * CF::CH;
-          const int64_t d = d0 + c;
-          if (d < D && srcs[which]) src = srcs[which] + ((b * D + d) * L + t);
-        } else {
-          const int rr = r - 3 * CF::CH, which = rr / CF::N, n = rr - which * CF::N;
-          src = srcs[3 + which] + ((b * CF::N + n) * L + t);
-        }
+  const int64_t L = a.seqlen;
+  for (int i = threadIdx.x; i < CF::RAW_ROWS * CF::T; i += CF::NT) {
+    const int r = i / CF::T, tt = i - r * CF::T;
+    const int64_t t = t0 + tt;
+    E val = zero_elem<E>();
+    if (t < L) {
+      if (r < 3 * CF::CH) {
+        const int which = r / CF::CH, c = r - which * CF::CH;
+        const int64_t d = d0 + c;
+        const void* base = which == 0 ? a.u : (which == 1 ? a.delta : a.z);
+        if (d < a.dim && base) val = static_cast<const E*>(base)[(b * a.dim + d) * L + t];
+      } else {
+        const int rr = r - 3 * CF::CH, which = rr / CF::N, n = rr - which * CF::N;
+        val = static_cast<const E*>(which == 0 ? a.B : a.C)[(b * CF::N + n) * L + t];
       }
-      if (src) cp_async16(dst, src);
-      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
-    cp_async_commit();
-  } else {
-    for (int i = tid; i < CF::RAW_ROWS * CF::T; i += CF::NT) {
-      const int r = i / CF::T, tt = i - r * CF::T;
-      const int64_t t = t0 + tt;
-      E val = zero_elem<E>();
-      if (t < L) {
-        if (r < 3 * CF::CH) {
-          const int which = r / CF::CH, c = r - which * CF::CH;
-          const int64_t d = d0 + c;
-          if (d < D && srcs[which]) val = srcs[which][(b * D + d) * L + t];
-        } else {
-          const int rr = r - 3 * CF::CH, which = rr / CF::N, n = rr - which * CF::N;
-          val = srcs[3 + which][(b * CF::N + n) * L + t];
-        }
-      }
-      raw[r * CF::RS + tt] = val;
-    }
+    raw[r * CF::T + tt] = val;
   }
 }
 
 // ------------------------------------------------------------- phase 1 ---
 
-template <class CF>
+template <class CF, bool kFull>
 __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem* raw,
-                                       float4* dw, float* bc, const float* s_bias,
-                                       int64_t d0, int64_t t0) {
+                                       float4* dwD, float4* dwW, unsigned char* bc,
+                                       const float* s_bias, int64_t d0, int64_t t0) {
+  using E = typename CF::Elem;
   const int tid = threadIdx.x;
-  constexpr int QPR = CF::T / 4;
-  const int64_t L = a.seqlen;
-  for (int i = tid; i < CF::CH * QPR; i += CF::NT) {
-    const int c = i / QPR, q = i - c * QPR;
-    const float4 dl = load4_f32(raw + (CF::CH + c) * CF::RS + 4 * q);
-    const float4 uu = load4_f32(raw + c * CF::RS + 4 * q);
+#pragma unroll
+  for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+    const int i = tid + it * CF::NT;
+    const int c = i / CF::QPR, q = i - c * CF::QPR;
+    const float4 dl = load4_f32(raw + (CF::CH + c) * CF::T + 4 * q);
+    const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
     const float bias = s_bias[c];
-    const bool chan_ok = d0 + c < a.dim;
-    float dv[4] = {dl.x, dl.y, dl.z, dl.w};
-    float uv[4] = {uu.x, uu.y, uu.z, uu.w};
+    const float dv[4] = {dl.x, dl.y, dl.z, dl.w};
+    const float uv[4] = {uu.x, uu.y, uu.z, uu.w};
     float delt[4], w[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const bool ok = chan_ok && (t0 + 4 * q + k < L);
       float x = dv[k] + bias;
-      x = a.softplus ? softplus_f32(x) : x;
-      delt[k] = ok ? x : 0.f;  // padding steps: A_bar = 1, B_bar u = 0 (state unchanged)
-      w[k] = delt[k] * uv[k];
+      x = a.softplus ? softplus_fast(x) : x;
+      if constexpr (!kFull) {
+        // padding steps and channels: A_bar = 1, B_bar u = 0 (state unchanged)
+        if (d0 + c >= a.dim || t0 + 4 * q + k >= a.seqlen) x = 0.f;
+      }
+      delt[k] = x;
+      w[k] = x * uv[k];
     }
-    dw[(2 * q) * CF::DW_STRIDE + c] = make_float4(delt[0], w[0], delt[1], w[1]);
-    dw[(2 * q + 1) * CF::DW_STRIDE + c] = make_float4(delt[2], w[2], delt[3], w[3]);
+    dwD[q * CF::DW_STRIDE + c] = make_float4(delt[0], delt[1], delt[2], delt[3]);
+    dwW[q * CF::DW_STRIDE + c] = make_float4(w[0], w[1], w[2], w[3]);
   }
-  // B and C: [n][t] staged rows -> [t][group j][B (G values), C (G values)]
-  for (int i = tid; i < 2 * CF::N * QPR; i += CF::NT) {
-    const int r = i / QPR, q = i - r * QPR;
-    const int which = r / CF::N, n = r - which * CF::N;
-    const float4 v = load4_f32(raw + (3 * CF::CH + r) * CF::RS + 4 * q);
-    const int j = n / CF::G, g = n - j * CF::G;
-    float* col = bc + (4 * q) * CF::BC_STRIDE + j * 2 * CF::G + which * CF::G + g;
-    col[0] = v.x;
-    col[CF::BC_STRIDE] = v.y;
-    col[2 * CF::BC_STRIDE] = v.z;
-    col[3 * CF::BC_STRIDE] = v.w;
+  // B and C rows [n][t] -> [t][n/4][B0..B3, C0..C3]
+  const E* rawB = raw + 3 * CF::CH * CF::T;
+  const E* rawC = rawB + CF::N * CF::T;
+  if constexpr (CF::ES == 2) {
+    constexpr int TP = CF::T / 2;  // timestep pairs (one 32-bit word per row)
+    const uint32_t* B32 = reinterpret_cast<const uint32_t*>(rawB);
+    const uint32_t* C32 = reinterpret_cast<const uint32_t*>(rawC);
+    for (int i = tid; i < (CF::N / 4) * TP; i += CF::NT) {
+      const int nb = i / TP, tp = i - nb * TP;
+      uint32_t bw[4], cw[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        bw[r] = B32[(4 * nb + r) * TP + tp];
+        cw[r] = C32[(4 * nb + r) * TP + tp];
+      }
+      uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + nb * CF::BC_BLOCK);
+      uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + nb * CF::BC_BLOCK);
+      *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(bw[2], bw[3], 0x5410),
+                         __byte_perm(cw[0], cw[1], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
+      *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(bw[2], bw[3], 0x7632),
+                         __byte_perm(cw[0], cw[1], 0x7632), __byte_perm(cw[2], cw[3], 0x7632));
+    }
+  } else {
+    const float* fb = reinterpret_cast<const float*>(rawB);
+    const float* fc = reinterpret_cast<const float*>(rawC);
+    for (int i = tid; i < (CF::N / 4) * CF::T; i += CF::NT) {
+      const int nb = i / CF::T, t = i - nb * CF::T;
+      float4* dst = reinterpret_cast<float4*>(bc + t * CF::BC_ROW + nb * CF::BC_BLOCK);
+      dst[0] = make_float4(fb[(4 * nb) * CF::T + t], fb[(4 * nb + 1) * CF::T + t],
+                           fb[(4 * nb + 2) * CF::T + t], fb[(4 * nb + 3) * CF::T + t]);
+      dst[1] = make_float4(fc[(4 * nb) * CF::T + t], fc[(4 * nb + 1) * CF::T + t],
+                           fc[(4 * nb + 2) * CF::T + t], fc[(4 * nb + 3) * CF::T + t]);
+    }
   }
 }
 
 // ------------------------------------------------------------- phase 2 ---
 
-// Sum the four per-lane partial readouts over the K lanes of a channel and
-// store the full sums for timesteps t..t+3 into the channel's sy row.
-template <int K>
-__device__ __forceinline__ void reduce_store4(float s0, float s1, float s2, float s3,
-                                              float* sy_t, int j) {
-  if constexpr (K == 1) {
-    *reinterpret_cast<float4*>(sy_t) = make_float4(s0, s1, s2, s3);
-  } else if constexpr (K == 2) {
-    const bool hi = j & 1;
-    float k0 = hi ? s2 : s0, k1 = hi ? s3 : s1;
-    const float o0 = hi ? s0 : s2, o1 = hi ? s1 : s3;
-    k0 += __shfl_xor_sync(kFullMask, o0, 1);
-    k1 += __shfl_xor_sync(kFullMask, o1, 1);
-    *reinterpret_cast<float2*>(sy_t + 2 * j) = make_float2(k0, k1);
+// B and C of one 4-state block at one timestep, as fp32 pairs.
+template <class CF>
+__device__ __forceinline__ void bc_block(const unsigned char* p, float2& b01, float2& b23,
+                                         float2& c01, float2& c23) {
+  if constexpr (CF::ES == 2) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    b01 = bf16x2_to_float2(v.x);
+    b23 = bf16x2_to_float2(v.y);
+    c01 = bf16x2_to_float2(v.z);
+    c23 = bf16x2_to_float2(v.w);
   } else {
-#pragma unroll
-    for (int m = K / 2; m >= 4; m /= 2) {
-      s0 += __shfl_xor_sync(kFullMask, s0, m);
-      s1 += __shfl_xor_sync(kFullMask, s1, m);
-      s2 += __shfl_xor_sync(kFullMask, s2, m);
-      s3 += __shfl_xor_sync(kFullMask, s3, m);
-    }
-    const bool b1 = j & 2;
-    float k0 = b1 ? s2 : s0, k1 = b1 ? s3 : s1;
-    const float o0 = b1 ? s0 : s2, o1 = b1 ? s1 : s3;
-    k0 += __shfl_xor_sync(kFullMask, o0, 2);
-    k1 += __shfl_xor_sync(kFullMask, o1, 2);
-    const bool b0 = j & 1;
-    float kk = b0 ? k1 : k0;
-    const float oo = b0 ? k0 : k1;
-    kk += __shfl_xor_sync(kFullMask, oo, 1);
-    if (j < 4) sy_t[j] = kk;
+    const float4 vb = reinterpret_cast<const float4*>(p)[0];
+    const float4 vc = reinterpret_cast<const float4*>(p)[1];
+    b01 = make_float2(vb.x, vb.y);
+    b23 = make_float2(vb.z, vb.w);
+    c01 = make_float2(vc.x, vc.y);
+    c23 = make_float2(vc.z, vc.w);
   }
 }
 
+// The recurrence for this lane's G states over the chunk, two states per
+// packed fp32x2 operation.  Each lane writes its partial readout
+// sum_{n in lane} C_t[n] h_t[n] for four timesteps at a time (one 16-byte
+// store); phase 3 adds the K partials of a channel.  The time loop carries
+// no cross-lane dependency, so the ex2 of later steps can issue while
+// earlier steps' FMA chains drain.
 template <class CF>
-__device__ __forceinline__ void phase2(const float4* dw, const float* bc, float* sy,
-                                       float (&h)[CF::G], const float (&a2)[CF::G],
+__device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
+                                       const unsigned char* bc, float* sy,
+                                       float2 (&h)[CF::G / 2], const float2 (&a2)[CF::G / 2],
                                        int c, int j) {
-  constexpr int G = CF::G;
-  const float* bcj = bc + j * 2 * G;
-  float* syc = sy + c * CF::SY_STRIDE;
-#pragma unroll 1
-  for (int t = 0; t < CF::T; t += 4) {
+  constexpr int NB = CF::G / 4;  // 4-state blocks per lane
+  const unsigned char* bcj = bc + j * NB * CF::BC_BLOCK;
+  float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE;
+#pragma unroll 2
+  for (int q = 0; q < CF::QPR; ++q) {
+    const float4 D4 = dwD[q * CF::DW_STRIDE + c];
+    const float4 W4 = dwW[q * CF::DW_STRIDE + c];
+    const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
+    const float ws[4] = {W4.x, W4.y, W4.z, W4.w};
     float s[4];
 #pragma unroll
-    for (int k2 = 0; k2 < 4; k2 += 2) {
-      const float4 p = dw[((t + k2) >> 1) * CF::DW_STRIDE + c];
+    for (int k = 0; k < 4; ++k) {
+      const unsigned char* row = bcj + (4 * q + k) * CF::BC_ROW;
+      const float2 dl2 = make_float2(dls[k], dls[k]);
+      const float2 w2 = make_float2(ws[k], ws[k]);
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        const float dl = kk ? p.z : p.x;
-        const float w = kk ? p.w : p.y;
-        const float* row = bcj + (t + k2 + kk) * CF::BC_STRIDE;
-        float Bv[G], Cv[G];
-        if constexpr (G % 4 == 0) {
-#pragma unroll
-          for (int g = 0; g < G; g += 4) {
-            const float4 bq = *reinterpret_cast<const float4*>(row + g);
-            const float4 cq = *reinterpret_cast<const float4*>(row + G + g);
-            Bv[g] = bq.x; Bv[g + 1] = bq.y; Bv[g + 2] = bq.z; Bv[g + 3] = bq.w;
-            Cv[g] = cq.x; Cv[g + 1] = cq.y; Cv[g + 2] = cq.z; Cv[g + 3] = cq.w;
-          }
-        } else {
-#pragma unroll
-          for (int g = 0; g < G; ++g) { Bv[g] = row[g]; Cv[g] = row[G + g]; }
-        }
-        float acc = 0.f;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float abar = ex2_approx(dl * a2[g]);
-          h[g] = fmaf(abar, h[g], w * Bv[g]);
-          acc = fmaf(Cv[g], h[g], acc);
-        }
-        s[k2 + kk] = acc;
+      for (int nb = 0; nb < NB; ++nb) {
+        float2 b01, b23, c01, c23;
+        bc_block<CF>(row + nb * CF::BC_BLOCK, b01, b23, c01, c23);
+        const float2 x01 = __fmul2_rn(dl2, a2[2 * nb]);
+        const float2 x23 = __fmul2_rn(dl2, a2[2 * nb + 1]);
+        const float2 e01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+        const float2 e23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+        h[2 * nb] = __ffma2_rn(e01, h[2 * nb], __fmul2_rn(w2, b01));
+        h[2 * nb + 1] = __ffma2_rn(e23, h[2 * nb + 1], __fmul2_rn(w2, b23));
+        acc = __ffma2_rn(c01, h[2 * nb], acc);
+        acc = __ffma2_rn(c23, h[2 * nb + 1], acc);
       }
+      s[k] = acc.x + acc.y;
     }
-    reduce_store4<CF::K>(s[0], s[1], s[2], s[3], syc + t, j);
+    *reinterpret_cast<float4*>(syr + 4 * q) = make_float4(s[0], s[1], s[2], s[3]);
   }
 }
 
 // ------------------------------------------------------------- phase 3 ---
 
-template <class CF>
+template <class CF, bool kFull>
 __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem* raw,
                                        const float* sy, const float* s_D,
                                        int64_t b, int64_t d0, int64_t t0, bool has_z) {
   const int tid = threadIdx.x;
-  constexpr int QPR = CF::T / 4;
   const int64_t L = a.seqlen, D = a.dim;
-  for (int i = tid; i < CF::CH * QPR; i += CF::NT) {
-    const int c = i / QPR, q = i - c * QPR;
+#pragma unroll
+  for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+    const int i = tid + it * CF::NT;
+    const int c = i / CF::QPR, q = i - c * CF::QPR;
     const int64_t d = d0 + c, t = t0 + 4 * q;
-    if (d >= D || t >= L) continue;
-    const float4 s = *reinterpret_cast<const float4*>(sy + c * CF::SY_STRIDE + 4 * q);
-    const float4 uu = load4_f32(raw + c * CF::RS + 4 * q);
+    if constexpr (!kFull) {
+      if (d >= D || t >= L) continue;
+    }
+    float4 s = *reinterpret_cast<const float4*>(sy + (c * CF::K) * CF::SY_STRIDE + 4 * q);
+#pragma unroll
+    for (int jj = 1; jj < CF::K; ++jj) {
+      const float4 o = *reinterpret_cast<const float4*>(sy + (c * CF::K + jj) * CF::SY_STRIDE + 4 * q);
+      s.x += o.x; s.y += o.y; s.z += o.z; s.w += o.w;
+    }
+    const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
     const float Dd = s_D[c];
     float y[4] = {fmaf(Dd, uu.x, s.x), fmaf(Dd, uu.y, s.y), fmaf(Dd, uu.z, s.z), fmaf(Dd, uu.w, s.w)};
     if (has_z) {
-      const float4 zz = load4_f32(raw + (2 * CF::CH + c) * CF::RS + 4 * q);
-      y[0] *= silu_f32(zz.x);
-      y[1] *= silu_f32(zz.y);
-      y[2] *= silu_f32(zz.z);
-      y[3] *= silu_f32(zz.w);
+      const float4 zz = load4_f32(raw + (2 * CF::CH + c) * CF::T + 4 * q);
+      y[0] *= silu_fast(zz.x);
+      y[1] *= silu_fast(zz.y);
+      y[2] *= silu_fast(zz.z);
+      y[3] *= silu_fast(zz.w);
     }
     float* dst = a.y + (b * D + d) * L + t;
-    if (a.vec && t + 3 < L) {
+    if (a.vec && (kFull || t + 3 < L)) {  // 16-byte stores only on aligned rows
       *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
     } else {
 #pragma unroll
@@ -287,68 +335,114 @@ __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem
 // -------------------------------------------------------------- kernel ---
 
 template <class CF>
-__global__ void __launch_bounds__(CF::NT) scan_fwd_chunked_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(CF::NT, 1)
+    scan_fwd_chunked_kernel(const FwdArgs a, const __grid_constant__ FwdMaps maps) {
   using E = typename CF::Elem;
-  extern __shared__ __align__(16) unsigned char smem[];
-  E* raw0 = reinterpret_cast<E*>(smem);
-  E* raw1 = reinterpret_cast<E*>(smem + CF::RAW_BYTES);
-  float4* dw = reinterpret_cast<float4*>(smem + 2 * CF::RAW_BYTES);
-  float* bc = reinterpret_cast<float*>(smem + 2 * CF::RAW_BYTES + CF::DW_BYTES);
-  float* sy = reinterpret_cast<float*>(smem + 2 * CF::RAW_BYTES + CF::DW_BYTES + CF::BC_BYTES);
+  extern __shared__ __align__(128) unsigned char smem_dyn[];
+  // TMA destinations want 128-byte alignment; the dynamic window follows the
+  // static arrays, so align its base explicitly (SMEM_BYTES has the slack).
+  unsigned char* smem = smem_dyn + ((128u - (smem_u32(smem_dyn) & 127u)) & 127u);
+  unsigned char* raw[2] = {smem, smem + CF::OFF_RAW1};
+  float4* dwD = reinterpret_cast<float4*>(smem + CF::OFF_DWD);
+  float4* dwW = reinterpret_cast<float4*>(smem + CF::OFF_DWW);
+  unsigned char* bc = smem + CF::OFF_BC;
+  float* sy = reinterpret_cast<float*>(smem + CF::OFF_SY);
   __shared__ float s_bias[CF::CH], s_D[CF::CH];
+  __shared__ __align__(8) uint64_t bars[2];
 
   const int64_t tiles_per_b = (a.dim + CF::CH - 1) / CF::CH;
   const int64_t b = blockIdx.x / tiles_per_b;
   const int64_t d0 = (blockIdx.x - b * tiles_per_b) * CF::CH;
   const int64_t L = a.seqlen;
   const bool has_z = a.z != nullptr;
+  const bool tma = a.vec != 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = warp * CF::CPW + lane / CF::K;  // this lane's channel within the CTA
   const int j = lane % CF::K;                   // this lane's state group
   const int64_t d = d0 + c;
   const bool chan_ok = d < a.dim;
+  const bool full_tile = d0 + CF::CH <= a.dim;
 
   for (int i = tid; i < CF::CH; i += CF::NT) {
     const int64_t dd = d0 + i;
     s_bias[i] = (dd < a.dim && a.delta_bias) ? a.delta_bias[dd] : 0.f;
     s_D[i] = (dd < a.dim && a.D) ? a.D[dd] : 0.f;
   }
+  if (tma && tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
 
-  float h[CF::G], a2[CF::G];
+  float2 h[CF::G / 2], a2[CF::G / 2];
 #pragma unroll
-  for (int g = 0; g < CF::G; ++g) {
-    h[g] = 0.f;
-    a2[g] = chan_ok ? a.A[d * CF::N + j * CF::G + g] * 1.4426950408889634f : 0.f;
+  for (int g = 0; g < CF::G / 2; ++g) {
+    h[g] = make_float2(0.f, 0.f);
+    a2[g] = chan_ok ? make_float2(a.A[d * CF::N + j * CF::G + 2 * g] * 1.4426950408889634f,
+                                  a.A[d * CF::N + j * CF::G + 2 * g + 1] * 1.4426950408889634f)
+                    : make_float2(0.f, 0.f);
   }
 
   const int64_t nchunks = (L + CF::T - 1) / CF::T;
-  load_chunk<CF>(a, raw0, b, d0, 0);
-  if (nchunks > 1) load_chunk<CF>(a, raw1, b, d0, CF::T);
-  // wait for chunk 0 only: chunk 1's group may stay in flight
-  if (a.vec) {
-    if (nchunks > 1) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-    else cp_async_wait_all();
+  bool ok = true;  // false once a bounded wait has given up (error word set)
+  auto full_chunk = [&](int64_t k) { return full_tile && (k + 1) * CF::T <= L; };
+  auto stage_in = [&](int64_t k) {  // make chunk k resident in raw[k & 1]
+    if (tma) {
+      ok = ok && mbar_wait_bounded(&bars[k & 1], (uint32_t)((k >> 1) & 1), kTmaSpinLimit);
+    } else {
+      load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw[k & 1]), b, d0, k * CF::T);
+    }
+  };
+  auto run_phase1 = [&](int64_t k) {
+    const E* r = reinterpret_cast<const E*>(raw[k & 1]);
+    if (full_chunk(k)) phase1<CF, true>(a, r, dwD, dwW, bc, s_bias, d0, k * CF::T);
+    else phase1<CF, false>(a, r, dwD, dwW, bc, s_bias, d0, k * CF::T);
+  };
+
+  if (tma && tid == 0) {
+    tma_chunk<CF>(maps, raw[0], &bars[0], (int32_t)b, (int32_t)d0, 0, has_z);
+    if (nchunks > 1) tma_chunk<CF>(maps, raw[1], &bars[1], (int32_t)b, (int32_t)d0, CF::T, has_z);
   }
-  __syncthreads();
-  phase1<CF>(a, raw0, dw, bc, s_bias, d0, 0);
+  // On a timed-out wait: wait (bounded) for every copy this CTA still has in
+  // flight, so that none lands in shared memory after the CTA has left.
+  auto drain_and_exit = [&](int64_t first, int64_t last) {
+    if (tma)
+      for (int64_t kk = first; kk <= last && kk < nchunks; ++kk)
+        mbar_wait_bounded(&bars[kk & 1], (uint32_t)((kk >> 1) & 1), kTmaSpinLimit);
+  };
+  stage_in(0);
+  if (!__syncthreads_and(ok)) {
+    drain_and_exit(0, 1);
+    return;
+  }
+  run_phase1(0);
   __syncthreads();
 
   for (int64_t k = 0; k < nchunks; ++k) {
-    E* cur = (k & 1) ? raw1 : raw0;
-    E* nxt = (k & 1) ? raw0 : raw1;
-    phase2<CF>(dw, bc, sy, h, a2, c, j);
-    if (a.vec) cp_async_wait_all();  // chunk k+1 has landed
+    phase2<CF>(dwD, dwW, bc, sy, h, a2, c, j);
+    if (k + 1 < nchunks) stage_in(k + 1);
+    if (!__syncthreads_and(ok)) {
+      drain_and_exit(k + 1, k + 1);
+      return;
+    }
+    const E* cur = reinterpret_cast<const E*>(raw[k & 1]);
+    if (full_chunk(k)) phase3<CF, true>(a, cur, sy, s_D, b, d0, k * CF::T, has_z);
+    else phase3<CF, false>(a, cur, sy, s_D, b, d0, k * CF::T, has_z);
+    if (k + 1 < nchunks) run_phase1(k + 1);
     __syncthreads();
-    phase3<CF>(a, cur, sy, s_D, b, d0, k * CF::T, has_z);
-    if (k + 1 < nchunks) phase1<CF>(a, nxt, dw, bc, s_bias, d0, (k + 1) * CF::T);
-    __syncthreads();
-    if (k + 2 < nchunks) load_chunk<CF>(a, cur, b, d0, (k + 2) * CF::T);
+    if (tma && tid == 0 && k + 2 < nchunks)
+      tma_chunk<CF>(maps, raw[k & 1], &bars[k & 1], (int32_t)b, (int32_t)d0,
+                    (int32_t)((k + 2) * CF::T), has_z);
   }
 
   if (a.last_state && chan_ok) {
     float* dst = a.last_state + ((b * a.dim + d) * CF::N + j * CF::G);
 #pragma unroll
-    for (int g = 0; g < CF::G; ++g) dst[g] = h[g];
+    for (int g = 0; g < CF::G / 2; ++g) {
+      dst[2 * g] = h[g].x;
+      dst[2 * g + 1] = h[g].y;
+    }
   }
 }
 

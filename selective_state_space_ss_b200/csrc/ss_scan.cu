@@ -1,6 +1,7 @@
 // ss_scan.cu -- host side of libssscan.so: argument checks, kernel choice and
 // launch for the C ABI declared in include/ss_scan.h.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <climits>
 #include <cstdint>
@@ -11,16 +12,57 @@
 
 namespace ssscan {
 
-// Device error word: a kernel that gives up a bounded wait ORs in a code;
-// ss_last_device_error reads and clears it.
-__device__ unsigned int g_error_word = 0;
-
 namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (so the library needs no link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    tried = true;
+  }
+  return fn;
+}
+
+// 3-D map over a [batch][rows][L] tensor, box [1][box_rows][box_t], zero fill
+// out of bounds, no swizzle, no multicast.
+bool encode_3d(CUtensorMap* m, const void* ptr, bool bf16, int64_t L, int64_t rows,
+               int64_t batch, int box_t, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t es = bf16 ? 2 : 4;
+  const cuuint64_t dims[3] = {(cuuint64_t)L, (cuuint64_t)rows, (cuuint64_t)batch};
+  const cuuint64_t strides[2] = {(cuuint64_t)L * es, (cuuint64_t)L * (cuuint64_t)rows * es};
+  const cuuint32_t box[3] = {(cuuint32_t)box_t, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+             const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class CF>
-ss_status launch_chunked(const FwdArgs& a, cudaStream_t stream) {
+bool encode_maps(const FwdArgs& a, FwdMaps* m) {
+  const bool bf16 = sizeof(typename CF::Elem) == 2;
+  if (a.seqlen >= INT32_MAX || a.dim >= INT32_MAX || a.batch >= INT32_MAX) return false;
+  bool ok = encode_3d(&m->u, a.u, bf16, a.seqlen, a.dim, a.batch, CF::T, CF::CH) &&
+            encode_3d(&m->delta, a.delta, bf16, a.seqlen, a.dim, a.batch, CF::T, CF::CH) &&
+            encode_3d(&m->z, a.z ? a.z : a.u, bf16, a.seqlen, a.dim, a.batch, CF::T, CF::CH) &&
+            encode_3d(&m->B, a.B, bf16, a.seqlen, CF::N, a.batch, CF::T, CF::N) &&
+            encode_3d(&m->C, a.C, bf16, a.seqlen, CF::N, a.batch, CF::T, CF::N);
+  return ok;
+}
+
+template <class CF>
+ss_status launch_chunked(FwdArgs a, cudaStream_t stream) {
   static bool configured = false;  // one attribute call per instantiation and process
   auto kern = scan_fwd_chunked_kernel<CF>;
   if (!configured) {
@@ -32,15 +74,32 @@ ss_status launch_chunked(const FwdArgs& a, cudaStream_t stream) {
   const int64_t tiles = (a.dim + CF::CH - 1) / CF::CH;
   const int64_t blocks = tiles * a.batch;
   if (blocks > INT_MAX) return SS_ERR_INVALID_ARG;
-  kern<<<(unsigned)blocks, CF::NT, CF::SMEM_BYTES, stream>>>(a);
+  FwdMaps maps;
+  memset(&maps, 0, sizeof maps);
+  if (a.vec && !encode_maps<CF>(a, &maps)) a.vec = 0;  // element-wise loads instead
+  kern<<<(unsigned)blocks, CF::NT, CF::SMEM_BYTES, stream>>>(a, maps);
   return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
+// Launch shapes (lanes per channel K, warps per CTA, chunk length T) per
+// state size; the macros exist so that tuning builds can override them.
+#ifndef SS_N16_K
+#define SS_N16_K 4
+#endif
+#ifndef SS_N16_W
+#define SS_N16_W 4
+#endif
+#ifndef SS_N16_T
+#define SS_N16_T 32
+#endif
+
 template <typename E>
 ss_status dispatch_dtype(const FwdArgs& a, int N, cudaStream_t stream) {
+  // FwdArgs is passed by value so that the launch may switch it to the
+  // element-wise path when a tensor map cannot be encoded.
   switch (N) {
-    case 16: return launch_chunked<ChunkedCfg<E, 16, 4, 4, 64>>(a, stream);
-    case 32: return launch_chunked<ChunkedCfg<E, 32, 4, 4, 64>>(a, stream);
+    case 16: return launch_chunked<ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T>>(a, stream);
+    case 32: return launch_chunked<ChunkedCfg<E, 32, 4, 4, 32>>(a, stream);
     case 64: return launch_chunked<ChunkedCfg<E, 64, 8, 8, 32>>(a, stream);
     case 128: return launch_chunked<ChunkedCfg<E, 128, 8, 8, 32>>(a, stream);
     default: return SS_ERR_UNSUPPORTED;
