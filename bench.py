@@ -37,6 +37,7 @@ L2_BYTES = 126 * 1024 * 1024
 NUM_SMS = 148
 MUFU_EX2_PER_CLK_PER_SM = 16  # ex2 results per clock per SM (special-function unit)
 KERNEL_SOURCES = ("selective_state_space_ss_b200/csrc/ss_scan.cu",
+                  "selective_state_space_ss_b200/csrc/pointwise.cuh",
                   "selective_state_space_ss_b200/csrc/scan_fwd_chunked.cuh",
                   "selective_state_space_ss_b200/csrc/scan_common.cuh")
 

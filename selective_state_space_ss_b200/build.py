@@ -50,6 +50,16 @@ def build(force: bool = False, ptxas_verbose: bool = False, out: str | None = No
     return target
 
 
+def build_probe() -> str:
+    """Compile the standalone issue-rate probe (probe_rates.cu) next to the library."""
+    out = os.path.join(PKG, "probe_rates")
+    src = os.path.join(CSRC, "probe_rates.cu")
+    if not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        subprocess.check_call([NVCC, *ARCH, "-O3", "-o", out, src])
+    return out
+
+
 if __name__ == "__main__":
+    build_probe()
     build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv)
     print(LIB)

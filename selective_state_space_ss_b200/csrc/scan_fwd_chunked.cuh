@@ -80,7 +80,10 @@ struct ChunkedCfg {
   static constexpr int DW_STRIDE = CH + 1;           // float4 per quad row (odd: conflict-free)
   static constexpr int DW_BYTES = QPR * DW_STRIDE * 16;
   static constexpr int BC_BLOCK = 8 * ES;            // B0..B3, C0..C3
-  static constexpr int BC_ROW = (N / 4) * BC_BLOCK;  // bytes per timestep
+  static constexpr int BC_DATA = (N / 4) * BC_BLOCK; // bytes of one timestep
+  // Row pitch: a quarter-warp of the transpose writes rows 2tp and 2tp+2;
+  // a pitch of 32 mod 64 bytes puts them on opposite halves of the banks.
+  static constexpr int BC_ROW = (BC_DATA % 128 == 64) ? BC_DATA + 32 : BC_DATA;
   static constexpr int BC_BYTES = T * BC_ROW;
   static constexpr int SY_STRIDE = T + 4;            // floats per (channel, lane) row
   static constexpr int SY_BYTES = CH * K * SY_STRIDE * 4;
@@ -91,6 +94,9 @@ struct ChunkedCfg {
   static constexpr int OFF_SY = OFF_BC + BC_BYTES;
   static constexpr int SMEM_USED = OFF_SY + SY_BYTES;
   static constexpr int SMEM_BYTES = SMEM_USED + 128;  // slack to align the base to 128 bytes
+  // CTAs per SM the register budget must allow (shared memory permitting)
+  static constexpr int MIN_CTAS = (227 * 1024 / (SMEM_USED + 128 + 1024)) < 5
+                                      ? (227 * 1024 / (SMEM_USED + 128 + 1024)) : 5;
   static constexpr int ITEMS = CH * QPR;             // (channel, quad) items per chunk
   static constexpr int ITEMS_PER_THREAD = (ITEMS + NT - 1) / NT;
 
@@ -192,8 +198,9 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     constexpr int TP = CF::T / 2;  // timestep pairs (one 32-bit word per row)
     const uint32_t* B32 = reinterpret_cast<const uint32_t*>(rawB);
     const uint32_t* C32 = reinterpret_cast<const uint32_t*>(rawC);
-    for (int i = tid; i < (CF::N / 4) * TP; i += CF::NT) {
-      const int nb = i / TP, tp = i - nb * TP;
+    constexpr int NB4 = CF::N / 4;
+    for (int i = tid; i < NB4 * TP; i += CF::NT) {
+      const int tp = i / NB4, nb = i - tp * NB4;
       uint32_t bw[4], cw[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
@@ -335,14 +342,15 @@ __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem
 // -------------------------------------------------------------- kernel ---
 
 template <class CF>
-__global__ void __launch_bounds__(CF::NT, 1)
+__global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     scan_fwd_chunked_kernel(const FwdArgs a, const __grid_constant__ FwdMaps maps) {
   using E = typename CF::Elem;
   extern __shared__ __align__(128) unsigned char smem_dyn[];
   // TMA destinations want 128-byte alignment; the dynamic window follows the
   // static arrays, so align its base explicitly (SMEM_BYTES has the slack).
   unsigned char* smem = smem_dyn + ((128u - (smem_u32(smem_dyn) & 127u)) & 127u);
-  unsigned char* raw[2] = {smem, smem + CF::OFF_RAW1};
+  // stage k & 1 of the raw tiles (pointer arithmetic: no indexed local array)
+  auto raw = [&](int64_t k) { return smem + (k & 1) * CF::OFF_RAW1; };
   float4* dwD = reinterpret_cast<float4*>(smem + CF::OFF_DWD);
   float4* dwW = reinterpret_cast<float4*>(smem + CF::OFF_DWW);
   unsigned char* bc = smem + CF::OFF_BC;
@@ -391,18 +399,18 @@ __global__ void __launch_bounds__(CF::NT, 1)
     if (tma) {
       ok = ok && mbar_wait_bounded(&bars[k & 1], (uint32_t)((k >> 1) & 1), kTmaSpinLimit);
     } else {
-      load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw[k & 1]), b, d0, k * CF::T);
+      load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw(k)), b, d0, k * CF::T);
     }
   };
   auto run_phase1 = [&](int64_t k) {
-    const E* r = reinterpret_cast<const E*>(raw[k & 1]);
+    const E* r = reinterpret_cast<const E*>(raw(k));
     if (full_chunk(k)) phase1<CF, true>(a, r, dwD, dwW, bc, s_bias, d0, k * CF::T);
     else phase1<CF, false>(a, r, dwD, dwW, bc, s_bias, d0, k * CF::T);
   };
 
   if (tma && tid == 0) {
-    tma_chunk<CF>(maps, raw[0], &bars[0], (int32_t)b, (int32_t)d0, 0, has_z);
-    if (nchunks > 1) tma_chunk<CF>(maps, raw[1], &bars[1], (int32_t)b, (int32_t)d0, CF::T, has_z);
+    tma_chunk<CF>(maps, raw(0), &bars[0], (int32_t)b, (int32_t)d0, 0, has_z);
+    if (nchunks > 1) tma_chunk<CF>(maps, raw(1), &bars[1], (int32_t)b, (int32_t)d0, CF::T, has_z);
   }
   // On a timed-out wait: wait (bounded) for every copy this CTA still has in
   // flight, so that none lands in shared memory after the CTA has left.
@@ -426,13 +434,13 @@ __global__ void __launch_bounds__(CF::NT, 1)
       drain_and_exit(k + 1, k + 1);
       return;
     }
-    const E* cur = reinterpret_cast<const E*>(raw[k & 1]);
+    const E* cur = reinterpret_cast<const E*>(raw(k));
     if (full_chunk(k)) phase3<CF, true>(a, cur, sy, s_D, b, d0, k * CF::T, has_z);
     else phase3<CF, false>(a, cur, sy, s_D, b, d0, k * CF::T, has_z);
     if (k + 1 < nchunks) run_phase1(k + 1);
     __syncthreads();
     if (tma && tid == 0 && k + 2 < nchunks)
-      tma_chunk<CF>(maps, raw[k & 1], &bars[k & 1], (int32_t)b, (int32_t)d0,
+      tma_chunk<CF>(maps, raw(k), &bars[k & 1], (int32_t)b, (int32_t)d0,
                     (int32_t)((k + 2) * CF::T), has_z);
   }
 
