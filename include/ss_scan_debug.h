@@ -1,0 +1,46 @@
+/*
+ * ss_scan_debug.h -- test hooks of libssscan.so.  Not for production use.
+ *
+ * Each setting is picked up by the NEXT ss_scan_fwd call in the process and
+ * then cleared (ss_scan_workspace_bytes honours a pending worker count, so a
+ * test can size the workspace for it).  They exist so that tests can drive the
+ * load-balanced schedule and its bounded carry waits on small problems:
+ *
+ *   SS_DEBUG_FORCE_WORKERS  value = number of CTAs that share the work (>= 1;
+ *                           capped at the number of channel groups), so ranges
+ *                           split channel groups and carries are handed over.
+ *   SS_DEBUG_SKIP_PUBLISH   value = worker index whose carry is never published:
+ *                           its successor's bounded wait runs out, the kernel
+ *                           returns without hanging and ss_last_device_error
+ *                           reports SS_ERR_TIMEOUT.  The outputs of that call
+ *                           are then unspecified.
+ *   SS_DEBUG_SPIN_LIMIT     value = polls (with back-off) before a carry wait
+ *                           gives up, so that test finishes quickly.
+ *   SS_DEBUG_CLEAR          value ignored: drop every pending setting.
+ *
+ * Returns SS_OK, or SS_ERR_INVALID_ARG for an unknown `what`.  Host-only,
+ * thread-safe, launches nothing.
+ */
+#ifndef SS_SCAN_DEBUG_H_
+#define SS_SCAN_DEBUG_H_
+
+#include "ss_scan.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  SS_DEBUG_CLEAR = 0,
+  SS_DEBUG_FORCE_WORKERS = 1,
+  SS_DEBUG_SKIP_PUBLISH = 2,
+  SS_DEBUG_SPIN_LIMIT = 3
+};
+
+ss_status ss_debug_inject(int what, long long value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS_SCAN_DEBUG_H_ */

@@ -7,6 +7,10 @@ lazily on the first call, and a missing library raises: there is no CPU path.
 """
 from ._native import (  # noqa: F401
     EXPORTED,
+    SS_DEBUG_CLEAR,
+    SS_DEBUG_FORCE_WORKERS,
+    SS_DEBUG_SKIP_PUBLISH,
+    SS_DEBUG_SPIN_LIMIT,
     SS_BF16,
     SS_ERR_CUDA,
     SS_ERR_INVALID_ARG,
@@ -17,6 +21,7 @@ from ._native import (  # noqa: F401
     SSError,
     library_path,
     load_library,
+    ss_debug_inject,
     ss_last_device_error,
     ss_scan_fwd,
     ss_scan_workspace_bytes,

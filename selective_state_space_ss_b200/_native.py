@@ -22,7 +22,10 @@ SS_OK, SS_ERR_INVALID_ARG, SS_ERR_UNSUPPORTED, SS_ERR_CUDA, SS_ERR_TIMEOUT = ran
 SS_F32, SS_BF16 = 0, 1
 
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
-            "ss_last_device_error")
+            "ss_last_device_error", "ss_debug_inject")
+
+# test hooks (include/ss_scan_debug.h)
+SS_DEBUG_CLEAR, SS_DEBUG_FORCE_WORKERS, SS_DEBUG_SKIP_PUBLISH, SS_DEBUG_SPIN_LIMIT = range(4)
 
 
 class SSError(RuntimeError):
@@ -56,6 +59,8 @@ def load_library():
         lib.ss_status_string.restype = ctypes.c_char_p
         lib.ss_last_device_error.argtypes = [vp]
         lib.ss_last_device_error.restype = ci
+        lib.ss_debug_inject.argtypes = [ci, ctypes.c_longlong]
+        lib.ss_debug_inject.restype = ci
         _lib = lib
         return lib
 
@@ -80,6 +85,13 @@ def _stream_handle(stream, device) -> int:
 def ss_last_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error status."""
     return load_library().ss_last_device_error(_stream_handle(stream, None))
+
+
+def ss_debug_inject(what: int, value: int = 0) -> None:
+    """Test hook for the next ss_scan_fwd call (see include/ss_scan_debug.h)."""
+    st = load_library().ss_debug_inject(int(what), int(value))
+    if st != SS_OK:
+        raise SSError(st, "ss_debug_inject")
 
 
 def _ptr(t):

@@ -164,7 +164,8 @@ __device__ __forceinline__ void load_chunk_scalar(const FwdArgs& a, typename CF:
 template <class CF, bool kFull>
 __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem* raw,
                                        float4* dwD, float4* dwW, unsigned char* bc,
-                                       const float* s_bias, int64_t d0, int64_t t0) {
+                                       const float (&bias_it)[CF::ITEMS_PER_THREAD],
+                                       int64_t d0, int64_t t0) {
   using E = typename CF::Elem;
   const int tid = threadIdx.x;
 #pragma unroll
@@ -173,7 +174,7 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     const int c = i / CF::QPR, q = i - c * CF::QPR;
     const float4 dl = load4_f32(raw + (CF::CH + c) * CF::T + 4 * q);
     const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
-    const float bias = s_bias[c];
+    const float bias = bias_it[it];
     const float dv[4] = {dl.x, dl.y, dl.z, dl.w};
     const float uv[4] = {uu.x, uu.y, uu.z, uu.w};
     float delt[4], w[4];
@@ -300,7 +301,7 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
 
 template <class CF, bool kFull>
 __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem* raw,
-                                       const float* sy, const float* s_D,
+                                       const float* sy, const float (&D_it)[CF::ITEMS_PER_THREAD],
                                        int64_t b, int64_t d0, int64_t t0, bool has_z) {
   const int tid = threadIdx.x;
   const int64_t L = a.seqlen, D = a.dim;
@@ -319,7 +320,7 @@ __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem
       s.x += o.x; s.y += o.y; s.z += o.z; s.w += o.w;
     }
     const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
-    const float Dd = s_D[c];
+    const float Dd = D_it[it];
     float y[4] = {fmaf(Dd, uu.x, s.x), fmaf(Dd, uu.y, s.y), fmaf(Dd, uu.z, s.z), fmaf(Dd, uu.w, s.w)};
     if (has_z) {
       const float4 zz = load4_f32(raw + (2 * CF::CH + c) * CF::T + 4 * q);
@@ -339,118 +340,354 @@ __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem
   }
 }
 
+// ------------------------------------------------------------ schedule ---
+
+// Work is the sequence of (channel group, chunk) units, group-major; worker w
+// (one CTA) owns units [w U / W, (w+1) U / W).  A range can start inside a
+// group (its "suffix" piece needs the state at that chunk from worker w-1)
+// and end inside a group (its "prefix" piece hands its final state to worker
+// w+1).  Each worker runs its prefix piece first (it starts from h = 0 and
+// publishes as early as possible), then its whole groups, then its suffix
+// piece, so the carry it waits for was produced at the very start of its
+// predecessor's run.  The host keeps every range at least one group long, so
+// no piece needs a carry in and hands one out at once.
+struct Sched {
+  int64_t units;        // groups x chunks per group
+  int64_t nk;           // chunks per group
+  int64_t tiles_per_b;  // channel tiles per batch row
+  float* carries;       // [workers][CH * N] published prefix states (nullable)
+  unsigned long long* flags;  // [workers] epoch of the published carry
+  unsigned long long epoch;   // unique per launch, so stale flags never match
+  uint32_t spin_limit;        // polls before a carry wait gives up
+  int skip_publish;           // test hook: this worker never publishes (-1: none)
+};
+
+// Walks one worker's chunk sequence without divisions: the three pieces
+// (prefix, whole groups, suffix) are set up once per CTA; advancing is a few
+// compares.  All fields are uniform across the CTA.
+struct Cursor {
+  int32_t g, c;        // channel group, chunk index within the group
+  int32_t b, tile;     // batch row, channel tile of group g
+  int32_t piece;       // 0 prefix, 1 whole groups, 2 suffix, 3 done
+  int64_t left;        // chunks left in the current piece
+  int64_t len;         // length of the current piece
+  // piece descriptors (same for every cursor of the CTA); scalars, so that
+  // nothing here is indexed at run time
+  int32_t g0, g1, g2, c2;
+  int64_t n0, n1, n2;
+  int32_t nk, tiles;
+
+  __device__ __forceinline__ void seat(int32_t gg, int32_t cc) {
+    g = gg;
+    c = cc;
+    b = gg / tiles;  // only when a piece starts
+    tile = gg - b * tiles;
+  }
+  __device__ __forceinline__ void enter(int32_t p) {
+    if (p == 0 && n0 == 0) p = 1;
+    if (p == 1 && n1 == 0) p = 2;
+    if (p == 2 && n2 == 0) p = 3;
+    piece = p;
+    if (p == 0) { len = n0; seat(g0, 0); }
+    else if (p == 1) { len = n1; seat(g1, 0); }
+    else if (p == 2) { len = n2; seat(g2, c2); }
+    left = len;
+  }
+  __device__ __forceinline__ void init(const Sched& s, int64_t u0, int64_t u1) {
+    nk = (int32_t)s.nk;
+    tiles = (int32_t)s.tiles_per_b;
+    const int64_t gfull0 = (u0 + s.nk - 1) / s.nk;
+    g0 = (int32_t)(u1 / s.nk);  n0 = u1 % s.nk;
+    g1 = (int32_t)gfull0;       n1 = (u1 / s.nk - gfull0) * s.nk;
+    g2 = (int32_t)(u0 / s.nk);  c2 = (int32_t)(u0 % s.nk);
+    n2 = c2 ? s.nk - c2 : 0;
+    enter(0);
+  }
+  __device__ __forceinline__ void advance() {
+    if (--left == 0) {
+      enter(piece + 1);
+      return;
+    }
+    if (++c == nk) {
+      c = 0;
+      ++g;
+      if (++tile == tiles) {
+        tile = 0;
+        ++b;
+      }
+    }
+  }
+  __device__ __forceinline__ bool first() const { return c == 0 || left == len; }
+  __device__ __forceinline__ bool carry_in() const { return piece == 2 && left == len; }
+  __device__ __forceinline__ bool carry_out() const { return piece == 0 && left == 1; }
+  __device__ __forceinline__ bool last() const { return c == nk - 1; }
+};
+
+// Bounded wait for worker `src`'s carry of this launch (one thread).
+__device__ __forceinline__ bool wait_carry(const Sched& s, int src) {
+  const unsigned long long* f = s.flags + src;
+  for (uint32_t i = 0; i < s.spin_limit; ++i) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(f) : "memory");
+    if (v == s.epoch) return true;
+    __nanosleep(i < 64 ? 32 : 256);
+  }
+  atomicOr(&g_error_word, kErrLookback);
+  return false;
+}
+
+__device__ __forceinline__ void publish_carry(const Sched& s, int w) {
+  unsigned long long* f = s.flags + w;
+  asm volatile("st.release.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(s.epoch) : "memory");
+}
+
 // -------------------------------------------------------------- kernel ---
 
-template <class CF>
+// kMulti = false: one channel group per CTA (gridDim = groups), a plain loop
+// over its chunks.  kMulti = true: balanced ranges with carry handoff.
+template <class CF, bool kMulti>
 __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
-    scan_fwd_chunked_kernel(const FwdArgs a, const __grid_constant__ FwdMaps maps) {
+    scan_fwd_chunked_kernel(const FwdArgs a, const __grid_constant__ FwdMaps maps,
+                            const Sched sched) {
   using E = typename CF::Elem;
   extern __shared__ __align__(128) unsigned char smem_dyn[];
   // TMA destinations want 128-byte alignment; the dynamic window follows the
   // static arrays, so align its base explicitly (SMEM_BYTES has the slack).
   unsigned char* smem = smem_dyn + ((128u - (smem_u32(smem_dyn) & 127u)) & 127u);
-  // stage k & 1 of the raw tiles (pointer arithmetic: no indexed local array)
-  auto raw = [&](int64_t k) { return smem + (k & 1) * CF::OFF_RAW1; };
+  // stage j & 1 of the raw tiles (pointer arithmetic: no indexed local array)
+  auto raw = [&](int64_t j) { return smem + (j & 1) * CF::OFF_RAW1; };
   float4* dwD = reinterpret_cast<float4*>(smem + CF::OFF_DWD);
   float4* dwW = reinterpret_cast<float4*>(smem + CF::OFF_DWW);
   unsigned char* bc = smem + CF::OFF_BC;
   float* sy = reinterpret_cast<float*>(smem + CF::OFF_SY);
-  __shared__ float s_bias[CF::CH], s_D[CF::CH];
   __shared__ __align__(8) uint64_t bars[2];
 
-  const int64_t tiles_per_b = (a.dim + CF::CH - 1) / CF::CH;
-  const int64_t b = blockIdx.x / tiles_per_b;
-  const int64_t d0 = (blockIdx.x - b * tiles_per_b) * CF::CH;
+  const int w = blockIdx.x;
+  const int64_t u0 = sched.units * w / gridDim.x;
+  const int64_t u1 = sched.units * (w + 1) / gridDim.x;
+  const int64_t nseq = u1 - u0;
   const int64_t L = a.seqlen;
   const bool has_z = a.z != nullptr;
   const bool tma = a.vec != 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = warp * CF::CPW + lane / CF::K;  // this lane's channel within the CTA
   const int j = lane % CF::K;                   // this lane's state group
-  const int64_t d = d0 + c;
-  const bool chan_ok = d < a.dim;
-  const bool full_tile = d0 + CF::CH <= a.dim;
 
-  for (int i = tid; i < CF::CH; i += CF::NT) {
-    const int64_t dd = d0 + i;
-    s_bias[i] = (dd < a.dim && a.delta_bias) ? a.delta_bias[dd] : 0.f;
-    s_D[i] = (dd < a.dim && a.D) ? a.D[dd] : 0.f;
-  }
   if (tma && tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     fence_mbar_init();
   }
   __syncthreads();
+  if (nseq <= 0) return;
 
-  float2 h[CF::G / 2], a2[CF::G / 2];
+  if constexpr (!kMulti) {
+    // ---- one channel group per CTA: chunk q of group w is unit q ----
+    const int64_t b = w / sched.tiles_per_b;
+    const int64_t d0 = (w - b * sched.tiles_per_b) * CF::CH;
+    const int64_t d = d0 + c;
+    const bool chan_ok = d < a.dim;
+    const bool full_tile = d0 + CF::CH <= a.dim;
+    float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
 #pragma unroll
-  for (int g = 0; g < CF::G / 2; ++g) {
-    h[g] = make_float2(0.f, 0.f);
-    a2[g] = chan_ok ? make_float2(a.A[d * CF::N + j * CF::G + 2 * g] * 1.4426950408889634f,
-                                  a.A[d * CF::N + j * CF::G + 2 * g + 1] * 1.4426950408889634f)
-                    : make_float2(0.f, 0.f);
+    for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+      const int64_t di = d0 + (tid + it * CF::NT) / CF::QPR;
+      bias_it[it] = (a.delta_bias && di < a.dim) ? __ldg(a.delta_bias + di) : 0.f;
+      D_it[it] = (a.D && di < a.dim) ? __ldg(a.D + di) : 0.f;
+    }
+    float2 h[CF::G / 2], a2[CF::G / 2];
+#pragma unroll
+    for (int g = 0; g < CF::G / 2; ++g) {
+      const int n = j * CF::G + 2 * g;
+      h[g] = make_float2(0.f, 0.f);
+      a2[g] = chan_ok ? make_float2(__ldg(a.A + d * CF::N + n) * 1.4426950408889634f,
+                                    __ldg(a.A + d * CF::N + n + 1) * 1.4426950408889634f)
+                      : make_float2(0.f, 0.f);
+    }
+    bool ok = true;
+    auto full_chunk = [&](int64_t k) { return full_tile && (k + 1) * CF::T <= L; };
+    auto stage_in = [&](int64_t k) {
+      if (tma) ok = ok && mbar_wait_bounded(&bars[k & 1], (uint32_t)((k >> 1) & 1), kTmaSpinLimit);
+      else load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw(k)), b, d0, k * CF::T);
+    };
+    auto run_phase1 = [&](int64_t k) {
+      const E* rp = reinterpret_cast<const E*>(raw(k));
+      if (full_chunk(k)) phase1<CF, true>(a, rp, dwD, dwW, bc, bias_it, d0, k * CF::T);
+      else phase1<CF, false>(a, rp, dwD, dwW, bc, bias_it, d0, k * CF::T);
+    };
+    auto drain = [&](int64_t first, int64_t last) {
+      if (tma)
+        for (int64_t kk = first; kk <= last && kk < nseq; ++kk)
+          mbar_wait_bounded(&bars[kk & 1], (uint32_t)((kk >> 1) & 1), kTmaSpinLimit);
+    };
+    if (tma && tid == 0) {
+      tma_chunk<CF>(maps, raw(0), &bars[0], (int32_t)b, (int32_t)d0, 0, has_z);
+      if (nseq > 1) tma_chunk<CF>(maps, raw(1), &bars[1], (int32_t)b, (int32_t)d0, CF::T, has_z);
+    }
+    stage_in(0);
+    if (!__syncthreads_and(ok)) {
+      drain(0, 1);
+      return;
+    }
+    run_phase1(0);
+    __syncthreads();
+    for (int64_t k = 0; k < nseq; ++k) {
+      phase2<CF>(dwD, dwW, bc, sy, h, a2, c, j);
+      if (k + 1 < nseq) stage_in(k + 1);
+      if (!__syncthreads_and(ok)) {
+        drain(k + 1, k + 1);
+        return;
+      }
+      const E* rc = reinterpret_cast<const E*>(raw(k));
+      if (full_chunk(k)) phase3<CF, true>(a, rc, sy, D_it, b, d0, k * CF::T, has_z);
+      else phase3<CF, false>(a, rc, sy, D_it, b, d0, k * CF::T, has_z);
+      if (k + 1 < nseq) run_phase1(k + 1);
+      __syncthreads();
+      if (tma && tid == 0 && k + 2 < nseq)
+        tma_chunk<CF>(maps, raw(k), &bars[k & 1], (int32_t)b, (int32_t)d0,
+                      (int32_t)((k + 2) * CF::T), has_z);
+    }
+    if (a.last_state && chan_ok) {
+      float* dst = a.last_state + ((b * a.dim + d) * CF::N + j * CF::G);
+#pragma unroll
+      for (int g = 0; g < CF::G / 2; ++g) {
+        dst[2 * g] = h[g].x;
+        dst[2 * g + 1] = h[g].y;
+      }
+    }
+    return;
   }
 
-  const int64_t nchunks = (L + CF::T - 1) / CF::T;
+  // three cursors over the same sequence: the chunk in the recurrence (cur),
+  // the one being prepared (prep, one ahead) and the one being fetched (fetch)
+  Cursor cur, prep, fetch;
+  cur.init(sched, u0, u1);
+  prep = cur;
+  fetch = cur;
+
+  float2 h[CF::G / 2], a2[CF::G / 2];
+  float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
+  int32_t bias_g = -1, D_g = -1;  // group whose bias / D are cached
   bool ok = true;  // false once a bounded wait has given up (error word set)
-  auto full_chunk = [&](int64_t k) { return full_tile && (k + 1) * CF::T <= L; };
-  auto stage_in = [&](int64_t k) {  // make chunk k resident in raw[k & 1]
+
+  auto d0_of = [&](const Cursor& r) { return (int64_t)r.tile * CF::CH; };
+  auto full_chunk = [&](const Cursor& r) {
+    return d0_of(r) + CF::CH <= a.dim && ((int64_t)r.c + 1) * CF::T <= L;
+  };
+  auto issue = [&](int64_t jj) {  // one thread: TMA loads of sequence chunk jj (= fetch)
+    tma_chunk<CF>(maps, raw(jj), &bars[jj & 1], fetch.b, (int32_t)d0_of(fetch), fetch.c * CF::T,
+                  has_z);
+  };
+  auto stage_in = [&](int64_t jj, const Cursor& r) {  // make chunk jj resident in raw(jj)
     if (tma) {
-      ok = ok && mbar_wait_bounded(&bars[k & 1], (uint32_t)((k >> 1) & 1), kTmaSpinLimit);
+      ok = ok && mbar_wait_bounded(&bars[jj & 1], (uint32_t)((jj >> 1) & 1), kTmaSpinLimit);
     } else {
-      load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw(k)), b, d0, k * CF::T);
+      load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw(jj)), r.b, d0_of(r), (int64_t)r.c * CF::T);
     }
   };
-  auto run_phase1 = [&](int64_t k) {
-    const E* r = reinterpret_cast<const E*>(raw(k));
-    if (full_chunk(k)) phase1<CF, true>(a, r, dwD, dwW, bc, s_bias, d0, k * CF::T);
-    else phase1<CF, false>(a, r, dwD, dwW, bc, s_bias, d0, k * CF::T);
+  auto load_items = [&](const float* src, const Cursor& r, float (&dst)[CF::ITEMS_PER_THREAD]) {
+#pragma unroll
+    for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+      const int64_t d = d0_of(r) + (tid + it * CF::NT) / CF::QPR;
+      dst[it] = (src && d < a.dim) ? __ldg(src + d) : 0.f;
+    }
+  };
+  auto run_phase1 = [&](int64_t jj) {  // jj = prep's chunk
+    if (prep.g != bias_g) {
+      load_items(a.delta_bias, prep, bias_it);
+      bias_g = prep.g;
+    }
+    const E* rp = reinterpret_cast<const E*>(raw(jj));
+    if (full_chunk(prep)) phase1<CF, true>(a, rp, dwD, dwW, bc, bias_it, d0_of(prep), (int64_t)prep.c * CF::T);
+    else phase1<CF, false>(a, rp, dwD, dwW, bc, bias_it, d0_of(prep), (int64_t)prep.c * CF::T);
+  };
+  // On a timed-out wait: wait (bounded) for every copy this CTA still has in
+  // flight, so that none lands in shared memory after the CTA has left.
+  auto drain = [&](int64_t first, int64_t last) {
+    if (tma)
+      for (int64_t kk = first; kk <= last && kk < nseq; ++kk)
+        mbar_wait_bounded(&bars[kk & 1], (uint32_t)((kk >> 1) & 1), kTmaSpinLimit);
   };
 
   if (tma && tid == 0) {
-    tma_chunk<CF>(maps, raw(0), &bars[0], (int32_t)b, (int32_t)d0, 0, has_z);
-    if (nchunks > 1) tma_chunk<CF>(maps, raw(1), &bars[1], (int32_t)b, (int32_t)d0, CF::T, has_z);
+    issue(0);
+    fetch.advance();
+    if (nseq > 1) {
+      issue(1);
+      fetch.advance();
+    }
   }
-  // On a timed-out wait: wait (bounded) for every copy this CTA still has in
-  // flight, so that none lands in shared memory after the CTA has left.
-  auto drain_and_exit = [&](int64_t first, int64_t last) {
-    if (tma)
-      for (int64_t kk = first; kk <= last && kk < nchunks; ++kk)
-        mbar_wait_bounded(&bars[kk & 1], (uint32_t)((kk >> 1) & 1), kTmaSpinLimit);
-  };
-  stage_in(0);
+  stage_in(0, prep);
   if (!__syncthreads_and(ok)) {
-    drain_and_exit(0, 1);
+    drain(0, 1);
     return;
   }
   run_phase1(0);
+  prep.advance();
   __syncthreads();
 
-  for (int64_t k = 0; k < nchunks; ++k) {
+  for (int64_t q = 0; q < nseq; ++q) {
+    const int64_t d0 = d0_of(cur), d = d0 + c;
+    const bool chan_ok = d < a.dim;
+    if (cur.first()) {
+      // a new piece: this lane's A values, and h from 0 or the predecessor's carry
+      bool have = true;
+      const bool cin_here = cur.carry_in();
+      if (cin_here) {
+        if (tid == 0) have = wait_carry(sched, w - 1);
+        have = __syncthreads_and(have);  // also orders the carry reads after the wait
+      }
+      const float* cin = have && cin_here ? sched.carries + (int64_t)(w - 1) * CF::CH * CF::N : nullptr;
+#pragma unroll
+      for (int g = 0; g < CF::G / 2; ++g) {
+        const int n = j * CF::G + 2 * g;
+        a2[g] = chan_ok ? make_float2(__ldg(a.A + d * CF::N + n) * 1.4426950408889634f,
+                                      __ldg(a.A + d * CF::N + n + 1) * 1.4426950408889634f)
+                        : make_float2(0.f, 0.f);
+        h[g] = cin ? make_float2(__ldcg(cin + c * CF::N + n), __ldcg(cin + c * CF::N + n + 1))
+                   : make_float2(0.f, 0.f);
+      }
+      ok = ok && have;
+    }
     phase2<CF>(dwD, dwW, bc, sy, h, a2, c, j);
-    if (k + 1 < nchunks) stage_in(k + 1);
+    const bool cout_here = cur.carry_out();
+    if (cout_here) {
+      float* dst = sched.carries + (int64_t)w * CF::CH * CF::N + c * CF::N + j * CF::G;
+#pragma unroll
+      for (int g = 0; g < CF::G / 2; ++g) __stcg(reinterpret_cast<float2*>(dst) + g, h[g]);
+      __threadfence();
+    }
+    if (cur.last() && a.last_state && chan_ok) {
+      float* dst = a.last_state + (((int64_t)cur.b * a.dim + d) * CF::N + j * CF::G);
+#pragma unroll
+      for (int g = 0; g < CF::G / 2; ++g) {
+        dst[2 * g] = h[g].x;
+        dst[2 * g + 1] = h[g].y;
+      }
+    }
+    if (q + 1 < nseq) stage_in(q + 1, prep);
     if (!__syncthreads_and(ok)) {
-      drain_and_exit(k + 1, k + 1);
+      drain(q + 1, q + 1);
       return;
     }
-    const E* cur = reinterpret_cast<const E*>(raw(k));
-    if (full_chunk(k)) phase3<CF, true>(a, cur, sy, s_D, b, d0, k * CF::T, has_z);
-    else phase3<CF, false>(a, cur, sy, s_D, b, d0, k * CF::T, has_z);
-    if (k + 1 < nchunks) run_phase1(k + 1);
-    __syncthreads();
-    if (tma && tid == 0 && k + 2 < nchunks)
-      tma_chunk<CF>(maps, raw(k), &bars[k & 1], (int32_t)b, (int32_t)d0,
-                    (int32_t)((k + 2) * CF::T), has_z);
-  }
-
-  if (a.last_state && chan_ok) {
-    float* dst = a.last_state + ((b * a.dim + d) * CF::N + j * CF::G);
-#pragma unroll
-    for (int g = 0; g < CF::G / 2; ++g) {
-      dst[2 * g] = h[g].x;
-      dst[2 * g + 1] = h[g].y;
+    if (cout_here && tid == 0 && w != sched.skip_publish) publish_carry(sched, w);
+    if (cur.g != D_g) {
+      load_items(a.D, cur, D_it);
+      D_g = cur.g;
     }
+    const E* rc = reinterpret_cast<const E*>(raw(q));
+    if (full_chunk(cur)) phase3<CF, true>(a, rc, sy, D_it, cur.b, d0, (int64_t)cur.c * CF::T, has_z);
+    else phase3<CF, false>(a, rc, sy, D_it, cur.b, d0, (int64_t)cur.c * CF::T, has_z);
+    if (q + 1 < nseq) {
+      run_phase1(q + 1);
+      prep.advance();
+    }
+    __syncthreads();
+    if (tma && tid == 0 && q + 2 < nseq) {
+      issue(q + 2);
+      fetch.advance();
+    }
+    cur.advance();
   }
 }
 

@@ -3,11 +3,14 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+#include <chrono>
 #include <climits>
 #include <cstdint>
 #include <cstring>
 
 #include "ss_scan.h"
+#include "ss_scan_debug.h"
 #include "scan_fwd_chunked.cuh"
 
 namespace ssscan {
@@ -61,23 +64,116 @@ bool encode_maps(const FwdArgs& a, FwdMaps* m) {
   return ok;
 }
 
+// Test hooks (ss_scan_debug.h): consumed by the next ss_scan_fwd call.
+std::atomic<long long> g_dbg_workers{0};
+std::atomic<long long> g_dbg_skip_publish{-1};
+std::atomic<long long> g_dbg_spin_limit{0};
+
+constexpr uint32_t kCarrySpinLimit = 1u << 22;  // ~1 s of polling with back-off
+
+// A launch-unique 64-bit epoch: carry flags written by earlier launches (or
+// arbitrary bytes in a fresh workspace) never equal it.
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> ctr{
+      (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() *
+      0x9E3779B97F4A7C15ULL};
+  return ctr.fetch_add(0x9E3779B97F4A7C15ULL) | 1ULL;
+}
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// How the work is cut: `workers` CTAs, each an equal contiguous range of
+// (channel group, chunk) units.  workers == groups means one group per CTA and
+// no carries; fewer workers balance the load across SMs with carry handoff.
+struct Plan {
+  int workers = 0;
+  int64_t groups = 0, nk = 0, tiles = 0;
+  size_t carry_bytes = 0, ws_bytes = 0;
+};
+
 template <class CF>
-ss_status launch_chunked(FwdArgs a, cudaStream_t stream) {
-  static bool configured = false;  // one attribute call per instantiation and process
-  auto kern = scan_fwd_chunked_kernel<CF>;
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) !=
-        cudaSuccess)
-      return SS_ERR_CUDA;
-    configured = true;
+bool configure_kernel() {
+  static int state = 0;  // 0 unknown, 1 ok, -1 failed
+  if (state == 0)
+    state = (cudaFuncSetAttribute(scan_fwd_chunked_kernel<CF, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) ==
+                 cudaSuccess &&
+             cudaFuncSetAttribute(scan_fwd_chunked_kernel<CF, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) ==
+                 cudaSuccess)
+                ? 1
+                : -1;
+  return state == 1;
+}
+
+template <class CF>
+bool make_plan(int64_t batch, int64_t dim, int64_t seqlen, Plan* p) {
+  if (!configure_kernel<CF>()) return false;
+  p->tiles = (dim + CF::CH - 1) / CF::CH;
+  p->groups = batch * p->tiles;
+  p->nk = (seqlen + CF::T - 1) / CF::T;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_fwd_chunked_kernel<CF, true>, CF::NT,
+                                                    CF::SMEM_BYTES) != cudaSuccess || occ < 1)
+    return false;
+  const int64_t sms = device_sms();
+  if (sms < 1) return false;
+  // One group per CTA (the plain loop) unless the work is between one and two
+  // waves of CTAs with the second at most half full: then one persistent CTA
+  // per resident slot, with balanced ranges and carry handoff, instead of a
+  // nearly empty extra round.  (Measured: the balanced loop costs ~7 % per
+  // chunk in bookkeeping; at 2-3 CTAs per SM fewer, balanced workers lose more
+  // in occupancy than the tail costs; over several waves the block scheduler
+  // already spreads the tail.)
+  const int64_t slots = sms * occ;
+  int64_t w = p->groups;
+  if (p->groups > slots && p->groups < 2 * slots && 2 * (p->groups - slots) <= slots) w = slots;
+  const long long forced = g_dbg_workers.load();
+  if (forced > 0) w = forced < p->groups ? forced : p->groups;
+  if (w > INT_MAX || p->groups > INT32_MAX || p->nk > INT32_MAX) return false;
+  p->workers = (int)w;
+  if (p->workers < p->groups) {
+    p->carry_bytes = align256((size_t)p->workers * CF::CH * CF::N * sizeof(float));
+    p->ws_bytes = p->carry_bytes + align256((size_t)p->workers * sizeof(unsigned long long));
   }
-  const int64_t tiles = (a.dim + CF::CH - 1) / CF::CH;
-  const int64_t blocks = tiles * a.batch;
-  if (blocks > INT_MAX) return SS_ERR_INVALID_ARG;
+  return true;
+}
+
+template <class CF>
+ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
+  Plan p;
+  if (!make_plan<CF>(a.batch, a.dim, a.seqlen, &p)) return SS_ERR_CUDA;
+  if (p.ws_bytes > 0 && (!workspace || workspace_bytes < p.ws_bytes ||
+                         !aligned(workspace, 256)))
+    return SS_ERR_INVALID_ARG;
   FwdMaps maps;
   memset(&maps, 0, sizeof maps);
   if (a.vec && !encode_maps<CF>(a, &maps)) a.vec = 0;  // element-wise loads instead
-  kern<<<(unsigned)blocks, CF::NT, CF::SMEM_BYTES, stream>>>(a, maps);
+  Sched sc;
+  sc.units = p.groups * p.nk;
+  sc.nk = p.nk;
+  sc.tiles_per_b = p.tiles;
+  sc.carries = p.ws_bytes ? static_cast<float*>(workspace) : nullptr;
+  sc.flags = p.ws_bytes ? reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) +
+                                                                 p.carry_bytes)
+                        : nullptr;
+  sc.epoch = next_epoch();
+  const long long spin = g_dbg_spin_limit.exchange(0);
+  sc.spin_limit = spin > 0 ? (uint32_t)spin : kCarrySpinLimit;
+  sc.skip_publish = (int)g_dbg_skip_publish.exchange(-1);
+  g_dbg_workers.store(0);
+  if (p.workers == p.groups)
+    scan_fwd_chunked_kernel<CF, false><<<(unsigned)p.workers, CF::NT, CF::SMEM_BYTES, stream>>>(a, maps, sc);
+  else
+    scan_fwd_chunked_kernel<CF, true><<<(unsigned)p.workers, CF::NT, CF::SMEM_BYTES, stream>>>(a, maps, sc);
   return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
@@ -94,16 +190,37 @@ ss_status launch_chunked(FwdArgs a, cudaStream_t stream) {
 #endif
 
 template <typename E>
-ss_status dispatch_dtype(const FwdArgs& a, int N, cudaStream_t stream) {
-  // FwdArgs is passed by value so that the launch may switch it to the
-  // element-wise path when a tensor map cannot be encoded.
+using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T>;
+template <typename E>
+using Cfg32 = ChunkedCfg<E, 32, 4, 4, 32>;
+template <typename E>
+using Cfg64 = ChunkedCfg<E, 64, 8, 8, 32>;
+template <typename E>
+using Cfg128 = ChunkedCfg<E, 128, 8, 8, 32>;
+
+template <typename E>
+ss_status dispatch_dtype(const FwdArgs& a, int N, void* ws, size_t wsb, cudaStream_t stream) {
   switch (N) {
-    case 16: return launch_chunked<ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T>>(a, stream);
-    case 32: return launch_chunked<ChunkedCfg<E, 32, 4, 4, 32>>(a, stream);
-    case 64: return launch_chunked<ChunkedCfg<E, 64, 8, 8, 32>>(a, stream);
-    case 128: return launch_chunked<ChunkedCfg<E, 128, 8, 8, 32>>(a, stream);
+    case 16: return launch_chunked<Cfg16<E>>(a, ws, wsb, stream);
+    case 32: return launch_chunked<Cfg32<E>>(a, ws, wsb, stream);
+    case 64: return launch_chunked<Cfg64<E>>(a, ws, wsb, stream);
+    case 128: return launch_chunked<Cfg128<E>>(a, ws, wsb, stream);
     default: return SS_ERR_UNSUPPORTED;
   }
+}
+
+template <typename E>
+bool plan_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N, size_t* bytes) {
+  Plan p;
+  bool ok = false;
+  switch (N) {
+    case 16: ok = make_plan<Cfg16<E>>(batch, dim, seqlen, &p); break;
+    case 32: ok = make_plan<Cfg32<E>>(batch, dim, seqlen, &p); break;
+    case 64: ok = make_plan<Cfg64<E>>(batch, dim, seqlen, &p); break;
+    case 128: ok = make_plan<Cfg128<E>>(batch, dim, seqlen, &p); break;
+  }
+  *bytes = p.ws_bytes;
+  return ok;
 }
 
 bool supported_dstate(int n) { return n == 16 || n == 32 || n == 64 || n == 128; }
@@ -135,10 +252,6 @@ ss_status ss_scan_fwd(const void* u, const void* delta, const float* A, const vo
   const void* f_ptrs[5] = {A, D, delta_bias, y_out, last_state_out};
   for (const void* p : f_ptrs)
     if (p && !aligned(p, 4)) return SS_ERR_INVALID_ARG;
-  const size_t need = ss_scan_workspace_bytes(batch, dim, seqlen, dstate);
-  if (need == (size_t)-1) return SS_ERR_INVALID_ARG;
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
-    return SS_ERR_INVALID_ARG;
 
   FwdArgs a;
   a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
@@ -152,13 +265,33 @@ ss_status ss_scan_fwd(const void* u, const void* delta, const float* A, const vo
   if (!aligned(y_out, 16)) vec = false;
   a.vec = vec ? 1 : 0;
 
-  if (in_dtype == SS_F32) return dispatch_dtype<float>(a, dstate, stream);
-  return dispatch_dtype<__nv_bfloat16>(a, dstate, stream);
+  if (in_dtype == SS_F32) return dispatch_dtype<float>(a, dstate, workspace, workspace_bytes, stream);
+  return dispatch_dtype<__nv_bfloat16>(a, dstate, workspace, workspace_bytes, stream);
 }
 
 size_t ss_scan_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int dstate) {
   if (batch < 1 || dim < 1 || seqlen < 1 || !supported_dstate(dstate)) return (size_t)-1;
-  return 0;
+  if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
+    return (size_t)-1;
+  size_t f32 = 0, bf16 = 0;  // enough for either input dtype
+  if (!plan_bytes<float>(batch, dim, seqlen, dstate, &f32) ||
+      !plan_bytes<__nv_bfloat16>(batch, dim, seqlen, dstate, &bf16))
+    return (size_t)-1;
+  return f32 > bf16 ? f32 : bf16;
+}
+
+ss_status ss_debug_inject(int what, long long value) {
+  switch (what) {
+    case SS_DEBUG_FORCE_WORKERS: g_dbg_workers.store(value); return SS_OK;
+    case SS_DEBUG_SKIP_PUBLISH: g_dbg_skip_publish.store(value); return SS_OK;
+    case SS_DEBUG_SPIN_LIMIT: g_dbg_spin_limit.store(value); return SS_OK;
+    case SS_DEBUG_CLEAR:
+      g_dbg_workers.store(0);
+      g_dbg_skip_publish.store(-1);
+      g_dbg_spin_limit.store(0);
+      return SS_OK;
+  }
+  return SS_ERR_INVALID_ARG;
 }
 
 const char* ss_status_string(ss_status s) {

@@ -40,6 +40,11 @@ def test_exports_every_declared_symbol(lib):
     assert set(N.EXPORTED) <= declared
 
 
+def test_debug_inject_rejects_unknown_code(lib):
+    assert lib.ss_debug_inject(99, 0) == N.SS_ERR_INVALID_ARG
+    assert lib.ss_debug_inject(N.SS_DEBUG_CLEAR, 0) == N.SS_OK
+
+
 def test_status_strings(lib):
     for s in range(5):
         assert N.ss_status_string(s).startswith("SS_")
@@ -82,11 +87,12 @@ def test_misaligned(lib, field, addr, dt):
     assert _call(lib, **{field: addr, "dt": dt}) == N.SS_ERR_INVALID_ARG
 
 
-def test_workspace_query(lib):
-    assert N.ss_scan_workspace_bytes(8, 1536, 2048, 16) >= 0
+def test_workspace_query_rejects_bad_sizes(lib):
+    # (valid sizes need the device's SM count, so they are covered by the GPU tests)
     with pytest.raises(N.SSError):
         N.ss_scan_workspace_bytes(8, 1536, 2048, 17)
     assert lib.ss_scan_workspace_bytes(0, 1, 1, 16) == ctypes.c_size_t(-1).value
+    assert lib.ss_scan_workspace_bytes(1, 1, 0, 16) == ctypes.c_size_t(-1).value
 
 
 def test_binding_refuses_cpu_tensors():

@@ -1,0 +1,80 @@
+"""The load-balanced schedule: CTAs own equal ranges of (channel group, chunk)
+units, split groups hand their state to the next CTA through the workspace, and
+those waits are bounded.  Forced worker counts exercise the handoff on small
+shapes; a skipped publish exercises the timeout path (no hang, no fault: the
+kernel gives up, reports SS_ERR_TIMEOUT and the next call is correct)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle  # noqa: E402
+import selective_state_space_ss_b200 as ss  # noqa: E402
+from selective_state_space_ss_b200 import inputs as I  # noqa: E402
+from tests.helpers import TOL, rel_err, run_gpu, to_device  # noqa: E402
+
+
+def _check(w, x, y, h):
+    yr, hr = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                             x["delta_bias"], softplus=w.softplus)
+    assert rel_err(y.cpu().numpy(), yr) <= TOL[w.dtype]
+    assert rel_err(h.cpu().numpy(), hr) <= TOL[w.dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [16, 32, 64, 128])
+@pytest.mark.parametrize("L,workers", [(1000, 3), (4097, 5), (256, 7), (33, 2), (8, 4)])
+def test_forced_split_parity(dtype, N, L, workers):
+    # 5 batch rows x 40 channels: several channel groups per row, a partial
+    # last group, ranges that start and end inside groups
+    w = I.Workload(f"split_{dtype}_{N}_{L}", 5, 40, L, N, dtype)
+    x = I.make_inputs(w, seed=L + N)
+    xd = to_device(x)
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, workers)
+    need = ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    y, h = run_gpu(xd, workspace=ws)
+    assert ss.ss_last_device_error() == ss.SS_OK
+    _check(w, x, y, h)
+
+
+def test_split_workspace_is_reused_across_calls():
+    w = I.Workload("reuse", 4, 64, 700, 16, "bf16")
+    x = I.make_inputs(w, seed=11)
+    xd = to_device(x)
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 3)
+    ws = torch.full((ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate),), 0xAB,
+                    dtype=torch.uint8, device="cuda")
+    for _ in range(3):  # stale flags from earlier calls must never be taken as fresh
+        ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 3)
+        y, h = run_gpu(xd, workspace=ws)
+        assert ss.ss_last_device_error() == ss.SS_OK
+        _check(w, x, y, h)
+
+
+def test_carry_wait_times_out_cleanly():
+    w = I.Workload("timeout", 4, 64, 512, 16, "bf16")
+    x = I.make_inputs(w, seed=12)
+    xd = to_device(x)
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 3)
+    ws = torch.empty(ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate),
+                     dtype=torch.uint8, device="cuda")
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 3)
+    ss.ss_debug_inject(ss.SS_DEBUG_SKIP_PUBLISH, 1)   # worker 2 waits for a carry that never comes
+    ss.ss_debug_inject(ss.SS_DEBUG_SPIN_LIMIT, 2000)
+    run_gpu(xd, workspace=ws)
+    assert ss.ss_last_device_error() == ss.SS_ERR_TIMEOUT
+    assert ss.ss_last_device_error() == ss.SS_OK  # read-and-clear
+    # the context is intact and the next call is right
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 3)
+    y, h = run_gpu(xd, workspace=ws)
+    assert ss.ss_last_device_error() == ss.SS_OK
+    _check(w, x, y, h)
+
+
+def test_debug_hooks_clear():
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 2)
+    ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
+    w = I.Workload("clear", 1, 8, 64, 16, "f32")
+    assert ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate) == 0
