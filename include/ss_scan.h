@@ -20,9 +20,10 @@
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers, caller-owned, contiguous, with
  *    the fastest axis last as written ([B,D,L] means L fastest).
- *  - The library never allocates device memory, never synchronises the
- *    stream (except ss_last_device_error) and keeps no state beyond one
- *    device-side error word per device.
+ *  - The library never allocates device memory at run time, never
+ *    synchronises the stream (except ss_last_device_error) and keeps no state
+ *    beyond one device-side error word per device (and the static scratch
+ *    array of ss_scan_fwd_noalloc, part of the loaded module).
  *  - Calls are asynchronous on `stream` (0 = the legacy default stream).
  *  - Arguments are checked on the host before any launch; a rejected call
  *    launches nothing and touches no buffer.
@@ -42,7 +43,8 @@ extern "C" {
 typedef enum {
   SS_OK = 0,
   SS_ERR_INVALID_ARG = 1, /* null required pointer, bad size, bad alignment, workspace too small */
-  SS_ERR_UNSUPPORTED = 2, /* dstate not in {16, 32, 64, 128}, or unknown dtype */
+  SS_ERR_UNSUPPORTED = 2, /* dstate not in {16, 32, 64, 128}, unknown dtype, or more
+                             scratch than ss_scan_fwd_noalloc holds */
   SS_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
   SS_ERR_TIMEOUT = 4      /* a bounded inter-block wait gave up (see ss_last_device_error) */
 } ss_status;
@@ -82,6 +84,44 @@ ss_status ss_scan_fwd(const void* u, const void* delta, const float* A,
                       int64_t batch, int64_t dim, int64_t seqlen, int dstate,
                       ss_dtype in_dtype, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * ss_scan_fwd_noalloc -- ss_scan_fwd for callers that cannot allocate device
+ * memory at the point of the call: for example a plugin running inside a host
+ * framework that owns every device allocation (a cudaMalloc of its own would
+ * bypass that pool and its accounting), or a latency-critical path where the
+ * implicit synchronisation of cudaMalloc/cudaFree is not acceptable.  The
+ * method on the pages has no counterpart of this entry point; it only changes
+ * where the scratch memory comes from.
+ *
+ * Arguments, layouts, results and errors are those of ss_scan_fwd, minus the
+ * workspace.  The scratch the scan may need (the carries handed between CTAs
+ * of the load-balanced schedule) lives in one static device array of
+ * SS_NOALLOC_SCRATCH_BYTES that the library owns; every GPU that loads the
+ * library holds it until the process exits.  This entry point calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *
+ *  - The first call on a device (with that device current) looks the array's
+ *    device address up once; make that first call before any stream capture.
+ *  - Problems whose schedule needs more scratch than SS_NOALLOC_SCRATCH_BYTES
+ *    (ss_scan_workspace_bytes(...) larger than it) are rejected with
+ *    SS_ERR_UNSUPPORTED and nothing is launched.
+ *  - Every call shares the one array and it keeps the last call's contents;
+ *    nothing in it has to start at zero (hand-over flags carry a per-launch
+ *    value, so stale contents are never taken as fresh).  Calls that overlap
+ *    on the GPU (two streams, or two host threads) race on the array: issue
+ *    them one after another on a stream, or use ss_scan_fwd with separate
+ *    workspaces.
+ */
+#define SS_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+ss_status ss_scan_fwd_noalloc(const void* u, const void* delta, const float* A,
+                              const void* B, const void* C, const float* D,
+                              const void* z, const float* delta_bias,
+                              int softplus_flag, float* y_out,
+                              float* last_state_out, int64_t batch,
+                              int64_t dim, int64_t seqlen, int dstate,
+                              ss_dtype in_dtype, cudaStream_t stream);
 
 /* Bytes of workspace ss_scan_fwd needs for these sizes on the current device
  * (0 when the chosen kernel needs none).  Returns (size_t)-1 for sizes that

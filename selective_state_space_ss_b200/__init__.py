@@ -17,6 +17,7 @@ from ._native import (  # noqa: F401
     SS_ERR_TIMEOUT,
     SS_ERR_UNSUPPORTED,
     SS_F32,
+    SS_NOALLOC_SCRATCH_BYTES,
     SS_OK,
     SSError,
     library_path,
@@ -24,6 +25,7 @@ from ._native import (  # noqa: F401
     ss_debug_inject,
     ss_last_device_error,
     ss_scan_fwd,
+    ss_scan_fwd_noalloc,
     ss_scan_workspace_bytes,
     ss_status_string,
 )

@@ -22,7 +22,10 @@ SS_OK, SS_ERR_INVALID_ARG, SS_ERR_UNSUPPORTED, SS_ERR_CUDA, SS_ERR_TIMEOUT = ran
 SS_F32, SS_BF16 = 0, 1
 
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
-            "ss_last_device_error", "ss_debug_inject")
+            "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc")
+
+# bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
+SS_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 # test hooks (include/ss_scan_debug.h)
 SS_DEBUG_CLEAR, SS_DEBUG_FORCE_WORKERS, SS_DEBUG_SKIP_PUBLISH, SS_DEBUG_SPIN_LIMIT = range(4)
@@ -61,6 +64,9 @@ def load_library():
         lib.ss_last_device_error.restype = ci
         lib.ss_debug_inject.argtypes = [ci, ctypes.c_longlong]
         lib.ss_debug_inject.restype = ci
+        lib.ss_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp,
+                                            i64, i64, i64, ci, ci, vp]
+        lib.ss_scan_fwd_noalloc.restype = ci
         _lib = lib
         return lib
 
@@ -157,4 +163,44 @@ def ss_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
                          _stream_handle(stream, device))
     if st != SS_OK:
         raise SSError(st, "ss_scan_fwd")
+    return y_out, last_state_out
+
+
+def ss_scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                        y_out=None, last_state_out=None, stream=None):
+    """ss_scan_fwd without a workspace: the library's static scratch array is used.
+
+    For callers that cannot allocate device memory where they call the scan.
+    The library allocates nothing; y_out and last_state_out must then be given
+    (they are allocated with torch here only when missing).  Raises SSError
+    with SS_ERR_UNSUPPORTED when the problem needs more scratch than
+    SS_NOALLOC_SCRATCH_BYTES.  Overlapping calls on the GPU race on the array.
+    """
+    lib = load_library()
+    device = u.device
+    if device.type != "cuda":
+        raise ValueError("ss_scan_fwd_noalloc runs on CUDA tensors only (no CPU fallback)")
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    in_types = (torch.float32, torch.bfloat16)
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _check_dev(name, t, device, in_types, (batch, dim, L))
+    for name, t in (("B", B), ("C", C)):
+        _check_dev(name, t, device, in_types, (batch, N, L))
+    if len({t.dtype for t in (u, delta, B, C, z) if t is not None}) != 1:
+        raise ValueError("u, delta, B, C and z must share one dtype")
+    _check_dev("A", A, device, (torch.float32,), (dim, N))
+    _check_dev("D", D, device, (torch.float32,), (dim,))
+    _check_dev("delta_bias", delta_bias, device, (torch.float32,), (dim,))
+    if y_out is None:
+        y_out = torch.empty((batch, dim, L), dtype=torch.float32, device=device)
+    _check_dev("y_out", y_out, device, (torch.float32,), (batch, dim, L))
+    _check_dev("last_state_out", last_state_out, device, (torch.float32,), (batch, dim, N))
+    dt = SS_F32 if u.dtype == torch.float32 else SS_BF16
+    st = lib.ss_scan_fwd_noalloc(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                 _ptr(delta_bias), int(bool(softplus)), _ptr(y_out),
+                                 _ptr(last_state_out), batch, dim, L, N, dt,
+                                 _stream_handle(stream, device))
+    if st != SS_OK:
+        raise SSError(st, "ss_scan_fwd_noalloc")
     return y_out, last_state_out

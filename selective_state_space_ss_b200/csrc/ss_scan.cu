@@ -230,6 +230,17 @@ bool supported_dstate(int n) { return n == 16 || n == 32 || n == 64 || n == 128;
 
 using namespace ssscan;
 
+// Scratch of ss_scan_fwd_noalloc: one file-scope device array, held by every
+// GPU that loads the library.  Host code must not use its name as an address
+// (it is a host-side stand-in); ss_scan_fwd_noalloc looks up the device
+// address once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SS_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 128;
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+}  // namespace
+
 extern "C" {
 
 ss_status ss_scan_fwd(const void* u, const void* delta, const float* A, const void* B,
@@ -267,6 +278,28 @@ ss_status ss_scan_fwd(const void* u, const void* delta, const float* A, const vo
 
   if (in_dtype == SS_F32) return dispatch_dtype<float>(a, dstate, workspace, workspace_bytes, stream);
   return dispatch_dtype<__nv_bfloat16>(a, dstate, workspace, workspace_bytes, stream);
+}
+
+ss_status ss_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B,
+                              const void* C, const float* D, const void* z,
+                              const float* delta_bias, int softplus_flag, float* y_out,
+                              float* last_state_out, int64_t batch, int64_t dim, int64_t seqlen,
+                              int dstate, ss_dtype in_dtype, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SS_ERR_UNSUPPORTED;
+  void* scratch = g_noalloc_ptr[dev].load();
+  if (!scratch) {  // once per device, with that device current
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch)
+      return SS_ERR_CUDA;
+    g_noalloc_ptr[dev].store(scratch);
+  }
+  const size_t need = ss_scan_workspace_bytes(batch, dim, seqlen, dstate);
+  if (need != (size_t)-1 && need > SS_NOALLOC_SCRATCH_BYTES) return SS_ERR_UNSUPPORTED;
+  // (invalid sizes fall through: ss_scan_fwd rejects them with its own status)
+  return ss_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, y_out, last_state_out,
+                     batch, dim, seqlen, dstate, in_dtype, scratch, SS_NOALLOC_SCRATCH_BYTES,
+                     stream);
 }
 
 size_t ss_scan_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int dstate) {
