@@ -56,4 +56,80 @@ __device__ __forceinline__ float silu_fast(float z) {
   return z * (z >= 0.f ? r : e * r);
 }
 
+// 2^x for x <= 0 on the FMA pipe (no special-function unit): x is clamped
+// to -126 (2^-126 ~ 1.2e-38 stands for 0 here), split as x = k + f with
+// k = round(x) by the 1.5 * 2^23 magic-number rounding and f in [-0.5, 0.5];
+// 2^f is the degree-6 fit of csrc/fit_poly.py (max rel err 9.7e-8) and 2^k is
+// put straight into the exponent field.
+__device__ __forceinline__ float2 exp2_neg_fma2(float2 x) {
+  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 j = __fadd2_rn(x, magic);
+  const float2 k = __fadd2_rn(j, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(k, make_float2(-1.f, -1.f), x);
+  float2 p = make_float2(1.533757750e-04f, 1.533757750e-04f);
+  p = __ffma2_rn(p, f, make_float2(1.339985989e-03f, 1.339985989e-03f));
+  p = __ffma2_rn(p, f, make_float2(9.618519805e-03f, 9.618519805e-03f));
+  p = __ffma2_rn(p, f, make_float2(5.550329015e-02f, 5.550329015e-02f));
+  p = __ffma2_rn(p, f, make_float2(2.402264625e-01f, 2.402264625e-01f));
+  p = __ffma2_rn(p, f, make_float2(6.931471825e-01f, 6.931471825e-01f));
+  p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
+  // bits of j are 0x4B400000 + k; (k + 127) << 23 is the exponent of 2^k
+  const int kx = __float_as_int(j.x) - 0x4B400000 + 127;
+  const int ky = __float_as_int(j.y) - 0x4B400000 + 127;
+  return __fmul2_rn(p, make_float2(__int_as_float(kx << 23), __int_as_float(ky << 23)));
+}
+
+// ---- packed forms: two independent elements per fp32x2 operation ----
+
+__device__ __forceinline__ float2 fabs2(float2 v) { return make_float2(fabsf(v.x), fabsf(v.y)); }
+
+// log1p(e)/e polynomial (same constants as log1p_unit) on a pair.
+__device__ __forceinline__ float2 log1p_unit2(float2 e) {
+  float2 p = make_float2(5.105825607e-03f, 5.105825607e-03f);
+  p = __ffma2_rn(p, e, make_float2(-2.899195626e-02f, -2.899195626e-02f));
+  p = __ffma2_rn(p, e, make_float2(7.738073915e-02f, 7.738073915e-02f));
+  p = __ffma2_rn(p, e, make_float2(-1.359059960e-01f, -1.359059960e-01f));
+  p = __ffma2_rn(p, e, make_float2(1.907130927e-01f, 1.907130927e-01f));
+  p = __ffma2_rn(p, e, make_float2(-2.483394593e-01f, -2.483394593e-01f));
+  p = __ffma2_rn(p, e, make_float2(3.331793547e-01f, 3.331793547e-01f));
+  p = __ffma2_rn(p, e, make_float2(-4.999943674e-01f, -4.999943674e-01f));
+  p = __ffma2_rn(p, e, make_float2(9.999999404e-01f, 9.999999404e-01f));
+  return __fmul2_rn(p, e);
+}
+
+#ifndef SS_POINTWISE_MUFU
+#define SS_POINTWISE_MUFU 3  // special-function ops per element in softplus + SiLU
+#endif
+
+// softplus on a pair (same math as softplus_fast).
+__device__ __forceinline__ float2 softplus_fast2(float2 x) {
+  const float2 t = __fmul2_rn(fabs2(x), make_float2(-1.4426950408889634f, -1.4426950408889634f));
+#if SS_POINTWISE_MUFU >= 3
+  const float2 e = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+#else
+  const float2 e = exp2_neg_fma2(t);
+#endif
+  return __fadd2_rn(make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)), log1p_unit2(e));
+}
+
+// SiLU on a pair (same math as silu_fast).
+__device__ __forceinline__ float2 silu_fast2(float2 z) {
+  const float2 t = __fmul2_rn(fabs2(z), make_float2(-1.4426950408889634f, -1.4426950408889634f));
+#if SS_POINTWISE_MUFU >= 2
+  const float2 e = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+#else
+  const float2 e = exp2_neg_fma2(t);
+#endif
+  const float2 d = __fadd2_rn(e, make_float2(1.f, 1.f));
+#if SS_POINTWISE_MUFU >= 3
+  const float2 r = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+#else
+  const float2 r = make_float2(rcp_1_2(d.x), rcp_1_2(d.y));
+#endif
+  const float2 er = __fmul2_rn(e, r);
+  const float2 sg = make_float2(z.x >= 0.f ? r.x : er.x, z.y >= 0.f ? r.y : er.y);
+  return __fmul2_rn(z, sg);
+}
+
 }  // namespace ssscan

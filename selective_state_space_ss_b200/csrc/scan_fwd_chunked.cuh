@@ -60,7 +60,12 @@ struct FwdMaps {
 
 constexpr uint32_t kTmaSpinLimit = 1u << 24;
 
-template <typename Tin, int N_, int K_, int NWARPS_, int T_>
+// Tin: input dtype; N: states per channel; K: lanes per channel; NWARPS: warps
+// per CTA; T: timesteps per chunk; WT: warps that split each chunk in time
+// (1: every warp walks the whole chunk for its own channels; >1: WT warps
+// share one set of channels, each scanning T/WT consecutive steps of the
+// chunk, joined with the pages' associative operator).
+template <typename Tin, int N_, int K_, int NWARPS_, int T_, int WT_ = 1>
 struct ChunkedCfg {
   using Elem = Tin;
   static constexpr int N = N_;            // states per channel
@@ -68,8 +73,11 @@ struct ChunkedCfg {
   static constexpr int G = N / K;         // states per lane
   static constexpr int NWARPS = NWARPS_;
   static constexpr int T = T_;            // timesteps per chunk
+  static constexpr int WT = WT_;          // time-split warps per channel set
+  static constexpr int WC = NWARPS / WT;  // warps across channels
+  static constexpr int TW = T / WT;       // steps per warp per chunk
   static constexpr int CPW = 32 / K;      // channels per warp
-  static constexpr int CH = NWARPS * CPW; // channels per CTA
+  static constexpr int CH = WC * CPW;     // channels per CTA
   static constexpr int NT = NWARPS * 32;
   static constexpr int ES = (int)sizeof(Tin);
   static constexpr int QPR = T / 4;                  // 4-step quads per row
@@ -92,22 +100,36 @@ struct ChunkedCfg {
   static constexpr int OFF_DWW = OFF_DWD + DW_BYTES;
   static constexpr int OFF_BC = OFF_DWW + DW_BYTES;
   static constexpr int OFF_SY = OFF_BC + BC_BYTES;
-  static constexpr int SMEM_USED = OFF_SY + SY_BYTES;
+  // time-split aggregates: (prod A_bar, local end state) per warp and lane state
+  static constexpr int AGG_FLOATS = WT > 1 ? WT * WC * 32 * G : 0;
+  static constexpr int OFF_AGG = OFF_SY + SY_BYTES;
+  static constexpr int SMEM_USED = OFF_AGG + 2 * AGG_FLOATS * 4;
   static constexpr int SMEM_BYTES = SMEM_USED + 128;  // slack to align the base to 128 bytes
   // CTAs per SM the register budget must allow (shared memory permitting)
-  static constexpr int MIN_CTAS = (227 * 1024 / (SMEM_USED + 128 + 1024)) < 5
-                                      ? (227 * 1024 / (SMEM_USED + 128 + 1024)) : 5;
+  // (at most 512 threads' worth: a 128-register budget per thread)
+  static constexpr int SMEM_CTAS = 227 * 1024 / (SMEM_USED + 128 + 1024);
+  static constexpr int THREAD_CTAS = 512 / NT > 0 ? 512 / NT : 1;
+  static constexpr int MIN_CTAS = SMEM_CTAS < THREAD_CTAS ? SMEM_CTAS : THREAD_CTAS;
   static constexpr int ITEMS = CH * QPR;             // (channel, quad) items per chunk
   static constexpr int ITEMS_PER_THREAD = (ITEMS + NT - 1) / NT;
 
   static_assert(N % K == 0 && 32 % K == 0, "lane split");
+  static_assert(NWARPS % WT == 0 && T % (4 * WT) == 0, "time split");
   static_assert(G % 4 == 0, "a lane holds whole 4-state blocks");
   static_assert(T % 8 == 0 && (T * ES) % 16 == 0 && T <= 256 && CH <= 256, "TMA box");
   static_assert(ACT_TILE % 128 == 0 && SEL_TILE % 128 == 0, "TMA destinations 128-byte aligned");
   static_assert(DW_BYTES % 16 == 0 && BC_BYTES % 16 == 0, "alignment");
-  static_assert(ITEMS % NT == 0, "whole items per thread");
+  static_assert(ITEMS % NT == 0 || ITEMS < NT, "whole items per thread");
+  static constexpr bool ITEM_GUARD = ITEMS < NT;  // some threads have no item
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
+
+// Quads of timesteps the recurrence loop is unrolled by (tuning builds may
+// override it).
+#ifndef SS_PHASE2_UNROLL
+#define SS_PHASE2_UNROLL 2
+#endif
+constexpr int kPhase2Unroll = SS_PHASE2_UNROLL;
 
 // Both halves of a packed bf16 pair as fp32 (exact).
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
@@ -171,24 +193,28 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
 #pragma unroll
   for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
     const int i = tid + it * CF::NT;
+    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
     const int c = i / CF::QPR, q = i - c * CF::QPR;
     const float4 dl = load4_f32(raw + (CF::CH + c) * CF::T + 4 * q);
     const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
     const float bias = bias_it[it];
-    const float dv[4] = {dl.x, dl.y, dl.z, dl.w};
-    const float uv[4] = {uu.x, uu.y, uu.z, uu.w};
-    float delt[4], w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float x = dv[k] + bias;
-      x = a.softplus ? softplus_fast(x) : x;
-      if constexpr (!kFull) {
-        // padding steps and channels: A_bar = 1, B_bar u = 0 (state unchanged)
-        if (d0 + c >= a.dim || t0 + 4 * q + k >= a.seqlen) x = 0.f;
-      }
-      delt[k] = x;
-      w[k] = x * uv[k];
+    const float2 b2 = make_float2(bias, bias);
+    float2 x01 = __fadd2_rn(make_float2(dl.x, dl.y), b2);
+    float2 x23 = __fadd2_rn(make_float2(dl.z, dl.w), b2);
+    if (a.softplus) {
+      x01 = softplus_fast2(x01);
+      x23 = softplus_fast2(x23);
     }
+    float delt[4] = {x01.x, x01.y, x23.x, x23.y};
+    if constexpr (!kFull) {
+      // padding steps and channels: A_bar = 1, B_bar u = 0 (state unchanged)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (d0 + c >= a.dim || t0 + 4 * q + k >= a.seqlen) delt[k] = 0.f;
+    }
+    const float2 w01 = __fmul2_rn(make_float2(delt[0], delt[1]), make_float2(uu.x, uu.y));
+    const float2 w23 = __fmul2_rn(make_float2(delt[2], delt[3]), make_float2(uu.z, uu.w));
+    const float w[4] = {w01.x, w01.y, w23.x, w23.y};
     dwD[q * CF::DW_STRIDE + c] = make_float4(delt[0], delt[1], delt[2], delt[3]);
     dwW[q * CF::DW_STRIDE + c] = make_float4(w[0], w[1], w[2], w[3]);
   }
@@ -265,13 +291,46 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
   constexpr int NB = CF::G / 4;  // 4-state blocks per lane
   const unsigned char* bcj = bc + j * NB * CF::BC_BLOCK;
   float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE;
-#pragma unroll 2
+#pragma unroll kPhase2Unroll
   for (int q = 0; q < CF::QPR; ++q) {
     const float4 D4 = dwD[q * CF::DW_STRIDE + c];
     const float4 W4 = dwW[q * CF::DW_STRIDE + c];
     const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
     const float ws[4] = {W4.x, W4.y, W4.z, W4.w};
     float s[4];
+#if defined(SS_PHASE2_EXP_FIRST)
+    // all ex2 of the quad first, then the four dependent update chains
+    float2 ee[4][CF::G / 2], wb[4][CF::G / 2], cc[4][CF::G / 2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const unsigned char* row = bcj + (4 * q + k) * CF::BC_ROW;
+      const float2 dl2 = make_float2(dls[k], dls[k]);
+      const float2 w2 = make_float2(ws[k], ws[k]);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        float2 b01, b23, c01, c23;
+        bc_block<CF>(row + nb * CF::BC_BLOCK, b01, b23, c01, c23);
+        const float2 x01 = __fmul2_rn(dl2, a2[2 * nb]);
+        const float2 x23 = __fmul2_rn(dl2, a2[2 * nb + 1]);
+        ee[k][2 * nb] = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+        ee[k][2 * nb + 1] = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+        wb[k][2 * nb] = __fmul2_rn(w2, b01);
+        wb[k][2 * nb + 1] = __fmul2_rn(w2, b23);
+        cc[k][2 * nb] = c01;
+        cc[k][2 * nb + 1] = c23;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int g = 0; g < CF::G / 2; ++g) {
+        h[g] = __ffma2_rn(ee[k][g], h[g], wb[k][g]);
+        acc = __ffma2_rn(cc[k][g], h[g], acc);
+      }
+      s[k] = acc.x + acc.y;
+    }
+#else
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const unsigned char* row = bcj + (4 * q + k) * CF::BC_ROW;
@@ -293,7 +352,106 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
       }
       s[k] = acc.x + acc.y;
     }
+#endif
     *reinterpret_cast<float4*>(syr + 4 * q) = make_float4(s[0], s[1], s[2], s[3]);
+  }
+}
+
+// The time-split recurrence (WT > 1).  Warp wt scans steps
+// [wt TW, (wt+1) TW) of the chunk from h = 0 while tracking the product of
+// its decays P_t = prod A_bar and the fix-up coefficients Q_t = C_t P_t; the
+// WT warps then swap their aggregates (P_end, h_end) through shared memory and
+// each folds the chunk's carry-in through the aggregates before it with the
+// operator (a1,b1) then (a2,b2) = (a2 a1, a2 b1 + b2) ("Mamba 选择性机制",
+// sec. 3.1), which gives its own carry-in h_in exactly: h_t = local h_t +
+// P_t h_in, so the readout is corrected by sum_n Q_t[n] h_in[n].  Every warp
+// folds all WT aggregates, so all of them leave with the chunk's carry-out in
+// h.  No ex2 is evaluated twice.
+template <class CF>
+__device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dwW,
+                                             const unsigned char* bc, float* sy, float* aggP,
+                                             float* aggH, float2 (&h)[CF::G / 2],
+                                             const float2 (&a2)[CF::G / 2], int c, int j, int wt,
+                                             int lane_g) {
+  constexpr int NB = CF::G / 4;
+  constexpr int G2 = CF::G / 2;
+  const unsigned char* bcj = bc + j * NB * CF::BC_BLOCK;
+  float2 hl[G2], P[G2];
+#pragma unroll
+  for (int g = 0; g < G2; ++g) {
+    hl[g] = make_float2(0.f, 0.f);
+    P[g] = make_float2(1.f, 1.f);
+  }
+  float2 Q[CF::TW][G2];
+  float s[CF::TW];
+#pragma unroll
+  for (int q = 0; q < CF::TW / 4; ++q) {
+    const int qq = wt * (CF::TW / 4) + q;
+    const float4 D4 = dwD[qq * CF::DW_STRIDE + c];
+    const float4 W4 = dwW[qq * CF::DW_STRIDE + c];
+    const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
+    const float ws[4] = {W4.x, W4.y, W4.z, W4.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = 4 * q + k;
+      const unsigned char* row = bcj + (4 * qq + k) * CF::BC_ROW;
+      const float2 dl2 = make_float2(dls[k], dls[k]);
+      const float2 w2 = make_float2(ws[k], ws[k]);
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        float2 b01, b23, c01, c23;
+        bc_block<CF>(row + nb * CF::BC_BLOCK, b01, b23, c01, c23);
+        const float2 x01 = __fmul2_rn(dl2, a2[2 * nb]);
+        const float2 x23 = __fmul2_rn(dl2, a2[2 * nb + 1]);
+        const float2 e01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+        const float2 e23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+        hl[2 * nb] = __ffma2_rn(e01, hl[2 * nb], __fmul2_rn(w2, b01));
+        hl[2 * nb + 1] = __ffma2_rn(e23, hl[2 * nb + 1], __fmul2_rn(w2, b23));
+        P[2 * nb] = __fmul2_rn(e01, P[2 * nb]);
+        P[2 * nb + 1] = __fmul2_rn(e23, P[2 * nb + 1]);
+        acc = __ffma2_rn(c01, hl[2 * nb], acc);
+        acc = __ffma2_rn(c23, hl[2 * nb + 1], acc);
+        Q[t][2 * nb] = __fmul2_rn(c01, P[2 * nb]);
+        Q[t][2 * nb + 1] = __fmul2_rn(c23, P[2 * nb + 1]);
+      }
+      s[t] = acc.x + acc.y;
+    }
+  }
+  // publish this warp's aggregate: [wt][lane in channel set][state]
+  float2* myP = reinterpret_cast<float2*>(aggP + (wt * CF::WC * 32 + lane_g) * CF::G);
+  float2* myH = reinterpret_cast<float2*>(aggH + (wt * CF::WC * 32 + lane_g) * CF::G);
+#pragma unroll
+  for (int g = 0; g < G2; ++g) {
+    myP[g] = P[g];
+    myH[g] = hl[g];
+  }
+  __syncthreads();
+  float2 hin[G2];
+#pragma unroll
+  for (int v = 0; v < CF::WT; ++v) {
+    if (v == wt) {
+#pragma unroll
+      for (int g = 0; g < G2; ++g) hin[g] = h[g];
+    }
+    const float2* vP = reinterpret_cast<const float2*>(aggP + (v * CF::WC * 32 + lane_g) * CF::G);
+    const float2* vH = reinterpret_cast<const float2*>(aggH + (v * CF::WC * 32 + lane_g) * CF::G);
+#pragma unroll
+    for (int g = 0; g < G2; ++g) h[g] = __ffma2_rn(vP[g], h[g], vH[g]);
+  }
+  float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE + wt * CF::TW;
+#pragma unroll
+  for (int q = 0; q < CF::TW / 4; ++q) {
+    float out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = 4 * q + k;
+      float2 fix = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int g = 0; g < G2; ++g) fix = __ffma2_rn(Q[t][g], hin[g], fix);
+      out[k] = s[t] + (fix.x + fix.y);
+    }
+    *reinterpret_cast<float4*>(syr + 4 * q) = make_float4(out[0], out[1], out[2], out[3]);
   }
 }
 
@@ -308,27 +466,31 @@ __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem
 #pragma unroll
   for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
     const int i = tid + it * CF::NT;
+    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
     const int c = i / CF::QPR, q = i - c * CF::QPR;
     const int64_t d = d0 + c, t = t0 + 4 * q;
     if constexpr (!kFull) {
       if (d >= D || t >= L) continue;
     }
-    float4 s = *reinterpret_cast<const float4*>(sy + (c * CF::K) * CF::SY_STRIDE + 4 * q);
+    const float4 s0 = *reinterpret_cast<const float4*>(sy + (c * CF::K) * CF::SY_STRIDE + 4 * q);
+    float2 s01 = make_float2(s0.x, s0.y), s23 = make_float2(s0.z, s0.w);
 #pragma unroll
     for (int jj = 1; jj < CF::K; ++jj) {
       const float4 o = *reinterpret_cast<const float4*>(sy + (c * CF::K + jj) * CF::SY_STRIDE + 4 * q);
-      s.x += o.x; s.y += o.y; s.z += o.z; s.w += o.w;
+      s01 = __fadd2_rn(s01, make_float2(o.x, o.y));
+      s23 = __fadd2_rn(s23, make_float2(o.z, o.w));
     }
     const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
     const float Dd = D_it[it];
-    float y[4] = {fmaf(Dd, uu.x, s.x), fmaf(Dd, uu.y, s.y), fmaf(Dd, uu.z, s.z), fmaf(Dd, uu.w, s.w)};
+    const float2 D2 = make_float2(Dd, Dd);
+    float2 y01 = __ffma2_rn(D2, make_float2(uu.x, uu.y), s01);
+    float2 y23 = __ffma2_rn(D2, make_float2(uu.z, uu.w), s23);
     if (has_z) {
       const float4 zz = load4_f32(raw + (2 * CF::CH + c) * CF::T + 4 * q);
-      y[0] *= silu_fast(zz.x);
-      y[1] *= silu_fast(zz.y);
-      y[2] *= silu_fast(zz.z);
-      y[3] *= silu_fast(zz.w);
+      y01 = __fmul2_rn(y01, silu_fast2(make_float2(zz.x, zz.y)));
+      y23 = __fmul2_rn(y23, silu_fast2(make_float2(zz.z, zz.w)));
     }
+    const float y[4] = {y01.x, y01.y, y23.x, y23.y};
     float* dst = a.y + (b * D + d) * L + t;
     if (a.vec && (kFull || t + 3 < L)) {  // 16-byte stores only on aligned rows
       *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
@@ -460,6 +622,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   float4* dwW = reinterpret_cast<float4*>(smem + CF::OFF_DWW);
   unsigned char* bc = smem + CF::OFF_BC;
   float* sy = reinterpret_cast<float*>(smem + CF::OFF_SY);
+  float* aggP = reinterpret_cast<float*>(smem + CF::OFF_AGG);
+  float* aggH = aggP + CF::AGG_FLOATS;
   __shared__ __align__(8) uint64_t bars[2];
 
   const int w = blockIdx.x;
@@ -470,8 +634,15 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   const bool has_z = a.z != nullptr;
   const bool tma = a.vec != 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = warp * CF::CPW + lane / CF::K;  // this lane's channel within the CTA
-  const int j = lane % CF::K;                   // this lane's state group
+  const int wc = warp % CF::WC, wt = warp / CF::WC;  // channel warp, time-split slot
+  const int c = wc * CF::CPW + lane / CF::K;     // this lane's channel within the CTA
+  const int j = lane % CF::K;                    // this lane's state group
+  const int lane_g = wc * 32 + lane;             // lane within its channel set
+  const bool writer = wt == 0;  // time-split warps hold the same carry: one writes it
+  auto run_phase2 = [&](float2 (&hh)[CF::G / 2], const float2 (&aa)[CF::G / 2]) {
+    if constexpr (CF::WT == 1) phase2<CF>(dwD, dwW, bc, sy, hh, aa, c, j);
+    else phase2_split<CF>(dwD, dwW, bc, sy, aggP, aggH, hh, aa, c, j, wt, lane_g);
+  };
 
   if (tma && tid == 0) {
     mbar_init(&bars[0], 1);
@@ -532,7 +703,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     run_phase1(0);
     __syncthreads();
     for (int64_t k = 0; k < nseq; ++k) {
-      phase2<CF>(dwD, dwW, bc, sy, h, a2, c, j);
+      run_phase2(h, a2);
       if (k + 1 < nseq) stage_in(k + 1);
       if (!__syncthreads_and(ok)) {
         drain(k + 1, k + 1);
@@ -547,7 +718,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
         tma_chunk<CF>(maps, raw(k), &bars[k & 1], (int32_t)b, (int32_t)d0,
                       (int32_t)((k + 2) * CF::T), has_z);
     }
-    if (a.last_state && chan_ok) {
+    if (a.last_state && chan_ok && writer) {
       float* dst = a.last_state + ((b * a.dim + d) * CF::N + j * CF::G);
 #pragma unroll
       for (int g = 0; g < CF::G / 2; ++g) {
@@ -649,15 +820,15 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
       }
       ok = ok && have;
     }
-    phase2<CF>(dwD, dwW, bc, sy, h, a2, c, j);
+    run_phase2(h, a2);
     const bool cout_here = cur.carry_out();
-    if (cout_here) {
+    if (cout_here && writer) {
       float* dst = sched.carries + (int64_t)w * CF::CH * CF::N + c * CF::N + j * CF::G;
 #pragma unroll
       for (int g = 0; g < CF::G / 2; ++g) __stcg(reinterpret_cast<float2*>(dst) + g, h[g]);
       __threadfence();
     }
-    if (cur.last() && a.last_state && chan_ok) {
+    if (cur.last() && a.last_state && chan_ok && writer) {
       float* dst = a.last_state + (((int64_t)cur.b * a.dim + d) * CF::N + j * CF::G);
 #pragma unroll
       for (int g = 0; g < CF::G / 2; ++g) {

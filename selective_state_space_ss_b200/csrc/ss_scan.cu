@@ -198,11 +198,42 @@ using Cfg64 = ChunkedCfg<E, 64, 8, 8, 32>;
 template <typename E>
 using Cfg128 = ChunkedCfg<E, 128, 8, 8, 32>;
 
+// Time-split shapes for problems with too few channels to fill the GPU: one
+// warp's worth of channels (8) per CTA, 8 warps splitting each chunk in time.
+#ifndef SS_SPLIT16_W
+#define SS_SPLIT16_W 8
+#endif
+#ifndef SS_SPLIT16_T
+#define SS_SPLIT16_T 128
+#endif
+#ifndef SS_SPLIT16_WT
+#define SS_SPLIT16_WT 8
+#endif
+template <typename E>
+using Split16 = ChunkedCfg<E, 16, 4, SS_SPLIT16_W, SS_SPLIT16_T, SS_SPLIT16_WT>;
+template <typename E>
+using Split32 = ChunkedCfg<E, 32, 4, 8, 32, 8>;
+
+// The time split costs ~1.5 extra instructions per (step, state); take it only
+// when the channel-parallel shape would leave SMs idle.
+template <class CF>
+bool too_few_groups(int64_t batch, int64_t dim) {
+#ifdef SS_SPLIT_ALWAYS
+  return true;
+#endif
+  const int64_t groups = batch * ((dim + CF::CH - 1) / CF::CH);
+  return groups < device_sms();
+}
+
 template <typename E>
 ss_status dispatch_dtype(const FwdArgs& a, int N, void* ws, size_t wsb, cudaStream_t stream) {
   switch (N) {
-    case 16: return launch_chunked<Cfg16<E>>(a, ws, wsb, stream);
-    case 32: return launch_chunked<Cfg32<E>>(a, ws, wsb, stream);
+    case 16:
+      if (too_few_groups<Cfg16<E>>(a.batch, a.dim)) return launch_chunked<Split16<E>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg16<E>>(a, ws, wsb, stream);
+    case 32:
+      if (too_few_groups<Cfg32<E>>(a.batch, a.dim)) return launch_chunked<Split32<E>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg32<E>>(a, ws, wsb, stream);
     case 64: return launch_chunked<Cfg64<E>>(a, ws, wsb, stream);
     case 128: return launch_chunked<Cfg128<E>>(a, ws, wsb, stream);
     default: return SS_ERR_UNSUPPORTED;
@@ -214,8 +245,14 @@ bool plan_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N, size_t* bytes
   Plan p;
   bool ok = false;
   switch (N) {
-    case 16: ok = make_plan<Cfg16<E>>(batch, dim, seqlen, &p); break;
-    case 32: ok = make_plan<Cfg32<E>>(batch, dim, seqlen, &p); break;
+    case 16:
+      ok = too_few_groups<Cfg16<E>>(batch, dim) ? make_plan<Split16<E>>(batch, dim, seqlen, &p)
+                                                : make_plan<Cfg16<E>>(batch, dim, seqlen, &p);
+      break;
+    case 32:
+      ok = too_few_groups<Cfg32<E>>(batch, dim) ? make_plan<Split32<E>>(batch, dim, seqlen, &p)
+                                                : make_plan<Cfg32<E>>(batch, dim, seqlen, &p);
+      break;
     case 64: ok = make_plan<Cfg64<E>>(batch, dim, seqlen, &p); break;
     case 128: ok = make_plan<Cfg128<E>>(batch, dim, seqlen, &p); break;
   }
