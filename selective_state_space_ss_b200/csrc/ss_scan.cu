@@ -193,10 +193,28 @@ template <typename E>
 using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T>;
 template <typename E>
 using Cfg32 = ChunkedCfg<E, 32, 4, 4, 32>;
+#ifndef SS_N64_K
+#define SS_N64_K 4
+#endif
+#ifndef SS_N64_W
+#define SS_N64_W 4
+#endif
+#ifndef SS_N64_T
+#define SS_N64_T 32
+#endif
+#ifndef SS_N128_K
+#define SS_N128_K 16
+#endif
+#ifndef SS_N128_W
+#define SS_N128_W 8
+#endif
+#ifndef SS_N128_T
+#define SS_N128_T 32
+#endif
 template <typename E>
-using Cfg64 = ChunkedCfg<E, 64, 8, 8, 32>;
+using Cfg64 = ChunkedCfg<E, 64, SS_N64_K, SS_N64_W, SS_N64_T>;
 template <typename E>
-using Cfg128 = ChunkedCfg<E, 128, 8, 8, 32>;
+using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T>;
 
 // Time-split shapes for problems with too few channels to fill the GPU: one
 // warp's worth of channels (8) per CTA, 8 warps splitting each chunk in time.

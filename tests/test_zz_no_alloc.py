@@ -70,16 +70,18 @@ def test_noalloc_matches_workspace_entry_point(shape, dtype, workers):
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
     ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
-    # N = 128 with a few hundred channel groups: the balanced schedule's carries
-    # exceed the static array
-    b, d, L, n = 10, 1024, 64, 128
-    need = ss.ss_scan_workspace_bytes(b, d, L, n)
-    if need <= N.SS_NOALLOC_SCRATCH_BYTES:
-        pytest.skip(f"schedule on this device needs only {need} bytes")
-    w = I.Workload("noalloc_big", b, d, L, n, "bf16")
-    xd = to_device(I.make_inputs(w, seed=5))
-    y = torch.zeros(b, d, L, device="cuda")
-    h = torch.zeros(b, d, n, device="cuda")
-    assert _noalloc_cabi(xd, y, h) == N.SS_ERR_UNSUPPORTED
-    torch.cuda.synchronize()
-    assert torch.count_nonzero(y).item() == 0  # nothing was launched
+    # 640 channel groups at N = 64 shared by 600 CTAs: 600 carries of
+    # 32 x 64 fp32 states (~4.9 MB) do not fit the static array
+    b, d, L, n = 20, 1024, 64, 64
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 600)
+    try:
+        assert ss.ss_scan_workspace_bytes(b, d, L, n) > N.SS_NOALLOC_SCRATCH_BYTES
+        w = I.Workload("noalloc_big", b, d, L, n, "bf16")
+        xd = to_device(I.make_inputs(w, seed=5))
+        y = torch.zeros(b, d, L, device="cuda")
+        h = torch.zeros(b, d, n, device="cuda")
+        assert _noalloc_cabi(xd, y, h) == N.SS_ERR_UNSUPPORTED
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(y).item() == 0  # nothing was launched
+    finally:
+        ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
