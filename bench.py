@@ -137,6 +137,28 @@ def _dist_env():
     return world, rank, local
 
 
+def rank_seed(rank: int, s: int) -> int:
+    """Seed of input set s on `rank`: every rank scans its own batch (weak scaling)."""
+    return 1000 + 17 * rank + s
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Largest elapsed time over all ranks (the job ends with the slowest rank)."""
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(elements_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job elements per second: all ranks' work over the slowest rank's time."""
+    return elements_per_rank * world * steps / (ms_max * 1e-3)
+
+
 def run_gpu_arm(args, w: I.Workload):
     import torch
     import torch.distributed as dist
@@ -158,7 +180,7 @@ def run_gpu_arm(args, w: I.Workload):
     # more than one L2 capacity ago (flushing is not needed then)
     per_set = w.algorithmic_bytes()
     nsets = max(1, -(-4 * L2_BYTES // per_set))
-    host = [I.make_inputs(w, seed=1000 + 17 * rank + s) for s in range(nsets)]
+    host = [I.make_inputs(w, seed=rank_seed(rank, s)) for s in range(nsets)]
 
     def to_dev(x):
         out = {}
@@ -200,13 +222,9 @@ def run_gpu_arm(args, w: I.Workload):
         torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_per_step = ms_max / args.steps
-    value = w.elements * world * args.steps / (ms_max * 1e-3)
+    value = job_throughput(w.elements, world, args.steps, ms_max)
 
     # end to end through the public call: pinned host inputs -> device -> scan -> y back to host
     ex = host[0]
@@ -246,10 +264,8 @@ def run_gpu_arm(args, w: I.Workload):
     f1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = w.elements * world * e2e_steps / (float(te.item()) * 1e-3)
+    e2e_value = job_throughput(w.elements, world, e2e_steps,
+                               max_over_ranks(f0.elapsed_time(f1), world, dev))
 
     if world > 1:
         dist.destroy_process_group()

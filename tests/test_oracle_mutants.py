@@ -1,0 +1,73 @@
+"""The oracle's pins have teeth: each plausible slip, planted in a copy of the
+oracle's C source (on the CPU), must make at least one pin in
+test_oracle_pins.py fail.  The real oracle is not touched."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ss_oracle.c")
+
+# (name, original text, mutated text)
+MUTANTS = [
+    ("B_bar without Delta", "h[n] = a_bar * h[n] + dt * b_t * ut;", "h[n] = a_bar * h[n] + b_t * ut;"),
+    ("sign of A", "exp(dt * (double)J->A[d * N + n])", "exp(-dt * (double)J->A[d * N + n])"),
+    ("B and C swapped", "const double b_t = widen(J->B,", "const double b_t = widen(J->C,"),
+    ("bias outside the softplus",
+     "const double dt = J->softplus_flag ? softplus64(x) : x;",
+     "const double dt = J->softplus_flag ? softplus64(x - bias) + bias : x;"),
+    ("readout before the update",
+     "h[n] = a_bar * h[n] + dt * b_t * ut;\n      s += c_t * h[n];",
+     "s += c_t * h[n];\n      h[n] = a_bar * h[n] + dt * b_t * ut;"),
+    ("gate misses the skip term",
+     "    s += Dd * ut;\n    if (J->z) s *= silu64(widen(J->z, J->dtype, row + t));",
+     "    if (J->z) s *= silu64(widen(J->z, J->dtype, row + t));\n    s += Dd * ut;"),
+    ("A indexed [n][d]", "J->A[d * N + n]", "J->A[n * J->dim + d]"),
+    ("state not carried", "h[n] = a_bar * h[n] + dt * b_t * ut;", "h[n] = a_bar * 0.0 + dt * b_t * ut;"),
+]
+
+PIN_CALLS = [
+    lambda: pins.test_lti_closed_form(False),
+    lambda: pins.test_lti_closed_form(True),
+    pins.test_tree_fold_equals_serial_oracle,
+    pins.test_hold_limit_exact_zero_delta,
+    pins.test_hold_limit_softplus_with_bias,
+    pins.test_reset_limit,
+    lambda: pins.test_bruteforce_unrolled(5),
+    pins.test_prefix_sum_special_case,
+    pins.test_index_plumbing_single_impulse,
+]
+
+
+def _build_mutant(tmp_path, old, new):
+    text = open(SRC).read()
+    assert old in text, f"mutation target not found: {old!r}"
+    src = tmp_path / "mutant.c"
+    src.write_text(text.replace(old, new, 1))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                           "-ffp-contract=off", "-o", str(lib), str(src), "-lm", "-lpthread"])
+    return str(lib)
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, monkeypatch, name, old, new):
+    path = _build_mutant(tmp_path, old, new)
+    real = oracle._load()
+    lib = ctypes.CDLL(path)
+    for fn in ("oracle_scan_fwd", "oracle_softplus", "oracle_silu"):
+        f = getattr(lib, fn)
+        f.argtypes = getattr(real, fn).argtypes
+        f.restype = getattr(real, fn).restype
+    monkeypatch.setattr(oracle, "_lib", lib)
+    failed = []
+    for call in PIN_CALLS:
+        try:
+            call()
+        except AssertionError:
+            failed.append(call)
+    assert failed, f"no pin caught the mutant '{name}'"
