@@ -183,17 +183,19 @@ __device__ __forceinline__ void load_chunk_scalar(const FwdArgs& a, typename CF:
 
 // ------------------------------------------------------------- phase 1 ---
 
-template <class CF, bool kFull>
+// Runs on NTH threads (tid in [0, NTH)): all threads of a CTA, or its helper
+// warps in the warp-specialised kernel.
+template <class CF, bool kFull, int NTH = CF::NT>
 __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem* raw,
                                        float4* dwD, float4* dwW, unsigned char* bc,
-                                       const float (&bias_it)[CF::ITEMS_PER_THREAD],
-                                       int64_t d0, int64_t t0) {
+                                       const float (&bias_it)[(CF::ITEMS + NTH - 1) / NTH],
+                                       int64_t d0, int64_t t0, int tid = threadIdx.x) {
   using E = typename CF::Elem;
-  const int tid = threadIdx.x;
+  constexpr int IPT = (CF::ITEMS + NTH - 1) / NTH;
 #pragma unroll
-  for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
-    const int i = tid + it * CF::NT;
-    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
+  for (int it = 0; it < IPT; ++it) {
+    const int i = tid + it * NTH;
+    if (CF::ITEMS % NTH != 0 && i >= CF::ITEMS) break;
     const int c = i / CF::QPR, q = i - c * CF::QPR;
     const float4 dl = load4_f32(raw + (CF::CH + c) * CF::T + 4 * q);
     const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
@@ -226,7 +228,7 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     const uint32_t* B32 = reinterpret_cast<const uint32_t*>(rawB);
     const uint32_t* C32 = reinterpret_cast<const uint32_t*>(rawC);
     constexpr int NB4 = CF::N / 4;
-    for (int i = tid; i < NB4 * TP; i += CF::NT) {
+    for (int i = tid; i < NB4 * TP; i += NTH) {
       const int tp = i / NB4, nb = i - tp * NB4;
       uint32_t bw[4], cw[4];
 #pragma unroll
@@ -244,7 +246,7 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
   } else {
     const float* fb = reinterpret_cast<const float*>(rawB);
     const float* fc = reinterpret_cast<const float*>(rawC);
-    for (int i = tid; i < (CF::N / 4) * CF::T; i += CF::NT) {
+    for (int i = tid; i < (CF::N / 4) * CF::T; i += NTH) {
       const int nb = i / CF::T, t = i - nb * CF::T;
       float4* dst = reinterpret_cast<float4*>(bc + t * CF::BC_ROW + nb * CF::BC_BLOCK);
       dst[0] = make_float4(fb[(4 * nb) * CF::T + t], fb[(4 * nb + 1) * CF::T + t],
@@ -457,16 +459,18 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
 
 // ------------------------------------------------------------- phase 3 ---
 
-template <class CF, bool kFull>
+template <class CF, bool kFull, int NTH = CF::NT>
 __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem* raw,
-                                       const float* sy, const float (&D_it)[CF::ITEMS_PER_THREAD],
-                                       int64_t b, int64_t d0, int64_t t0, bool has_z) {
-  const int tid = threadIdx.x;
+                                       const float* sy,
+                                       const float (&D_it)[(CF::ITEMS + NTH - 1) / NTH],
+                                       int64_t b, int64_t d0, int64_t t0, bool has_z,
+                                       int tid = threadIdx.x) {
   const int64_t L = a.seqlen, D = a.dim;
+  constexpr int IPT = (CF::ITEMS + NTH - 1) / NTH;
 #pragma unroll
-  for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
-    const int i = tid + it * CF::NT;
-    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
+  for (int it = 0; it < IPT; ++it) {
+    const int i = tid + it * NTH;
+    if (CF::ITEMS % NTH != 0 && i >= CF::ITEMS) break;
     const int c = i / CF::QPR, q = i - c * CF::QPR;
     const int64_t d = d0 + c, t = t0 + 4 * q;
     if constexpr (!kFull) {

@@ -166,3 +166,15 @@ def test_device_error_word_clear():
     w = I.Workload("err", 1, 8, 40, 16, "f32")
     run_gpu(to_device(I.make_inputs(w, seed=1)))
     assert ss_last_device_error() == SS_OK
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("L", [7, 100, 1001, 2048])
+def test_wide_shapes_warp_specialised_path(dtype, L):
+    """Enough channel groups (5 x ceil(1000/32) = 160) to fill the SMs, so N = 16
+    runs the warp-specialised kernel: partial last channel tile, ragged tails,
+    odd L (element-wise loads)."""
+    w = I.Workload(f"wide_{dtype}_L{L}", 5, 1000, L, 16, dtype)
+    rng = np.random.default_rng(L)
+    channels = np.unique(np.concatenate([[0, 999, 1000, 4999], rng.choice(5000, 300, replace=False)]))
+    _parity(w, seed=L + 7, channels=channels)
