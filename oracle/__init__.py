@@ -47,7 +47,7 @@ def _load():
             vp, i64 = ctypes.c_void_p, ctypes.c_int64
             lib.oracle_scan_fwd.argtypes = [
                 vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
-                i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, ctypes.c_int]
+                i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, vp, ctypes.c_int]
             lib.oracle_scan_fwd.restype = ctypes.c_int
             lib.oracle_softplus.argtypes = [ctypes.c_double]
             lib.oracle_softplus.restype = ctypes.c_double
@@ -72,13 +72,15 @@ def _stored(a, name):
 
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
-             softplus=True, channels=None, nthreads=None):
+             softplus=True, channels=None, nthreads=None, h0=None):
     """Serial fp64 selective scan.
 
     u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; all float32 or all
     bf16 bits (uint16).  A: [dim, N] float32; D, delta_bias: [dim] float32.
     channels: optional 1-D int array of flat channel ids (b*dim + d); then
-    only those rows are computed.  Returns (y, last_state) as float64 with
+    only those rows are computed.  h0: optional [batch, dim, N] initial state
+    (widened to float64; the scan starts from zero without it).
+    Returns (y, last_state) as float64 with
     shapes [batch, dim, L] / [batch, dim, N], or [len(channels), L] /
     [len(channels), N] when channels is given.
     """
@@ -103,6 +105,10 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
         raise ValueError("A must be [dim, N]")
     D = None if D is None else np.ascontiguousarray(D, dtype=np.float32)
     delta_bias = None if delta_bias is None else np.ascontiguousarray(delta_bias, dtype=np.float32)
+    if h0 is not None:
+        h0 = np.ascontiguousarray(h0, dtype=np.float64)
+        if h0.shape != (batch, dim, N):
+            raise ValueError("h0 must be [batch, dim, N]")
     if channels is not None:
         channels = np.ascontiguousarray(channels, dtype=np.int64)
         nch = channels.size
@@ -117,10 +123,27 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     rc = _load().oracle_scan_fwd(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(softplus)), dt, batch, dim, L, N,
-        _ptr(channels), nch, _ptr(y), _ptr(h), int(nthreads))
+        _ptr(channels), nch, _ptr(y), _ptr(h), _ptr(h0), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_scan_fwd rejected its arguments")
     return y, h
+
+
+def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+              softplus=True, nthreads=None):
+    """One recurrent (decode) step: the scan over a single token started from
+    the carried state.
+
+    state: [batch, dim, N] (any float dtype, widened to float64); u, delta, z:
+    [batch, dim]; B, C: [batch, N]; the rest as in scan_fwd.  Returns
+    (y [batch, dim], new_state [batch, dim, N]) as float64.
+    """
+    y, h = scan_fwd(np.asarray(u)[..., None], np.asarray(delta)[..., None], A,
+                    np.asarray(B)[..., None], np.asarray(C)[..., None], D=D,
+                    z=None if z is None else np.asarray(z)[..., None],
+                    delta_bias=delta_bias, softplus=softplus, nthreads=nthreads,
+                    h0=state)
+    return y[..., 0], h
 
 
 def softplus(x: float) -> float:

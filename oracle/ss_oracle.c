@@ -9,7 +9,7 @@
  * What it computes is the plain serial recurrence of the selective SSM,
  * widened exactly from the stored input dtype to double:
  *
- *   for every (b, d):  h[n] = 0
+ *   for every (b, d):  h[n] = h0[b,d,n]  (0 when no initial state is given)
  *     for t = 0 .. L-1:
  *       Delta  = softplus(delta[b,d,t] + delta_bias[d])   (or without softplus)
  *       h[n]   = exp(Delta * A[d,n]) * h[n] + Delta * B[b,n,t] * u[b,d,t]
@@ -39,6 +39,11 @@
  *  - softplus_flag == 0 means Delta = delta + delta_bias.
  *  - SiLU(z) = z / (1 + exp(-z)).
  *  - a null D, delta_bias or z means zero skip, zero bias and no gate.
+ *  - an initial state h0 replaces the zero state of the pure-PyTorch module;
+ *    the pages keep h between calls for recurrent (one token at a time)
+ *    inference ("从Transformer的痛点说起 ... Mamba", sec. 5.1 table and
+ *    sec. 6.3, fourth note), and one such step is this recurrence with L = 1
+ *    started from the carried state.
  */
 #include <math.h>
 #include <pthread.h>
@@ -75,6 +80,7 @@ typedef struct {
   int64_t n_channels;
   double* y;          /* [n_channels, seqlen] */
   double* last_state; /* [n_channels, dstate] or NULL */
+  const double* h0;   /* [batch, dim, dstate] initial state or NULL (zero) */
   int64_t next;       /* work counter (guarded by mu) */
   pthread_mutex_t mu;
 } job_t;
@@ -91,7 +97,7 @@ static void run_channel(const job_t* J, int64_t slot, double* h) {
   const double Dd = J->D ? (double)J->D[d] : 0.0;
   double* yrow = J->y + slot * L;
 
-  for (int n = 0; n < N; ++n) h[n] = 0.0;
+  for (int n = 0; n < N; ++n) h[n] = J->h0 ? J->h0[flat * N + n] : 0.0;
   for (int64_t t = 0; t < L; ++t) {
     const double x = widen(J->delta, J->dtype, row + t) + bias;
     const double dt = J->softplus_flag ? softplus64(x) : x;
@@ -137,6 +143,9 @@ static void* worker(void* arg) {
  *               channel ids; y and last_state then hold only those rows.
  * y           : [n_channels, seqlen] double
  * last_state  : [n_channels, dstate] double (nullable)
+ * h0          : [batch, dim, dstate] double initial state, indexed by the
+ *               full flat channel id even when `channels` is given (nullable:
+ *               the state starts at zero)
  * nthreads    : worker threads (>= 1)
  */
 int oracle_scan_fwd(const void* u, const void* delta, const float* A,
@@ -144,7 +153,8 @@ int oracle_scan_fwd(const void* u, const void* delta, const float* A,
                     const void* z, const float* delta_bias, int softplus_flag,
                     int dtype, int64_t batch, int64_t dim, int64_t seqlen,
                     int dstate, const int64_t* channels, int64_t n_channels,
-                    double* y, double* last_state, int nthreads) {
+                    double* y, double* last_state, const double* h0,
+                    int nthreads) {
   if (!u || !delta || !A || !B || !C || !y) return -1;
   if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0) return -1;
   if (dtype != 0 && dtype != 1) return -1;
@@ -163,7 +173,7 @@ int oracle_scan_fwd(const void* u, const void* delta, const float* A,
   J.softplus_flag = softplus_flag; J.dtype = dtype;
   J.batch = batch; J.dim = dim; J.seqlen = seqlen; J.dstate = dstate;
   J.channels = channels; J.n_channels = n_channels;
-  J.y = y; J.last_state = last_state; J.next = 0;
+  J.y = y; J.last_state = last_state; J.h0 = h0; J.next = 0;
   pthread_mutex_init(&J.mu, NULL);
 
   pthread_t tids[512];

@@ -28,6 +28,9 @@ MUTANTS = [
      "    if (J->z) s *= silu64(widen(J->z, J->dtype, row + t));\n    s += Dd * ut;"),
     ("A indexed [n][d]", "J->A[d * N + n]", "J->A[n * J->dim + d]"),
     ("state not carried", "h[n] = a_bar * h[n] + dt * b_t * ut;", "h[n] = a_bar * 0.0 + dt * b_t * ut;"),
+    ("initial state ignored", "h[n] = J->h0 ? J->h0[flat * N + n] : 0.0;", "h[n] = 0.0;"),
+    ("initial state indexed [b][n][d]", "J->h0[flat * N + n]", "J->h0[(b * N + n) * J->dim + d]"),
+    ("initial state indexed [n][b][d]", "J->h0[flat * N + n]", "J->h0[n * J->batch * J->dim + flat]"),
 ]
 
 PIN_CALLS = [
@@ -40,6 +43,8 @@ PIN_CALLS = [
     lambda: pins.test_bruteforce_unrolled(5),
     pins.test_prefix_sum_special_case,
     pins.test_index_plumbing_single_impulse,
+    pins.test_initial_state_free_decay_closed_form,
+    lambda: pins.test_initial_state_bruteforce(3),
 ]
 
 

@@ -338,6 +338,112 @@ def test_index_plumbing_single_impulse():
             assert np.all(y[b, d, 1:L - 1] == 0.0)
 
 
+# ------------------------------------------------------- initial state -----
+# A carried state h0 stands for the recurrent mode of the pages: inference
+# keeps h and feeds one token at a time ("从Transformer的痛点说起 ... Mamba",
+# sec. 5.1 table and sec. 6.3).
+
+def _distinct_h0(batch, dim, N):
+    b = np.arange(batch)[:, None, None]
+    d = np.arange(dim)[None, :, None]
+    n = np.arange(N)[None, None, :]
+    return (1.0 + 0.5 * b + 0.125 * d + 2.0 * n) * np.where((b + d + n) % 2 == 0, 1.0, -1.0)
+
+
+def test_initial_state_free_decay_closed_form():
+    """u = 0 and a constant Delta: the state only decays, h_t[n] =
+    e^{(t+1) Delta A[d,n]} h0[b,d,n], evaluated directly (no products), and
+    y_t = (C_t . h_t) SiLU(z_t).  h0, A and C are distinct per index, so a
+    transposed or shifted initial-state index lands on a wrong value."""
+    rng = np.random.default_rng(21)
+    batch, dim, L, N = 2, 3, 40, 5
+    A = _f32(-(0.05 + 0.1 * np.arange(dim)[:, None] + 0.37 * np.arange(N)[None, :]))
+    dl = _f32(0.02 + 0.03 * np.arange(dim)).astype(np.float64)
+    delta = _f32(np.broadcast_to(dl[None, :, None], (batch, dim, L)))
+    u = np.zeros((batch, dim, L), np.float32)
+    B = _f32(rng.normal(size=(batch, N, L)))
+    C = _f32(rng.normal(size=(batch, N, L)))
+    z = _f32(rng.normal(size=(batch, dim, L)))
+    Dv = _f32(rng.normal(size=dim))
+    h0 = _distinct_h0(batch, dim, N)
+    y, h = oracle.scan_fwd(u, delta, A, B, C, D=Dv, z=z, softplus=False, h0=h0)
+    A64 = A.astype(np.float64)
+    for t in range(L):
+        ht = np.exp((t + 1) * dl[None, :, None] * A64[None]) * h0
+        ref = np.einsum("bn,bdn->bd", C[:, :, t].astype(np.float64), ht)
+        ref = ref * np.vectorize(oracle.silu)(z[:, :, t].astype(np.float64))
+        assert _rel(y[:, :, t], ref) < 1e-14
+    assert _rel(h, np.exp(L * dl[None, :, None] * A64[None]) * h0) < 1e-14
+
+
+@pytest.mark.parametrize("L", [1, 3, 5])
+def test_initial_state_bruteforce(L):
+    """h_t = (prod_{k<=t} A_bar_k) h0 + sum_{s<=t} (prod_{s<k<=t} A_bar_k) Delta_s B_s u_s
+    with explicit products, softplus and bias on, gate and skip on."""
+    rng = np.random.default_rng(200 + L)
+    batch, dim, N = 2, 3, 4
+    c = _rand_case(rng, batch, dim, L, N)
+    c["A"] = _f32(-rng.uniform(0.1, 3.0, size=(dim, N)))
+    delta = _f32(rng.normal(scale=0.5, size=(batch, dim, L)))
+    bias = _f32(rng.uniform(-4, 0, size=dim))
+    h0 = rng.normal(size=(batch, dim, N))
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                           delta_bias=bias, softplus=True, h0=h0)
+    for b in range(batch):
+        for d in range(dim):
+            dl = [oracle.softplus(float(delta[b, d, t]) + float(bias[d])) for t in range(L)]
+            for t in range(L):
+                acc = 0.0
+                hts = []
+                for n in range(N):
+                    a = float(c["A"][d, n])
+                    lead = 1.0
+                    for k in range(t + 1):
+                        lead *= math.exp(dl[k] * a)
+                    hn = lead * h0[b, d, n]
+                    for s in range(t + 1):
+                        prod = 1.0
+                        for k in range(s + 1, t + 1):
+                            prod *= math.exp(dl[k] * a)
+                        hn += prod * dl[s] * float(c["B"][b, n, s]) * float(c["u"][b, d, s])
+                    hts.append(hn)
+                    acc += float(c["C"][b, n, t]) * hn
+                ref = (acc + float(c["D"][d]) * float(c["u"][b, d, t])) * oracle.silu(float(c["z"][b, d, t]))
+                assert y[b, d, t] == pytest.approx(ref, rel=1e-13, abs=1e-15)
+            assert np.allclose(h[b, d], hts, rtol=1e-13, atol=1e-15)
+
+
+def test_split_sequence_equals_whole():
+    """Scanning [0, P) and then [P, L) from the first part's final state gives
+    the whole scan's outputs on [P, L) and its final state (the carried state is
+    all the past the recurrence keeps)."""
+    w = I.Workload("t", 2, 5, 77, 16, "bf16")
+    x = I.make_inputs(w, seed=12)
+    P = 30
+    cut = lambda k, a, b: np.ascontiguousarray(x[k][:, :, a:b])
+    y, h = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"])
+    y1, h1 = oracle.scan_fwd(cut("u", 0, P), cut("delta", 0, P), x["A"], cut("B", 0, P), cut("C", 0, P),
+                             x["D"], cut("z", 0, P), x["delta_bias"])
+    y2, h2 = oracle.scan_fwd(cut("u", P, 77), cut("delta", P, 77), x["A"], cut("B", P, 77),
+                             cut("C", P, 77), x["D"], cut("z", P, 77), x["delta_bias"], h0=h1)
+    assert np.array_equal(y1, y[:, :, :P])
+    assert _rel(y2, y[:, :, P:]) < 1e-13
+    assert _rel(h2, h) < 1e-13
+
+
+def test_step_chain_equals_scan():
+    """L single-token steps from h0 = 0 reproduce the scan over the L tokens."""
+    w = I.Workload("t", 2, 4, 9, 8, "f32")
+    x = I.make_inputs(w, seed=5)
+    y, h = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"])
+    state = np.zeros((2, 4, 8))
+    for t in range(9):
+        yt, state = oracle.scan_step(state, x["u"][:, :, t], x["delta"][:, :, t], x["A"], x["B"][:, :, t],
+                                     x["C"][:, :, t], x["D"], x["z"][:, :, t], x["delta_bias"])
+        assert np.array_equal(yt, y[:, :, t])
+    assert np.array_equal(state, h)
+
+
 # ------------------------------------------------------- host plumbing -----
 
 def test_channel_subset_matches_full():
