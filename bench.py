@@ -1,9 +1,12 @@
 """Benchmark of the fused selective-scan forward (one B200 per rank).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py --op step [--workload step_...]     (the recurrent decode step)
 
 A step is one pass of the whole hot path (ss_scan_fwd: discretise, scan,
 read out, gate, store y and the final state) over one batch of the workload.
+With `--op step` a step is one ss_scan_step call: every sequence of the batch
+advances its carried state by one token.
 Rank 0 prints one JSON line.  Multi-GPU runs (torchrun, one rank per GPU)
 shard nothing: every rank scans its own full batch of the workload, with no
 data-path collective (weak scaling); the only collectives are the timing
@@ -36,10 +39,11 @@ UNIT = "elements/s"
 L2_BYTES = 126 * 1024 * 1024
 NUM_SMS = 148
 MUFU_EX2_PER_CLK_PER_SM = 16  # ex2 results per clock per SM (special-function unit)
-KERNEL_SOURCES = ("selective_state_space_ss_b200/csrc/ss_scan.cu",
-                  "selective_state_space_ss_b200/csrc/pointwise.cuh",
-                  "selective_state_space_ss_b200/csrc/scan_fwd_chunked.cuh",
-                  "selective_state_space_ss_b200/csrc/scan_common.cuh")
+_CSRC = "selective_state_space_ss_b200/csrc/"
+KERNEL_SOURCES = tuple(_CSRC + f for f in ("ss_scan.cu", "pointwise.cuh", "scan_fwd_chunked.cuh",
+                                           "scan_common.cuh"))
+STEP_KERNEL_SOURCES = tuple(_CSRC + f for f in ("ss_scan.cu", "pointwise.cuh", "scan_step.cuh",
+                                                "scan_common.cuh"))
 
 
 def peaks():
@@ -53,22 +57,22 @@ def peaks():
     return p
 
 
-def kernel_hash() -> str:
+def kernel_hash(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, sources=KERNEL_SOURCES):
     """DRAM bytes per launch from a committed ncu summary, if taken on this kernel source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f).get(workload)
-    if not rec or rec.get("kernel_hash") != kernel_hash():
+    if not rec or rec.get("kernel_hash") != kernel_hash(sources):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -275,6 +279,123 @@ def run_gpu_arm(args, w: I.Workload):
                 nsets=nsets, host=host[0])
 
 
+STEP_METRIC = "selective-scan decode step (B·D) channel-steps/s and % of HBM roofline"
+STEP_UNIT = "channel-steps/s"
+
+
+def run_step_arm(args, w: I.Workload):
+    """One decode step per timed iteration; the state stays on the device."""
+    import torch
+
+    from selective_state_space_ss_b200 import load_library, ss_scan_step
+
+    _, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    load_library()
+    stream = torch.cuda.current_stream(dev)
+    nsets = max(1, -(-4 * L2_BYTES // I.step_bytes(w)))
+    host = [I.make_step_inputs(w, seed=rank_seed(rank, s)) for s in range(nsets)]
+
+    def to_dev(x):
+        return {k: (None if v is None else
+                    (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
+                     else torch.from_numpy(v)).to(dev)) for k, v in x.items()}
+
+    sets = [to_dev(x) for x in host]
+    ys = [torch.empty((w.batch, w.dim), dtype=torch.float32, device=dev) for _ in sets]
+
+    def step(i, st):
+        s = i % nsets
+        x = sets[s]
+        ss_scan_step(x["state"], x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+                     delta_bias=x["delta_bias"], softplus=w.softplus, y_out=ys[s], stream=st)
+
+    for i in range(args.warmup):
+        step(i, stream)
+    torch.cuda.synchronize()
+    # a step takes tens of microseconds, about what one Python call costs: the
+    # timed steps replay a CUDA graph of one step per input set, so the GPU
+    # never waits on the host
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(nsets):
+            step(i, None)  # the capture stream
+    torch.cuda.synchronize()
+    reps = max(1, -(-args.steps // nsets))
+    steps = reps * nsets
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+
+    # end to end: the token's inputs from pinned host memory, the step, y back;
+    # the carried state lives on the device between tokens
+    tok_keys = ("u", "delta", "z", "B", "C")
+    pinned = {k: (torch.from_numpy(host[0][k].view(np.int16)).view(torch.bfloat16)
+                  if host[0][k].dtype == np.uint16 else torch.from_numpy(host[0][k])).pin_memory()
+              for k in tok_keys if host[0][k] is not None}
+    y_host = torch.empty((w.batch, w.dim), dtype=torch.float32).pin_memory()
+    x0 = sets[0]
+    dbuf = {k: torch.empty_like(v, device=dev) for k, v in pinned.items()}
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dbuf[k].copy_(v, non_blocking=True)
+        y = ss_scan_step(x0["state"], dbuf["u"], dbuf["delta"], x0["A"], dbuf["B"], dbuf["C"],
+                         D=x0["D"], z=dbuf.get("z"), delta_bias=x0["delta_bias"], softplus=w.softplus,
+                         y_out=ys[0], stream=stream)
+        y_host.copy_(y, non_blocking=True)
+
+    n_e2e = max(3, min(args.steps, 50))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / n_e2e
+    chans = w.batch * w.dim
+    p = peaks()
+    achieved = I.step_bytes(w) / (ms * 1e-3) / 1e9
+    line = {"metric": STEP_METRIC, "value": chans / (ms * 1e-3), "unit": STEP_UNIT, "n_gpus": 1,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
+                       "in_dtype": w.dtype, "state_dtype": "f32", "y_dtype": "f32",
+                       "l2": "inputs and states rotated over sets totalling >= 4x L2; no flush"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": p["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / p["hbm_gbs"],
+                         "traffic": profiled_traffic(w.name, STEP_KERNEL_SOURCES),
+                         "bytes_per_step": I.step_bytes(w), "peak_source": f"HBM copy, {p['source']}"},
+            "e2e": {"value": chans / (e2e_ms * 1e-3), "unit": STEP_UNIT,
+                    "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in pinned.values()),
+                    "d2h_bytes_per_step": y_host.numel() * 4},
+            "gpu_launches": steps, "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        import oracle
+
+        x = host[0]
+        cores = os.cpu_count() or 1
+        reps, t0 = 0, time.perf_counter()
+        while reps < 1 or (time.perf_counter() - t0 < 5.0 and reps < 50):
+            oracle.scan_step(x["state"], x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                             x["delta_bias"], softplus=w.softplus, nthreads=cores)
+            reps += 1
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": reps * chans / dt, "unit": STEP_UNIT, "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{reps} full steps of {chans} channels, fp64, {cores} threads"}
+    return line
+
+
 def roofline(w: I.Workload, kernel_ms: float):
     p = peaks()
     t_hbm = w.algorithmic_bytes() / (p["hbm_gbs"] * 1e9)
@@ -364,13 +485,23 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--op", default="scan", choices=["scan", "step"])
+    ap.add_argument("--workload", default=None,
+                    choices=sorted(I.WORKLOADS) + sorted(I.STEP_WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    w = I.WORKLOADS[args.workload]
+    if args.op == "step":
+        if args.impl != "native" or args.gpus != 1:
+            ap.error("--op step runs the native arm on one GPU")
+        w = I.STEP_WORKLOADS[args.workload or "step_b128_d8192_n16_bf16"]
+        print(json.dumps(run_step_arm(args, w)), flush=True)
+        return
+    if args.workload in I.STEP_WORKLOADS:
+        ap.error("decode-step workloads run with --op step")
+    w = I.WORKLOADS[args.workload or DEFAULT_WORKLOAD]
 
     if args.impl == "reference":
         line = run_reference_arm(args, w)

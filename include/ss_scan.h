@@ -86,6 +86,63 @@ ss_status ss_scan_fwd(const void* u, const void* delta, const float* A,
                       size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * ss_scan_fwd_from_state -- ss_scan_fwd started from a carried state instead
+ * of zero: h[n] = initial_state[b,d,n] before t = 0.  This continues a
+ * sequence across calls (a long prompt fed in pieces, or a prompt after
+ * earlier turns of a dialogue); the pages keep h between calls for recurrent
+ * inference ("从Transformer的痛点说起 ... Mamba", sec. 5.1 table and sec. 6.3).
+ * Scanning [0, P) and then [P, L) from the first call's last_state gives the
+ * outputs of one call over [0, L), up to fp32 rounding.
+ *
+ *  initial_state [batch, dim, dstate]  float32, nullable (then exactly
+ *                ss_scan_fwd).  It may be the same buffer as last_state_out
+ *                (the state is then advanced in place); any other overlap
+ *                with an output is not allowed.
+ *
+ * Every other argument, layout, result and error is that of ss_scan_fwd; the
+ * workspace size is the same ss_scan_workspace_bytes(...).
+ */
+ss_status ss_scan_fwd_from_state(const void* u, const void* delta, const float* A,
+                                 const void* B, const void* C, const float* D,
+                                 const void* z, const float* delta_bias,
+                                 int softplus_flag, const float* initial_state,
+                                 float* y_out, float* last_state_out,
+                                 int64_t batch, int64_t dim, int64_t seqlen,
+                                 int dstate, ss_dtype in_dtype, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * ss_scan_step -- one recurrent (decode) step: the same recurrence over a
+ * single token, advancing a carried state in place ("从Transformer的痛点说起
+ * ... Mamba", sec. 5.1 table: O(1) work and memory per generated token;
+ * sec. 6.3: the state h is kept per sample between steps).  For every b, d, n:
+ *
+ *   Delta      = softplus(delta[b,d] + delta_bias[d])  (or without softplus)
+ *   state[b,d,n] <- exp(Delta * A[d,n]) * state[b,d,n] + Delta * B[b,n] * u[b,d]
+ *   y[b,d]     = (sum_n C[b,n] * state[b,d,n] + D[d] * u[b,d]) * SiLU(z[b,d])
+ *
+ *  u, delta, z   [batch, dim]          in_dtype     (z nullable: no gate)
+ *  A             [dim, dstate]         float32
+ *  B, C          [batch, dstate]       in_dtype
+ *  D, delta_bias [dim]                 float32      (nullable: 0)
+ *  state         [batch, dim, dstate]  float32, read and written in place
+ *  y_out         [batch, dim]          float32 (written); must not overlap state
+ *  batch, dim >= 1, batch*dim*dstate <= 2^56, dim*dstate < 2^31;
+ *  dstate 16, 32, 64 or 128
+ *
+ * Device pointers, caller-owned, contiguous, each aligned to its element
+ * size; 16-byte aligned state and A and (4 * element size)-aligned B and C
+ * take vector loads, anything else element-wise loads (correct, slower).
+ * No workspace.  Returns SS_OK after the launch, or an error code with nothing
+ * launched (SS_ERR_INVALID_ARG, SS_ERR_UNSUPPORTED, SS_ERR_CUDA).
+ */
+ss_status ss_scan_step(const void* u, const void* delta, const float* A,
+                       const void* B, const void* C, const float* D,
+                       const void* z, const float* delta_bias, int softplus_flag,
+                       float* state, float* y_out, int64_t batch, int64_t dim,
+                       int dstate, ss_dtype in_dtype, cudaStream_t stream);
+
+/*
  * ss_scan_fwd_noalloc -- ss_scan_fwd for callers that cannot allocate device
  * memory at the point of the call: for example a plugin running inside a host
  * framework that owns every device allocation (a cudaMalloc of its own would

@@ -1,7 +1,8 @@
 /*
  * ss_scan_debug.h -- test hooks of libssscan.so.  Not for production use.
  *
- * Each setting is picked up by the NEXT ss_scan_fwd call in the process and
+ * Each setting is picked up by the NEXT ss_scan_fwd (SS_DEBUG_STEP_SIMPLE:
+ * ss_scan_step) call in the process and
  * then cleared (ss_scan_workspace_bytes honours a pending worker count, so a
  * test can size the workspace for it).  They exist so that tests can drive the
  * load-balanced schedule and its bounded carry waits on small problems:
@@ -16,6 +17,9 @@
  *                           are then unspecified.
  *   SS_DEBUG_SPIN_LIMIT     value = polls (with back-off) before a carry wait
  *                           gives up, so that test finishes quickly.
+ *   SS_DEBUG_STEP_SIMPLE    value != 0: the next ss_scan_step call takes the
+ *                           plain-load kernel even where the bulk-copy
+ *                           pipeline applies, so both are tested on one shape.
  *   SS_DEBUG_CLEAR          value ignored: drop every pending setting.
  *
  * Returns SS_OK, or SS_ERR_INVALID_ARG for an unknown `what`.  Host-only,
@@ -34,7 +38,8 @@ enum {
   SS_DEBUG_CLEAR = 0,
   SS_DEBUG_FORCE_WORKERS = 1,
   SS_DEBUG_SKIP_PUBLISH = 2,
-  SS_DEBUG_SPIN_LIMIT = 3
+  SS_DEBUG_SPIN_LIMIT = 3,
+  SS_DEBUG_STEP_SIMPLE = 4
 };
 
 ss_status ss_debug_inject(int what, long long value);

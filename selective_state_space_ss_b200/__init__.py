@@ -1,4 +1,4 @@
-"""B200-native S6 selective-scan forward.
+"""B200-native S6 selective scan: the fused forward and the recurrent step.
 
 The compute lives in libssscan.so (hand-written sm_100a CUDA, C ABI in
 include/ss_scan.h); this package is its Python binding plus the seeded input
@@ -11,6 +11,7 @@ from ._native import (  # noqa: F401
     SS_DEBUG_FORCE_WORKERS,
     SS_DEBUG_SKIP_PUBLISH,
     SS_DEBUG_SPIN_LIMIT,
+    SS_DEBUG_STEP_SIMPLE,
     SS_BF16,
     SS_ERR_CUDA,
     SS_ERR_INVALID_ARG,
@@ -25,7 +26,9 @@ from ._native import (  # noqa: F401
     ss_debug_inject,
     ss_last_device_error,
     ss_scan_fwd,
+    ss_scan_fwd_from_state,
     ss_scan_fwd_noalloc,
+    ss_scan_step,
     ss_scan_workspace_bytes,
     ss_status_string,
 )

@@ -22,13 +22,15 @@ SS_OK, SS_ERR_INVALID_ARG, SS_ERR_UNSUPPORTED, SS_ERR_CUDA, SS_ERR_TIMEOUT = ran
 SS_F32, SS_BF16 = 0, 1
 
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
-            "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc")
+            "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc",
+            "ss_scan_fwd_from_state", "ss_scan_step")
 
 # bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
 SS_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 # test hooks (include/ss_scan_debug.h)
-SS_DEBUG_CLEAR, SS_DEBUG_FORCE_WORKERS, SS_DEBUG_SKIP_PUBLISH, SS_DEBUG_SPIN_LIMIT = range(4)
+(SS_DEBUG_CLEAR, SS_DEBUG_FORCE_WORKERS, SS_DEBUG_SKIP_PUBLISH, SS_DEBUG_SPIN_LIMIT,
+ SS_DEBUG_STEP_SIMPLE) = range(5)
 
 
 class SSError(RuntimeError):
@@ -67,6 +69,11 @@ def load_library():
         lib.ss_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp,
                                             i64, i64, i64, ci, ci, vp]
         lib.ss_scan_fwd_noalloc.restype = ci
+        lib.ss_scan_fwd_from_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp,
+                                               i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
+        lib.ss_scan_fwd_from_state.restype = ci
+        lib.ss_scan_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, i64, i64, ci, ci, vp]
+        lib.ss_scan_step.restype = ci
         _lib = lib
         return lib
 
@@ -94,7 +101,7 @@ def ss_last_device_error(stream=None) -> int:
 
 
 def ss_debug_inject(what: int, value: int = 0) -> None:
-    """Test hook for the next ss_scan_fwd call (see include/ss_scan_debug.h)."""
+    """Test hook for the next ss_scan_fwd / ss_scan_step call (include/ss_scan_debug.h)."""
     st = load_library().ss_debug_inject(int(what), int(value))
     if st != SS_OK:
         raise SSError(st, "ss_debug_inject")
@@ -117,21 +124,10 @@ def _check_dev(name, t, device, dtypes, shape=None):
         raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
 
 
-def ss_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                y_out=None, last_state_out=None, return_last_state=True,
-                workspace=None, stream=None):
-    """Fused selective-scan forward on the GPU.
-
-    u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; one dtype, float32 or
-    bfloat16.  A: [dim, N] float32; D, delta_bias: [dim] float32 (optional).
-    Returns (y [batch, dim, L] float32, last_state [batch, dim, N] float32 or
-    None).  Output and workspace tensors are allocated with torch when not
-    given; the library itself allocates nothing.
-    """
-    lib = load_library()
+def _fwd_operands(u, delta, A, B, C, D, z, delta_bias):
     device = u.device
     if device.type != "cuda":
-        raise ValueError("ss_scan_fwd runs on CUDA tensors only (no CPU fallback)")
+        raise ValueError("the scan runs on CUDA tensors only (no CPU fallback)")
     if u.dim() != 3 or B.dim() != 3:
         raise ValueError("u must be [batch, dim, L] and B [batch, N, L]")
     batch, dim, L = u.shape
@@ -146,6 +142,13 @@ def ss_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
     _check_dev("A", A, device, (torch.float32,), (dim, N))
     _check_dev("D", D, device, (torch.float32,), (dim,))
     _check_dev("delta_bias", delta_bias, device, (torch.float32,), (dim,))
+    return device, batch, dim, L, N
+
+
+def _fwd_call(name, initial_state, u, delta, A, B, C, D, z, delta_bias, softplus, y_out,
+              last_state_out, return_last_state, workspace, stream):
+    lib = load_library()
+    device, batch, dim, L, N = _fwd_operands(u, delta, A, B, C, D, z, delta_bias)
     if y_out is None:
         y_out = torch.empty((batch, dim, L), dtype=torch.float32, device=device)
     _check_dev("y_out", y_out, device, (torch.float32,), (batch, dim, L))
@@ -157,13 +160,80 @@ def ss_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     dt = SS_F32 if u.dtype == torch.float32 else SS_BF16
-    st = lib.ss_scan_fwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-                         _ptr(delta_bias), int(bool(softplus)), _ptr(y_out), _ptr(last_state_out),
-                         batch, dim, L, N, dt, _ptr(workspace), ws_bytes,
-                         _stream_handle(stream, device))
+    head = (_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus)))
+    tail = (_ptr(y_out), _ptr(last_state_out), batch, dim, L, N, dt, _ptr(workspace), ws_bytes,
+            _stream_handle(stream, device))
+    if name == "ss_scan_fwd":
+        st = lib.ss_scan_fwd(*head, *tail)
+    else:
+        _check_dev("initial_state", initial_state, device, (torch.float32,), (batch, dim, N))
+        st = lib.ss_scan_fwd_from_state(*head, _ptr(initial_state), *tail)
     if st != SS_OK:
-        raise SSError(st, "ss_scan_fwd")
+        raise SSError(st, name)
     return y_out, last_state_out
+
+
+def ss_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                y_out=None, last_state_out=None, return_last_state=True,
+                workspace=None, stream=None):
+    """Fused selective-scan forward on the GPU.
+
+    u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; one dtype, float32 or
+    bfloat16.  A: [dim, N] float32; D, delta_bias: [dim] float32 (optional).
+    Returns (y [batch, dim, L] float32, last_state [batch, dim, N] float32 or
+    None).  Output and workspace tensors are allocated with torch when not
+    given; the library itself allocates nothing.
+    """
+    return _fwd_call("ss_scan_fwd", None, u, delta, A, B, C, D, z, delta_bias, softplus, y_out,
+                     last_state_out, return_last_state, workspace, stream)
+
+
+def ss_scan_fwd_from_state(initial_state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                           softplus=True, y_out=None, last_state_out=None,
+                           return_last_state=True, workspace=None, stream=None):
+    """ss_scan_fwd started from initial_state [batch, dim, N] float32 (None:
+    zero).  last_state_out may be initial_state itself (in-place advance)."""
+    return _fwd_call("ss_scan_fwd_from_state", initial_state, u, delta, A, B, C, D, z,
+                     delta_bias, softplus, y_out, last_state_out, return_last_state, workspace,
+                     stream)
+
+
+def ss_scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                 y_out=None, stream=None):
+    """One recurrent (decode) step; advances state [batch, dim, N] float32 in place.
+
+    u, delta, z: [batch, dim]; B, C: [batch, N]; float32 or bfloat16.
+    Returns y [batch, dim] float32.
+    """
+    lib = load_library()
+    device = state.device
+    if device.type != "cuda":
+        raise ValueError("ss_scan_step runs on CUDA tensors only (no CPU fallback)")
+    if state.dim() != 3:
+        raise ValueError("state must be [batch, dim, N]")
+    batch, dim, N = state.shape
+    _check_dev("state", state, device, (torch.float32,), (batch, dim, N))
+    in_types = (torch.float32, torch.bfloat16)
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _check_dev(name, t, device, in_types, (batch, dim))
+    for name, t in (("B", B), ("C", C)):
+        _check_dev(name, t, device, in_types, (batch, N))
+    if len({t.dtype for t in (u, delta, B, C, z) if t is not None}) != 1:
+        raise ValueError("u, delta, B, C and z must share one dtype")
+    _check_dev("A", A, device, (torch.float32,), (dim, N))
+    _check_dev("D", D, device, (torch.float32,), (dim,))
+    _check_dev("delta_bias", delta_bias, device, (torch.float32,), (dim,))
+    if y_out is None:
+        y_out = torch.empty((batch, dim), dtype=torch.float32, device=device)
+    _check_dev("y_out", y_out, device, (torch.float32,), (batch, dim))
+    dt = SS_F32 if u.dtype == torch.float32 else SS_BF16
+    st = lib.ss_scan_step(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                          _ptr(delta_bias), int(bool(softplus)), _ptr(state), _ptr(y_out),
+                          batch, dim, N, dt, _stream_handle(stream, device))
+    if st != SS_OK:
+        raise SSError(st, "ss_scan_step")
+    return y_out
 
 
 def ss_scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,

@@ -47,6 +47,7 @@ struct FwdArgs {
   const float* delta_bias;  // nullable
   float* y;
   float* last_state;  // nullable
+  const float* h0;    // [batch, dim, N] initial state, nullable (zero); may be last_state
   int64_t batch, dim, seqlen;
   int softplus;
   int vec;  // 1: TMA path (16-byte aligned rows); 0: element-wise loads
@@ -674,7 +675,9 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
 #pragma unroll
     for (int g = 0; g < CF::G / 2; ++g) {
       const int n = j * CF::G + 2 * g;
-      h[g] = make_float2(0.f, 0.f);
+      // plain loads: h0 may be the last_state buffer this kernel writes
+      const float* h0 = a.h0 + (b * a.dim + d) * CF::N + n;
+      h[g] = (a.h0 && chan_ok) ? make_float2(h0[0], h0[1]) : make_float2(0.f, 0.f);
       a2[g] = chan_ok ? make_float2(__ldg(a.A + d * CF::N + n) * 1.4426950408889634f,
                                     __ldg(a.A + d * CF::N + n + 1) * 1.4426950408889634f)
                       : make_float2(0.f, 0.f);
@@ -819,8 +822,14 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
         a2[g] = chan_ok ? make_float2(__ldg(a.A + d * CF::N + n) * 1.4426950408889634f,
                                       __ldg(a.A + d * CF::N + n + 1) * 1.4426950408889634f)
                         : make_float2(0.f, 0.f);
-        h[g] = cin ? make_float2(__ldcg(cin + c * CF::N + n), __ldcg(cin + c * CF::N + n + 1))
-                   : make_float2(0.f, 0.f);
+        if (cin)
+          h[g] = make_float2(__ldcg(cin + c * CF::N + n), __ldcg(cin + c * CF::N + n + 1));
+        else if (a.h0 && chan_ok) {  // a piece that starts the group (chunk 0)
+          const float* h0 = a.h0 + ((int64_t)cur.b * a.dim + d) * CF::N + n;
+          h[g] = make_float2(h0[0], h0[1]);
+        }
+        else
+          h[g] = make_float2(0.f, 0.f);
       }
       ok = ok && have;
     }

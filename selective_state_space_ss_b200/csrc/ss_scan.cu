@@ -12,6 +12,7 @@
 #include "ss_scan.h"
 #include "ss_scan_debug.h"
 #include "scan_fwd_chunked.cuh"
+#include "scan_step.cuh"
 
 namespace ssscan {
 
@@ -68,6 +69,7 @@ bool encode_maps(const FwdArgs& a, FwdMaps* m) {
 std::atomic<long long> g_dbg_workers{0};
 std::atomic<long long> g_dbg_skip_publish{-1};
 std::atomic<long long> g_dbg_spin_limit{0};
+std::atomic<long long> g_dbg_step_simple{0};
 
 constexpr uint32_t kCarrySpinLimit = 1u << 22;  // ~1 s of polling with back-off
 
@@ -280,6 +282,93 @@ bool plan_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N, size_t* bytes
 
 bool supported_dstate(int n) { return n == 16 || n == 32 || n == 64 || n == 128; }
 
+template <typename E, int N>
+ss_status launch_step(const StepArgs& a, bool vec, cudaStream_t stream) {
+  constexpr int64_t per_block = kStepThreads * kStepUnits;
+  const int64_t bx = (a.dim * (N / 4) + per_block - 1) / per_block;
+  if (bx > INT_MAX) return SS_ERR_INVALID_ARG;
+  const dim3 grid((unsigned)bx, (unsigned)(a.batch < 65535 ? a.batch : 65535));
+  if (vec) scan_step_kernel<E, N, true><<<grid, kStepThreads, 0, stream>>>(a);
+  else scan_step_kernel<E, N, false><<<grid, kStepThreads, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+// The bulk-copy pipeline: persistent CTAs, as many as fit on the device at once.
+template <typename E, int N>
+ss_status launch_step_pipe(const StepArgs& a, cudaStream_t stream) {
+  using CF = StepPipeCfg<E, N>;
+  static int state = 0;  // 0 unknown, 1 ok, -1 failed
+  static int occ = 0;
+  if (state == 0) {
+    state = (cudaFuncSetAttribute(scan_step_pipe_kernel<E, N>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) ==
+                 cudaSuccess &&
+             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_step_pipe_kernel<E, N>, CF::NT,
+                                                           CF::SMEM_BYTES) == cudaSuccess &&
+             occ > 0)
+                ? 1
+                : -1;
+  }
+  if (state != 1) return SS_ERR_CUDA;
+  StepPipeSched sc;
+  sc.tiles_per_row = (a.dim + CF::TILE_CH - 1) / CF::TILE_CH;
+  sc.items = sc.tiles_per_row * a.batch;
+  const int64_t slots = (int64_t)device_sms() * occ;
+  if (slots < 1) return SS_ERR_CUDA;
+  const int64_t grid = sc.items < slots ? sc.items : slots;
+  scan_step_pipe_kernel<E, N><<<(unsigned)grid, CF::NT, CF::SMEM_BYTES, stream>>>(a, sc);
+  return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+template <typename E>
+ss_status dispatch_step(const StepArgs& a, int N, bool vec, bool pipe, cudaStream_t stream) {
+  switch (N) {
+    case 16: return pipe ? launch_step_pipe<E, 16>(a, stream) : launch_step<E, 16>(a, vec, stream);
+    case 32: return pipe ? launch_step_pipe<E, 32>(a, stream) : launch_step<E, 32>(a, vec, stream);
+    case 64: return pipe ? launch_step_pipe<E, 64>(a, stream) : launch_step<E, 64>(a, vec, stream);
+    case 128: return pipe ? launch_step_pipe<E, 128>(a, stream) : launch_step<E, 128>(a, vec, stream);
+    default: return SS_ERR_UNSUPPORTED;
+  }
+}
+
+ss_status scan_fwd_impl(const void* u, const void* delta, const float* A, const void* B,
+                        const void* C, const float* D, const void* z, const float* delta_bias,
+                        int softplus_flag, const float* h0, float* y_out, float* last_state_out,
+                        int64_t batch, int64_t dim, int64_t seqlen, int dstate,
+                        ss_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  if (!u || !delta || !A || !B || !C || !y_out) return SS_ERR_INVALID_ARG;
+  if (batch < 1 || dim < 1 || seqlen < 1) return SS_ERR_INVALID_ARG;
+  if (in_dtype != SS_F32 && in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED;
+  if (!supported_dstate(dstate)) return SS_ERR_UNSUPPORTED;
+  // batch*dim*seqlen and batch*dstate*seqlen must stay far from int64 overflow
+  if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
+    return SS_ERR_INVALID_ARG;
+  if (batch * (int64_t)dstate > (INT64_C(1) << 62) / seqlen) return SS_ERR_INVALID_ARG;
+  const size_t es = in_dtype == SS_F32 ? 4 : 2;
+  const void* in_ptrs[5] = {u, delta, z, B, C};
+  for (const void* p : in_ptrs)
+    if (p && !aligned(p, es)) return SS_ERR_INVALID_ARG;
+  const void* f_ptrs[6] = {A, D, delta_bias, y_out, last_state_out, h0};
+  for (const void* p : f_ptrs)
+    if (p && !aligned(p, 4)) return SS_ERR_INVALID_ARG;
+
+  FwdArgs a;
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.A = A; a.D = D; a.delta_bias = delta_bias;
+  a.y = y_out; a.last_state = last_state_out; a.h0 = h0;
+  a.batch = batch; a.dim = dim; a.seqlen = seqlen;
+  a.softplus = softplus_flag != 0;
+  bool vec = ((size_t)seqlen * es) % 16 == 0;
+  for (const void* p : in_ptrs)
+    if (p && !aligned(p, 16)) vec = false;
+  if (!aligned(y_out, 16)) vec = false;
+  a.vec = vec ? 1 : 0;
+
+  if (in_dtype == SS_F32) return dispatch_dtype<float>(a, dstate, workspace, workspace_bytes, stream);
+  return dispatch_dtype<__nv_bfloat16>(a, dstate, workspace, workspace_bytes, stream);
+}
+
 }  // namespace
 }  // namespace ssscan
 
@@ -303,36 +392,54 @@ ss_status ss_scan_fwd(const void* u, const void* delta, const float* A, const vo
                       int softplus_flag, float* y_out, float* last_state_out, int64_t batch,
                       int64_t dim, int64_t seqlen, int dstate, ss_dtype in_dtype,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  if (!u || !delta || !A || !B || !C || !y_out) return SS_ERR_INVALID_ARG;
-  if (batch < 1 || dim < 1 || seqlen < 1) return SS_ERR_INVALID_ARG;
+  return scan_fwd_impl(u, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, y_out,
+                       last_state_out, batch, dim, seqlen, dstate, in_dtype, workspace,
+                       workspace_bytes, stream);
+}
+
+ss_status ss_scan_fwd_from_state(const void* u, const void* delta, const float* A,
+                                 const void* B, const void* C, const float* D, const void* z,
+                                 const float* delta_bias, int softplus_flag,
+                                 const float* initial_state, float* y_out, float* last_state_out,
+                                 int64_t batch, int64_t dim, int64_t seqlen, int dstate,
+                                 ss_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+  return scan_fwd_impl(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y_out,
+                       last_state_out, batch, dim, seqlen, dstate, in_dtype, workspace,
+                       workspace_bytes, stream);
+}
+
+ss_status ss_scan_step(const void* u, const void* delta, const float* A, const void* B,
+                       const void* C, const float* D, const void* z, const float* delta_bias,
+                       int softplus_flag, float* state, float* y_out, int64_t batch, int64_t dim,
+                       int dstate, ss_dtype in_dtype, cudaStream_t stream) {
+  if (!u || !delta || !A || !B || !C || !state || !y_out) return SS_ERR_INVALID_ARG;
+  if (batch < 1 || dim < 1) return SS_ERR_INVALID_ARG;
   if (in_dtype != SS_F32 && in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED;
   if (!supported_dstate(dstate)) return SS_ERR_UNSUPPORTED;
-  // batch*dim*seqlen and batch*dstate*seqlen must stay far from int64 overflow
-  if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
-    return SS_ERR_INVALID_ARG;
-  if (batch * (int64_t)dstate > (INT64_C(1) << 62) / seqlen) return SS_ERR_INVALID_ARG;
+  if (batch > (INT64_C(1) << 56) / dim / dstate) return SS_ERR_INVALID_ARG;
+  if (dim * dstate > INT32_MAX) return SS_ERR_INVALID_ARG;  // one row's state indexes in 32 bits
   const size_t es = in_dtype == SS_F32 ? 4 : 2;
   const void* in_ptrs[5] = {u, delta, z, B, C};
   for (const void* p : in_ptrs)
     if (p && !aligned(p, es)) return SS_ERR_INVALID_ARG;
-  const void* f_ptrs[5] = {A, D, delta_bias, y_out, last_state_out};
+  const void* f_ptrs[5] = {A, D, delta_bias, state, y_out};
   for (const void* p : f_ptrs)
     if (p && !aligned(p, 4)) return SS_ERR_INVALID_ARG;
-
-  FwdArgs a;
+  StepArgs a;
   a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.A = A; a.D = D; a.delta_bias = delta_bias;
-  a.y = y_out; a.last_state = last_state_out;
-  a.batch = batch; a.dim = dim; a.seqlen = seqlen;
+  a.state = state; a.y = y_out;
+  a.batch = batch; a.dim = dim;
   a.softplus = softplus_flag != 0;
-  bool vec = ((size_t)seqlen * es) % 16 == 0;
+  const bool vec = aligned(state, 16) && aligned(A, 16) && aligned(B, 4 * es) && aligned(C, 4 * es);
+  // bulk copies need 16-byte aligned sources and sizes: every row of u, delta
+  // and z (dim * es bytes) and the state, B, C and A bases
+  bool pipe = vec && (dim * (int64_t)es) % 16 == 0 && g_dbg_step_simple.exchange(0) == 0;
   for (const void* p : in_ptrs)
-    if (p && !aligned(p, 16)) vec = false;
-  if (!aligned(y_out, 16)) vec = false;
-  a.vec = vec ? 1 : 0;
-
-  if (in_dtype == SS_F32) return dispatch_dtype<float>(a, dstate, workspace, workspace_bytes, stream);
-  return dispatch_dtype<__nv_bfloat16>(a, dstate, workspace, workspace_bytes, stream);
+    if (p && !aligned(p, 16)) pipe = false;
+  if (in_dtype == SS_F32) return dispatch_step<float>(a, dstate, vec, pipe, stream);
+  return dispatch_step<__nv_bfloat16>(a, dstate, vec, pipe, stream);
 }
 
 ss_status ss_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B,
@@ -373,7 +480,9 @@ ss_status ss_debug_inject(int what, long long value) {
     case SS_DEBUG_FORCE_WORKERS: g_dbg_workers.store(value); return SS_OK;
     case SS_DEBUG_SKIP_PUBLISH: g_dbg_skip_publish.store(value); return SS_OK;
     case SS_DEBUG_SPIN_LIMIT: g_dbg_spin_limit.store(value); return SS_OK;
+    case SS_DEBUG_STEP_SIMPLE: g_dbg_step_simple.store(value); return SS_OK;
     case SS_DEBUG_CLEAR:
+      g_dbg_step_simple.store(0);
       g_dbg_workers.store(0);
       g_dbg_skip_publish.store(-1);
       g_dbg_spin_limit.store(0);

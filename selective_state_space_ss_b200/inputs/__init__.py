@@ -13,6 +13,12 @@ described in "从Transformer的痛点说起 ... Mamba", sec. 4.2 and 6.2):
   A[d, n] = -(n + 1) * (1 + 0.1 U) with U ~ U(0, 1);
   D[d] ~ N(0, 1).
 Activations use the layout [batch, dim, L] and B, C use [batch, N, L], L fastest.
+
+A carried state (initial state of a continued scan, or the state a decode step
+advances) is drawn as N(0, 1) fp32 [batch, dim, N]: the magnitude of a state
+after many steps of unit-variance inputs with Delta*B*u of order 0.01-1.
+Decode-step workloads are Workload objects with seqlen = 1 (one token per
+channel); their tensors drop the L axis.
 """
 from __future__ import annotations
 
@@ -31,7 +37,7 @@ _lock = threading.Lock()
 _lib = None
 
 # stream ids: one independent counter-based stream per tensor
-STREAM = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "A": 6, "D": 7, "dt": 8}
+STREAM = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "A": 6, "D": 7, "dt": 8, "h0": 9}
 
 
 def build(force: bool = False) -> str:
@@ -164,3 +170,43 @@ def make_inputs(w: Workload, seed: int = 1234, nthreads: int | None = None) -> d
     else:
         x["delta_bias"] = None
     return x
+
+
+def make_state(batch: int, dim: int, dstate: int, seed: int = 1234, scale: float = 1.0,
+               nthreads: int | None = None) -> np.ndarray:
+    """A carried state [batch, dim, dstate] float32, N(0, scale^2)."""
+    return fill(seed, STREAM["h0"], (batch, dim, dstate), scale=scale, nthreads=nthreads)
+
+
+def make_step_inputs(w: Workload, seed: int = 1234, nthreads: int | None = None) -> dict:
+    """Inputs of one decode step: make_inputs at seqlen 1 with the L axis
+    dropped (u, delta, z [batch, dim]; B, C [batch, N]) plus the carried
+    state [batch, dim, N] under key "state"."""
+    if w.seqlen != 1:
+        raise ValueError("a decode-step workload has seqlen 1")
+    x = make_inputs(w, seed=seed, nthreads=nthreads)
+    for k in ("u", "delta", "z", "B", "C"):
+        if x[k] is not None:
+            x[k] = np.ascontiguousarray(x[k][..., 0])
+    x["state"] = make_state(w.batch, w.dim, w.dstate, seed=seed, nthreads=nthreads)
+    return x
+
+
+def step_bytes(w: Workload) -> int:
+    """Bytes one decode step must move: the state read and written once, the
+    token's inputs, B and C, A, D and the bias, and y."""
+    es = 4 if w.dtype == "f32" else 2
+    ch = w.batch * w.dim
+    n_act = 2 + (1 if w.with_z else 0)
+    rd = ch * w.dstate * 4 + n_act * ch * es + 2 * w.batch * w.dstate * es
+    rd += w.dim * w.dstate * 4 + w.dim * 4 * ((1 if w.with_D else 0) + (1 if w.with_bias else 0))
+    wr = ch * w.dstate * 4 + ch * 4
+    return rd + wr
+
+
+# Decode-step workloads: a batch of sequences advancing one token through one
+# layer of a Mamba-6.9B-wide model (d_model 4096, expand 2: dim 8192).
+STEP_WORKLOADS = {
+    "step_b128_d8192_n16_bf16": Workload("step_b128_d8192_n16_bf16", 128, 8192, 1, 16, "bf16"),
+    "step_b128_d8192_n16_f32": Workload("step_b128_d8192_n16_f32", 128, 8192, 1, 16, "f32"),
+}

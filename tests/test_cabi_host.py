@@ -87,6 +87,48 @@ def test_misaligned(lib, field, addr, dt):
     assert _call(lib, **{field: addr, "dt": dt}) == N.SS_ERR_INVALID_ARG
 
 
+def _call_state(lib, **over):
+    a = dict(u=0x10000, delta=0x20000, A=0x30000, B=0x40000, C=0x50000, D=None, z=None,
+             bias=None, sp=1, h0=0x70000, y=0x60000, h=None, batch=1, dim=1, L=8, N=16,
+             dt=N.SS_F32, ws=None, wsb=0)
+    a.update(over)
+    return lib.ss_scan_fwd_from_state(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                                      a["bias"], a["sp"], a["h0"], a["y"], a["h"], a["batch"],
+                                      a["dim"], a["L"], a["N"], a["dt"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(u=None), N.SS_ERR_INVALID_ARG), (dict(y=None), N.SS_ERR_INVALID_ARG),
+    (dict(h0=0x70002), N.SS_ERR_INVALID_ARG), (dict(L=0), N.SS_ERR_INVALID_ARG),
+    (dict(N=24), N.SS_ERR_UNSUPPORTED), (dict(dt=5), N.SS_ERR_UNSUPPORTED)])
+def test_from_state_rejections(lib, over, status):
+    assert _call_state(lib, **over) == status
+
+
+def _call_step(lib, **over):
+    a = dict(u=0x10000, delta=0x20000, A=0x30000, B=0x40000, C=0x50000, D=None, z=None,
+             bias=None, sp=1, state=0x70000, y=0x60000, batch=1, dim=1, N=16, dt=N.SS_F32)
+    a.update(over)
+    return lib.ss_scan_step(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
+                            a["sp"], a["state"], a["y"], a["batch"], a["dim"], a["N"], a["dt"], None)
+
+
+@pytest.mark.parametrize("field", ["u", "delta", "A", "B", "C", "state", "y"])
+def test_step_null_required_pointer(lib, field):
+    assert _call_step(lib, **{field: None}) == N.SS_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(batch=0), N.SS_ERR_INVALID_ARG), (dict(dim=-3), N.SS_ERR_INVALID_ARG),
+    (dict(batch=1 << 40, dim=1 << 20), N.SS_ERR_INVALID_ARG),
+    (dict(dim=1 << 28), N.SS_ERR_INVALID_ARG),
+    (dict(N=8), N.SS_ERR_UNSUPPORTED), (dict(N=256), N.SS_ERR_UNSUPPORTED),
+    (dict(dt=2), N.SS_ERR_UNSUPPORTED), (dict(state=0x70002), N.SS_ERR_INVALID_ARG),
+    (dict(u=0x10001, dt=N.SS_BF16), N.SS_ERR_INVALID_ARG), (dict(D=0x80002), N.SS_ERR_INVALID_ARG)])
+def test_step_rejections(lib, over, status):
+    assert _call_step(lib, **over) == status
+
+
 def test_workspace_query_rejects_bad_sizes(lib):
     # (valid sizes need the device's SM count, so they are covered by the GPU tests)
     with pytest.raises(N.SSError):
@@ -101,3 +143,10 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 2, 8)
     with pytest.raises(ValueError):
         N.ss_scan_fwd(x, x, torch.zeros(2, 16), torch.zeros(1, 16, 8), torch.zeros(1, 16, 8))
+    with pytest.raises(ValueError):
+        N.ss_scan_fwd_from_state(torch.zeros(1, 2, 16), x, x, torch.zeros(2, 16),
+                                 torch.zeros(1, 16, 8), torch.zeros(1, 16, 8))
+    t = torch.zeros(1, 2)
+    with pytest.raises(ValueError):
+        N.ss_scan_step(torch.zeros(1, 2, 16), t, t, torch.zeros(2, 16), torch.zeros(1, 16),
+                       torch.zeros(1, 16))
