@@ -47,7 +47,7 @@ def _load():
             vp, i64 = ctypes.c_void_p, ctypes.c_int64
             lib.oracle_scan_fwd.argtypes = [
                 vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
-                i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, vp, ctypes.c_int]
+                i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int]
             lib.oracle_scan_fwd.restype = ctypes.c_int
             lib.oracle_softplus.argtypes = [ctypes.c_double]
             lib.oracle_softplus.restype = ctypes.c_double
@@ -72,7 +72,8 @@ def _stored(a, name):
 
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
-             softplus=True, channels=None, nthreads=None, h0=None):
+             softplus=True, channels=None, nthreads=None, h0=None, conv_weight=None,
+             conv_bias=None):
     """Serial fp64 selective scan.
 
     u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; all float32 or all
@@ -80,6 +81,9 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     channels: optional 1-D int array of flat channel ids (b*dim + d); then
     only those rows are computed.  h0: optional [batch, dim, N] initial state
     (widened to float64; the scan starts from zero without it).
+    conv_weight: optional [dim, W] float32 taps of the causal depthwise
+    convolution; u then holds the convolution's input x and the scan runs on
+    SiLU(conv(x) + conv_bias).  conv_bias: optional [dim] float32.
     Returns (y, last_state) as float64 with
     shapes [batch, dim, L] / [batch, dim, N], or [len(channels), L] /
     [len(channels), N] when channels is given.
@@ -109,6 +113,17 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
         h0 = np.ascontiguousarray(h0, dtype=np.float64)
         if h0.shape != (batch, dim, N):
             raise ValueError("h0 must be [batch, dim, N]")
+    conv_w = conv_b = None
+    width = 0
+    if conv_weight is not None:
+        conv_w = np.ascontiguousarray(conv_weight, dtype=np.float32)
+        if conv_w.ndim != 2 or conv_w.shape[0] != dim:
+            raise ValueError("conv_weight must be [dim, W]")
+        width = conv_w.shape[1]
+        if conv_bias is not None:
+            conv_b = np.ascontiguousarray(conv_bias, dtype=np.float32)
+            if conv_b.shape != (dim,):
+                raise ValueError("conv_bias must be [dim]")
     if channels is not None:
         channels = np.ascontiguousarray(channels, dtype=np.int64)
         nch = channels.size
@@ -123,7 +138,8 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     rc = _load().oracle_scan_fwd(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(softplus)), dt, batch, dim, L, N,
-        _ptr(channels), nch, _ptr(y), _ptr(h), _ptr(h0), int(nthreads))
+        _ptr(channels), nch, _ptr(y), _ptr(h), _ptr(h0), _ptr(conv_w), _ptr(conv_b), width,
+        int(nthreads))
     if rc != 0:
         raise ValueError("oracle_scan_fwd rejected its arguments")
     return y, h

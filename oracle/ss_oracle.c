@@ -39,6 +39,12 @@
  *  - softplus_flag == 0 means Delta = delta + delta_bias.
  *  - SiLU(z) = z / (1 + exp(-z)).
  *  - a null D, delta_bias or z means zero skip, zero bias and no gate.
+ *  - with a short convolution (same page, sec. 3.3 block diagram and the
+ *    sec. 4.2 code: a depthwise Conv1d of width W, padding W-1, cut to the
+ *    first L outputs, then SiLU), the scan's input is
+ *      u[b,d,t] = SiLU(conv_bias[d] + sum_{k<W} conv_w[d,k] x[b,d,t-(W-1)+k]),
+ *    with x = 0 before t = 0 (Conv1d is a cross-correlation, so tap W-1
+ *    meets the current token).
  *  - an initial state h0 replaces the zero state of the pure-PyTorch module;
  *    the pages keep h between calls for recurrent (one token at a time)
  *    inference ("从Transformer的痛点说起 ... Mamba", sec. 5.1 table and
@@ -81,11 +87,27 @@ typedef struct {
   double* y;          /* [n_channels, seqlen] */
   double* last_state; /* [n_channels, dstate] or NULL */
   const double* h0;   /* [batch, dim, dstate] initial state or NULL (zero) */
+  const float* conv_w; /* [dim, conv_width] or NULL: u is the scan input itself */
+  const float* conv_b; /* [dim] or NULL */
+  int conv_width;
   int64_t next;       /* work counter (guarded by mu) */
   pthread_mutex_t mu;
 } job_t;
 
 /* One (b, d) channel: the serial recurrence, nothing reordered. */
+/* The scan's input at step t of one channel: u itself, or the SiLU of the
+ * causal depthwise convolution of x (stored in J->u) at t. */
+static double scan_input(const job_t* J, int64_t row, int64_t d, int64_t t) {
+  if (!J->conv_w) return widen(J->u, J->dtype, row + t);
+  const int W = J->conv_width;
+  double acc = J->conv_b ? (double)J->conv_b[d] : 0.0;
+  for (int k = 0; k < W; ++k) {
+    const int64_t s = t - (W - 1) + k;
+    if (s >= 0) acc += (double)J->conv_w[d * W + k] * widen(J->u, J->dtype, row + s);
+  }
+  return silu64(acc);
+}
+
 static void run_channel(const job_t* J, int64_t slot, double* h) {
   const int64_t flat = J->channels ? J->channels[slot] : slot;
   const int64_t b = flat / J->dim, d = flat % J->dim;
@@ -101,7 +123,7 @@ static void run_channel(const job_t* J, int64_t slot, double* h) {
   for (int64_t t = 0; t < L; ++t) {
     const double x = widen(J->delta, J->dtype, row + t) + bias;
     const double dt = J->softplus_flag ? softplus64(x) : x;
-    const double ut = widen(J->u, J->dtype, row + t);
+    const double ut = scan_input(J, row, d, t);
     double s = 0.0;
     for (int n = 0; n < N; ++n) {
       const double a_bar = exp(dt * (double)J->A[d * N + n]);
@@ -136,7 +158,8 @@ static void* worker(void* arg) {
 /*
  * oracle_scan_fwd: returns 0 on success, -1 on a bad argument.
  *
- * u, delta, z : [batch, dim, seqlen] in `dtype` (0 f32, 1 bf16), L fastest
+ * u, delta, z : [batch, dim, seqlen] in `dtype` (0 f32, 1 bf16), L fastest;
+ *               with conv_w, u holds the convolution's input x
  * B, C        : [batch, dstate, seqlen] in `dtype`
  * A           : [dim, dstate] f32;  D, delta_bias: [dim] f32 (nullable)
  * channels    : NULL for every channel (b*dim+d order), else n_channels flat
@@ -146,6 +169,9 @@ static void* worker(void* arg) {
  * h0          : [batch, dim, dstate] double initial state, indexed by the
  *               full flat channel id even when `channels` is given (nullable:
  *               the state starts at zero)
+ * conv_w      : [dim, conv_width] f32 taps of the short convolution, or NULL
+ * conv_b      : [dim] f32 convolution bias (nullable)
+ * conv_width  : 1..64 when conv_w is given
  * nthreads    : worker threads (>= 1)
  */
 int oracle_scan_fwd(const void* u, const void* delta, const float* A,
@@ -154,10 +180,12 @@ int oracle_scan_fwd(const void* u, const void* delta, const float* A,
                     int dtype, int64_t batch, int64_t dim, int64_t seqlen,
                     int dstate, const int64_t* channels, int64_t n_channels,
                     double* y, double* last_state, const double* h0,
+                    const float* conv_w, const float* conv_b, int conv_width,
                     int nthreads) {
   if (!u || !delta || !A || !B || !C || !y) return -1;
   if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0) return -1;
   if (dtype != 0 && dtype != 1) return -1;
+  if (conv_w && (conv_width < 1 || conv_width > 64)) return -1;
   if (!channels) n_channels = batch * dim;
   if (n_channels <= 0) return -1;
   if (channels)
@@ -174,6 +202,7 @@ int oracle_scan_fwd(const void* u, const void* delta, const float* A,
   J.batch = batch; J.dim = dim; J.seqlen = seqlen; J.dstate = dstate;
   J.channels = channels; J.n_channels = n_channels;
   J.y = y; J.last_state = last_state; J.h0 = h0; J.next = 0;
+  J.conv_w = conv_w; J.conv_b = conv_b; J.conv_width = conv_w ? conv_width : 0;
   pthread_mutex_init(&J.mu, NULL);
 
   pthread_t tids[512];

@@ -11,8 +11,9 @@
 // buffered on mbarriers, so the next chunk's copy overlaps this chunk's math):
 //   phase 1  per element: Delta = softplus(delta + bias), w = Delta * u, kept
 //            as float4 of four timesteps; B_t and C_t transposed from their
-//            [n][t] rows into [t][4-state block][B0..B3, C0..C3] in the input
-//            dtype, so one 16-byte load gives a lane four states' B and C;
+//            [n][t] rows into [t][state pair][B_lo, B_hi, C_lo, C_hi] in the
+//            input dtype, so a lane's states' B and C are one contiguous run
+//            (one 16-byte load for four bf16 states);
 //   phase 2  per (channel, state): A_bar = 2^(Delta * A * log2 e),
 //            h = A_bar * h + w * B_t[n], and the lane's partial readout
 //            sum_n C_t[n] h[n], in packed fp32x2 arithmetic; B_t and C_t are
@@ -88,7 +89,8 @@ struct ChunkedCfg {
   static constexpr int RAW_BYTES = RAW_ROWS * T * ES;
   static constexpr int DW_STRIDE = CH + 1;           // float4 per quad row (odd: conflict-free)
   static constexpr int DW_BYTES = QPR * DW_STRIDE * 16;
-  static constexpr int BC_BLOCK = 8 * ES;            // B0..B3, C0..C3
+  static constexpr int PAIR_BYTES = 4 * ES;          // one state pair: B_lo, B_hi, C_lo, C_hi
+  static constexpr int BC_BLOCK = 2 * PAIR_BYTES;    // two pairs: four states
   static constexpr int BC_DATA = (N / 4) * BC_BLOCK; // bytes of one timestep
   // Row pitch: a quarter-warp of the transpose writes rows 2tp and 2tp+2;
   // a pitch of 32 mod 64 bytes puts them on opposite halves of the banks.
@@ -116,7 +118,7 @@ struct ChunkedCfg {
 
   static_assert(N % K == 0 && 32 % K == 0, "lane split");
   static_assert(NWARPS % WT == 0 && T % (4 * WT) == 0, "time split");
-  static_assert(G % 4 == 0, "a lane holds whole 4-state blocks");
+  static_assert(G % 2 == 0, "a lane holds whole state pairs");
   static_assert(T % 8 == 0 && (T * ES) % 16 == 0 && T <= 256 && CH <= 256, "TMA box");
   static_assert(ACT_TILE % 128 == 0 && SEL_TILE % 128 == 0, "TMA destinations 128-byte aligned");
   static_assert(DW_BYTES % 16 == 0 && BC_BYTES % 16 == 0, "alignment");
@@ -221,7 +223,7 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     dwD[q * CF::DW_STRIDE + c] = make_float4(delt[0], delt[1], delt[2], delt[3]);
     dwW[q * CF::DW_STRIDE + c] = make_float4(w[0], w[1], w[2], w[3]);
   }
-  // B and C rows [n][t] -> [t][n/4][B0..B3, C0..C3]
+  // B and C rows [n][t] -> [t][n/2 pairs][B_2p, B_2p+1, C_2p, C_2p+1]
   const E* rawB = raw + 3 * CF::CH * CF::T;
   const E* rawC = rawB + CF::N * CF::T;
   if constexpr (CF::ES == 2) {
@@ -239,10 +241,10 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
       }
       uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + nb * CF::BC_BLOCK);
       uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + nb * CF::BC_BLOCK);
-      *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(bw[2], bw[3], 0x5410),
-                         __byte_perm(cw[0], cw[1], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
-      *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(bw[2], bw[3], 0x7632),
-                         __byte_perm(cw[0], cw[1], 0x7632), __byte_perm(cw[2], cw[3], 0x7632));
+      *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(cw[0], cw[1], 0x5410),
+                         __byte_perm(bw[2], bw[3], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
+      *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(cw[0], cw[1], 0x7632),
+                         __byte_perm(bw[2], bw[3], 0x7632), __byte_perm(cw[2], cw[3], 0x7632));
     }
   } else {
     const float* fb = reinterpret_cast<const float*>(rawB);
@@ -251,8 +253,8 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
       const int nb = i / CF::T, t = i - nb * CF::T;
       float4* dst = reinterpret_cast<float4*>(bc + t * CF::BC_ROW + nb * CF::BC_BLOCK);
       dst[0] = make_float4(fb[(4 * nb) * CF::T + t], fb[(4 * nb + 1) * CF::T + t],
-                           fb[(4 * nb + 2) * CF::T + t], fb[(4 * nb + 3) * CF::T + t]);
-      dst[1] = make_float4(fc[(4 * nb) * CF::T + t], fc[(4 * nb + 1) * CF::T + t],
+                           fc[(4 * nb) * CF::T + t], fc[(4 * nb + 1) * CF::T + t]);
+      dst[1] = make_float4(fb[(4 * nb + 2) * CF::T + t], fb[(4 * nb + 3) * CF::T + t],
                            fc[(4 * nb + 2) * CF::T + t], fc[(4 * nb + 3) * CF::T + t]);
     }
   }
@@ -260,23 +262,36 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
 
 // ------------------------------------------------------------- phase 2 ---
 
-// B and C of one 4-state block at one timestep, as fp32 pairs.
-template <class CF>
-__device__ __forceinline__ void bc_block(const unsigned char* p, float2& b01, float2& b23,
-                                         float2& c01, float2& c23) {
+// B and C of NP consecutive state pairs at one timestep, as fp32 pairs; p
+// points at the first pair (16-byte loads where the pairs allow).
+template <class CF, int NP>
+__device__ __forceinline__ void bc_pairs(const unsigned char* p, float2 (&b)[NP],
+                                         float2 (&c)[NP]) {
   if constexpr (CF::ES == 2) {
-    const uint4 v = *reinterpret_cast<const uint4*>(p);
-    b01 = bf16x2_to_float2(v.x);
-    b23 = bf16x2_to_float2(v.y);
-    c01 = bf16x2_to_float2(v.z);
-    c23 = bf16x2_to_float2(v.w);
+    if constexpr (NP % 2 == 0) {
+#pragma unroll
+      for (int i = 0; i < NP / 2; ++i) {
+        const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+        b[2 * i] = bf16x2_to_float2(v.x);
+        c[2 * i] = bf16x2_to_float2(v.y);
+        b[2 * i + 1] = bf16x2_to_float2(v.z);
+        c[2 * i + 1] = bf16x2_to_float2(v.w);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const uint2 v = reinterpret_cast<const uint2*>(p)[i];
+        b[i] = bf16x2_to_float2(v.x);
+        c[i] = bf16x2_to_float2(v.y);
+      }
+    }
   } else {
-    const float4 vb = reinterpret_cast<const float4*>(p)[0];
-    const float4 vc = reinterpret_cast<const float4*>(p)[1];
-    b01 = make_float2(vb.x, vb.y);
-    b23 = make_float2(vb.z, vb.w);
-    c01 = make_float2(vc.x, vc.y);
-    c23 = make_float2(vc.z, vc.w);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const float4 v = reinterpret_cast<const float4*>(p)[i];
+      b[i] = make_float2(v.x, v.y);
+      c[i] = make_float2(v.z, v.w);
+    }
   }
 }
 
@@ -291,8 +306,8 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
                                        const unsigned char* bc, float* sy,
                                        float2 (&h)[CF::G / 2], const float2 (&a2)[CF::G / 2],
                                        int c, int j) {
-  constexpr int NB = CF::G / 4;  // 4-state blocks per lane
-  const unsigned char* bcj = bc + j * NB * CF::BC_BLOCK;
+  constexpr int G2 = CF::G / 2;  // state pairs per lane
+  const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
   float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE;
 #pragma unroll kPhase2Unroll
   for (int q = 0; q < CF::QPR; ++q) {
@@ -303,31 +318,25 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
     float s[4];
 #if defined(SS_PHASE2_EXP_FIRST)
     // all ex2 of the quad first, then the four dependent update chains
-    float2 ee[4][CF::G / 2], wb[4][CF::G / 2], cc[4][CF::G / 2];
+    float2 ee[4][G2], wb[4][G2], cc[4][G2];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const unsigned char* row = bcj + (4 * q + k) * CF::BC_ROW;
       const float2 dl2 = make_float2(dls[k], dls[k]);
       const float2 w2 = make_float2(ws[k], ws[k]);
+      float2 bb[G2];
+      bc_pairs<CF, G2>(bcj + (4 * q + k) * CF::BC_ROW, bb, cc[k]);
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        float2 b01, b23, c01, c23;
-        bc_block<CF>(row + nb * CF::BC_BLOCK, b01, b23, c01, c23);
-        const float2 x01 = __fmul2_rn(dl2, a2[2 * nb]);
-        const float2 x23 = __fmul2_rn(dl2, a2[2 * nb + 1]);
-        ee[k][2 * nb] = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
-        ee[k][2 * nb + 1] = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-        wb[k][2 * nb] = __fmul2_rn(w2, b01);
-        wb[k][2 * nb + 1] = __fmul2_rn(w2, b23);
-        cc[k][2 * nb] = c01;
-        cc[k][2 * nb + 1] = c23;
+      for (int g = 0; g < G2; ++g) {
+        const float2 x = __fmul2_rn(dl2, a2[g]);
+        ee[k][g] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        wb[k][g] = __fmul2_rn(w2, bb[g]);
       }
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int g = 0; g < CF::G / 2; ++g) {
+      for (int g = 0; g < G2; ++g) {
         h[g] = __ffma2_rn(ee[k][g], h[g], wb[k][g]);
         acc = __ffma2_rn(cc[k][g], h[g], acc);
       }
@@ -336,22 +345,17 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
 #else
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const unsigned char* row = bcj + (4 * q + k) * CF::BC_ROW;
       const float2 dl2 = make_float2(dls[k], dls[k]);
       const float2 w2 = make_float2(ws[k], ws[k]);
+      float2 bb[G2], cc[G2];
+      bc_pairs<CF, G2>(bcj + (4 * q + k) * CF::BC_ROW, bb, cc);
       float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        float2 b01, b23, c01, c23;
-        bc_block<CF>(row + nb * CF::BC_BLOCK, b01, b23, c01, c23);
-        const float2 x01 = __fmul2_rn(dl2, a2[2 * nb]);
-        const float2 x23 = __fmul2_rn(dl2, a2[2 * nb + 1]);
-        const float2 e01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
-        const float2 e23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-        h[2 * nb] = __ffma2_rn(e01, h[2 * nb], __fmul2_rn(w2, b01));
-        h[2 * nb + 1] = __ffma2_rn(e23, h[2 * nb + 1], __fmul2_rn(w2, b23));
-        acc = __ffma2_rn(c01, h[2 * nb], acc);
-        acc = __ffma2_rn(c23, h[2 * nb + 1], acc);
+      for (int g = 0; g < G2; ++g) {
+        const float2 x = __fmul2_rn(dl2, a2[g]);
+        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        h[g] = __ffma2_rn(e, h[g], __fmul2_rn(w2, bb[g]));
+        acc = __ffma2_rn(cc[g], h[g], acc);
       }
       s[k] = acc.x + acc.y;
     }
@@ -376,9 +380,8 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
                                              float* aggH, float2 (&h)[CF::G / 2],
                                              const float2 (&a2)[CF::G / 2], int c, int j, int wt,
                                              int lane_g) {
-  constexpr int NB = CF::G / 4;
   constexpr int G2 = CF::G / 2;
-  const unsigned char* bcj = bc + j * NB * CF::BC_BLOCK;
+  const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
   float2 hl[G2], P[G2];
 #pragma unroll
   for (int g = 0; g < G2; ++g) {
@@ -401,22 +404,16 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
       const float2 dl2 = make_float2(dls[k], dls[k]);
       const float2 w2 = make_float2(ws[k], ws[k]);
       float2 acc = make_float2(0.f, 0.f);
+      float2 bb[G2], cc[G2];
+      bc_pairs<CF, G2>(row, bb, cc);
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        float2 b01, b23, c01, c23;
-        bc_block<CF>(row + nb * CF::BC_BLOCK, b01, b23, c01, c23);
-        const float2 x01 = __fmul2_rn(dl2, a2[2 * nb]);
-        const float2 x23 = __fmul2_rn(dl2, a2[2 * nb + 1]);
-        const float2 e01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
-        const float2 e23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-        hl[2 * nb] = __ffma2_rn(e01, hl[2 * nb], __fmul2_rn(w2, b01));
-        hl[2 * nb + 1] = __ffma2_rn(e23, hl[2 * nb + 1], __fmul2_rn(w2, b23));
-        P[2 * nb] = __fmul2_rn(e01, P[2 * nb]);
-        P[2 * nb + 1] = __fmul2_rn(e23, P[2 * nb + 1]);
-        acc = __ffma2_rn(c01, hl[2 * nb], acc);
-        acc = __ffma2_rn(c23, hl[2 * nb + 1], acc);
-        Q[t][2 * nb] = __fmul2_rn(c01, P[2 * nb]);
-        Q[t][2 * nb + 1] = __fmul2_rn(c23, P[2 * nb + 1]);
+      for (int g = 0; g < G2; ++g) {
+        const float2 x = __fmul2_rn(dl2, a2[g]);
+        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        hl[g] = __ffma2_rn(e, hl[g], __fmul2_rn(w2, bb[g]));
+        P[g] = __fmul2_rn(e, P[g]);
+        acc = __ffma2_rn(cc[g], hl[g], acc);
+        Q[t][g] = __fmul2_rn(cc[g], P[g]);
       }
       s[t] = acc.x + acc.y;
     }

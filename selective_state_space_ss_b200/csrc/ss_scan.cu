@@ -193,8 +193,17 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
 
 template <typename E>
 using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T>;
+#ifndef SS_N32_K
+#define SS_N32_K 4
+#endif
+#ifndef SS_N32_W
+#define SS_N32_W 4
+#endif
+#ifndef SS_N32_T
+#define SS_N32_T 32
+#endif
 template <typename E>
-using Cfg32 = ChunkedCfg<E, 32, 4, 4, 32>;
+using Cfg32 = ChunkedCfg<E, 32, SS_N32_K, SS_N32_W, SS_N32_T>;
 #ifndef SS_N64_K
 #define SS_N64_K 4
 #endif

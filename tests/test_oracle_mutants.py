@@ -31,6 +31,11 @@ MUTANTS = [
     ("initial state ignored", "h[n] = J->h0 ? J->h0[flat * N + n] : 0.0;", "h[n] = 0.0;"),
     ("initial state indexed [b][n][d]", "J->h0[flat * N + n]", "J->h0[(b * N + n) * J->dim + d]"),
     ("initial state indexed [n][b][d]", "J->h0[flat * N + n]", "J->h0[n * J->batch * J->dim + flat]"),
+    ("conv taps reversed", "J->conv_w[d * W + k]", "J->conv_w[d * W + (W - 1 - k)]"),
+    ("conv taps indexed [k][d]", "J->conv_w[d * W + k]", "J->conv_w[k * J->dim + d]"),
+    ("conv window shifted", "const int64_t s = t - (W - 1) + k;", "const int64_t s = t - W + k;"),
+    ("conv bias dropped", "double acc = J->conv_b ? (double)J->conv_b[d] : 0.0;", "double acc = 0.0;"),
+    ("conv output without SiLU", "  return silu64(acc);", "  return acc;"),
 ]
 
 PIN_CALLS = [
@@ -45,6 +50,8 @@ PIN_CALLS = [
     pins.test_index_plumbing_single_impulse,
     pins.test_initial_state_free_decay_closed_form,
     lambda: pins.test_initial_state_bruteforce(3),
+    lambda: pins.test_conv_prologue_matches_numpy_convolution(4),
+    pins.test_conv_prologue_impulse_taps,
 ]
 
 

@@ -444,6 +444,100 @@ def test_step_chain_equals_scan():
     assert np.array_equal(state, h)
 
 
+# ------------------------------------------------ short convolution -------
+# The block's depthwise Conv1d of width W, padding W-1, cut to L outputs, then
+# SiLU ("从Transformer的痛点说起 ... Mamba", sec. 3.3 diagram and sec. 4.2 code).
+# With B = 0 the state stays zero and y = D u, so y exposes u itself.
+
+def _conv_case(rng, batch, dim, L, N, W):
+    c = _rand_case(rng, batch, dim, L, N)
+    c["B"] = np.zeros_like(c["B"])
+    c["D"] = np.ones(dim, np.float32)
+    c["w"] = _f32(rng.normal(size=(dim, W)))
+    c["b"] = _f32(rng.normal(size=dim))
+    return c
+
+
+@pytest.mark.parametrize("W", [1, 2, 4, 7])
+def test_conv_prologue_matches_numpy_convolution(W):
+    """u = SiLU(causal conv + bias), the conv from numpy's full convolution with
+    the taps reversed (Conv1d is a cross-correlation), cut to the first L."""
+    rng = np.random.default_rng(300 + W)
+    batch, dim, L, N = 2, 5, 40, 4
+    c = _conv_case(rng, batch, dim, L, N, W)
+    delta = _f32(rng.normal(size=(batch, dim, L)))
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], softplus=True,
+                           conv_weight=c["w"], conv_bias=c["b"])
+    assert np.all(h == 0.0)
+    x64 = c["u"].astype(np.float64)
+    for b in range(batch):
+        for d in range(dim):
+            pre = np.convolve(x64[b, d], c["w"][d, ::-1].astype(np.float64))[:L] + float(c["b"][d])
+            ref = pre / (1.0 + np.exp(-pre))
+            assert _rel(y[b, d], ref) < 1e-14
+
+
+def test_conv_prologue_impulse_taps():
+    """x = one impulse per (b, d) at step s: u_t = SiLU(w[d, W-1-(t-s)] x_s + bias)
+    for t in [s, s+W-1] and SiLU(bias) elsewhere; taps, bias and impulse size
+    differ per index, so a reversed, shifted or transposed tap lands wrong."""
+    batch, dim, L, N, W = 2, 3, 16, 4, 4
+    rng = np.random.default_rng(12)
+    c = _conv_case(rng, batch, dim, L, N, W)
+    c["w"] = _f32(0.5 + np.arange(dim)[:, None] * 0.25 + np.arange(W)[None, :] * 1.5)
+    c["b"] = _f32(-0.3 + 0.1 * np.arange(dim))
+    x = np.zeros((batch, dim, L), np.float32)
+    starts = np.array([[3, 7, 12], [0, 5, 9]])
+    for b in range(batch):
+        for d in range(dim):
+            x[b, d, starts[b, d]] = 1.0 + b + 0.5 * d
+    delta = np.zeros((batch, dim, L), np.float32)
+    y, _ = oracle.scan_fwd(x, delta, c["A"], c["B"], c["C"], D=c["D"], softplus=False,
+                           conv_weight=c["w"], conv_bias=c["b"])
+    for b in range(batch):
+        for d in range(dim):
+            s0, xs, bias = starts[b, d], float(x[b, d, starts[b, d]]), float(c["b"][d])
+            for t in range(L):
+                k = W - 1 - (t - s0)
+                pre = bias + (float(c["w"][d, k]) * xs if 0 <= k < W else 0.0)
+                assert y[b, d, t] == pytest.approx(oracle.silu(pre), rel=1e-15, abs=1e-300)
+
+
+def test_conv_prologue_feeds_the_scan():
+    """With the convolution on, the scan sees u = SiLU(conv): brute-force
+    products over that u (width 3, full B, C, gate and skip)."""
+    rng = np.random.default_rng(44)
+    batch, dim, L, N, W = 1, 2, 5, 3, 3
+    c = _rand_case(rng, batch, dim, L, N)
+    c["A"] = _f32(-rng.uniform(0.1, 2.0, size=(dim, N)))
+    w = _f32(rng.normal(size=(dim, W)))
+    cb = _f32(rng.normal(size=dim))
+    delta = _f32(rng.normal(scale=0.5, size=(batch, dim, L)))
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                           softplus=True, conv_weight=w, conv_bias=cb)
+    for d in range(dim):
+        xs = [float(v) for v in c["u"][0, d]]
+        us = []
+        for t in range(L):
+            pre = float(cb[d]) + sum(float(w[d, k]) * xs[t - (W - 1) + k]
+                                     for k in range(W) if t - (W - 1) + k >= 0)
+            us.append(oracle.silu(pre))
+        dl = [oracle.softplus(float(delta[0, d, t])) for t in range(L)]
+        for t in range(L):
+            acc = 0.0
+            for n in range(N):
+                a = float(c["A"][d, n])
+                hn = 0.0
+                for s_ in range(t + 1):
+                    prod = 1.0
+                    for k in range(s_ + 1, t + 1):
+                        prod *= math.exp(dl[k] * a)
+                    hn += prod * dl[s_] * float(c["B"][0, n, s_]) * us[s_]
+                acc += float(c["C"][0, n, t]) * hn
+            ref = (acc + float(c["D"][d]) * us[t]) * oracle.silu(float(c["z"][0, d, t]))
+            assert y[0, d, t] == pytest.approx(ref, rel=1e-13, abs=1e-15)
+
+
 # ------------------------------------------------------- host plumbing -----
 
 def test_channel_subset_matches_full():
