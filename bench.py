@@ -42,8 +42,8 @@ MUFU_EX2_PER_CLK_PER_SM = 16  # ex2 results per clock per SM (special-function u
 _CSRC = "selective_state_space_ss_b200/csrc/"
 KERNEL_SOURCES = tuple(_CSRC + f for f in ("ss_scan.cu", "pointwise.cuh", "scan_fwd_chunked.cuh",
                                            "scan_common.cuh"))
-STEP_KERNEL_SOURCES = tuple(_CSRC + f for f in ("ss_scan.cu", "pointwise.cuh", "scan_step.cuh",
-                                                "scan_common.cuh"))
+# (the step kernels' launch shapes are constants of scan_step.cuh)
+STEP_KERNEL_SOURCES = tuple(_CSRC + f for f in ("pointwise.cuh", "scan_step.cuh", "scan_common.cuh"))
 
 
 def peaks():
@@ -167,7 +167,7 @@ def run_gpu_arm(args, w: I.Workload):
     import torch
     import torch.distributed as dist
 
-    from selective_state_space_ss_b200 import ss_scan_fwd, load_library
+    from selective_state_space_ss_b200 import load_library, ss_scan_fwd, ss_scan_fwd_conv
 
     world, rank, local = _dist_env()
     torch.cuda.set_device(local)
@@ -200,13 +200,24 @@ def run_gpu_arm(args, w: I.Workload):
     sets = [to_dev(x) for x in host]
     ys = [torch.empty((w.batch, w.dim, w.seqlen), dtype=torch.float32, device=dev) for _ in sets]
     hs = [torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev) for _ in sets]
+    conv = None
+    if args.conv:  # u = SiLU(conv1d(x)) inside the kernel; x takes u's place
+        cw, cb = I.make_conv(w.dim, args.conv, seed=rank_seed(rank, 99))
+        conv = (torch.from_numpy(cw).to(dev), torch.from_numpy(cb).to(dev))
+        host[0]["conv"] = (cw, cb)
+
+    def scan(x, y_out, h_out):
+        if conv is None:
+            return ss_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+                               delta_bias=x["delta_bias"], softplus=w.softplus, y_out=y_out,
+                               last_state_out=h_out, stream=stream)
+        return ss_scan_fwd_conv(x["u"], conv[0], x["delta"], x["A"], x["B"], x["C"], D=x["D"],
+                                z=x["z"], delta_bias=x["delta_bias"], conv_bias=conv[1],
+                                softplus=w.softplus, y_out=y_out, last_state_out=h_out, stream=stream)
 
     def step(i):
         s = i % nsets
-        x = sets[s]
-        ss_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
-                    delta_bias=x["delta_bias"], softplus=w.softplus, y_out=ys[s], last_state_out=hs[s],
-                    stream=stream)
+        scan(sets[s], ys[s], hs[s])
 
     def barrier():
         if world > 1:
@@ -234,6 +245,8 @@ def run_gpu_arm(args, w: I.Workload):
     ex = host[0]
     pinned = {}
     for k, v in ex.items():
+        if k == "conv":
+            continue
         if v is None:
             pinned[k] = None
         else:
@@ -250,9 +263,7 @@ def run_gpu_arm(args, w: I.Workload):
         for k, v in pinned.items():
             if v is not None:
                 dbuf[k].copy_(v, non_blocking=True)
-        y, h = ss_scan_fwd(dbuf["u"], dbuf["delta"], dbuf["A"], dbuf["B"], dbuf["C"], D=dbuf["D"],
-                           z=dbuf["z"], delta_bias=dbuf["delta_bias"], softplus=w.softplus,
-                           y_out=ys[0], last_state_out=hs[0], stream=stream)
+        y, h = scan(dbuf, ys[0], hs[0])
         y_host.copy_(y, non_blocking=True)
         h_host.copy_(h, non_blocking=True)
 
@@ -433,8 +444,10 @@ def oracle_sample(w: I.Workload, x: dict, target_s: float):
     while True:
         ch = np.sort(rng.choice(nch, take, replace=False))
         t0 = time.perf_counter()
+        cw, cb = x.get("conv", (None, None))
         oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
-                        softplus=w.softplus, channels=ch, nthreads=cores)
+                        softplus=w.softplus, channels=ch, nthreads=cores, conv_weight=cw,
+                        conv_bias=cb)
         dt = time.perf_counter() - t0
         if dt >= target_s or take == nch:
             return take, dt, cores
@@ -473,9 +486,10 @@ def run_reference_arm(args, w: I.Workload):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def config_of(w: I.Workload, world: int):
-    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate,
-            "in_dtype": w.dtype, "state_dtype": "f32", "y_dtype": "f32",
+def config_of(w: I.Workload, world: int, conv: int = 0):
+    return {"workload": w.name + (f"+conv{conv}" if conv else ""), "batch": w.batch,
+            "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate,
+            "in_dtype": w.dtype, "state_dtype": "f32", "y_dtype": "f32", "conv_width": conv,
             "parallelism": f"replicas x{world} (independent batch per GPU, no collective)",
             "l2": "inputs rotated over sets totalling >= 4x L2 (126 MB); no flush"}
 
@@ -490,6 +504,8 @@ def main():
                     choices=sorted(I.WORKLOADS) + sorted(I.STEP_WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--conv", type=int, default=0,
+                    help="fuse the short causal conv1d + SiLU of this width (1-4) into the scan")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -516,7 +532,7 @@ def main():
     line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": r["world"],
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": config_of(w, r["world"]), "roofline": roof,
+            "data": "synthetic", "config": config_of(w, r["world"], args.conv), "roofline": roof,
             "e2e": r["e2e"], "gpu_launches": args.steps, "clocks": r["clocks"]}
     if r["world"] == 1 and not args.no_cpu_baseline:
         take, dt, cores = oracle_sample(w, r["host"], target_s=10.0)

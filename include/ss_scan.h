@@ -112,6 +112,36 @@ ss_status ss_scan_fwd_from_state(const void* u, const void* delta, const float* 
                                  size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * ss_scan_fwd_conv -- ss_scan_fwd whose input u is formed inside the kernel
+ * from the block's short convolution: the causal depthwise Conv1d of width W
+ * (padding W-1, cut to the first L outputs) followed by SiLU
+ * ("从Transformer的痛点说起 ... Mamba", sec. 3.3 block diagram and the sec. 4.2
+ * code), so the convolved activation never goes through HBM:
+ *
+ *   u[b,d,t] = SiLU(conv_bias[d] + sum_{k<W} conv_weight[d,k] x[b,d,t-(W-1)+k]),
+ *   x[b,d,t] = 0 for t < 0 (tap W-1 meets the current token).
+ *
+ *  x            [batch, dim, seqlen]  in_dtype   (takes the place of u)
+ *  conv_weight  [dim, conv_width]     float32    (required)
+ *  conv_bias    [dim]                 float32    (nullable: 0)
+ *  conv_width   1..4 (others: SS_ERR_UNSUPPORTED)
+ *
+ * The scan starts from h = 0 and from x = 0 before t = 0.  Every other
+ * argument, layout, result and error is that of ss_scan_fwd (u there is the
+ * convolution's output, here computed); D multiplies that output, as in the
+ * sec. 4.2 code.  The workspace size is ss_scan_workspace_bytes(...).
+ */
+ss_status ss_scan_fwd_conv(const void* x, const float* conv_weight,
+                           const float* conv_bias, int conv_width,
+                           const void* delta, const float* A, const void* B,
+                           const void* C, const float* D, const void* z,
+                           const float* delta_bias, int softplus_flag,
+                           float* y_out, float* last_state_out, int64_t batch,
+                           int64_t dim, int64_t seqlen, int dstate,
+                           ss_dtype in_dtype, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * ss_scan_step -- one recurrent (decode) step: the same recurrence over a
  * single token, advancing a carried state in place ("从Transformer的痛点说起
  * ... Mamba", sec. 5.1 table: O(1) work and memory per generated token;

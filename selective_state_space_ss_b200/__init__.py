@@ -26,6 +26,7 @@ from ._native import (  # noqa: F401
     ss_debug_inject,
     ss_last_device_error,
     ss_scan_fwd,
+    ss_scan_fwd_conv,
     ss_scan_fwd_from_state,
     ss_scan_fwd_noalloc,
     ss_scan_step,

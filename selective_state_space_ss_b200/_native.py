@@ -23,7 +23,7 @@ SS_F32, SS_BF16 = 0, 1
 
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
             "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc",
-            "ss_scan_fwd_from_state", "ss_scan_step")
+            "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv")
 
 # bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
 SS_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -73,6 +73,9 @@ def load_library():
                                                i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
         lib.ss_scan_fwd_from_state.restype = ci
         lib.ss_scan_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, i64, i64, ci, ci, vp]
+        lib.ss_scan_fwd_conv.argtypes = [vp, vp, vp, ci, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp,
+                                         i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
+        lib.ss_scan_fwd_conv.restype = ci
         lib.ss_scan_step.restype = ci
         _lib = lib
         return lib
@@ -166,6 +169,15 @@ def _fwd_call(name, initial_state, u, delta, A, B, C, D, z, delta_bias, softplus
             _stream_handle(stream, device))
     if name == "ss_scan_fwd":
         st = lib.ss_scan_fwd(*head, *tail)
+    elif name == "ss_scan_fwd_conv":
+        cw, cb = initial_state
+        _check_dev("conv_weight", cw, device, (torch.float32,))
+        _check_dev("conv_bias", cb, device, (torch.float32,), (dim,))
+        if cw.dim() != 2 or cw.shape[0] != dim:
+            raise ValueError("conv_weight must be [dim, W]")
+        st = lib.ss_scan_fwd_conv(_ptr(u), _ptr(cw), _ptr(cb), cw.shape[1], _ptr(delta), _ptr(A),
+                                  _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+                                  int(bool(softplus)), *tail)
     else:
         _check_dev("initial_state", initial_state, device, (torch.float32,), (batch, dim, N))
         st = lib.ss_scan_fwd_from_state(*head, _ptr(initial_state), *tail)
@@ -195,6 +207,18 @@ def ss_scan_fwd_from_state(initial_state, u, delta, A, B, C, D=None, z=None, del
     """ss_scan_fwd started from initial_state [batch, dim, N] float32 (None:
     zero).  last_state_out may be initial_state itself (in-place advance)."""
     return _fwd_call("ss_scan_fwd_from_state", initial_state, u, delta, A, B, C, D, z,
+                     delta_bias, softplus, y_out, last_state_out, return_last_state, workspace,
+                     stream)
+
+
+def ss_scan_fwd_conv(x, conv_weight, delta, A, B, C, D=None, z=None, delta_bias=None,
+                     conv_bias=None, softplus=True, y_out=None, last_state_out=None,
+                     return_last_state=True, workspace=None, stream=None):
+    """ss_scan_fwd with u = SiLU(causal depthwise conv1d(x) + conv_bias) formed
+    in the kernel.  x: [batch, dim, L] (float32 or bfloat16); conv_weight:
+    [dim, W] float32 with W in 1..4 (tap W-1 meets the current token);
+    conv_bias: [dim] float32 (optional)."""
+    return _fwd_call("ss_scan_fwd_conv", (conv_weight, conv_bias), x, delta, A, B, C, D, z,
                      delta_bias, softplus, y_out, last_state_out, return_last_state, workspace,
                      stream)
 

@@ -49,6 +49,11 @@ struct FwdArgs {
   float* y;
   float* last_state;  // nullable
   const float* h0;    // [batch, dim, N] initial state, nullable (zero); may be last_state
+  // fused short convolution (kernels built with CONV): u holds the
+  // convolution's input x; conv_w [dim, conv_width <= kConvTaps], conv_b [dim]
+  const float* conv_w;
+  const float* conv_b;  // nullable
+  int conv_width;
   int64_t batch, dim, seqlen;
   int softplus;
   int vec;  // 1: TMA path (16-byte aligned rows); 0: element-wise loads
@@ -61,13 +66,16 @@ struct FwdMaps {
 };
 
 constexpr uint32_t kTmaSpinLimit = 1u << 24;
+constexpr int kConvTaps = 4;  // widest fused convolution
 
 // Tin: input dtype; N: states per channel; K: lanes per channel; NWARPS: warps
 // per CTA; T: timesteps per chunk; WT: warps that split each chunk in time
 // (1: every warp walks the whole chunk for its own channels; >1: WT warps
 // share one set of channels, each scanning T/WT consecutive steps of the
-// chunk, joined with the pages' associative operator).
-template <typename Tin, int N_, int K_, int NWARPS_, int T_, int WT_ = 1>
+// chunk, joined with the pages' associative operator).  CONV: the u input is
+// the pre-convolution x, staged with HALO earlier steps per row, and phase 1
+// forms u = SiLU(conv(x) + bias).
+template <typename Tin, int N_, int K_, int NWARPS_, int T_, int WT_ = 1, bool CONV_ = false>
 struct ChunkedCfg {
   using Elem = Tin;
   static constexpr int N = N_;            // states per channel
@@ -83,10 +91,20 @@ struct ChunkedCfg {
   static constexpr int NT = NWARPS * 32;
   static constexpr int ES = (int)sizeof(Tin);
   static constexpr int QPR = T / 4;                  // 4-step quads per row
-  static constexpr int RAW_ROWS = 3 * CH + 2 * N;    // u, delta, z rows then B, C rows
-  static constexpr int ACT_TILE = CH * T * ES;       // one activation tile (bytes)
+  static constexpr bool CONV = CONV_;
+  // x steps staged before the chunk: >= kConvTaps - 1, and a whole number of
+  // 16-byte units so that the shifted TMA box stays aligned
+  static constexpr int HALO = CONV ? 8 : 0;
+  static constexpr int XT = T + HALO;                // u (or x) row length
+  static constexpr int ACT_TILE = CH * T * ES;       // one delta or z tile (bytes)
+  static constexpr int X_TILE = CH * XT * ES;        // the u (or x) tile (bytes)
   static constexpr int SEL_TILE = N * T * ES;        // one B or C tile (bytes)
-  static constexpr int RAW_BYTES = RAW_ROWS * T * ES;
+  // raw stage: [u or x: CH rows of XT][delta: CH x T][z: CH x T][B: N x T][C: N x T]
+  static constexpr int OFF_DELTA_T = X_TILE;
+  static constexpr int OFF_Z_T = X_TILE + ACT_TILE;
+  static constexpr int OFF_B_T = X_TILE + 2 * ACT_TILE;
+  static constexpr int OFF_C_T = OFF_B_T + SEL_TILE;
+  static constexpr int RAW_BYTES = OFF_C_T + SEL_TILE;
   static constexpr int DW_STRIDE = CH + 1;           // float4 per quad row (odd: conflict-free)
   static constexpr int DW_BYTES = QPR * DW_STRIDE * 16;
   static constexpr int PAIR_BYTES = 4 * ES;          // one state pair: B_lo, B_hi, C_lo, C_hi
@@ -106,7 +124,10 @@ struct ChunkedCfg {
   // time-split aggregates: (prod A_bar, local end state) per warp and lane state
   static constexpr int AGG_FLOATS = WT > 1 ? WT * WC * 32 * G : 0;
   static constexpr int OFF_AGG = OFF_SY + SY_BYTES;
-  static constexpr int SMEM_USED = OFF_AGG + 2 * AGG_FLOATS * 4;
+  // CONV: u = SiLU(conv) per (quad, channel), for phase 3's D u
+  static constexpr int SU_BYTES = CONV ? DW_BYTES : 0;
+  static constexpr int OFF_SU = OFF_AGG + 2 * AGG_FLOATS * 4;
+  static constexpr int SMEM_USED = OFF_SU + SU_BYTES;
   static constexpr int SMEM_BYTES = SMEM_USED + 128;  // slack to align the base to 128 bytes
   // CTAs per SM the register budget must allow (shared memory permitting)
   // (at most 512 threads' worth: a 128-register budget per thread)
@@ -120,7 +141,10 @@ struct ChunkedCfg {
   static_assert(NWARPS % WT == 0 && T % (4 * WT) == 0, "time split");
   static_assert(G % 2 == 0, "a lane holds whole state pairs");
   static_assert(T % 8 == 0 && (T * ES) % 16 == 0 && T <= 256 && CH <= 256, "TMA box");
-  static_assert(ACT_TILE % 128 == 0 && SEL_TILE % 128 == 0, "TMA destinations 128-byte aligned");
+  static_assert(ACT_TILE % 128 == 0 && SEL_TILE % 128 == 0 && X_TILE % 128 == 0,
+                "TMA destinations 128-byte aligned");
+  static_assert(!CONV || ((HALO * ES) % 16 == 0 && HALO >= kConvTaps - 1 && XT <= 256),
+                "convolution halo");
   static_assert(DW_BYTES % 16 == 0 && BC_BYTES % 16 == 0, "alignment");
   static_assert(ITEMS % NT == 0 || ITEMS < NT, "whole items per thread");
   static constexpr bool ITEM_GUARD = ITEMS < NT;  // some threads have no item
@@ -143,7 +167,7 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
 
 template <class CF>
 __device__ __forceinline__ uint32_t chunk_tx_bytes(bool has_z) {
-  return (has_z ? 3 : 2) * CF::ACT_TILE + 2 * CF::SEL_TILE;
+  return CF::X_TILE + (has_z ? 2 : 1) * CF::ACT_TILE + 2 * CF::SEL_TILE;
 }
 
 // Issue the TMA loads of chunk t0 into one raw stage (one thread).
@@ -152,56 +176,98 @@ __device__ __forceinline__ void tma_chunk(const FwdMaps& m, unsigned char* raw, 
                                           int32_t b, int32_t d0, int32_t t0, bool has_z) {
   fence_proxy_async_smem();
   mbar_arrive_expect_tx(bar, chunk_tx_bytes<CF>(has_z));
-  tma_load_3d(raw, &m.u, bar, t0, d0, b);
-  tma_load_3d(raw + CF::ACT_TILE, &m.delta, bar, t0, d0, b);
-  if (has_z) tma_load_3d(raw + 2 * CF::ACT_TILE, &m.z, bar, t0, d0, b);
-  tma_load_3d(raw + 3 * CF::ACT_TILE, &m.B, bar, t0, 0, b);
-  tma_load_3d(raw + 3 * CF::ACT_TILE + CF::SEL_TILE, &m.C, bar, t0, 0, b);
+  // the x box starts HALO steps early (zero fill before t = 0); HALO * size
+  // is a multiple of 16 bytes, so the start stays 16-byte aligned
+  tma_load_3d(raw, &m.u, bar, t0 - CF::HALO, d0, b);
+  tma_load_3d(raw + CF::OFF_DELTA_T, &m.delta, bar, t0, d0, b);
+  if (has_z) tma_load_3d(raw + CF::OFF_Z_T, &m.z, bar, t0, d0, b);
+  tma_load_3d(raw + CF::OFF_B_T, &m.B, bar, t0, 0, b);
+  tma_load_3d(raw + CF::OFF_C_T, &m.C, bar, t0, 0, b);
 }
 
-// Element-wise fallback for rows that TMA cannot address (all threads).
+// Element-wise fallback for rows that TMA cannot address (all threads); the
+// same stage layout as tma_chunk, zeros outside the tensors.
 template <class CF>
 __device__ __forceinline__ void load_chunk_scalar(const FwdArgs& a, typename CF::Elem* raw,
                                                   int64_t b, int64_t d0, int64_t t0) {
   using E = typename CF::Elem;
   const int64_t L = a.seqlen;
-  for (int i = threadIdx.x; i < CF::RAW_ROWS * CF::T; i += CF::NT) {
+  // u (or x with its halo): CH rows of XT steps from t0 - HALO
+  for (int i = threadIdx.x; i < CF::CH * CF::XT; i += CF::NT) {
+    const int c = i / CF::XT, tt = i - c * CF::XT;
+    const int64_t t = t0 - CF::HALO + tt, d = d0 + c;
+    E val = zero_elem<E>();
+    if (t >= 0 && t < L && d < a.dim) val = static_cast<const E*>(a.u)[(b * a.dim + d) * L + t];
+    raw[i] = val;
+  }
+  // delta, z, B, C: [2 CH + 2 N] rows of T steps
+  E* rest = raw + CF::CH * CF::XT;
+  for (int i = threadIdx.x; i < (2 * CF::CH + 2 * CF::N) * CF::T; i += CF::NT) {
     const int r = i / CF::T, tt = i - r * CF::T;
     const int64_t t = t0 + tt;
     E val = zero_elem<E>();
     if (t < L) {
-      if (r < 3 * CF::CH) {
+      if (r < 2 * CF::CH) {
         const int which = r / CF::CH, c = r - which * CF::CH;
         const int64_t d = d0 + c;
-        const void* base = which == 0 ? a.u : (which == 1 ? a.delta : a.z);
+        const void* base = which == 0 ? a.delta : a.z;
         if (d < a.dim && base) val = static_cast<const E*>(base)[(b * a.dim + d) * L + t];
       } else {
-        const int rr = r - 3 * CF::CH, which = rr / CF::N, n = rr - which * CF::N;
+        const int rr = r - 2 * CF::CH, which = rr / CF::N, n = rr - which * CF::N;
         val = static_cast<const E*>(which == 0 ? a.B : a.C)[(b * CF::N + n) * L + t];
       }
     }
-    raw[r * CF::T + tt] = val;
+    rest[i] = val;
   }
 }
 
 // ------------------------------------------------------------- phase 1 ---
 
-// Runs on NTH threads (tid in [0, NTH)): all threads of a CTA, or its helper
-// warps in the warp-specialised kernel.
-template <class CF, bool kFull, int NTH = CF::NT>
+// Per (channel, 4-step quad) item, spread over the CTA's threads.  The same
+// item-to-thread map is used by phase 3, so a thread's per-channel constants
+// (bias, convolution taps, D) stay in its registers.
+template <class CF>
+struct ConvRegs {  // per-item convolution taps, right-aligned: tap kConvTaps-1 meets step t
+  float w[CF::CONV ? CF::ITEMS_PER_THREAD : 1][kConvTaps];
+  float b[CF::CONV ? CF::ITEMS_PER_THREAD : 1];
+};
+
+template <class CF, bool kFull>
 __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem* raw,
-                                       float4* dwD, float4* dwW, unsigned char* bc,
-                                       const float (&bias_it)[(CF::ITEMS + NTH - 1) / NTH],
-                                       int64_t d0, int64_t t0, int tid = threadIdx.x) {
+                                       float4* dwD, float4* dwW, float4* su, unsigned char* bc,
+                                       const float (&bias_it)[CF::ITEMS_PER_THREAD],
+                                       const ConvRegs<CF>& cv, int64_t d0, int64_t t0) {
   using E = typename CF::Elem;
-  constexpr int IPT = (CF::ITEMS + NTH - 1) / NTH;
+  const int tid = threadIdx.x;
+  const E* rawD = raw + CF::CH * CF::XT;
 #pragma unroll
-  for (int it = 0; it < IPT; ++it) {
-    const int i = tid + it * NTH;
-    if (CF::ITEMS % NTH != 0 && i >= CF::ITEMS) break;
+  for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+    const int i = tid + it * CF::NT;
+    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
     const int c = i / CF::QPR, q = i - c * CF::QPR;
-    const float4 dl = load4_f32(raw + (CF::CH + c) * CF::T + 4 * q);
-    const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
+    const float4 dl = load4_f32(rawD + c * CF::T + 4 * q);
+    float4 uu;
+    if constexpr (CF::CONV) {
+      // u = SiLU(b + sum_k w[k] x[t - (kConvTaps-1) + k]); the row holds x from
+      // step t0 - HALO, so steps t0+4q-4 .. t0+4q+3 are elements 4q+HALO-4 ..
+      const E* xr = raw + c * CF::XT + 4 * q + CF::HALO - 4;
+      const float4 xa = load4_f32(xr), xb = load4_f32(xr + 4);
+      const float win[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      float o[4];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        float acc = cv.b[it];
+#pragma unroll
+        for (int k = 0; k < kConvTaps; ++k) acc = fmaf(cv.w[it][k], win[k4 + 5 - kConvTaps + k], acc);
+        o[k4] = acc;
+      }
+      const float2 u01 = silu_fast2(make_float2(o[0], o[1]));
+      const float2 u23 = silu_fast2(make_float2(o[2], o[3]));
+      uu = make_float4(u01.x, u01.y, u23.x, u23.y);
+      su[q * CF::DW_STRIDE + c] = uu;
+    } else {
+      uu = load4_f32(raw + c * CF::XT + 4 * q);
+    }
     const float bias = bias_it[it];
     const float2 b2 = make_float2(bias, bias);
     float2 x01 = __fadd2_rn(make_float2(dl.x, dl.y), b2);
@@ -224,14 +290,14 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     dwW[q * CF::DW_STRIDE + c] = make_float4(w[0], w[1], w[2], w[3]);
   }
   // B and C rows [n][t] -> [t][n/2 pairs][B_2p, B_2p+1, C_2p, C_2p+1]
-  const E* rawB = raw + 3 * CF::CH * CF::T;
-  const E* rawC = rawB + CF::N * CF::T;
+  const E* rawB = raw + CF::OFF_B_T / CF::ES;
+  const E* rawC = raw + CF::OFF_C_T / CF::ES;
   if constexpr (CF::ES == 2) {
     constexpr int TP = CF::T / 2;  // timestep pairs (one 32-bit word per row)
     const uint32_t* B32 = reinterpret_cast<const uint32_t*>(rawB);
     const uint32_t* C32 = reinterpret_cast<const uint32_t*>(rawC);
     constexpr int NB4 = CF::N / 4;
-    for (int i = tid; i < NB4 * TP; i += NTH) {
+    for (int i = tid; i < NB4 * TP; i += CF::NT) {
       const int tp = i / NB4, nb = i - tp * NB4;
       uint32_t bw[4], cw[4];
 #pragma unroll
@@ -249,7 +315,7 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
   } else {
     const float* fb = reinterpret_cast<const float*>(rawB);
     const float* fc = reinterpret_cast<const float*>(rawC);
-    for (int i = tid; i < (CF::N / 4) * CF::T; i += NTH) {
+    for (int i = tid; i < (CF::N / 4) * CF::T; i += CF::NT) {
       const int nb = i / CF::T, t = i - nb * CF::T;
       float4* dst = reinterpret_cast<float4*>(bc + t * CF::BC_ROW + nb * CF::BC_BLOCK);
       dst[0] = make_float4(fb[(4 * nb) * CF::T + t], fb[(4 * nb + 1) * CF::T + t],
@@ -457,18 +523,18 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
 
 // ------------------------------------------------------------- phase 3 ---
 
-template <class CF, bool kFull, int NTH = CF::NT>
+template <class CF, bool kFull>
 __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem* raw,
-                                       const float* sy,
-                                       const float (&D_it)[(CF::ITEMS + NTH - 1) / NTH],
-                                       int64_t b, int64_t d0, int64_t t0, bool has_z,
-                                       int tid = threadIdx.x) {
+                                       const float* sy, const float4* su,
+                                       const float (&D_it)[CF::ITEMS_PER_THREAD], int64_t b,
+                                       int64_t d0, int64_t t0, bool has_z) {
   const int64_t L = a.seqlen, D = a.dim;
-  constexpr int IPT = (CF::ITEMS + NTH - 1) / NTH;
+  const int tid = threadIdx.x;
+  const typename CF::Elem* rawZ = raw + CF::OFF_Z_T / CF::ES;
 #pragma unroll
-  for (int it = 0; it < IPT; ++it) {
-    const int i = tid + it * NTH;
-    if (CF::ITEMS % NTH != 0 && i >= CF::ITEMS) break;
+  for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+    const int i = tid + it * CF::NT;
+    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
     const int c = i / CF::QPR, q = i - c * CF::QPR;
     const int64_t d = d0 + c, t = t0 + 4 * q;
     if constexpr (!kFull) {
@@ -482,13 +548,15 @@ __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem
       s01 = __fadd2_rn(s01, make_float2(o.x, o.y));
       s23 = __fadd2_rn(s23, make_float2(o.z, o.w));
     }
-    const float4 uu = load4_f32(raw + c * CF::T + 4 * q);
+    float4 uu;
+    if constexpr (CF::CONV) uu = su[q * CF::DW_STRIDE + c];
+    else uu = load4_f32(raw + c * CF::XT + 4 * q);
     const float Dd = D_it[it];
     const float2 D2 = make_float2(Dd, Dd);
     float2 y01 = __ffma2_rn(D2, make_float2(uu.x, uu.y), s01);
     float2 y23 = __ffma2_rn(D2, make_float2(uu.z, uu.w), s23);
     if (has_z) {
-      const float4 zz = load4_f32(raw + (2 * CF::CH + c) * CF::T + 4 * q);
+      const float4 zz = load4_f32(rawZ + c * CF::T + 4 * q);
       y01 = __fmul2_rn(y01, silu_fast2(make_float2(zz.x, zz.y)));
       y23 = __fmul2_rn(y23, silu_fast2(make_float2(zz.z, zz.w)));
     }
@@ -605,6 +673,26 @@ __device__ __forceinline__ void publish_carry(const Sched& s, int w) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(s.epoch) : "memory");
 }
 
+// This thread's convolution taps for its items of channel tile d0, placed
+// right-aligned in kConvTaps slots (zeros before a shorter filter).
+template <class CF>
+__device__ __forceinline__ void load_conv_regs(const FwdArgs& a, int64_t d0, ConvRegs<CF>& cv) {
+  if constexpr (CF::CONV) {
+    const int W = a.conv_width;
+#pragma unroll
+    for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+      const int64_t d = d0 + (threadIdx.x + it * CF::NT) / CF::QPR;
+      const bool ok = d < a.dim;
+#pragma unroll
+      for (int k = 0; k < kConvTaps; ++k) {
+        const int src = k - (kConvTaps - W);
+        cv.w[it][k] = (ok && src >= 0) ? __ldg(a.conv_w + d * W + src) : 0.f;
+      }
+      cv.b[it] = (ok && a.conv_b) ? __ldg(a.conv_b + d) : 0.f;
+    }
+  }
+}
+
 // -------------------------------------------------------------- kernel ---
 
 // kMulti = false: one channel group per CTA (gridDim = groups), a plain loop
@@ -626,6 +714,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   float* sy = reinterpret_cast<float*>(smem + CF::OFF_SY);
   float* aggP = reinterpret_cast<float*>(smem + CF::OFF_AGG);
   float* aggH = aggP + CF::AGG_FLOATS;
+  float4* su = reinterpret_cast<float4*>(smem + CF::OFF_SU);  // CONV only
   __shared__ __align__(8) uint64_t bars[2];
 
   const int w = blockIdx.x;
@@ -662,12 +751,14 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     const bool chan_ok = d < a.dim;
     const bool full_tile = d0 + CF::CH <= a.dim;
     float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
+    ConvRegs<CF> cv;
 #pragma unroll
     for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
       const int64_t di = d0 + (tid + it * CF::NT) / CF::QPR;
       bias_it[it] = (a.delta_bias && di < a.dim) ? __ldg(a.delta_bias + di) : 0.f;
       D_it[it] = (a.D && di < a.dim) ? __ldg(a.D + di) : 0.f;
     }
+    load_conv_regs<CF>(a, d0, cv);
     float2 h[CF::G / 2], a2[CF::G / 2];
 #pragma unroll
     for (int g = 0; g < CF::G / 2; ++g) {
@@ -687,8 +778,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     };
     auto run_phase1 = [&](int64_t k) {
       const E* rp = reinterpret_cast<const E*>(raw(k));
-      if (full_chunk(k)) phase1<CF, true>(a, rp, dwD, dwW, bc, bias_it, d0, k * CF::T);
-      else phase1<CF, false>(a, rp, dwD, dwW, bc, bias_it, d0, k * CF::T);
+      if (full_chunk(k)) phase1<CF, true>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0, k * CF::T);
+      else phase1<CF, false>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0, k * CF::T);
     };
     auto drain = [&](int64_t first, int64_t last) {
       if (tma)
@@ -714,8 +805,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
         return;
       }
       const E* rc = reinterpret_cast<const E*>(raw(k));
-      if (full_chunk(k)) phase3<CF, true>(a, rc, sy, D_it, b, d0, k * CF::T, has_z);
-      else phase3<CF, false>(a, rc, sy, D_it, b, d0, k * CF::T, has_z);
+      if (full_chunk(k)) phase3<CF, true>(a, rc, sy, su, D_it, b, d0, k * CF::T, has_z);
+      else phase3<CF, false>(a, rc, sy, su, D_it, b, d0, k * CF::T, has_z);
       if (k + 1 < nseq) run_phase1(k + 1);
       __syncthreads();
       if (tma && tid == 0 && k + 2 < nseq)
@@ -742,7 +833,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
 
   float2 h[CF::G / 2], a2[CF::G / 2];
   float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
-  int32_t bias_g = -1, D_g = -1;  // group whose bias / D are cached
+  ConvRegs<CF> cv;
+  int32_t bias_g = -1, D_g = -1;  // group whose bias (and taps) / D are cached
   bool ok = true;  // false once a bounded wait has given up (error word set)
 
   auto d0_of = [&](const Cursor& r) { return (int64_t)r.tile * CF::CH; };
@@ -770,11 +862,13 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   auto run_phase1 = [&](int64_t jj) {  // jj = prep's chunk
     if (prep.g != bias_g) {
       load_items(a.delta_bias, prep, bias_it);
+      load_conv_regs<CF>(a, d0_of(prep), cv);
       bias_g = prep.g;
     }
     const E* rp = reinterpret_cast<const E*>(raw(jj));
-    if (full_chunk(prep)) phase1<CF, true>(a, rp, dwD, dwW, bc, bias_it, d0_of(prep), (int64_t)prep.c * CF::T);
-    else phase1<CF, false>(a, rp, dwD, dwW, bc, bias_it, d0_of(prep), (int64_t)prep.c * CF::T);
+    const int64_t t0 = (int64_t)prep.c * CF::T;
+    if (full_chunk(prep)) phase1<CF, true>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0_of(prep), t0);
+    else phase1<CF, false>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0_of(prep), t0);
   };
   // On a timed-out wait: wait (bounded) for every copy this CTA still has in
   // flight, so that none lands in shared memory after the CTA has left.
@@ -857,8 +951,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
       D_g = cur.g;
     }
     const E* rc = reinterpret_cast<const E*>(raw(q));
-    if (full_chunk(cur)) phase3<CF, true>(a, rc, sy, D_it, cur.b, d0, (int64_t)cur.c * CF::T, has_z);
-    else phase3<CF, false>(a, rc, sy, D_it, cur.b, d0, (int64_t)cur.c * CF::T, has_z);
+    if (full_chunk(cur)) phase3<CF, true>(a, rc, sy, su, D_it, cur.b, d0, (int64_t)cur.c * CF::T, has_z);
+    else phase3<CF, false>(a, rc, sy, su, D_it, cur.b, d0, (int64_t)cur.c * CF::T, has_z);
     if (q + 1 < nseq) {
       run_phase1(q + 1);
       prep.advance();

@@ -19,6 +19,10 @@ advances) is drawn as N(0, 1) fp32 [batch, dim, N]: the magnitude of a state
 after many steps of unit-variance inputs with Delta*B*u of order 0.01-1.
 Decode-step workloads are Workload objects with seqlen = 1 (one token per
 channel); their tensors drop the L axis.
+
+The short convolution's taps [dim, W] and bias [dim] are U(-1/sqrt(W),
+1/sqrt(W)), the default initialisation of a depthwise Conv1d of width W; its
+input x takes the place of u (N(0, 1)).
 """
 from __future__ import annotations
 
@@ -37,7 +41,8 @@ _lock = threading.Lock()
 _lib = None
 
 # stream ids: one independent counter-based stream per tensor
-STREAM = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "A": 6, "D": 7, "dt": 8, "h0": 9}
+STREAM = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "A": 6, "D": 7, "dt": 8, "h0": 9,
+          "conv_w": 10, "conv_b": 11}
 
 
 def build(force: bool = False) -> str:
@@ -210,3 +215,11 @@ STEP_WORKLOADS = {
     "step_b128_d8192_n16_bf16": Workload("step_b128_d8192_n16_bf16", 128, 8192, 1, 16, "bf16"),
     "step_b128_d8192_n16_f32": Workload("step_b128_d8192_n16_f32", 128, 8192, 1, 16, "f32"),
 }
+
+
+def make_conv(dim: int, width: int, seed: int = 1234) -> tuple[np.ndarray, np.ndarray]:
+    """Taps [dim, width] and bias [dim] of the short depthwise convolution."""
+    r = 1.0 / np.sqrt(width)
+    w = fill(seed, STREAM["conv_w"], (dim, width), kind="uniform", mean=-r, scale=2 * r)
+    b = fill(seed, STREAM["conv_b"], (dim,), kind="uniform", mean=-r, scale=2 * r)
+    return w, b

@@ -129,6 +129,26 @@ def test_step_rejections(lib, over, status):
     assert _call_step(lib, **over) == status
 
 
+def _call_conv(lib, **over):
+    a = dict(x=0x10000, cw=0x90000, cb=None, W=4, delta=0x20000, A=0x30000, B=0x40000,
+             C=0x50000, D=None, z=None, bias=None, sp=1, y=0x60000, h=None, batch=1, dim=1, L=8,
+             N=16, dt=N.SS_F32, ws=None, wsb=0)
+    a.update(over)
+    return lib.ss_scan_fwd_conv(a["x"], a["cw"], a["cb"], a["W"], a["delta"], a["A"], a["B"],
+                                a["C"], a["D"], a["z"], a["bias"], a["sp"], a["y"], a["h"],
+                                a["batch"], a["dim"], a["L"], a["N"], a["dt"], a["ws"], a["wsb"],
+                                None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(cw=None), N.SS_ERR_INVALID_ARG), (dict(x=None), N.SS_ERR_INVALID_ARG),
+    (dict(W=0), N.SS_ERR_UNSUPPORTED), (dict(W=5), N.SS_ERR_UNSUPPORTED),
+    (dict(cw=0x90002), N.SS_ERR_INVALID_ARG), (dict(cb=0x90006), N.SS_ERR_INVALID_ARG),
+    (dict(N=48), N.SS_ERR_UNSUPPORTED)])
+def test_conv_rejections(lib, over, status):
+    assert _call_conv(lib, **over) == status
+
+
 def test_workspace_query_rejects_bad_sizes(lib):
     # (valid sizes need the device's SM count, so they are covered by the GPU tests)
     with pytest.raises(N.SSError):
