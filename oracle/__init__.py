@@ -47,7 +47,8 @@ def _load():
             vp, i64 = ctypes.c_void_p, ctypes.c_int64
             lib.oracle_scan_fwd.argtypes = [
                 vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
-                i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int]
+                i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int]
             lib.oracle_scan_fwd.restype = ctypes.c_int
             lib.oracle_softplus.argtypes = [ctypes.c_double]
             lib.oracle_softplus.restype = ctypes.c_double
@@ -73,7 +74,7 @@ def _stored(a, name):
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
              softplus=True, channels=None, nthreads=None, h0=None, conv_weight=None,
-             conv_bias=None):
+             conv_bias=None, zoh=False):
     """Serial fp64 selective scan.
 
     u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; all float32 or all
@@ -84,6 +85,8 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     conv_weight: optional [dim, W] float32 taps of the causal depthwise
     convolution; u then holds the convolution's input x and the scan runs on
     SiLU(conv(x) + conv_bias).  conv_bias: optional [dim] float32.
+    zoh: exact zero-order hold, B_bar = expm1(Delta A) / A * B (Delta B where
+    A = 0), instead of the simplified Delta B.
     Returns (y, last_state) as float64 with
     shapes [batch, dim, L] / [batch, dim, N], or [len(channels), L] /
     [len(channels), N] when channels is given.
@@ -139,7 +142,7 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(softplus)), dt, batch, dim, L, N,
         _ptr(channels), nch, _ptr(y), _ptr(h), _ptr(h0), _ptr(conv_w), _ptr(conv_b), width,
-        int(nthreads))
+        int(bool(zoh)), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_scan_fwd rejected its arguments")
     return y, h

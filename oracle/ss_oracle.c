@@ -45,6 +45,10 @@
  *      u[b,d,t] = SiLU(conv_bias[d] + sum_{k<W} conv_w[d,k] x[b,d,t-(W-1)+k]),
  *    with x = 0 before t = 0 (Conv1d is a cross-correlation, so tap W-1
  *    meets the current token).
+ *  - exact zero-order hold (zoh != 0; same page, sec. 2.2, the form before its
+ *    simplification): B_bar = (Delta A)^-1 (exp(Delta A) - 1) Delta B, which
+ *    for diagonal A is expm1(Delta A[d,n]) / A[d,n] * B[b,n,t], and Delta B
+ *    where A[d,n] = 0 (its limit).  expm1 keeps it exact for small Delta A.
  *  - an initial state h0 replaces the zero state of the pure-PyTorch module;
  *    the pages keep h between calls for recurrent (one token at a time)
  *    inference ("从Transformer的痛点说起 ... Mamba", sec. 5.1 table and
@@ -90,6 +94,7 @@ typedef struct {
   const float* conv_w; /* [dim, conv_width] or NULL: u is the scan input itself */
   const float* conv_b; /* [dim] or NULL */
   int conv_width;
+  int zoh;            /* 1: exact zero-order hold for B_bar */
   int64_t next;       /* work counter (guarded by mu) */
   pthread_mutex_t mu;
 } job_t;
@@ -129,7 +134,9 @@ static void run_channel(const job_t* J, int64_t slot, double* h) {
       const double a_bar = exp(dt * (double)J->A[d * N + n]);
       const double b_t = widen(J->B, J->dtype, bc_base + (int64_t)n * L + t);
       const double c_t = widen(J->C, J->dtype, bc_base + (int64_t)n * L + t);
-      h[n] = a_bar * h[n] + dt * b_t * ut;
+      const double an = (double)J->A[d * N + n];
+      const double b_bar = (J->zoh && an != 0.0) ? expm1(dt * an) / an * b_t : dt * b_t;
+      h[n] = a_bar * h[n] + b_bar * ut;
       s += c_t * h[n];
     }
     s += Dd * ut;
@@ -172,6 +179,7 @@ static void* worker(void* arg) {
  * conv_w      : [dim, conv_width] f32 taps of the short convolution, or NULL
  * conv_b      : [dim] f32 convolution bias (nullable)
  * conv_width  : 1..64 when conv_w is given
+ * zoh         : nonzero for the exact zero-order-hold B_bar
  * nthreads    : worker threads (>= 1)
  */
 int oracle_scan_fwd(const void* u, const void* delta, const float* A,
@@ -181,7 +189,7 @@ int oracle_scan_fwd(const void* u, const void* delta, const float* A,
                     int dstate, const int64_t* channels, int64_t n_channels,
                     double* y, double* last_state, const double* h0,
                     const float* conv_w, const float* conv_b, int conv_width,
-                    int nthreads) {
+                    int zoh, int nthreads) {
   if (!u || !delta || !A || !B || !C || !y) return -1;
   if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0) return -1;
   if (dtype != 0 && dtype != 1) return -1;
@@ -203,6 +211,7 @@ int oracle_scan_fwd(const void* u, const void* delta, const float* A,
   J.channels = channels; J.n_channels = n_channels;
   J.y = y; J.last_state = last_state; J.h0 = h0; J.next = 0;
   J.conv_w = conv_w; J.conv_b = conv_b; J.conv_width = conv_w ? conv_width : 0;
+  J.zoh = zoh != 0;
   pthread_mutex_init(&J.mu, NULL);
 
   pthread_t tids[512];

@@ -14,20 +14,20 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "ss_oracle.c")
 
 # (name, original text, mutated text)
 MUTANTS = [
-    ("B_bar without Delta", "h[n] = a_bar * h[n] + dt * b_t * ut;", "h[n] = a_bar * h[n] + b_t * ut;"),
+    ("B_bar without Delta", ": dt * b_t;", ": b_t;"),
     ("sign of A", "exp(dt * (double)J->A[d * N + n])", "exp(-dt * (double)J->A[d * N + n])"),
     ("B and C swapped", "const double b_t = widen(J->B,", "const double b_t = widen(J->C,"),
     ("bias outside the softplus",
      "const double dt = J->softplus_flag ? softplus64(x) : x;",
      "const double dt = J->softplus_flag ? softplus64(x - bias) + bias : x;"),
     ("readout before the update",
-     "h[n] = a_bar * h[n] + dt * b_t * ut;\n      s += c_t * h[n];",
-     "s += c_t * h[n];\n      h[n] = a_bar * h[n] + dt * b_t * ut;"),
+     "h[n] = a_bar * h[n] + b_bar * ut;\n      s += c_t * h[n];",
+     "s += c_t * h[n];\n      h[n] = a_bar * h[n] + b_bar * ut;"),
     ("gate misses the skip term",
      "    s += Dd * ut;\n    if (J->z) s *= silu64(widen(J->z, J->dtype, row + t));",
      "    if (J->z) s *= silu64(widen(J->z, J->dtype, row + t));\n    s += Dd * ut;"),
     ("A indexed [n][d]", "J->A[d * N + n]", "J->A[n * J->dim + d]"),
-    ("state not carried", "h[n] = a_bar * h[n] + dt * b_t * ut;", "h[n] = a_bar * 0.0 + dt * b_t * ut;"),
+    ("state not carried", "h[n] = a_bar * h[n] + b_bar * ut;", "h[n] = a_bar * 0.0 + b_bar * ut;"),
     ("initial state ignored", "h[n] = J->h0 ? J->h0[flat * N + n] : 0.0;", "h[n] = 0.0;"),
     ("initial state indexed [b][n][d]", "J->h0[flat * N + n]", "J->h0[(b * N + n) * J->dim + d]"),
     ("initial state indexed [n][b][d]", "J->h0[flat * N + n]", "J->h0[n * J->batch * J->dim + flat]"),
@@ -36,6 +36,10 @@ MUTANTS = [
     ("conv window shifted", "const int64_t s = t - (W - 1) + k;", "const int64_t s = t - W + k;"),
     ("conv bias dropped", "double acc = J->conv_b ? (double)J->conv_b[d] : 0.0;", "double acc = 0.0;"),
     ("conv output without SiLU", "  return silu64(acc);", "  return acc;"),
+    ("zoh through exp - 1", "expm1(dt * an)", "(exp(dt * an) - 1.0)"),
+    ("zoh without the division by A", "expm1(dt * an) / an * b_t", "expm1(dt * an) * b_t"),
+    ("zoh with Delta twice", "expm1(dt * an) / an * b_t", "expm1(dt * an) / an * dt * b_t"),
+    ("zoh sign of A", "expm1(dt * an) / an * b_t", "expm1(-dt * an) / an * b_t"),
 ]
 
 PIN_CALLS = [
@@ -52,6 +56,8 @@ PIN_CALLS = [
     lambda: pins.test_initial_state_bruteforce(3),
     lambda: pins.test_conv_prologue_matches_numpy_convolution(4),
     pins.test_conv_prologue_impulse_taps,
+    pins.test_zoh_matches_ode_integration,
+    pins.test_zoh_small_delta_series,
 ]
 
 

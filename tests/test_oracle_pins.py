@@ -36,7 +36,7 @@ def test_softplus_identities():
     for x in (-35.0, -7.25, -1e-3, 0.3, 2.0, 19.5, 29.9, 30.1, 55.0):
         assert oracle.softplus(x) - oracle.softplus(-x) == pytest.approx(x, rel=1e-15, abs=1e-15)
     assert oracle.softplus(60.0) == 60.0
-    assert oracle.softplus(-40.0) == pytest.approx(math.exp(-40.0), rel=1e-15)
+    assert oracle.softplus(-40.0) == pytest.approx(math.exp(-40.0), rel=1e-15, abs=0)
     # monotone and positive
     xs = np.linspace(-50, 50, 1001)
     v = np.array([oracle.softplus(x) for x in xs])
@@ -49,9 +49,9 @@ def test_silu_identities():
     assert oracle.silu(0.0) == 0.0
     for z in (-20.0, -3.0, -0.5, 0.25, 1.0, 4.0, 30.0):
         assert oracle.silu(z) - oracle.silu(-z) == pytest.approx(z, rel=1e-15, abs=1e-15)
-    assert oracle.silu(50.0) == pytest.approx(50.0, rel=1e-20)
+    assert oracle.silu(50.0) == pytest.approx(50.0, rel=1e-20, abs=0)
     assert abs(oracle.silu(-50.0)) < 1e-19
-    assert oracle.silu(1.0) == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
+    assert oracle.silu(1.0) == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15, abs=0)
 
 
 # ------------------------------------------------------ LTI closed form ----
@@ -331,10 +331,11 @@ def test_index_plumbing_single_impulse():
             dl = float(bias[d])
             for n in range(N):
                 ref = math.exp((L - 1) * dl * float(A[d, n])) * dl * float(B[b, n, 0]) * float(u[b, d, 0])
-                assert h[b, d, n] == pytest.approx(ref, rel=1e-14)
+                assert h[b, d, n] == pytest.approx(ref, rel=1e-14, abs=0)
             # y_0 = D u_0 + C_0.h_0 (C_0 = 0); y_{L-1} = C_{L-1}.h_{L-1}
-            assert y[b, d, 0] == pytest.approx(float(Dv[d]) * float(u[b, d, 0]), rel=1e-15)
-            assert y[b, d, L - 1] == pytest.approx(float(np.dot(C[b, :, L - 1].astype(np.float64), h[b, d])), rel=1e-14)
+            assert y[b, d, 0] == pytest.approx(float(Dv[d]) * float(u[b, d, 0]), rel=1e-15, abs=0)
+            assert y[b, d, L - 1] == pytest.approx(float(np.dot(C[b, :, L - 1].astype(np.float64), h[b, d])),
+                                                   rel=1e-14, abs=0)
             assert np.all(y[b, d, 1:L - 1] == 0.0)
 
 
@@ -536,6 +537,80 @@ def test_conv_prologue_feeds_the_scan():
                 acc += float(c["C"][0, n, t]) * hn
             ref = (acc + float(c["D"][d]) * us[t]) * oracle.silu(float(c["z"][0, d, t]))
             assert y[0, d, t] == pytest.approx(ref, rel=1e-13, abs=1e-15)
+
+
+# ------------------------------------------------- exact zero-order hold ---
+# ZOH: the continuous system h' = A h + B x with the input held constant over
+# each step of length Delta ("从Transformer的痛点说起 ... Mamba", sec. 2.2).
+
+def _rk4_hold(a, b, x, dl, h, m=512):
+    """Integrate h' = a h + b x over [0, dl] with m classical RK4 steps (no exp)."""
+    k = dl / m
+    f = lambda v: a * v + b * x
+    for _ in range(m):
+        k1 = f(h)
+        k2 = f(h + 0.5 * k * k1)
+        k3 = f(h + 0.5 * k * k2)
+        k4 = f(h + k * k3)
+        h = h + k / 6.0 * (k1 + 2 * k2 + 2 * k3 + k4)
+    return h
+
+
+def test_zoh_matches_ode_integration():
+    """The exact-ZOH recurrence equals a fine Runge-Kutta integration of the
+    continuous system with each input held over its step (and the same
+    readout): B_bar is (Delta A)^-1 (e^{Delta A} - 1) Delta B."""
+    rng = np.random.default_rng(71)
+    batch, dim, L, N = 1, 2, 12, 3
+    c = _rand_case(rng, batch, dim, L, N)
+    c["A"] = _f32(-rng.uniform(0.2, 3.0, size=(dim, N)))
+    delta = _f32(rng.uniform(0.05, 0.6, size=(batch, dim, L)))
+    y, h = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], softplus=False, zoh=True)
+    for d in range(dim):
+        hs = np.zeros(N)
+        for t in range(L):
+            dl = float(delta[0, d, t])
+            for n in range(N):
+                hs[n] = _rk4_hold(float(c["A"][d, n]), float(c["B"][0, n, t]), float(c["u"][0, d, t]),
+                                  dl, hs[n])
+            ref = float(np.dot(c["C"][0, :, t].astype(np.float64), hs)) + float(c["D"][d]) * float(c["u"][0, d, t])
+            assert y[0, d, t] == pytest.approx(ref, rel=1e-9, abs=1e-12)
+        assert np.allclose(h[0, d], hs, rtol=1e-9, atol=1e-12)
+
+
+def test_zoh_small_delta_series():
+    """Delta A ~ 1e-9: B_bar = Delta B (1 + x/2 + x^2/6) to 1e-16, x = Delta A; an
+    e^x - 1 evaluation would lose half the digits here."""
+    rng = np.random.default_rng(72)
+    batch, dim, N = 1, 3, 4
+    A = _f32(-rng.uniform(0.5, 2.0, size=(dim, N)))
+    u = _f32(rng.normal(size=(batch, dim, 1)))
+    B = _f32(rng.normal(size=(batch, N, 1)))
+    C = np.zeros((batch, N, 1), np.float32)
+    delta = np.full((batch, dim, 1), 1e-9, np.float32)
+    _, h = oracle.scan_fwd(u, delta, A, B, C, softplus=False, zoh=True)
+    for d in range(dim):
+        dl = float(delta[0, d, 0])
+        for n in range(N):
+            x = dl * float(A[d, n])
+            ref = dl * (1.0 + x / 2 + x * x / 6) * float(B[0, n, 0]) * float(u[0, d, 0])
+            assert h[0, d, n] == pytest.approx(ref, rel=1e-15, abs=0)
+
+
+def test_zoh_limit_a_zero_and_simplified_form():
+    """A = 0: B_bar = Delta B exactly (the limit), so ZOH and the simplified form
+    agree bitwise on those states; with A != 0 they differ."""
+    rng = np.random.default_rng(73)
+    batch, dim, L, N = 2, 3, 20, 4
+    c = _rand_case(rng, batch, dim, L, N)
+    delta = _f32(rng.normal(scale=0.5, size=(batch, dim, L)))
+    A0 = np.zeros((dim, N), np.float32)
+    y1, h1 = oracle.scan_fwd(c["u"], delta, A0, c["B"], c["C"], D=c["D"], z=c["z"], zoh=True)
+    y2, h2 = oracle.scan_fwd(c["u"], delta, A0, c["B"], c["C"], D=c["D"], z=c["z"], zoh=False)
+    assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
+    y3, _ = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], z=c["z"], zoh=True)
+    y4, _ = oracle.scan_fwd(c["u"], delta, c["A"], c["B"], c["C"], D=c["D"], z=c["z"], zoh=False)
+    assert _rel(y3, y4) > 1e-3
 
 
 # ------------------------------------------------------- host plumbing -----
