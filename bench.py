@@ -167,7 +167,8 @@ def run_gpu_arm(args, w: I.Workload):
     import torch
     import torch.distributed as dist
 
-    from selective_state_space_ss_b200 import load_library, ss_scan_fwd, ss_scan_fwd_conv
+    from selective_state_space_ss_b200 import (load_library, ss_scan_fwd, ss_scan_fwd_conv,
+                                               ss_scan_fwd_zoh)
 
     world, rank, local = _dist_env()
     torch.cuda.set_device(local)
@@ -206,9 +207,13 @@ def run_gpu_arm(args, w: I.Workload):
         conv = (torch.from_numpy(cw).to(dev), torch.from_numpy(cb).to(dev))
         host[0]["conv"] = (cw, cb)
 
+    if args.zoh:
+        host[0]["zoh"] = True
+
     def scan(x, y_out, h_out):
         if conv is None:
-            return ss_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+            fn = ss_scan_fwd_zoh if args.zoh else ss_scan_fwd
+            return fn(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
                                delta_bias=x["delta_bias"], softplus=w.softplus, y_out=y_out,
                                last_state_out=h_out, stream=stream)
         return ss_scan_fwd_conv(x["u"], conv[0], x["delta"], x["A"], x["B"], x["C"], D=x["D"],
@@ -245,7 +250,7 @@ def run_gpu_arm(args, w: I.Workload):
     ex = host[0]
     pinned = {}
     for k, v in ex.items():
-        if k == "conv":
+        if k in ("conv", "zoh"):
             continue
         if v is None:
             pinned[k] = None
@@ -447,7 +452,7 @@ def oracle_sample(w: I.Workload, x: dict, target_s: float):
         cw, cb = x.get("conv", (None, None))
         oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
                         softplus=w.softplus, channels=ch, nthreads=cores, conv_weight=cw,
-                        conv_bias=cb)
+                        conv_bias=cb, zoh=x.get("zoh", False))
         dt = time.perf_counter() - t0
         if dt >= target_s or take == nch:
             return take, dt, cores
@@ -486,8 +491,9 @@ def run_reference_arm(args, w: I.Workload):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def config_of(w: I.Workload, world: int, conv: int = 0):
-    return {"workload": w.name + (f"+conv{conv}" if conv else ""), "batch": w.batch,
+def config_of(w: I.Workload, world: int, conv: int = 0, zoh: bool = False):
+    return {"workload": w.name + (f"+conv{conv}" if conv else "") + ("+zoh" if zoh else ""),
+            "b_bar": "exact zoh" if zoh else "delta*B", "batch": w.batch,
             "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate,
             "in_dtype": w.dtype, "state_dtype": "f32", "y_dtype": "f32", "conv_width": conv,
             "parallelism": f"replicas x{world} (independent batch per GPU, no collective)",
@@ -504,11 +510,14 @@ def main():
                     choices=sorted(I.WORKLOADS) + sorted(I.STEP_WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--zoh", action="store_true", help="exact zero-order-hold B_bar")
     ap.add_argument("--conv", type=int, default=0,
                     help="fuse the short causal conv1d + SiLU of this width (1-4) into the scan")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.conv and args.zoh:
+        ap.error("--conv and --zoh are separate kernel variants")
     if args.op == "step":
         if args.impl != "native" or args.gpus != 1:
             ap.error("--op step runs the native arm on one GPU")
@@ -532,7 +541,8 @@ def main():
     line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": r["world"],
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": config_of(w, r["world"], args.conv), "roofline": roof,
+            "data": "synthetic", "config": config_of(w, r["world"], args.conv, args.zoh),
+            "roofline": roof,
             "e2e": r["e2e"], "gpu_launches": args.steps, "clocks": r["clocks"]}
     if r["world"] == 1 and not args.no_cpu_baseline:
         take, dt, cores = oracle_sample(w, r["host"], target_s=10.0)

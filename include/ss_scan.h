@@ -112,6 +112,27 @@ ss_status ss_scan_fwd_from_state(const void* u, const void* delta, const float* 
                                  size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * ss_scan_fwd_zoh -- ss_scan_fwd with the exact zero-order-hold input matrix
+ * instead of its simplification ("从Transformer的痛点说起 ... Mamba", sec. 2.2:
+ * B_bar = (Delta A)^-1 (exp(Delta A) - I) Delta B, which implementations
+ * usually simplify to Delta B).  For diagonal A:
+ *
+ *   h[n] = exp(Delta_t A[d,n]) h[n] + (exp(Delta_t A[d,n]) - 1) / A[d,n] B[b,n,t] u[b,d,t]
+ *
+ * and Delta_t B[b,n,t] u[b,d,t] where A[d,n] = 0 (the limit).  Near
+ * Delta A = 0 the kernel takes (exp(x) - 1)/x from its Taylor series, so no
+ * cancellation reaches the state.  Arguments, layouts, results, errors and
+ * the workspace size are those of ss_scan_fwd.
+ */
+ss_status ss_scan_fwd_zoh(const void* u, const void* delta, const float* A,
+                          const void* B, const void* C, const float* D,
+                          const void* z, const float* delta_bias,
+                          int softplus_flag, float* y_out, float* last_state_out,
+                          int64_t batch, int64_t dim, int64_t seqlen, int dstate,
+                          ss_dtype in_dtype, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * ss_scan_fwd_conv -- ss_scan_fwd whose input u is formed inside the kernel
  * from the block's short convolution: the causal depthwise Conv1d of width W
  * (padding W-1, cut to the first L outputs) followed by SiLU

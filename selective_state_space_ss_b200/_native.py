@@ -23,7 +23,7 @@ SS_F32, SS_BF16 = 0, 1
 
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
             "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc",
-            "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv")
+            "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv", "ss_scan_fwd_zoh")
 
 # bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
 SS_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -76,6 +76,8 @@ def load_library():
         lib.ss_scan_fwd_conv.argtypes = [vp, vp, vp, ci, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp,
                                          i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
         lib.ss_scan_fwd_conv.restype = ci
+        lib.ss_scan_fwd_zoh.argtypes = lib.ss_scan_fwd.argtypes
+        lib.ss_scan_fwd_zoh.restype = ci
         lib.ss_scan_step.restype = ci
         _lib = lib
         return lib
@@ -169,6 +171,8 @@ def _fwd_call(name, initial_state, u, delta, A, B, C, D, z, delta_bias, softplus
             _stream_handle(stream, device))
     if name == "ss_scan_fwd":
         st = lib.ss_scan_fwd(*head, *tail)
+    elif name == "ss_scan_fwd_zoh":
+        st = lib.ss_scan_fwd_zoh(*head, *tail)
     elif name == "ss_scan_fwd_conv":
         cw, cb = initial_state
         _check_dev("conv_weight", cw, device, (torch.float32,))
@@ -209,6 +213,14 @@ def ss_scan_fwd_from_state(initial_state, u, delta, A, B, C, D=None, z=None, del
     return _fwd_call("ss_scan_fwd_from_state", initial_state, u, delta, A, B, C, D, z,
                      delta_bias, softplus, y_out, last_state_out, return_last_state, workspace,
                      stream)
+
+
+def ss_scan_fwd_zoh(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                    y_out=None, last_state_out=None, return_last_state=True, workspace=None,
+                    stream=None):
+    """ss_scan_fwd with the exact zero-order-hold B_bar = (exp(Delta A) - 1) / A * B."""
+    return _fwd_call("ss_scan_fwd_zoh", None, u, delta, A, B, C, D, z, delta_bias, softplus, y_out,
+                     last_state_out, return_last_state, workspace, stream)
 
 
 def ss_scan_fwd_conv(x, conv_weight, delta, A, B, C, D=None, z=None, delta_bias=None,

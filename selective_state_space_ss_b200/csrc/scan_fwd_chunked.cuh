@@ -74,8 +74,9 @@ constexpr int kConvTaps = 4;  // widest fused convolution
 // share one set of channels, each scanning T/WT consecutive steps of the
 // chunk, joined with the pages' associative operator).  CONV: the u input is
 // the pre-convolution x, staged with HALO earlier steps per row, and phase 1
-// forms u = SiLU(conv(x) + bias).
-template <typename Tin, int N_, int K_, int NWARPS_, int T_, int WT_ = 1, bool CONV_ = false>
+// forms u = SiLU(conv(x) + bias).  ZOH: exact zero-order-hold B_bar.
+template <typename Tin, int N_, int K_, int NWARPS_, int T_, int WT_ = 1, bool CONV_ = false,
+          bool ZOH_ = false>
 struct ChunkedCfg {
   using Elem = Tin;
   static constexpr int N = N_;            // states per channel
@@ -92,6 +93,7 @@ struct ChunkedCfg {
   static constexpr int ES = (int)sizeof(Tin);
   static constexpr int QPR = T / 4;                  // 4-step quads per row
   static constexpr bool CONV = CONV_;
+  static constexpr bool ZOH = ZOH_;
   // x steps staged before the chunk: >= kConvTaps - 1, and a whole number of
   // 16-byte units so that the shifted TMA box stays aligned
   static constexpr int HALO = CONV ? 8 : 0;
@@ -127,7 +129,10 @@ struct ChunkedCfg {
   // CONV: u = SiLU(conv) per (quad, channel), for phase 3's D u
   static constexpr int SU_BYTES = CONV ? DW_BYTES : 0;
   static constexpr int OFF_SU = OFF_AGG + 2 * AGG_FLOATS * 4;
-  static constexpr int SMEM_USED = OFF_SU + SU_BYTES;
+  // ZOH: 1 / Delta per (quad, channel)
+  static constexpr int DWI_BYTES = ZOH ? DW_BYTES : 0;
+  static constexpr int OFF_DWI = OFF_SU + SU_BYTES;
+  static constexpr int SMEM_USED = OFF_DWI + DWI_BYTES;
   static constexpr int SMEM_BYTES = SMEM_USED + 128;  // slack to align the base to 128 bytes
   // CTAs per SM the register budget must allow (shared memory permitting)
   // (at most 512 threads' worth: a 128-register budget per thread)
@@ -234,7 +239,8 @@ struct ConvRegs {  // per-item convolution taps, right-aligned: tap kConvTaps-1 
 
 template <class CF, bool kFull>
 __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem* raw,
-                                       float4* dwD, float4* dwW, float4* su, unsigned char* bc,
+                                       float4* dwD, float4* dwW, float4* dwI, float4* su,
+                                       unsigned char* bc,
                                        const float (&bias_it)[CF::ITEMS_PER_THREAD],
                                        const ConvRegs<CF>& cv, int64_t d0, int64_t t0) {
   using E = typename CF::Elem;
@@ -288,6 +294,9 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     const float w[4] = {w01.x, w01.y, w23.x, w23.y};
     dwD[q * CF::DW_STRIDE + c] = make_float4(delt[0], delt[1], delt[2], delt[3]);
     dwW[q * CF::DW_STRIDE + c] = make_float4(w[0], w[1], w[2], w[3]);
+    if constexpr (CF::ZOH)  // 1/0 = inf on padding steps: the series branch of phi takes them
+      dwI[q * CF::DW_STRIDE + c] = make_float4(rcp_approx(delt[0]), rcp_approx(delt[1]),
+                                               rcp_approx(delt[2]), rcp_approx(delt[3]));
   }
   // B and C rows [n][t] -> [t][n/2 pairs][B_2p, B_2p+1, C_2p, C_2p+1]
   const E* rawB = raw + CF::OFF_B_T / CF::ES;
@@ -361,6 +370,53 @@ __device__ __forceinline__ void bc_pairs(const unsigned char* p, float2 (&b)[NP]
   }
 }
 
+// Exact zero-order hold: B_bar u = phi(x) Delta u B with x = Delta A (natural
+// units) and phi(x) = (e^x - 1) / x = sum_k x^k / (k+1)!.  e = 2^(x log2 e) is
+// the decay the recurrence already has.  Near x = 0, e - 1 cancels, so phi
+// there comes from its Taylor series (in x2 = x log2 e, the argument of the
+// ex2; the degree-5 truncation error is below 1e-8 for |x2| < kZohSeriesMax);
+// elsewhere phi = (e - 1) (1/A) (1/Delta), whose rounding error is then below
+// 2e-6 relative.  A select (not a blend) keeps A = 0 (1/A stored as 0) and
+// padding steps (Delta = 0, 1/Delta = inf) on the series branch.
+constexpr float kZohSeriesMax = 0.25f;
+struct ZohSeries {  // phi(x2 ln 2) = sum_k c[k] x2^k, c[k] = ln2^k / (k+1)!
+  static constexpr double ln2 = 0.69314718055994530942;
+  __host__ __device__ static constexpr float c(int k) {
+    double v = 1.0, f = 1.0;
+    for (int i = 1; i <= k; ++i) {
+      v *= ln2;
+      f *= (double)(i + 1);
+    }
+    return (float)(v / f);
+  }
+};
+
+__device__ __forceinline__ float zoh_phi(float x2, float e, float inv_a, float inv_dl) {
+  constexpr float c0 = ZohSeries::c(0), c1 = ZohSeries::c(1), c2 = ZohSeries::c(2),
+                  c3 = ZohSeries::c(3), c4 = ZohSeries::c(4), c5 = ZohSeries::c(5);
+  float p = fmaf(c5, x2, c4);
+  p = fmaf(p, x2, c3);
+  p = fmaf(p, x2, c2);
+  p = fmaf(p, x2, c1);
+  p = fmaf(p, x2, c0);
+  const float big = (e - 1.f) * inv_a * inv_dl;
+  return fabsf(x2) < kZohSeriesMax ? p : big;
+}
+
+// The same on a pair of states (packed series and product, scalar selects).
+__device__ __forceinline__ float2 zoh_phi2(float2 x2, float2 e, float2 inv_a, float2 inv_dl) {
+  constexpr float c0 = ZohSeries::c(0), c1 = ZohSeries::c(1), c2 = ZohSeries::c(2),
+                  c3 = ZohSeries::c(3), c4 = ZohSeries::c(4), c5 = ZohSeries::c(5);
+  float2 p = __ffma2_rn(make_float2(c5, c5), x2, make_float2(c4, c4));
+  p = __ffma2_rn(p, x2, make_float2(c3, c3));
+  p = __ffma2_rn(p, x2, make_float2(c2, c2));
+  p = __ffma2_rn(p, x2, make_float2(c1, c1));
+  p = __ffma2_rn(p, x2, make_float2(c0, c0));
+  const float2 big = __fmul2_rn(__fmul2_rn(__fadd2_rn(e, make_float2(-1.f, -1.f)), inv_a), inv_dl);
+  return make_float2(fabsf(x2.x) < kZohSeriesMax ? p.x : big.x,
+                     fabsf(x2.y) < kZohSeriesMax ? p.y : big.y);
+}
+
 // The recurrence for this lane's G states over the chunk, two states per
 // packed fp32x2 operation.  Each lane writes its partial readout
 // sum_{n in lane} C_t[n] h_t[n] for four timesteps at a time (one 16-byte
@@ -368,10 +424,10 @@ __device__ __forceinline__ void bc_pairs(const unsigned char* p, float2 (&b)[NP]
 // no cross-lane dependency, so the ex2 of later steps can issue while
 // earlier steps' FMA chains drain.
 template <class CF>
-__device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
+__device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW, const float4* dwI,
                                        const unsigned char* bc, float* sy,
                                        float2 (&h)[CF::G / 2], const float2 (&a2)[CF::G / 2],
-                                       int c, int j) {
+                                       const float2 (&ia)[CF::G / 2], int c, int j) {
   constexpr int G2 = CF::G / 2;  // state pairs per lane
   const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
   float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE;
@@ -381,34 +437,12 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
     const float4 W4 = dwW[q * CF::DW_STRIDE + c];
     const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
     const float ws[4] = {W4.x, W4.y, W4.z, W4.w};
+    float idl[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (CF::ZOH) {
+      const float4 I4 = dwI[q * CF::DW_STRIDE + c];
+      idl[0] = I4.x; idl[1] = I4.y; idl[2] = I4.z; idl[3] = I4.w;
+    }
     float s[4];
-#if defined(SS_PHASE2_EXP_FIRST)
-    // all ex2 of the quad first, then the four dependent update chains
-    float2 ee[4][G2], wb[4][G2], cc[4][G2];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 dl2 = make_float2(dls[k], dls[k]);
-      const float2 w2 = make_float2(ws[k], ws[k]);
-      float2 bb[G2];
-      bc_pairs<CF, G2>(bcj + (4 * q + k) * CF::BC_ROW, bb, cc[k]);
-#pragma unroll
-      for (int g = 0; g < G2; ++g) {
-        const float2 x = __fmul2_rn(dl2, a2[g]);
-        ee[k][g] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        wb[k][g] = __fmul2_rn(w2, bb[g]);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int g = 0; g < G2; ++g) {
-        h[g] = __ffma2_rn(ee[k][g], h[g], wb[k][g]);
-        acc = __ffma2_rn(cc[k][g], h[g], acc);
-      }
-      s[k] = acc.x + acc.y;
-    }
-#else
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float2 dl2 = make_float2(dls[k], dls[k]);
@@ -420,12 +454,16 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
       for (int g = 0; g < G2; ++g) {
         const float2 x = __fmul2_rn(dl2, a2[g]);
         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        h[g] = __ffma2_rn(e, h[g], __fmul2_rn(w2, bb[g]));
+        float2 wb;
+        if constexpr (CF::ZOH)
+          wb = __fmul2_rn(__fmul2_rn(zoh_phi2(x, e, ia[g], make_float2(idl[k], idl[k])), w2), bb[g]);
+        else
+          wb = __fmul2_rn(w2, bb[g]);
+        h[g] = __ffma2_rn(e, h[g], wb);
         acc = __ffma2_rn(cc[g], h[g], acc);
       }
       s[k] = acc.x + acc.y;
     }
-#endif
     *reinterpret_cast<float4*>(syr + 4 * q) = make_float4(s[0], s[1], s[2], s[3]);
   }
 }
@@ -442,9 +480,11 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW,
 // h.  No ex2 is evaluated twice.
 template <class CF>
 __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dwW,
-                                             const unsigned char* bc, float* sy, float* aggP,
-                                             float* aggH, float2 (&h)[CF::G / 2],
-                                             const float2 (&a2)[CF::G / 2], int c, int j, int wt,
+                                             const float4* dwI, const unsigned char* bc,
+                                             float* sy, float* aggP, float* aggH,
+                                             float2 (&h)[CF::G / 2],
+                                             const float2 (&a2)[CF::G / 2],
+                                             const float2 (&ia)[CF::G / 2], int c, int j, int wt,
                                              int lane_g) {
   constexpr int G2 = CF::G / 2;
   const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
@@ -463,6 +503,11 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
     const float4 W4 = dwW[qq * CF::DW_STRIDE + c];
     const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
     const float ws[4] = {W4.x, W4.y, W4.z, W4.w};
+    float idl[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (CF::ZOH) {
+      const float4 I4 = dwI[qq * CF::DW_STRIDE + c];
+      idl[0] = I4.x; idl[1] = I4.y; idl[2] = I4.z; idl[3] = I4.w;
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int t = 4 * q + k;
@@ -476,7 +521,12 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
       for (int g = 0; g < G2; ++g) {
         const float2 x = __fmul2_rn(dl2, a2[g]);
         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        hl[g] = __ffma2_rn(e, hl[g], __fmul2_rn(w2, bb[g]));
+        float2 wb;
+        if constexpr (CF::ZOH)
+          wb = __fmul2_rn(__fmul2_rn(zoh_phi2(x, e, ia[g], make_float2(idl[k], idl[k])), w2), bb[g]);
+        else
+          wb = __fmul2_rn(w2, bb[g]);
+        hl[g] = __ffma2_rn(e, hl[g], wb);
         P[g] = __fmul2_rn(e, P[g]);
         acc = __ffma2_rn(cc[g], hl[g], acc);
         Q[t][g] = __fmul2_rn(cc[g], P[g]);
@@ -673,6 +723,19 @@ __device__ __forceinline__ void publish_carry(const Sched& s, int w) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(s.epoch) : "memory");
 }
 
+// A lane's decay constants for states n, n+1 of channel d: A log2 e (the ex2
+// argument per unit Delta) and, for the exact zero-order hold, 1/A (0 where
+// A = 0, which the series branch covers).
+template <class CF>
+__device__ __forceinline__ void load_decay(const FwdArgs& a, int64_t d, int n, bool chan_ok,
+                                           float2& a2, float2& ia) {
+  const float A0 = chan_ok ? __ldg(a.A + d * CF::N + n) : 0.f;
+  const float A1 = chan_ok ? __ldg(a.A + d * CF::N + n + 1) : 0.f;
+  a2 = make_float2(A0 * 1.4426950408889634f, A1 * 1.4426950408889634f);
+  ia = CF::ZOH ? make_float2(A0 != 0.f ? 1.f / A0 : 0.f, A1 != 0.f ? 1.f / A1 : 0.f)
+               : make_float2(0.f, 0.f);
+}
+
 // This thread's convolution taps for its items of channel tile d0, placed
 // right-aligned in kConvTaps slots (zeros before a shorter filter).
 template <class CF>
@@ -730,9 +793,11 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   const int j = lane % CF::K;                    // this lane's state group
   const int lane_g = wc * 32 + lane;             // lane within its channel set
   const bool writer = wt == 0;  // time-split warps hold the same carry: one writes it
-  auto run_phase2 = [&](float2 (&hh)[CF::G / 2], const float2 (&aa)[CF::G / 2]) {
-    if constexpr (CF::WT == 1) phase2<CF>(dwD, dwW, bc, sy, hh, aa, c, j);
-    else phase2_split<CF>(dwD, dwW, bc, sy, aggP, aggH, hh, aa, c, j, wt, lane_g);
+  float4* dwI = reinterpret_cast<float4*>(smem + CF::OFF_DWI);  // ZOH only
+  auto run_phase2 = [&](float2 (&hh)[CF::G / 2], const float2 (&aa)[CF::G / 2],
+                        const float2 (&ii)[CF::G / 2]) {
+    if constexpr (CF::WT == 1) phase2<CF>(dwD, dwW, dwI, bc, sy, hh, aa, ii, c, j);
+    else phase2_split<CF>(dwD, dwW, dwI, bc, sy, aggP, aggH, hh, aa, ii, c, j, wt, lane_g);
   };
 
   if (tma && tid == 0) {
@@ -759,16 +824,14 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
       D_it[it] = (a.D && di < a.dim) ? __ldg(a.D + di) : 0.f;
     }
     load_conv_regs<CF>(a, d0, cv);
-    float2 h[CF::G / 2], a2[CF::G / 2];
+    float2 h[CF::G / 2], a2[CF::G / 2], ia[CF::G / 2];
 #pragma unroll
     for (int g = 0; g < CF::G / 2; ++g) {
       const int n = j * CF::G + 2 * g;
       // plain loads: h0 may be the last_state buffer this kernel writes
       const float* h0 = a.h0 + (b * a.dim + d) * CF::N + n;
       h[g] = (a.h0 && chan_ok) ? make_float2(h0[0], h0[1]) : make_float2(0.f, 0.f);
-      a2[g] = chan_ok ? make_float2(__ldg(a.A + d * CF::N + n) * 1.4426950408889634f,
-                                    __ldg(a.A + d * CF::N + n + 1) * 1.4426950408889634f)
-                      : make_float2(0.f, 0.f);
+      load_decay<CF>(a, d, n, chan_ok, a2[g], ia[g]);
     }
     bool ok = true;
     auto full_chunk = [&](int64_t k) { return full_tile && (k + 1) * CF::T <= L; };
@@ -778,8 +841,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     };
     auto run_phase1 = [&](int64_t k) {
       const E* rp = reinterpret_cast<const E*>(raw(k));
-      if (full_chunk(k)) phase1<CF, true>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0, k * CF::T);
-      else phase1<CF, false>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0, k * CF::T);
+      if (full_chunk(k)) phase1<CF, true>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0, k * CF::T);
+      else phase1<CF, false>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0, k * CF::T);
     };
     auto drain = [&](int64_t first, int64_t last) {
       if (tma)
@@ -798,7 +861,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     run_phase1(0);
     __syncthreads();
     for (int64_t k = 0; k < nseq; ++k) {
-      run_phase2(h, a2);
+      run_phase2(h, a2, ia);
       if (k + 1 < nseq) stage_in(k + 1);
       if (!__syncthreads_and(ok)) {
         drain(k + 1, k + 1);
@@ -831,7 +894,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   prep = cur;
   fetch = cur;
 
-  float2 h[CF::G / 2], a2[CF::G / 2];
+  float2 h[CF::G / 2], a2[CF::G / 2], ia[CF::G / 2];
   float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
   ConvRegs<CF> cv;
   int32_t bias_g = -1, D_g = -1;  // group whose bias (and taps) / D are cached
@@ -867,8 +930,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     }
     const E* rp = reinterpret_cast<const E*>(raw(jj));
     const int64_t t0 = (int64_t)prep.c * CF::T;
-    if (full_chunk(prep)) phase1<CF, true>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0_of(prep), t0);
-    else phase1<CF, false>(a, rp, dwD, dwW, su, bc, bias_it, cv, d0_of(prep), t0);
+    if (full_chunk(prep)) phase1<CF, true>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0_of(prep), t0);
+    else phase1<CF, false>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0_of(prep), t0);
   };
   // On a timed-out wait: wait (bounded) for every copy this CTA still has in
   // flight, so that none lands in shared memory after the CTA has left.
@@ -910,9 +973,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
 #pragma unroll
       for (int g = 0; g < CF::G / 2; ++g) {
         const int n = j * CF::G + 2 * g;
-        a2[g] = chan_ok ? make_float2(__ldg(a.A + d * CF::N + n) * 1.4426950408889634f,
-                                      __ldg(a.A + d * CF::N + n + 1) * 1.4426950408889634f)
-                        : make_float2(0.f, 0.f);
+        load_decay<CF>(a, d, n, chan_ok, a2[g], ia[g]);
         if (cin)
           h[g] = make_float2(__ldcg(cin + c * CF::N + n), __ldcg(cin + c * CF::N + n + 1));
         else if (a.h0 && chan_ok) {  // a piece that starts the group (chunk 0)
@@ -924,7 +985,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
       }
       ok = ok && have;
     }
-    run_phase2(h, a2);
+    run_phase2(h, a2, ia);
     const bool cout_here = cur.carry_out();
     if (cout_here && writer) {
       float* dst = sched.carries + (int64_t)w * CF::CH * CF::N + c * CF::N + j * CF::G;

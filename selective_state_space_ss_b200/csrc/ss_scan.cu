@@ -191,8 +191,8 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
 #define SS_N16_T 32
 #endif
 
-template <typename E, bool CV = false>
-using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, 1, CV>;
+template <typename E, bool CV = false, bool Z = false>
+using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, 1, CV, Z>;
 #ifndef SS_N32_K
 #define SS_N32_K 4
 #endif
@@ -202,8 +202,8 @@ using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, 1, CV>;
 #ifndef SS_N32_T
 #define SS_N32_T 32
 #endif
-template <typename E, bool CV = false>
-using Cfg32 = ChunkedCfg<E, 32, SS_N32_K, SS_N32_W, SS_N32_T, 1, CV>;
+template <typename E, bool CV = false, bool Z = false>
+using Cfg32 = ChunkedCfg<E, 32, SS_N32_K, SS_N32_W, SS_N32_T, 1, CV, Z>;
 #ifndef SS_N64_K
 #define SS_N64_K 4
 #endif
@@ -222,10 +222,10 @@ using Cfg32 = ChunkedCfg<E, 32, SS_N32_K, SS_N32_W, SS_N32_T, 1, CV>;
 #ifndef SS_N128_T
 #define SS_N128_T 32
 #endif
-template <typename E, bool CV = false>
-using Cfg64 = ChunkedCfg<E, 64, SS_N64_K, SS_N64_W, SS_N64_T, 1, CV>;
-template <typename E, bool CV = false>
-using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T, 1, CV>;
+template <typename E, bool CV = false, bool Z = false>
+using Cfg64 = ChunkedCfg<E, 64, SS_N64_K, SS_N64_W, SS_N64_T, 1, CV, Z>;
+template <typename E, bool CV = false, bool Z = false>
+using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T, 1, CV, Z>;
 
 // Time-split shapes for problems with too few channels to fill the GPU: one
 // warp's worth of channels (8) per CTA, 8 warps splitting each chunk in time.
@@ -238,10 +238,10 @@ using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T, 1, CV>;
 #ifndef SS_SPLIT16_WT
 #define SS_SPLIT16_WT 8
 #endif
-template <typename E, bool CV = false>
-using Split16 = ChunkedCfg<E, 16, 4, SS_SPLIT16_W, SS_SPLIT16_T, SS_SPLIT16_WT, CV>;
-template <typename E, bool CV = false>
-using Split32 = ChunkedCfg<E, 32, 4, 8, 32, 8, CV>;
+template <typename E, bool CV = false, bool Z = false>
+using Split16 = ChunkedCfg<E, 16, 4, SS_SPLIT16_W, SS_SPLIT16_T, SS_SPLIT16_WT, CV, Z>;
+template <typename E, bool CV = false, bool Z = false>
+using Split32 = ChunkedCfg<E, 32, 4, 8, 32, 8, CV, Z>;
 
 // The time split costs ~1.5 extra instructions per (step, state); take it only
 // when the channel-parallel shape would leave SMs idle.
@@ -254,38 +254,38 @@ bool too_few_groups(int64_t batch, int64_t dim) {
   return groups < device_sms();
 }
 
-template <typename E, bool CV>
+template <typename E, bool CV, bool Z>
 ss_status dispatch_dtype(const FwdArgs& a, int N, void* ws, size_t wsb, cudaStream_t stream) {
   switch (N) {
     case 16:
-      if (too_few_groups<Cfg16<E, CV>>(a.batch, a.dim))
-        return launch_chunked<Split16<E, CV>>(a, ws, wsb, stream);
-      return launch_chunked<Cfg16<E, CV>>(a, ws, wsb, stream);
+      if (too_few_groups<Cfg16<E, CV, Z>>(a.batch, a.dim))
+        return launch_chunked<Split16<E, CV, Z>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg16<E, CV, Z>>(a, ws, wsb, stream);
     case 32:
-      if (too_few_groups<Cfg32<E, CV>>(a.batch, a.dim))
-        return launch_chunked<Split32<E, CV>>(a, ws, wsb, stream);
-      return launch_chunked<Cfg32<E, CV>>(a, ws, wsb, stream);
-    case 64: return launch_chunked<Cfg64<E, CV>>(a, ws, wsb, stream);
-    case 128: return launch_chunked<Cfg128<E, CV>>(a, ws, wsb, stream);
+      if (too_few_groups<Cfg32<E, CV, Z>>(a.batch, a.dim))
+        return launch_chunked<Split32<E, CV, Z>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg32<E, CV, Z>>(a, ws, wsb, stream);
+    case 64: return launch_chunked<Cfg64<E, CV, Z>>(a, ws, wsb, stream);
+    case 128: return launch_chunked<Cfg128<E, CV, Z>>(a, ws, wsb, stream);
     default: return SS_ERR_UNSUPPORTED;
   }
 }
 
-template <typename E, bool CV>
+template <typename E, bool CV, bool Z>
 bool plan_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N, size_t* bytes) {
   Plan p;
   bool ok = false;
   switch (N) {
     case 16:
-      ok = too_few_groups<Cfg16<E, CV>>(batch, dim) ? make_plan<Split16<E, CV>>(batch, dim, seqlen, &p)
-                                                    : make_plan<Cfg16<E, CV>>(batch, dim, seqlen, &p);
+      ok = too_few_groups<Cfg16<E, CV, Z>>(batch, dim) ? make_plan<Split16<E, CV, Z>>(batch, dim, seqlen, &p)
+                                                    : make_plan<Cfg16<E, CV, Z>>(batch, dim, seqlen, &p);
       break;
     case 32:
-      ok = too_few_groups<Cfg32<E, CV>>(batch, dim) ? make_plan<Split32<E, CV>>(batch, dim, seqlen, &p)
-                                                    : make_plan<Cfg32<E, CV>>(batch, dim, seqlen, &p);
+      ok = too_few_groups<Cfg32<E, CV, Z>>(batch, dim) ? make_plan<Split32<E, CV, Z>>(batch, dim, seqlen, &p)
+                                                    : make_plan<Cfg32<E, CV, Z>>(batch, dim, seqlen, &p);
       break;
-    case 64: ok = make_plan<Cfg64<E, CV>>(batch, dim, seqlen, &p); break;
-    case 128: ok = make_plan<Cfg128<E, CV>>(batch, dim, seqlen, &p); break;
+    case 64: ok = make_plan<Cfg64<E, CV, Z>>(batch, dim, seqlen, &p); break;
+    case 128: ok = make_plan<Cfg128<E, CV, Z>>(batch, dim, seqlen, &p); break;
   }
   *bytes = p.ws_bytes;
   return ok;
@@ -348,7 +348,7 @@ ss_status scan_fwd_impl(const void* u, const void* delta, const float* A, const 
                         int64_t batch, int64_t dim, int64_t seqlen, int dstate,
                         ss_dtype in_dtype, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream, const float* conv_w = nullptr,
-                        const float* conv_b = nullptr, int conv_width = 0) {
+                        const float* conv_b = nullptr, int conv_width = 0, bool zoh = false) {
   if (!u || !delta || !A || !B || !C || !y_out) return SS_ERR_INVALID_ARG;
   if (batch < 1 || dim < 1 || seqlen < 1) return SS_ERR_INVALID_ARG;
   if (in_dtype != SS_F32 && in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED;
@@ -379,12 +379,17 @@ ss_status scan_fwd_impl(const void* u, const void* delta, const float* A, const 
   if (!aligned(y_out, 16)) vec = false;
   a.vec = vec ? 1 : 0;
 
+  const bool f32 = in_dtype == SS_F32;
   if (conv_w) {
-    if (in_dtype == SS_F32) return dispatch_dtype<float, true>(a, dstate, workspace, workspace_bytes, stream);
-    return dispatch_dtype<__nv_bfloat16, true>(a, dstate, workspace, workspace_bytes, stream);
+    if (f32) return dispatch_dtype<float, true, false>(a, dstate, workspace, workspace_bytes, stream);
+    return dispatch_dtype<__nv_bfloat16, true, false>(a, dstate, workspace, workspace_bytes, stream);
   }
-  if (in_dtype == SS_F32) return dispatch_dtype<float, false>(a, dstate, workspace, workspace_bytes, stream);
-  return dispatch_dtype<__nv_bfloat16, false>(a, dstate, workspace, workspace_bytes, stream);
+  if (zoh) {
+    if (f32) return dispatch_dtype<float, false, true>(a, dstate, workspace, workspace_bytes, stream);
+    return dispatch_dtype<__nv_bfloat16, false, true>(a, dstate, workspace, workspace_bytes, stream);
+  }
+  if (f32) return dispatch_dtype<float, false, false>(a, dstate, workspace, workspace_bytes, stream);
+  return dispatch_dtype<__nv_bfloat16, false, false>(a, dstate, workspace, workspace_bytes, stream);
 }
 
 }  // namespace
@@ -425,6 +430,16 @@ ss_status ss_scan_fwd_from_state(const void* u, const void* delta, const float* 
   return scan_fwd_impl(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y_out,
                        last_state_out, batch, dim, seqlen, dstate, in_dtype, workspace,
                        workspace_bytes, stream);
+}
+
+ss_status ss_scan_fwd_zoh(const void* u, const void* delta, const float* A, const void* B,
+                          const void* C, const float* D, const void* z, const float* delta_bias,
+                          int softplus_flag, float* y_out, float* last_state_out, int64_t batch,
+                          int64_t dim, int64_t seqlen, int dstate, ss_dtype in_dtype,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return scan_fwd_impl(u, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, y_out,
+                       last_state_out, batch, dim, seqlen, dstate, in_dtype, workspace,
+                       workspace_bytes, stream, nullptr, nullptr, 0, true);
 }
 
 ss_status ss_scan_fwd_conv(const void* x, const float* conv_weight, const float* conv_bias,
@@ -499,12 +514,15 @@ size_t ss_scan_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int d
   if (batch < 1 || dim < 1 || seqlen < 1 || !supported_dstate(dstate)) return (size_t)-1;
   if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
     return (size_t)-1;
-  // enough for either input dtype, with or without the fused convolution
-  size_t need[4] = {0, 0, 0, 0};
-  if (!plan_bytes<float, false>(batch, dim, seqlen, dstate, &need[0]) ||
-      !plan_bytes<__nv_bfloat16, false>(batch, dim, seqlen, dstate, &need[1]) ||
-      !plan_bytes<float, true>(batch, dim, seqlen, dstate, &need[2]) ||
-      !plan_bytes<__nv_bfloat16, true>(batch, dim, seqlen, dstate, &need[3]))
+  // enough for either input dtype and every kernel variant (plain, fused
+  // convolution, exact zero-order hold)
+  size_t need[6] = {0, 0, 0, 0, 0, 0};
+  if (!plan_bytes<float, false, false>(batch, dim, seqlen, dstate, &need[0]) ||
+      !plan_bytes<__nv_bfloat16, false, false>(batch, dim, seqlen, dstate, &need[1]) ||
+      !plan_bytes<float, true, false>(batch, dim, seqlen, dstate, &need[2]) ||
+      !plan_bytes<__nv_bfloat16, true, false>(batch, dim, seqlen, dstate, &need[3]) ||
+      !plan_bytes<float, false, true>(batch, dim, seqlen, dstate, &need[4]) ||
+      !plan_bytes<__nv_bfloat16, false, true>(batch, dim, seqlen, dstate, &need[5]))
     return (size_t)-1;
   size_t m = 0;
   for (size_t v : need) m = v > m ? v : m;

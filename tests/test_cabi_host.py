@@ -149,6 +149,18 @@ def test_conv_rejections(lib, over, status):
     assert _call_conv(lib, **over) == status
 
 
+@pytest.mark.parametrize("over", [dict(u=None), dict(N=8), dict(L=0), dict(y=0x60002)])
+def test_zoh_rejections(lib, over):
+    a = dict(u=0x10000, delta=0x20000, A=0x30000, B=0x40000, C=0x50000, D=None, z=None,
+             bias=None, sp=1, y=0x60000, h=None, batch=1, dim=1, L=8, N=16, dt=N.SS_F32,
+             ws=None, wsb=0)
+    a.update(over)
+    st = lib.ss_scan_fwd_zoh(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
+                             a["sp"], a["y"], a["h"], a["batch"], a["dim"], a["L"], a["N"], a["dt"],
+                             a["ws"], a["wsb"], None)
+    assert st in (N.SS_ERR_INVALID_ARG, N.SS_ERR_UNSUPPORTED)
+
+
 def test_workspace_query_rejects_bad_sizes(lib):
     # (valid sizes need the device's SM count, so they are covered by the GPU tests)
     with pytest.raises(N.SSError):
