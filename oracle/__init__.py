@@ -50,6 +50,10 @@ def _load():
                 i64, i64, i64, ctypes.c_int, vp, i64, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int]
             lib.oracle_scan_fwd.restype = ctypes.c_int
+            lib.oracle_scan_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+                                            ctypes.c_int, i64, i64, i64, ctypes.c_int, vp, vp,
+                                            vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int]
+            lib.oracle_scan_bwd.restype = ctypes.c_int
             lib.oracle_softplus.argtypes = [ctypes.c_double]
             lib.oracle_softplus.restype = ctypes.c_double
             lib.oracle_silu.argtypes = [ctypes.c_double]
@@ -163,6 +167,49 @@ def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
                     delta_bias=delta_bias, softplus=softplus, nthreads=nthreads,
                     h0=state)
     return y[..., 0], h
+
+
+def scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, dy=None,
+             dlast=None, nthreads=None):
+    """Reverse-mode gradients of the scan (simplified B_bar, zero initial state).
+
+    Inputs as scan_fwd; dy: [batch, dim, L] gradient of the loss with respect
+    to y; dlast: optional [batch, dim, N] gradient with respect to the final
+    state.  Returns a dict of float64 arrays: du, ddelta, dz (None without z),
+    dA [dim, N], dB, dC [batch, N, L], dD, ddelta_bias [dim].
+    """
+    u, dt = _stored(u, "u")
+    delta, _ = _stored(delta, "delta")
+    B, _ = _stored(B, "B")
+    C, _ = _stored(C, "C")
+    if z is not None:
+        z, _ = _stored(z, "z")
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    A = np.ascontiguousarray(A, dtype=np.float32)
+    D = None if D is None else np.ascontiguousarray(D, dtype=np.float32)
+    delta_bias = None if delta_bias is None else np.ascontiguousarray(delta_bias, dtype=np.float32)
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    if dy.shape != (batch, dim, L):
+        raise ValueError("dy must be [batch, dim, L]")
+    if dlast is not None:
+        dlast = np.ascontiguousarray(dlast, dtype=np.float64)
+        if dlast.shape != (batch, dim, N):
+            raise ValueError("dlast must be [batch, dim, N]")
+    out = {"du": np.empty((batch, dim, L)), "ddelta": np.empty((batch, dim, L)),
+           "dz": np.empty((batch, dim, L)) if z is not None else None,
+           "dA": np.empty((dim, N)), "dB": np.empty((batch, N, L)), "dC": np.empty((batch, N, L)),
+           "dD": np.empty(dim), "ddelta_bias": np.empty(dim)}
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().oracle_scan_bwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        int(bool(softplus)), dt, batch, dim, L, N, _ptr(dy), _ptr(dlast), _ptr(out["du"]),
+        _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]),
+        _ptr(out["dD"]), _ptr(out["ddelta_bias"]), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_scan_bwd rejected its arguments")
+    return out
 
 
 def softplus(x: float) -> float:

@@ -227,3 +227,181 @@ int oracle_scan_fwd(const void* u, const void* delta, const float* A,
 /* The scalar pieces, exported so that tests can pin them one by one. */
 double oracle_softplus(double x) { return softplus64(x); }
 double oracle_silu(double z) { return silu64(z); }
+
+
+/* ------------------------------------------------------------- backward --
+ *
+ * Reverse-mode derivative of the simplified-B_bar scan (h0 = 0, no
+ * convolution) for a loss whose gradient with respect to y is dy (and, if
+ * given, dlast with respect to the final state).  Per channel the forward
+ * states h_t are recomputed and kept, then the adjoint g_t = dL/dh_t runs
+ * backwards in time:
+ *
+ *   q_t  = C_t . h_t + D u_t,   y_t = q_t SiLU(z_t)
+ *   dq_t = dy_t SiLU(z_t),      dz_t = dy_t q_t SiLU'(z_t)
+ *   g_t[n] = dq_t C_t[n] + a_{t+1}[n] g_{t+1}[n]   (+ dlast[n] at t = L-1)
+ *   with a_t[n] = exp(Delta_t A[n]):
+ *     dDelta_t = sum_n g_t[n] (B_t[n] u_t + A[n] a_t[n] h_{t-1}[n])
+ *     du_t     = dq_t D + sum_n g_t[n] Delta_t B_t[n]
+ *     dA[n]   += g_t[n] Delta_t a_t[n] h_{t-1}[n]
+ *     dB_t[n] += g_t[n] Delta_t u_t          (summed over channels d)
+ *     dC_t[n] += dq_t h_t[n]                 (summed over channels d)
+ *     dD      += dq_t u_t
+ *     ddelta_t = dDelta_t softplus'(x_t) = dDelta_t sigmoid(x_t)  (flag on)
+ *     dbias   += ddelta_t
+ * SiLU'(z) = s (1 + z (1 - s)), s = sigmoid(z).  The pages describe this
+ * backward only as recomputation instead of stored states ("Mamba 深度解读报告",
+ * sec. 3.3; "Mamba 选择性机制", sec. 3.4); the derivative itself is the chain
+ * rule applied to the forward above.
+ */
+typedef struct {
+  const void *u, *delta, *B, *C, *z;
+  const float *A, *D, *delta_bias;
+  const double *dy, *dlast;
+  int softplus_flag, dtype;
+  int64_t batch, dim, seqlen;
+  int dstate;
+  double *du, *ddelta, *dz;         /* [batch, dim, L] */
+  double *dA, *dB, *dC, *dD, *dbias; /* shared sums, merged under mu */
+  int64_t next;
+  pthread_mutex_t mu;
+} bjob_t;
+
+static double sigmoid64(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+static void bwd_channel(bjob_t* J, int64_t flat, double* hs, double* g, double* dA,
+                        double* dB, double* dC, double* dD, double* dbias) {
+  const int64_t b = flat / J->dim, d = flat % J->dim, L = J->seqlen;
+  const int N = J->dstate;
+  const int64_t row = (b * J->dim + d) * L, bc = b * (int64_t)N * L;
+  const double bias = J->delta_bias ? (double)J->delta_bias[d] : 0.0;
+  const double Dd = J->D ? (double)J->D[d] : 0.0;
+  /* forward, keeping h_t for every t */
+  for (int64_t t = 0; t < L; ++t) {
+    const double x = widen(J->delta, J->dtype, row + t) + bias;
+    const double dt = J->softplus_flag ? softplus64(x) : x;
+    const double ut = widen(J->u, J->dtype, row + t);
+    for (int n = 0; n < N; ++n) {
+      const double prev = t ? hs[(t - 1) * N + n] : 0.0;
+      hs[t * N + n] = exp(dt * (double)J->A[d * N + n]) * prev +
+                      dt * widen(J->B, J->dtype, bc + (int64_t)n * L + t) * ut;
+    }
+  }
+  /* adjoint, backwards */
+  for (int n = 0; n < N; ++n) g[n] = J->dlast ? J->dlast[flat * N + n] : 0.0;
+  for (int64_t t = L - 1; t >= 0; --t) {
+    const double x = widen(J->delta, J->dtype, row + t) + bias;
+    const double dt = J->softplus_flag ? softplus64(x) : x;
+    const double ut = widen(J->u, J->dtype, row + t);
+    double q = Dd * ut;
+    for (int n = 0; n < N; ++n) q += widen(J->C, J->dtype, bc + (int64_t)n * L + t) * hs[t * N + n];
+    double dq = J->dy[row + t];
+    if (J->z) {
+      const double zt = widen(J->z, J->dtype, row + t), sg = sigmoid64(zt);
+      J->dz[row + t] = J->dy[row + t] * q * sg * (1.0 + zt * (1.0 - sg));
+      dq = J->dy[row + t] * zt * sg;
+    }
+    double ddt = 0.0, du = dq * Dd;
+    *dD += dq * ut;
+    for (int n = 0; n < N; ++n) {
+      const double an = (double)J->A[d * N + n];
+      const double a = exp(dt * an);
+      const double bt = widen(J->B, J->dtype, bc + (int64_t)n * L + t);
+      const double ct = widen(J->C, J->dtype, bc + (int64_t)n * L + t);
+      const double prev = t ? hs[(t - 1) * N + n] : 0.0;
+      const double gt = g[n] + dq * ct; /* g[n] holds a_{t+1} g_{t+1} (+ dlast) */
+      ddt += gt * (bt * ut + an * a * prev);
+      du += gt * dt * bt;
+      dA[d * N + n] += gt * dt * a * prev;
+      dB[bc + (int64_t)n * L + t] += gt * dt * ut;
+      dC[bc + (int64_t)n * L + t] += dq * hs[t * N + n];
+      g[n] = a * gt;
+    }
+    const double dx = J->softplus_flag ? ddt * sigmoid64(x) : ddt;
+    J->ddelta[row + t] = dx;
+    J->du[row + t] = du;
+    dbias[d] += dx;
+  }
+}
+
+static void* bwd_worker(void* arg) {
+  bjob_t* J = (bjob_t*)arg;
+  const int N = J->dstate;
+  const int64_t L = J->seqlen, D = J->dim;
+  const size_t nbc = (size_t)J->batch * N * L;
+  double* hs = (double*)malloc(sizeof(double) * (size_t)L * N);
+  double* g = (double*)malloc(sizeof(double) * N);
+  double* dA = (double*)calloc((size_t)D * N, sizeof(double));
+  double* dB = (double*)calloc(nbc, sizeof(double));
+  double* dC = (double*)calloc(nbc, sizeof(double));
+  double* dD = (double*)calloc((size_t)D, sizeof(double));
+  double* dbias = (double*)calloc((size_t)D, sizeof(double));
+  if (hs && g && dA && dB && dC && dD && dbias) {
+    for (;;) {
+      pthread_mutex_lock(&J->mu);
+      const int64_t flat = J->next++;
+      pthread_mutex_unlock(&J->mu);
+      if (flat >= J->batch * D) break;
+      double dDd = 0.0;
+      bwd_channel(J, flat, hs, g, dA, dB, dC, &dDd, dbias);
+      dD[flat % D] += dDd;
+    }
+    pthread_mutex_lock(&J->mu);
+    for (int64_t i = 0; i < D * N; ++i) J->dA[i] += dA[i];
+    for (size_t i = 0; i < nbc; ++i) {
+      J->dB[i] += dB[i];
+      J->dC[i] += dC[i];
+    }
+    for (int64_t i = 0; i < D; ++i) {
+      J->dD[i] += dD[i];
+      J->dbias[i] += dbias[i];
+    }
+    pthread_mutex_unlock(&J->mu);
+  }
+  free(hs); free(g); free(dA); free(dB); free(dC); free(dD); free(dbias);
+  return NULL;
+}
+
+/*
+ * oracle_scan_bwd: returns 0, or -1 on a bad argument or memory shortage.
+ * Inputs as oracle_scan_fwd (every channel); dy [batch, dim, L] and dlast
+ * [batch, dim, N] (nullable) in double.  Outputs (double, overwritten):
+ * du, ddelta, dz [batch, dim, L] (dz ignored without z); dA [dim, N];
+ * dB, dC [batch, N, L]; dD, dbias [dim].
+ */
+int oracle_scan_bwd(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* delta_bias,
+                    int softplus_flag, int dtype, int64_t batch, int64_t dim, int64_t seqlen,
+                    int dstate, const double* dy, const double* dlast, double* du,
+                    double* ddelta, double* dz, double* dA, double* dB, double* dC,
+                    double* dD, double* dbias, int nthreads) {
+  if (!u || !delta || !A || !B || !C || !dy || !du || !ddelta || !dA || !dB || !dC || !dD ||
+      !dbias || (z && !dz))
+    return -1;
+  if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0) return -1;
+  if (dtype != 0 && dtype != 1) return -1;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 512) nthreads = 512;
+  memset(dA, 0, sizeof(double) * (size_t)(dim * dstate));
+  memset(dB, 0, sizeof(double) * (size_t)(batch * dstate * seqlen));
+  memset(dC, 0, sizeof(double) * (size_t)(batch * dstate * seqlen));
+  memset(dD, 0, sizeof(double) * (size_t)dim);
+  memset(dbias, 0, sizeof(double) * (size_t)dim);
+  bjob_t J;
+  memset(&J, 0, sizeof J);
+  J.u = u; J.delta = delta; J.B = B; J.C = C; J.z = z;
+  J.A = A; J.D = D; J.delta_bias = delta_bias; J.dy = dy; J.dlast = dlast;
+  J.softplus_flag = softplus_flag; J.dtype = dtype;
+  J.batch = batch; J.dim = dim; J.seqlen = seqlen; J.dstate = dstate;
+  J.du = du; J.ddelta = ddelta; J.dz = dz;
+  J.dA = dA; J.dB = dB; J.dC = dC; J.dD = dD; J.dbias = dbias;
+  pthread_mutex_init(&J.mu, NULL);
+  pthread_t tids[512];
+  int started = 0;
+  for (int i = 1; i < nthreads; ++i)
+    if (pthread_create(&tids[started], NULL, bwd_worker, &J) == 0) ++started;
+  bwd_worker(&J);
+  for (int i = 0; i < started; ++i) pthread_join(tids[i], NULL);
+  pthread_mutex_destroy(&J.mu);
+  return 0;
+}

@@ -40,6 +40,14 @@ MUTANTS = [
     ("zoh without the division by A", "expm1(dt * an) / an * b_t", "expm1(dt * an) * b_t"),
     ("zoh with Delta twice", "expm1(dt * an) / an * b_t", "expm1(dt * an) / an * dt * b_t"),
     ("zoh sign of A", "expm1(dt * an) / an * b_t", "expm1(-dt * an) / an * b_t"),
+    ("bwd carry not decayed", "g[n] = a * gt;", "g[n] = gt;"),
+    ("bwd dDelta misses the decay term", "ddt += gt * (bt * ut + an * a * prev);", "ddt += gt * bt * ut;"),
+    ("bwd dz with the sigmoid only", "q * sg * (1.0 + zt * (1.0 - sg));", "q * sg;"),
+    ("bwd dC from the previous state", "dC[bc + (int64_t)n * L + t] += dq * hs[t * N + n];",
+     "dC[bc + (int64_t)n * L + t] += dq * prev;"),
+    ("bwd softplus derivative dropped", "ddt * sigmoid64(x) : ddt", "ddt : ddt"),
+    ("bwd dA without Delta", "gt * dt * a * prev", "gt * a * prev"),
+    ("bwd du misses the skip", "du = dq * Dd;", "du = 0.0;"),
 ]
 
 PIN_CALLS = [
@@ -58,6 +66,7 @@ PIN_CALLS = [
     pins.test_conv_prologue_impulse_taps,
     pins.test_zoh_matches_ode_integration,
     pins.test_zoh_small_delta_series,
+    lambda: pins.test_backward_matches_finite_differences(True, True, True),
 ]
 
 
@@ -77,7 +86,7 @@ def test_pins_catch_mutant(tmp_path, monkeypatch, name, old, new):
     path = _build_mutant(tmp_path, old, new)
     real = oracle._load()
     lib = ctypes.CDLL(path)
-    for fn in ("oracle_scan_fwd", "oracle_softplus", "oracle_silu"):
+    for fn in ("oracle_scan_fwd", "oracle_scan_bwd", "oracle_softplus", "oracle_silu"):
         f = getattr(lib, fn)
         f.argtypes = getattr(real, fn).argtypes
         f.restype = getattr(real, fn).restype

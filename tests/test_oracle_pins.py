@@ -613,6 +613,81 @@ def test_zoh_limit_a_zero_and_simplified_form():
     assert _rel(y3, y4) > 1e-3
 
 
+# ------------------------------------------------------------- backward ----
+# The oracle's reverse-mode gradients against central finite differences of
+# the forward oracle itself (fp64 throughout; a perturbed float32 input is
+# stepped by exactly representable amounts).
+
+def _loss(x, dy, dlast, softplus):
+    y, h = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                           x["delta_bias"], softplus=softplus, nthreads=1)
+    v = float(np.sum(y * dy))
+    if dlast is not None:
+        v += float(np.sum(h * dlast))
+    return v
+
+
+def _fd_check(x, dy, dlast, softplus, rng, per_tensor=12):
+    g = oracle.scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
+                        softplus=softplus, dy=dy, dlast=dlast, nthreads=1)
+    names = {"u": "du", "delta": "ddelta", "z": "dz", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+             "delta_bias": "ddelta_bias"}
+    for key, gname in names.items():
+        if x[key] is None:
+            continue
+        arr = x[key]
+        flat = arr.reshape(-1)
+        idx = rng.choice(flat.size, min(per_tensor, flat.size), replace=False)
+        scale = float(np.max(np.abs(g[gname]))) + 1e-30
+        for i in idx:
+            orig = flat[i]
+            step = np.float32(1e-3 * max(1.0, abs(float(orig))))
+            hi, lo = np.float32(orig + step), np.float32(orig - step)
+            flat[i] = hi
+            f_hi = _loss(x, dy, dlast, softplus)
+            flat[i] = lo
+            f_lo = _loss(x, dy, dlast, softplus)
+            flat[i] = orig
+            fd = (f_hi - f_lo) / (float(hi) - float(lo))
+            got = float(g[gname].reshape(-1)[i])
+            assert abs(fd - got) <= 2e-5 * scale, f"{gname}[{i}]: fd {fd} vs {got}"
+
+
+@pytest.mark.parametrize("softplus,with_z,with_dlast", [(True, True, False), (True, True, True),
+                                                        (False, False, False)])
+def test_backward_matches_finite_differences(softplus, with_z, with_dlast):
+    rng = np.random.default_rng(90 + 2 * softplus + with_z + 4 * with_dlast)
+    batch, dim, L, N = 2, 3, 9, 4
+    c = _rand_case(rng, batch, dim, L, N)
+    c["A"] = _f32(-rng.uniform(0.2, 2.0, size=(dim, N)))
+    x = dict(u=c["u"], B=c["B"], C=c["C"], A=c["A"], D=c["D"], z=c["z"] if with_z else None,
+             delta_bias=_f32(rng.uniform(-1.5, -0.5, size=dim)))
+    if softplus:
+        x["delta"] = _f32(rng.normal(scale=0.5, size=(batch, dim, L)))
+    else:  # Delta = delta + bias must stay positive
+        x["delta"] = _f32(rng.uniform(1.6, 2.0, size=(batch, dim, L)))
+    dy = rng.normal(size=(batch, dim, L))
+    dlast = rng.normal(size=(batch, dim, N)) if with_dlast else None
+    _fd_check(x, dy, dlast, softplus, rng)
+
+
+def test_backward_linear_in_dy():
+    """The gradients are linear in the upstream gradient: grad(2 dy1 - dy2) =
+    2 grad(dy1) - grad(dy2), and zero for dy = 0 (without dlast)."""
+    w = I.Workload("t", 2, 4, 11, 8, "bf16")
+    x = I.make_inputs(w, seed=21)
+    rng = np.random.default_rng(3)
+    dy1, dy2 = rng.normal(size=(2, 4, 11)), rng.normal(size=(2, 4, 11))
+    args = (x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"])
+    g1 = oracle.scan_bwd(*args, dy=dy1)
+    g2 = oracle.scan_bwd(*args, dy=dy2)
+    g3 = oracle.scan_bwd(*args, dy=2 * dy1 - dy2)
+    g0 = oracle.scan_bwd(*args, dy=np.zeros_like(dy1))
+    for k in g1:  # dz = dy q SiLU'(z) is linear in dy as well
+        assert _rel(g3[k], 2 * g1[k] - g2[k]) < 1e-12, k
+        assert np.all(g0[k] == 0.0), k
+
+
 # ------------------------------------------------------- host plumbing -----
 
 def test_channel_subset_matches_full():
