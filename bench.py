@@ -412,6 +412,76 @@ def run_step_arm(args, w: I.Workload):
     return line
 
 
+BWD_METRIC = "selective-scan backward (B·L·D) elements/s and % of SFU roofline"
+
+
+def bwd_bytes(w: I.Workload) -> int:
+    """Bytes a backward must move: the forward's inputs and dy once; du, ddelta,
+    dz, dB, dC, dA, dD and the bias gradient once (fp32)."""
+    es = 4 if w.dtype == "f32" else 2
+    el = w.elements
+    rd = (3 * el + 2 * w.batch * w.dstate * w.seqlen) * es + el * 4 + w.dim * (w.dstate + 2) * 4
+    wr = 3 * el * 4 + 2 * w.batch * w.dstate * w.seqlen * 4 + w.dim * (w.dstate + 2) * 4
+    return rd + wr
+
+
+def run_bwd_arm(args, w: I.Workload):
+    """One backward per step (states recomputed inside), inputs rotated."""
+    import torch
+
+    from selective_state_space_ss_b200 import load_library, ss_scan_bwd, ss_scan_bwd_workspace_bytes
+
+    _, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    load_library()
+    stream = torch.cuda.current_stream(dev)
+    nsets = max(1, -(-4 * L2_BYTES // bwd_bytes(w)))
+    host = [I.make_inputs(w, seed=rank_seed(rank, s)) for s in range(nsets)]
+
+    def to_dev(x):
+        return {k: (None if v is None else
+                    (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
+                     else torch.from_numpy(v)).to(dev)) for k, v in x.items()}
+
+    sets = [to_dev(x) for x in host]
+    dys = [torch.from_numpy(I.fill(rank_seed(rank, s), 12, (w.batch, w.dim, w.seqlen))).to(dev)
+           for s in range(nsets)]
+    ws = torch.empty(ss_scan_bwd_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        x = sets[i % nsets]
+        ss_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], dys[i % nsets], D=x["D"], z=x["z"],
+                    delta_bias=x["delta_bias"], softplus=w.softplus, workspace=ws, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    p = peaks()
+    sfu_rate = NUM_SMS * MUFU_EX2_PER_CLK_PER_SM * p["sm_max_mhz"] * 1e6
+    exps = 2 * w.exps()  # a recomputing backward evaluates exp(Delta A) forward and backward
+    achieved = exps / (ms * 1e-3) / 1e9
+    line = {"metric": BWD_METRIC, "value": w.elements / (ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": dict(config_of(w, 1), op="backward"),
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": sfu_rate / 1e9, "unit": "Gexp2/s",
+                         "frac": achieved * 1e9 / sfu_rate, "traffic": None,
+                         "exps_per_step": exps, "hbm_bytes_per_step": bwd_bytes(w),
+                         "hbm_frac": bwd_bytes(w) / (ms * 1e-3) / 1e9 / p["hbm_gbs"]},
+            "gpu_launches": args.steps, "clocks": clk.summary()}
+    return line
+
+
 def roofline(w: I.Workload, kernel_ms: float):
     p = peaks()
     t_hbm = w.algorithmic_bytes() / (p["hbm_gbs"] * 1e9)
@@ -505,7 +575,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--op", default="scan", choices=["scan", "step"])
+    ap.add_argument("--op", default="scan", choices=["scan", "step", "bwd"])
     ap.add_argument("--workload", default=None,
                     choices=sorted(I.WORKLOADS) + sorted(I.STEP_WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
@@ -526,6 +596,12 @@ def main():
         return
     if args.workload in I.STEP_WORKLOADS:
         ap.error("decode-step workloads run with --op step")
+    if args.op == "bwd":
+        if args.impl != "native" or args.gpus != 1:
+            ap.error("--op bwd runs the native arm on one GPU")
+        print(json.dumps(run_bwd_arm(args, I.WORKLOADS[args.workload or DEFAULT_WORKLOAD])),
+              flush=True)
+        return
     w = I.WORKLOADS[args.workload or DEFAULT_WORKLOAD]
 
     if args.impl == "reference":

@@ -194,6 +194,50 @@ ss_status ss_scan_step(const void* u, const void* delta, const float* A,
                        int dstate, ss_dtype in_dtype, cudaStream_t stream);
 
 /*
+ * ss_scan_bwd -- gradients of ss_scan_fwd (simplified B_bar, zero initial
+ * state) for an upstream gradient dy of y (and optionally dlast_state of the
+ * final state).  The forward's states are not stored anywhere: the backward
+ * recomputes them from the inputs ("Mamba 深度解读报告", sec. 3.3;
+ * "Mamba 选择性机制", sec. 3.4), keeping only the state at the start of every
+ * 16-step chunk in the caller's workspace.  With a_t = exp(Delta_t A),
+ * q_t = C_t . h_t + D u_t, y_t = q_t SiLU(z_t) and the adjoint
+ * g_t = dL/dh_t = dq_t C_t + a_{t+1} g_{t+1}:
+ *
+ *   dz       = dy q SiLU'(z),           dq = dy SiLU(z)   (dq = dy without z)
+ *   du       = dq D + sum_n g Delta B
+ *   ddelta   = (sum_n g (B u + A a h_{t-1})) * softplus'(delta + bias)
+ *              (times 1 without the softplus)
+ *   dA[d,n]  = sum_{b,t} g Delta a h_{t-1}
+ *   dB, dC   = sum_d g Delta u,  sum_d dq h_t         [batch, dstate, seqlen]
+ *   dD[d]    = sum_{b,t} dq u,   ddelta_bias[d] = sum_{b,t} ddelta
+ *
+ * Inputs exactly as ss_scan_fwd; dy [batch, dim, seqlen] float32 (required);
+ * dlast_state [batch, dim, dstate] float32 (nullable: 0).  Outputs, all
+ * float32 and overwritten: du, ddelta [batch, dim, seqlen] (required); dz
+ * (required when z is given, ignored otherwise); dA [dim, dstate], dB, dC
+ * [batch, dstate, seqlen] (required); dD (nullable; ignored without D),
+ * ddelta_bias [dim] (nullable).  dA, dB, dC, dD and ddelta_bias are summed
+ * with atomic adds after the call zeroes them on `stream` (so their low bits
+ * may vary from call to call).  workspace: at least
+ * ss_scan_bwd_workspace_bytes(...) bytes, 256-byte aligned, caller-owned.
+ * Any element alignment; errors as ss_scan_fwd.
+ */
+ss_status ss_scan_bwd(const void* u, const void* delta, const float* A,
+                      const void* B, const void* C, const float* D,
+                      const void* z, const float* delta_bias, int softplus_flag,
+                      const float* dy, const float* dlast_state, float* du,
+                      float* ddelta, float* dA, float* dB, float* dC, float* dD,
+                      float* dz, float* ddelta_bias, int64_t batch, int64_t dim,
+                      int64_t seqlen, int dstate, ss_dtype in_dtype,
+                      void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
+/* Bytes of workspace ss_scan_bwd needs: 16 bytes x batch x dim x dstate x
+ * ceil(seqlen / 16) (rounded up), or (size_t)-1 for sizes it would reject. */
+size_t ss_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen,
+                                   int dstate);
+
+/*
  * ss_scan_fwd_noalloc -- ss_scan_fwd for callers that cannot allocate device
  * memory at the point of the call: for example a plugin running inside a host
  * framework that owns every device allocation (a cudaMalloc of its own would

@@ -1,4 +1,4 @@
-"""B200-native S6 selective scan: the fused forward and the recurrent step.
+"""B200-native S6 selective scan: the fused forward, its backward and the recurrent step.
 
 The compute lives in libssscan.so (hand-written sm_100a CUDA, C ABI in
 include/ss_scan.h); this package is its Python binding plus the seeded input
@@ -25,6 +25,8 @@ from ._native import (  # noqa: F401
     load_library,
     ss_debug_inject,
     ss_last_device_error,
+    ss_scan_bwd,
+    ss_scan_bwd_workspace_bytes,
     ss_scan_fwd,
     ss_scan_fwd_conv,
     ss_scan_fwd_from_state,

@@ -23,7 +23,8 @@ SS_F32, SS_BF16 = 0, 1
 
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
             "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc",
-            "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv", "ss_scan_fwd_zoh")
+            "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv", "ss_scan_fwd_zoh",
+            "ss_scan_bwd", "ss_scan_bwd_workspace_bytes")
 
 # bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
 SS_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -78,6 +79,11 @@ def load_library():
         lib.ss_scan_fwd_conv.restype = ci
         lib.ss_scan_fwd_zoh.argtypes = lib.ss_scan_fwd.argtypes
         lib.ss_scan_fwd_zoh.restype = ci
+        lib.ss_scan_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp, vp, vp, vp,
+                                    vp, vp, vp, i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
+        lib.ss_scan_bwd.restype = ci
+        lib.ss_scan_bwd_workspace_bytes.argtypes = [i64, i64, i64, ci]
+        lib.ss_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.ss_scan_step.restype = ci
         _lib = lib
         return lib
@@ -233,6 +239,48 @@ def ss_scan_fwd_conv(x, conv_weight, delta, A, B, C, D=None, z=None, delta_bias=
     return _fwd_call("ss_scan_fwd_conv", (conv_weight, conv_bias), x, delta, A, B, C, D, z,
                      delta_bias, softplus, y_out, last_state_out, return_last_state, workspace,
                      stream)
+
+
+def ss_scan_bwd_workspace_bytes(batch: int, dim: int, seqlen: int, dstate: int) -> int:
+    n = load_library().ss_scan_bwd_workspace_bytes(batch, dim, seqlen, dstate)
+    if n == ctypes.c_size_t(-1).value:
+        raise SSError(SS_ERR_INVALID_ARG, "ss_scan_bwd_workspace_bytes")
+    return n
+
+
+def ss_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=True,
+                dlast_state=None, workspace=None, stream=None):
+    """Gradients of ss_scan_fwd for an upstream dy [batch, dim, L] float32.
+
+    Returns a dict of float32 tensors: du, ddelta, dz (None without z), dA
+    [dim, N], dB, dC [batch, N, L], dD (None without D), ddelta_bias (None
+    without delta_bias).  The states are recomputed, not stored.
+    """
+    lib = load_library()
+    device, batch, dim, L, N = _fwd_operands(u, delta, A, B, C, D, z, delta_bias)
+    _check_dev("dy", dy, device, (torch.float32,), (batch, dim, L))
+    _check_dev("dlast_state", dlast_state, device, (torch.float32,), (batch, dim, N))
+    f32 = dict(dtype=torch.float32, device=device)
+    g = {"du": torch.empty((batch, dim, L), **f32), "ddelta": torch.empty((batch, dim, L), **f32),
+         "dz": torch.empty((batch, dim, L), **f32) if z is not None else None,
+         "dA": torch.empty((dim, N), **f32), "dB": torch.empty((batch, N, L), **f32),
+         "dC": torch.empty((batch, N, L), **f32),
+         "dD": torch.empty((dim,), **f32) if D is not None else None,
+         "ddelta_bias": torch.empty((dim,), **f32) if delta_bias is not None else None}
+    need = ss_scan_bwd_workspace_bytes(batch, dim, L, N)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    dt = SS_F32 if u.dtype == torch.float32 else SS_BF16
+    st = lib.ss_scan_bwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                         _ptr(delta_bias), int(bool(softplus)), _ptr(dy), _ptr(dlast_state),
+                         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]),
+                         _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddelta_bias"]),
+                         batch, dim, L, N, dt, _ptr(workspace), ws_bytes,
+                         _stream_handle(stream, device))
+    if st != SS_OK:
+        raise SSError(st, "ss_scan_bwd")
+    return g
 
 
 def ss_scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,

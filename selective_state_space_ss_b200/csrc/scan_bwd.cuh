@@ -1,0 +1,432 @@
+// scan_bwd.cuh -- backward of the selective scan with recomputation.
+//
+// The forward keeps no states ("Mamba 深度解读报告", sec. 3.3; "Mamba 选择性机制",
+// sec. 3.4: the backward recomputes them from the inputs instead of storing
+// them).  One CTA owns CH channels of one batch row and the whole sequence:
+//
+//  pass 1  forward over the sequence, writing only the state at the start of
+//          every chunk of T steps to the caller's workspace (CH x N floats
+//          per chunk);
+//  pass 2  over the chunks in reverse: recompute the chunk's states h_t from
+//          its checkpoint into shared memory, then run the adjoint
+//          g_t = dq_t C_t + a_{t+1} g_{t+1} backwards through the chunk with
+//          the carry in registers:
+//            dDelta_t = sum_n g_t (B_t u_t + A a_t h_{t-1}),
+//            du_t     = dq_t D + sum_n g_t Delta_t B_t,
+//            dA      += g_t Delta_t a_t h_{t-1},
+//            dB_t    += g_t Delta_t u_t   (over channels),
+//            dC_t    += dq_t h_t          (over channels),
+//          with dq_t = dy_t SiLU(z_t), dz_t = dy_t q_t SiLU'(z_t),
+//          q_t = C_t . h_t + D u_t, ddelta = dDelta softplus'(x).
+//
+// Lane layout: four states of one channel per lane (N/4 lanes per channel).
+// Per-channel sums over a lane's states go through shared memory; sums over
+// the CTA's channels (dB, dC) are reduced in shared memory and added to HBM
+// with one atomic per (state, step) per CTA; dA, dD and the bias gradient
+// with one atomic per channel state per CTA.  Those outputs are zeroed by
+// the host before the launch.
+#pragma once
+
+#include "pointwise.cuh"
+
+namespace ssscan {
+
+struct BwdArgs {
+  const void* u;
+  const void* delta;
+  const void* z;  // nullable
+  const void* B;
+  const void* C;
+  const float* A;
+  const float* D;           // nullable
+  const float* delta_bias;  // nullable
+  const float* dy;          // [batch, dim, L] fp32
+  const float* dlast;       // [batch, dim, N] fp32, nullable
+  float* du;                // [batch, dim, L]
+  float* ddelta;            // [batch, dim, L]
+  float* dz;                // [batch, dim, L], nullable (when z is)
+  float* dA;                // [dim, N], accumulated
+  float* dB;                // [batch, N, L], accumulated
+  float* dC;                // [batch, N, L], accumulated
+  float* dD;                // [dim], accumulated, nullable
+  float* dbias;             // [dim], accumulated, nullable
+  float* ckpt;              // workspace: [CTAs][chunks][CH * N]
+  int64_t batch, dim, seqlen;
+  int softplus;
+};
+
+template <typename Tin, int N_>
+struct BwdCfg {
+  using Elem = Tin;
+  static constexpr int N = N_;
+  static constexpr int G = 4;             // states per lane
+  static constexpr int K = N / G;         // lanes per channel
+  static constexpr int CPW = 32 / K;      // channels per warp
+  static constexpr int NWARPS = 4;
+  static constexpr int NT = NWARPS * 32;
+  static constexpr int CH = NWARPS * CPW; // channels per CTA
+  static constexpr int CHP = CH + 1;      // padded row of per-channel values
+  static constexpr int T = 16;            // steps per chunk
+  static constexpr int ITEMS = CH * T;    // (step, channel) items per chunk
+  static constexpr int IPT = (ITEMS + NT - 1) / NT;
+  static constexpr int STEP_FLOATS = CH * N;  // one step's states of the CTA
+  // staged inputs per thread (register prefetch of the next chunk)
+  static constexpr int ACT_PT = (CH * T + NT - 1) / NT;
+  static constexpr int SEL_PT = (N * T + NT - 1) / NT;
+  // shared memory (floats); per-channel values are [T][CHP] (step-major, so
+  // the lanes of a warp read consecutive channels), B and C are [T][N]
+  static constexpr int OFF_U = 0;
+  static constexpr int OFF_DL = OFF_U + T * CHP;        // delta, then Delta
+  static constexpr int OFF_Z = OFF_DL + T * CHP;
+  static constexpr int OFF_DY = OFF_Z + T * CHP;        // dy, then dq
+  static constexpr int OFF_W = OFF_DY + T * CHP;        // Delta u
+  static constexpr int OFF_SG = OFF_W + T * CHP;        // softplus'(x)
+  static constexpr int OFF_P1 = OFF_SG + T * CHP;       // per-channel sums (readout, dDelta)
+  static constexpr int OFF_P2 = OFF_P1 + T * CHP;       // per-channel sums (du)
+  static constexpr int NP = N + 4;                      // B, C row pitch (16-byte aligned)
+  static constexpr int OFF_B = (OFF_P2 + T * CHP + 3) / 4 * 4;  // [T][NP]
+  static constexpr int OFF_C = OFF_B + T * NP;
+  static constexpr int OFF_H = OFF_C + T * NP;          // [T][CH*N] states, then g Delta u
+  static constexpr int SMEM_FLOATS = OFF_H + T * STEP_FLOATS;
+  static constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
+  static_assert(N % G == 0 && 32 % K == 0, "lane split");
+  static_assert(ITEMS % NT == 0 || ITEMS < NT, "whole items per thread");
+  static constexpr bool ITEM_GUARD = ITEMS < NT;  // some threads have no item
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <typename E>
+__device__ __forceinline__ float ld_elem(const E* p, int64_t i) {
+  return to_f32(p[i]);
+}
+
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  return rcp_approx(1.f + ex2_approx(-x * 1.4426950408889634f));
+}
+
+// One chunk's inputs in registers (global loads issued early, stored to
+// shared memory once the previous chunk is done with it).  Activations are
+// read along t (coalesced): element r of a thread is (c, t) = (i / T, i % T),
+// i = tid + r * NT.
+template <class CF>
+struct BwdStage {
+  float u[CF::ACT_PT], dl[CF::ACT_PT], z[CF::ACT_PT], dy[CF::ACT_PT];
+  float b[CF::SEL_PT], c[CF::SEL_PT];
+};
+
+template <class CF, bool with_grad>
+__device__ __forceinline__ void bwd_fetch(const BwdArgs& a, BwdStage<CF>& st, int64_t b,
+                                          int64_t d0, int64_t t0) {
+  using E = typename CF::Elem;
+  const int64_t L = a.seqlen;
+#pragma unroll
+  for (int r = 0; r < CF::ACT_PT; ++r) {
+    const int i = threadIdx.x + r * CF::NT;
+    const int c = i / CF::T, tt = i - c * CF::T;
+    const int64_t d = d0 + c, t = t0 + tt;
+    const bool in = i < CF::CH * CF::T && d < a.dim && t < L;
+    const int64_t off = (b * a.dim + d) * L + t;
+    st.u[r] = in ? ld_elem(static_cast<const E*>(a.u), off) : 0.f;
+    st.dl[r] = in ? ld_elem(static_cast<const E*>(a.delta), off) : 0.f;
+    if (with_grad) {
+      st.z[r] = (in && a.z) ? ld_elem(static_cast<const E*>(a.z), off) : 0.f;
+      st.dy[r] = in ? a.dy[off] : 0.f;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < CF::SEL_PT; ++r) {
+    const int i = threadIdx.x + r * CF::NT;
+    const int n = i / CF::T, tt = i - n * CF::T;
+    const int64_t t = t0 + tt;
+    const bool in = i < CF::N * CF::T && t < L;
+    const int64_t off = (b * CF::N + n) * L + t;
+    st.b[r] = in ? ld_elem(static_cast<const E*>(a.B), off) : 0.f;
+    if (with_grad) st.c[r] = in ? ld_elem(static_cast<const E*>(a.C), off) : 0.f;
+  }
+}
+
+template <class CF, bool with_grad>
+__device__ __forceinline__ void bwd_store(const BwdStage<CF>& st, float* sm) {
+#pragma unroll
+  for (int r = 0; r < CF::ACT_PT; ++r) {
+    const int i = threadIdx.x + r * CF::NT;
+    if (i >= CF::CH * CF::T) break;
+    const int c = i / CF::T, tt = i - c * CF::T;
+    const int o = tt * CF::CHP + c;
+    sm[CF::OFF_U + o] = st.u[r];
+    sm[CF::OFF_DL + o] = st.dl[r];
+    if (with_grad) {
+      sm[CF::OFF_Z + o] = st.z[r];
+      sm[CF::OFF_DY + o] = st.dy[r];
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < CF::SEL_PT; ++r) {
+    const int i = threadIdx.x + r * CF::NT;
+    if (i >= CF::N * CF::T) break;
+    const int n = i / CF::T, tt = i - n * CF::T;
+    sm[CF::OFF_B + tt * CF::NP + n] = st.b[r];
+    if (with_grad) sm[CF::OFF_C + tt * CF::NP + n] = st.c[r];
+  }
+}
+
+// Per (step, channel) item: Delta (0 on padding), Delta u, softplus'(x).
+// Items are channel-fastest: item i is (t, c) = (i / CH, i % CH).
+template <class CF>
+__device__ __forceinline__ void bwd_discretise(const BwdArgs& a, float* sm, int64_t d0,
+                                               int64_t t0) {
+#pragma unroll
+  for (int it = 0; it < CF::IPT; ++it) {
+    const int i = threadIdx.x + it * CF::NT;
+    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
+    const int tt = i / CF::CH, c = i - tt * CF::CH;
+    const int o = tt * CF::CHP + c;
+    const int64_t d = d0 + c;
+    const bool in = d < a.dim && t0 + tt < a.seqlen;
+    const float x = sm[CF::OFF_DL + o] + ((a.delta_bias && d < a.dim) ? __ldg(a.delta_bias + d) : 0.f);
+    const float dl = in ? (a.softplus ? softplus_fast(x) : x) : 0.f;
+    sm[CF::OFF_DL + o] = dl;
+    sm[CF::OFF_W + o] = dl * sm[CF::OFF_U + o];
+    sm[CF::OFF_SG + o] = a.softplus ? sigmoid_fast(x) : 1.f;
+  }
+}
+
+// Sum over the K lanes of a channel (consecutive lanes of one warp).
+template <int K>
+__device__ __forceinline__ float lane_sum(float v) {
+#pragma unroll
+  for (int off = K / 2; off > 0; off >>= 1) v += __shfl_xor_sync(kFullMask, v, off);
+  return v;
+}
+
+template <class CF>
+__global__ void __launch_bounds__(CF::NT)
+    scan_bwd_kernel(const BwdArgs a) {
+  constexpr int N = CF::N, G = CF::G, K = CF::K, T = CF::T, CHP = CF::CHP;
+  extern __shared__ __align__(16) float sm[];
+  const int64_t tiles = (a.dim + CF::CH - 1) / CF::CH;
+  const int64_t b = blockIdx.x / tiles;
+  const int64_t d0 = (blockIdx.x - b * tiles) * CF::CH;
+  const int64_t L = a.seqlen;
+  const int64_t nk = (L + T - 1) / T;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = warp * CF::CPW + lane / K;  // this lane's channel
+  const int j = lane % K;                   // its state group
+  const int64_t d = d0 + c;
+  const bool chan_ok = d < a.dim;
+  float* ck = a.ckpt + (int64_t)blockIdx.x * nk * CF::STEP_FLOATS;
+  float* hb = sm + CF::OFF_H;
+
+  // decay constants of this lane's four states, as two packed pairs
+  float2 A2[2], An[2];
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const float a0 = chan_ok ? __ldg(a.A + d * N + j * G + 2 * p) : 0.f;
+    const float a1 = chan_ok ? __ldg(a.A + d * N + j * G + 2 * p + 1) : 0.f;
+    An[p] = make_float2(a0, a1);
+    A2[p] = make_float2(a0 * 1.4426950408889634f, a1 * 1.4426950408889634f);
+  }
+  BwdStage<CF> st;
+  auto ex2_pair = [](float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); };
+  auto ld_pairs = [](const float* p, float2 (&v)[2]) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    v[0] = make_float2(q.x, q.y);
+    v[1] = make_float2(q.z, q.w);
+  };
+  auto st_pairs = [](float* p, const float2 (&v)[2]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+  };
+  float* ck_lane = ck + c * N + j * G;        // this lane's slot in every checkpoint
+  float* hb_lane = hb + c * N + j * G;        // and in every step row of hb
+
+  // ---- pass 1: forward, checkpoint the state at every chunk start ----
+  float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  bwd_fetch<CF, false>(a, st, b, d0, 0);
+  for (int64_t k = 0; k < nk; ++k) {
+    st_pairs(ck_lane + k * CF::STEP_FLOATS, h);
+    bwd_store<CF, false>(st, sm);
+    if (k + 1 < nk) bwd_fetch<CF, false>(a, st, b, d0, (k + 1) * T);
+    __syncthreads();
+    bwd_discretise<CF>(a, sm, d0, k * T);
+    __syncthreads();
+#pragma unroll 4
+    for (int t = 0; t < T; ++t) {
+      const float dl = sm[CF::OFF_DL + t * CHP + c], w = sm[CF::OFF_W + t * CHP + c];
+      const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w);
+      float2 bb[2];
+      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
+#pragma unroll
+      for (int p = 0; p < 2; ++p)
+        h[p] = __ffma2_rn(ex2_pair(__fmul2_rn(dl2, A2[p])), h[p], __fmul2_rn(w2, bb[p]));
+    }
+    __syncthreads();
+  }
+
+  // ---- pass 2: chunks in reverse ----
+  float2 carry[2];
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const float* dl_ = a.dlast + (b * a.dim + d) * N + j * G + 2 * p;
+    carry[p] = (a.dlast && chan_ok) ? make_float2(dl_[0], dl_[1]) : make_float2(0.f, 0.f);
+  }
+  float2 dA_acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float dD_acc[CF::IPT], db_acc[CF::IPT];
+#pragma unroll
+  for (int it = 0; it < CF::IPT; ++it) dD_acc[it] = db_acc[it] = 0.f;
+
+  bwd_fetch<CF, true>(a, st, b, d0, (nk - 1) * T);
+  float2 ck_next[2];  // the checkpoint of the chunk to come, loaded a chunk early
+  ld_pairs(ck_lane + (nk - 1) * CF::STEP_FLOATS, ck_next);
+  for (int64_t k = nk - 1; k >= 0; --k) {
+    const int64_t t0 = k * T;
+    const float2 h_start[2] = {ck_next[0], ck_next[1]};
+    bwd_store<CF, true>(st, sm);
+    if (k > 0) {
+      bwd_fetch<CF, true>(a, st, b, d0, (k - 1) * T);
+      ld_pairs(ck_lane + (k - 1) * CF::STEP_FLOATS, ck_next);
+    }
+    __syncthreads();
+    bwd_discretise<CF>(a, sm, d0, t0);
+    __syncthreads();
+    // recompute the chunk's states from its checkpoint; channel readouts
+    float2 hs[2] = {h_start[0], h_start[1]};
+#pragma unroll 4
+    for (int t = 0; t < T; ++t) {
+      const float dl = sm[CF::OFF_DL + t * CHP + c], w = sm[CF::OFF_W + t * CHP + c];
+      const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w);
+      float2 bb[2], cc[2];
+      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
+      ld_pairs(sm + CF::OFF_C + t * CF::NP + j * G, cc);
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        hs[p] = __ffma2_rn(ex2_pair(__fmul2_rn(dl2, A2[p])), hs[p], __fmul2_rn(w2, bb[p]));
+        acc = __ffma2_rn(cc[p], hs[p], acc);
+      }
+      st_pairs(hb_lane + t * CF::STEP_FLOATS, hs);
+      const float part = lane_sum<K>(acc.x + acc.y);
+      if (j == 0) sm[CF::OFF_P1 + t * CHP + c] = part;
+    }
+    __syncthreads();
+    // per item: q, the gate's derivatives, dq
+#pragma unroll
+    for (int it = 0; it < CF::IPT; ++it) {
+      const int i = tid + it * CF::NT;
+      if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
+      const int tt = i / CF::CH, ci = i - tt * CF::CH;
+      const int o = tt * CHP + ci;
+      const int64_t di = d0 + ci, t = t0 + tt;
+      const bool in = di < a.dim && t < L;
+      const float Dd = (a.D && di < a.dim) ? __ldg(a.D + di) : 0.f;
+      const float uu = sm[CF::OFF_U + o];
+      const float q = sm[CF::OFF_P1 + o] + Dd * uu;
+      const float dy = sm[CF::OFF_DY + o];
+      float dq = dy;
+      if (a.z) {
+        const float zz = sm[CF::OFF_Z + o];
+        const float sg = sigmoid_fast(zz);
+        dq = dy * zz * sg;
+        if (in) a.dz[(b * a.dim + di) * L + t] = dy * q * sg * (1.f + zz * (1.f - sg));
+      }
+      sm[CF::OFF_DY + o] = dq;
+      if (in) dD_acc[it] = fmaf(dq, uu, dD_acc[it]);
+    }
+    __syncthreads();
+    // dC[b, n, t] += sum_c dq[t, c] h_t[c, n]
+    for (int i = tid; i < N * T; i += CF::NT) {
+      const int tt = i / N, n = i - tt * N;
+      if (t0 + tt >= L) continue;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int cc = 0; cc < CF::CH; ++cc)
+        acc = fmaf(sm[CF::OFF_DY + tt * CHP + cc], hb[tt * CF::STEP_FLOATS + cc * N + n], acc);
+      atomicAdd(a.dC + (b * N + n) * L + t0 + tt, acc);
+    }
+    __syncthreads();
+    // the adjoint, backwards through the chunk
+#pragma unroll 2
+    for (int t = T - 1; t >= 0; --t) {
+      const float dl = sm[CF::OFF_DL + t * CHP + c];
+      const float uu = sm[CF::OFF_U + t * CHP + c];
+      const float dq = sm[CF::OFF_DY + t * CHP + c];
+      const float2 dl2 = make_float2(dl, dl), uu2 = make_float2(uu, uu), dq2 = make_float2(dq, dq);
+      float2 bb[2], cc[2], prev[2];
+      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
+      ld_pairs(sm + CF::OFF_C + t * CF::NP + j * G, cc);
+      if (t > 0) {
+        ld_pairs(hb_lane + (t - 1) * CF::STEP_FLOATS, prev);
+      } else {
+        prev[0] = h_start[0];
+        prev[1] = h_start[1];
+      }
+      float2 ddl = make_float2(0.f, 0.f), dup = make_float2(0.f, 0.f), gdu[2];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float2 e = ex2_pair(__fmul2_rn(dl2, A2[p]));
+        const float2 gt = __ffma2_rn(dq2, cc[p], carry[p]);
+        const float2 eprev = __fmul2_rn(e, prev[p]);
+        ddl = __ffma2_rn(gt, __ffma2_rn(bb[p], uu2, __fmul2_rn(An[p], eprev)), ddl);
+        const float2 gdl = __fmul2_rn(gt, dl2);
+        dup = __ffma2_rn(gdl, bb[p], dup);
+        dA_acc[p] = __ffma2_rn(gdl, eprev, dA_acc[p]);
+        gdu[p] = __fmul2_rn(gdl, uu2);
+        carry[p] = __fmul2_rn(e, gt);
+      }
+      // h_t is no longer needed (its dC and its step's prev are done): reuse the slot
+      st_pairs(hb_lane + t * CF::STEP_FLOATS, gdu);
+      const float ddl_c = lane_sum<K>(ddl.x + ddl.y);
+      const float dup_c = lane_sum<K>(dup.x + dup.y);
+      if (j == 0) {
+        sm[CF::OFF_P1 + t * CHP + c] = ddl_c;
+        sm[CF::OFF_P2 + t * CHP + c] = dup_c;
+      }
+    }
+    __syncthreads();
+    // dB[b, n, t] += sum_c g Delta u
+    for (int i = tid; i < N * T; i += CF::NT) {
+      const int tt = i / N, n = i - tt * N;
+      if (t0 + tt >= L) continue;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int cc = 0; cc < CF::CH; ++cc) acc += hb[tt * CF::STEP_FLOATS + cc * N + n];
+      atomicAdd(a.dB + (b * N + n) * L + t0 + tt, acc);
+    }
+    // per item: du, ddelta, the bias gradient
+#pragma unroll
+    for (int it = 0; it < CF::IPT; ++it) {
+      const int i = tid + it * CF::NT;
+      if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
+      const int tt = i / CF::CH, ci = i - tt * CF::CH;
+      const int o = tt * CHP + ci;
+      const int64_t di = d0 + ci, t = t0 + tt;
+      if (di >= a.dim || t >= L) continue;
+      const float Dd = a.D ? __ldg(a.D + di) : 0.f;
+      const float dx = sm[CF::OFF_P1 + o] * sm[CF::OFF_SG + o];
+      const int64_t off = (b * a.dim + di) * L + t;
+      a.ddelta[off] = dx;
+      a.du[off] = fmaf(sm[CF::OFF_DY + o], Dd, sm[CF::OFF_P2 + o]);
+      db_acc[it] += dx;
+    }
+    __syncthreads();
+  }
+
+  // per-channel sums over this CTA's part of the batch
+  if (chan_ok) {
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      atomicAdd(a.dA + d * N + j * G + 2 * p, dA_acc[p].x);
+      atomicAdd(a.dA + d * N + j * G + 2 * p + 1, dA_acc[p].y);
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < CF::IPT; ++it) {
+    const int i = tid + it * CF::NT;
+    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
+    const int64_t di = d0 + (i - (i / CF::CH) * CF::CH);
+    if (di >= a.dim) continue;
+    if (a.dD) atomicAdd(a.dD + di, dD_acc[it]);
+    if (a.dbias) atomicAdd(a.dbias + di, db_acc[it]);
+  }
+}
+
+}  // namespace ssscan

@@ -13,6 +13,7 @@
 #include "ss_scan_debug.h"
 #include "scan_fwd_chunked.cuh"
 #include "scan_step.cuh"
+#include "scan_bwd.cuh"
 
 namespace ssscan {
 
@@ -342,6 +343,40 @@ ss_status dispatch_step(const StepArgs& a, int N, bool vec, bool pipe, cudaStrea
   }
 }
 
+template <typename E, int N>
+size_t bwd_ws_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
+  using CF = BwdCfg<E, N>;
+  const int64_t ctas = batch * ((dim + CF::CH - 1) / CF::CH);
+  const int64_t nk = (seqlen + CF::T - 1) / CF::T;
+  return align256((size_t)ctas * (size_t)nk * CF::STEP_FLOATS * sizeof(float));
+}
+
+template <typename E, int N>
+ss_status launch_bwd(const BwdArgs& a, size_t ws_bytes, cudaStream_t stream) {
+  using CF = BwdCfg<E, N>;
+  static int state = 0;
+  if (state == 0)
+    state = cudaFuncSetAttribute(scan_bwd_kernel<CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 CF::SMEM_BYTES) == cudaSuccess ? 1 : -1;
+  if (state != 1) return SS_ERR_CUDA;
+  if (ws_bytes < bwd_ws_bytes<E, N>(a.batch, a.dim, a.seqlen)) return SS_ERR_INVALID_ARG;
+  const int64_t ctas = a.batch * ((a.dim + CF::CH - 1) / CF::CH);
+  if (ctas > INT_MAX) return SS_ERR_INVALID_ARG;
+  scan_bwd_kernel<CF><<<(unsigned)ctas, CF::NT, CF::SMEM_BYTES, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+template <typename E>
+ss_status dispatch_bwd(const BwdArgs& a, int N, size_t ws_bytes, cudaStream_t stream) {
+  switch (N) {
+    case 16: return launch_bwd<E, 16>(a, ws_bytes, stream);
+    case 32: return launch_bwd<E, 32>(a, ws_bytes, stream);
+    case 64: return launch_bwd<E, 64>(a, ws_bytes, stream);
+    case 128: return launch_bwd<E, 128>(a, ws_bytes, stream);
+    default: return SS_ERR_UNSUPPORTED;
+  }
+}
+
 ss_status scan_fwd_impl(const void* u, const void* delta, const float* A, const void* B,
                         const void* C, const float* D, const void* z, const float* delta_bias,
                         int softplus_flag, const float* h0, float* y_out, float* last_state_out,
@@ -430,6 +465,62 @@ ss_status ss_scan_fwd_from_state(const void* u, const void* delta, const float* 
   return scan_fwd_impl(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y_out,
                        last_state_out, batch, dim, seqlen, dstate, in_dtype, workspace,
                        workspace_bytes, stream);
+}
+
+size_t ss_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int dstate) {
+  if (batch < 1 || dim < 1 || seqlen < 1 || !supported_dstate(dstate)) return (size_t)-1;
+  if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
+    return (size_t)-1;
+  switch (dstate) {  // the layout does not depend on the input dtype
+    case 16: return bwd_ws_bytes<float, 16>(batch, dim, seqlen);
+    case 32: return bwd_ws_bytes<float, 32>(batch, dim, seqlen);
+    case 64: return bwd_ws_bytes<float, 64>(batch, dim, seqlen);
+    default: return bwd_ws_bytes<float, 128>(batch, dim, seqlen);
+  }
+}
+
+ss_status ss_scan_bwd(const void* u, const void* delta, const float* A, const void* B,
+                      const void* C, const float* D, const void* z, const float* delta_bias,
+                      int softplus_flag, const float* dy, const float* dlast_state, float* du,
+                      float* ddelta, float* dA, float* dB, float* dC, float* dD, float* dz,
+                      float* ddelta_bias, int64_t batch, int64_t dim, int64_t seqlen, int dstate,
+                      ss_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
+  if (!u || !delta || !A || !B || !C || !dy || !du || !ddelta || !dA || !dB || !dC)
+    return SS_ERR_INVALID_ARG;
+  if (z && !dz) return SS_ERR_INVALID_ARG;
+  if (batch < 1 || dim < 1 || seqlen < 1) return SS_ERR_INVALID_ARG;
+  if (in_dtype != SS_F32 && in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED;
+  if (!supported_dstate(dstate)) return SS_ERR_UNSUPPORTED;
+  if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
+    return SS_ERR_INVALID_ARG;
+  if (batch * (int64_t)dstate > (INT64_C(1) << 62) / seqlen) return SS_ERR_INVALID_ARG;
+  const size_t es = in_dtype == SS_F32 ? 4 : 2;
+  const void* in_ptrs[5] = {u, delta, z, B, C};
+  for (const void* p : in_ptrs)
+    if (p && !aligned(p, es)) return SS_ERR_INVALID_ARG;
+  const void* f_ptrs[13] = {A, D, delta_bias, dy, dlast_state, du, ddelta, dA, dB, dC, dD, dz,
+                            ddelta_bias};
+  for (const void* p : f_ptrs)
+    if (p && !aligned(p, 4)) return SS_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return SS_ERR_INVALID_ARG;
+  // the sums over channels, steps and batch rows accumulate with atomics
+  if (cudaMemsetAsync(dA, 0, (size_t)dim * dstate * 4, stream) != cudaSuccess ||
+      cudaMemsetAsync(dB, 0, (size_t)(batch * dstate * seqlen) * 4, stream) != cudaSuccess ||
+      cudaMemsetAsync(dC, 0, (size_t)(batch * dstate * seqlen) * 4, stream) != cudaSuccess ||
+      (dD && cudaMemsetAsync(dD, 0, (size_t)dim * 4, stream) != cudaSuccess) ||
+      (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, (size_t)dim * 4, stream) != cudaSuccess))
+    return SS_ERR_CUDA;
+  BwdArgs a;
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.A = A; a.D = D; a.delta_bias = delta_bias; a.dy = dy; a.dlast = dlast_state;
+  a.du = du; a.ddelta = ddelta; a.dz = dz; a.dA = dA; a.dB = dB; a.dC = dC;
+  a.dD = D ? dD : nullptr; a.dbias = ddelta_bias;
+  a.ckpt = static_cast<float*>(workspace);
+  a.batch = batch; a.dim = dim; a.seqlen = seqlen;
+  a.softplus = softplus_flag != 0;
+  if (in_dtype == SS_F32) return dispatch_bwd<float>(a, dstate, workspace_bytes, stream);
+  return dispatch_bwd<__nv_bfloat16>(a, dstate, workspace_bytes, stream);
 }
 
 ss_status ss_scan_fwd_zoh(const void* u, const void* delta, const float* A, const void* B,

@@ -1,0 +1,95 @@
+"""GPU-vs-oracle parity for ss_scan_bwd (gradients with recomputation).
+
+Every gradient is compared with the fp64 oracle's reverse-mode sweep
+element by element, relative to its largest reference value.  Tolerance:
+TOL_BWD (see the design notes: fp32 recomputation of the states, fp32
+adjoint, and atomically ordered sums over channels, steps and batch rows).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle  # noqa: E402
+import selective_state_space_ss_b200 as ss  # noqa: E402
+from selective_state_space_ss_b200 import inputs as I  # noqa: E402
+from tests.helpers import rel_err, to_device  # noqa: E402
+
+TOL_BWD = {"f32": 1e-4, "bf16": 1e-4}
+NAMES = ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias")
+
+
+def _dy(w, seed):
+    return I.fill(seed, 12, (w.batch, w.dim, w.seqlen))
+
+
+def _run(w, x, dy, dlast=None, softplus=True):
+    xd = to_device(x)
+    g = ss.ss_scan_bwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], torch.from_numpy(dy).cuda(),
+                       D=xd["D"], z=xd["z"], delta_bias=xd["delta_bias"], softplus=softplus,
+                       dlast_state=None if dlast is None else torch.from_numpy(dlast).cuda())
+    assert ss.ss_last_device_error() == ss.SS_OK
+    r = oracle.scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
+                        softplus=softplus, dy=dy.astype(np.float64),
+                        dlast=None if dlast is None else dlast.astype(np.float64))
+    errs = {}
+    for k in NAMES:
+        if g[k] is None or r[k] is None:
+            assert (g[k] is None) == (r[k] is None or (k == "dD" and x["D"] is None)
+                                      or (k == "ddelta_bias" and x["delta_bias"] is None)), k
+            continue
+        errs[k] = rel_err(g[k].cpu().numpy(), r[k])
+    bad = {k: v for k, v in errs.items() if v > TOL_BWD[w.dtype]}
+    assert not bad, f"{w.name}: {bad} (all: {errs})"
+    return errs
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [16, 32, 64, 128])
+@pytest.mark.parametrize("L", [1, 15, 16, 17, 300])
+def test_bwd_small_shapes(dtype, N, L):
+    w = I.Workload(f"bwd_{dtype}_{N}_{L}", 2, 37, L, N, dtype)
+    x = I.make_inputs(w, seed=L + N)
+    _run(w, x, _dy(w, L))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bwd_with_final_state_gradient(dtype):
+    w = I.Workload(f"bwdlast_{dtype}", 3, 50, 200, 16, dtype)
+    x = I.make_inputs(w, seed=5)
+    dlast = I.fill(6, 13, (3, 50, 16))
+    _run(w, x, _dy(w, 7), dlast=dlast)
+
+
+@pytest.mark.parametrize("variant", ["no_z", "no_D", "no_bias", "no_softplus", "bare"])
+def test_bwd_optional_inputs(variant):
+    kw = {"no_z": dict(with_z=False), "no_D": dict(with_D=False),
+          "no_bias": dict(with_bias=False), "no_softplus": dict(softplus=False),
+          "bare": dict(with_z=False, with_D=False, with_bias=False, softplus=False)}[variant]
+    w = dataclasses.replace(I.Workload("bwdopt", 2, 70, 130, 32, "f32"), **kw)
+    x = I.make_inputs(w, seed=9)
+    if not w.softplus:  # Delta = delta + bias must stay positive and small
+        x["delta"] = (np.abs(x["delta"]) * 0.02 + 1e-3).astype(np.float32)
+        if x["delta_bias"] is not None:
+            x["delta_bias"] = np.full_like(x["delta_bias"], 1e-3)
+    _run(w, x, _dy(w, 10), softplus=w.softplus)
+
+
+def test_bwd_medium_workload():
+    # several CTAs per batch row (the sums over channels cross CTAs), 64 chunks
+    w = I.Workload("bwdmed", 2, 512, 1024, 16, "bf16")
+    x = I.make_inputs(w, seed=11)
+    _run(w, x, _dy(w, 12))
+
+
+def test_bwd_workspace_too_small():
+    w = I.Workload("bwdws", 1, 32, 64, 16, "f32")
+    xd = to_device(I.make_inputs(w, seed=1))
+    dy = torch.zeros(1, 32, 64, device="cuda")
+    need = ss.ss_scan_bwd_workspace_bytes(1, 32, 64, 16)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ss.SSError):
+        ss.ss_scan_bwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], dy, workspace=ws)
