@@ -42,7 +42,8 @@ MUFU_EX2_PER_CLK_PER_SM = 16  # ex2 results per clock per SM (special-function u
 _CSRC = "selective_state_space_ss_b200/csrc/"
 KERNEL_SOURCES = tuple(_CSRC + f for f in ("ss_scan.cu", "pointwise.cuh", "scan_fwd_chunked.cuh",
                                            "scan_common.cuh"))
-# (the step kernels' launch shapes are constants of scan_step.cuh)
+BWD_KERNEL_SOURCES = tuple(_CSRC + f for f in ("pointwise.cuh", "scan_bwd.cuh", "scan_common.cuh"))
+# (the step and backward kernels' launch shapes are constants of their headers)
 STEP_KERNEL_SOURCES = tuple(_CSRC + f for f in ("pointwise.cuh", "scan_step.cuh", "scan_common.cuh"))
 
 
@@ -475,7 +476,8 @@ def run_bwd_arm(args, w: I.Workload):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": dict(config_of(w, 1), op="backward"),
             "roofline": {"bound": "alu", "achieved": achieved, "peak": sfu_rate / 1e9, "unit": "Gexp2/s",
-                         "frac": achieved * 1e9 / sfu_rate, "traffic": None,
+                         "frac": achieved * 1e9 / sfu_rate,
+                         "traffic": profiled_traffic(w.name + "+bwd", BWD_KERNEL_SOURCES),
                          "exps_per_step": exps, "hbm_bytes_per_step": bwd_bytes(w),
                          "hbm_frac": bwd_bytes(w) / (ms * 1e-3) / 1e9 / p["hbm_gbs"]},
             "gpu_launches": args.steps, "clocks": clk.summary()}
