@@ -481,6 +481,32 @@ def run_bwd_arm(args, w: I.Workload):
                          "exps_per_step": exps, "hbm_bytes_per_step": bwd_bytes(w),
                          "hbm_frac": bwd_bytes(w) / (ms * 1e-3) / 1e9 / p["hbm_gbs"]},
             "gpu_launches": args.steps, "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        # the oracle's reverse sweep sums dB, dC over every channel of a row, so
+        # the sample is the first batch row with its first channels, full L
+        import dataclasses
+
+        import oracle
+
+        x = host[0]
+        cores = os.cpu_count() or 1
+        dims = w.dim
+        ws_ = dataclasses.replace(w, batch=1, dim=dims)
+        xs = {k: (None if v is None else np.ascontiguousarray(
+            v[:1, :dims] if k in ("u", "delta", "z") else v[:1] if k in ("B", "C")
+            else v[:dims])) for k, v in x.items()}
+        dy = I.fill(7, 12, (1, dims, w.seqlen)).astype(np.float64)
+        reps, t0 = 0, time.perf_counter()
+        while reps < 1 or (time.perf_counter() - t0 < 10.0 and reps < 100):
+            oracle.scan_bwd(xs["u"], xs["delta"], xs["A"], xs["B"], xs["C"], xs["D"], xs["z"],
+                            xs["delta_bias"], softplus=w.softplus, dy=dy, nthreads=cores)
+            reps += 1
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": reps * ws_.elements / dt, "unit": UNIT, "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"batch row 0 of {w.batch} ({dims} channels x full "
+                                          f"L={w.seqlen}), {reps} runs, fp64 reverse sweep, "
+                                          f"{cores} threads, {dt:.1f} s"}
     return line
 
 

@@ -114,18 +114,54 @@ struct BwdStage {
   float b[CF::SEL_PT], c[CF::SEL_PT];
 };
 
-template <class CF, bool with_grad>
-__device__ __forceinline__ void bwd_fetch(const BwdArgs& a, BwdStage<CF>& st, int64_t b,
-                                          int64_t d0, int64_t t0) {
-  using E = typename CF::Elem;
+// A thread's fixed element slots: staging slot r is activation element
+// (c, t) = (i / T, i % T) and B/C element (n, t) of every chunk, i = tid + r NT;
+// item slot it is (t, c) = (i / CH, i % CH).  Their row offsets, validity and
+// per-channel constants are computed once, so a chunk only adds t0.
+template <class CF>
+struct BwdSlots {
+  // staging slot r covers element (c, t) = (c0 + r NT/T, t_s) and B/C element
+  // (n0 + r NT/T, t_s): offsets are a base plus r times a row stride
+  int64_t act0, sel0, row;  // row = (NT / T) L
+  int c0, n0, t_s;
+  int64_t item[CF::IPT];    // (b dim + d) L + t of item slot it, or -1
+  float bias[CF::IPT], D[CF::IPT];
+};
+
+template <class CF>
+__device__ __forceinline__ void bwd_slots(const BwdArgs& a, int64_t b, int64_t d0,
+                                          BwdSlots<CF>& sl) {
+  static_assert(CF::NT % CF::T == 0, "staging slots advance by whole rows");
   const int64_t L = a.seqlen;
+  sl.c0 = threadIdx.x / CF::T;
+  sl.n0 = sl.c0;
+  sl.t_s = threadIdx.x - sl.c0 * CF::T;
+  sl.row = (int64_t)(CF::NT / CF::T) * L;
+  sl.act0 = (b * a.dim + d0 + sl.c0) * L + sl.t_s;
+  sl.sel0 = (b * CF::N + sl.n0) * L + sl.t_s;
+#pragma unroll
+  for (int it = 0; it < CF::IPT; ++it) {
+    const int i = threadIdx.x + it * CF::NT;
+    const int tt = i / CF::CH, c = i - tt * CF::CH;
+    const int64_t d = d0 + c;
+    const bool ok = (!CF::ITEM_GUARD || i < CF::ITEMS) && d < a.dim;
+    sl.item[it] = ok ? (b * a.dim + d) * L + tt : -1;
+    sl.bias[it] = (ok && a.delta_bias) ? __ldg(a.delta_bias + d) : 0.f;
+    sl.D[it] = (ok && a.D) ? __ldg(a.D + d) : 0.f;
+  }
+}
+
+template <class CF, bool with_grad>
+__device__ __forceinline__ void bwd_fetch(const BwdArgs& a, BwdStage<CF>& st,
+                                          const BwdSlots<CF>& sl, int64_t d0, int64_t t0) {
+  using E = typename CF::Elem;
+  constexpr int RS = CF::NT / CF::T;  // rows per slot step
+  const bool t_in = t0 + sl.t_s < a.seqlen;
 #pragma unroll
   for (int r = 0; r < CF::ACT_PT; ++r) {
-    const int i = threadIdx.x + r * CF::NT;
-    const int c = i / CF::T, tt = i - c * CF::T;
-    const int64_t d = d0 + c, t = t0 + tt;
-    const bool in = i < CF::CH * CF::T && d < a.dim && t < L;
-    const int64_t off = (b * a.dim + d) * L + t;
+    const int c = sl.c0 + r * RS;
+    const bool in = t_in && c < CF::CH && d0 + c < a.dim;
+    const int64_t off = sl.act0 + r * sl.row + t0;
     st.u[r] = in ? ld_elem(static_cast<const E*>(a.u), off) : 0.f;
     st.dl[r] = in ? ld_elem(static_cast<const E*>(a.delta), off) : 0.f;
     if (with_grad) {
@@ -135,11 +171,8 @@ __device__ __forceinline__ void bwd_fetch(const BwdArgs& a, BwdStage<CF>& st, in
   }
 #pragma unroll
   for (int r = 0; r < CF::SEL_PT; ++r) {
-    const int i = threadIdx.x + r * CF::NT;
-    const int n = i / CF::T, tt = i - n * CF::T;
-    const int64_t t = t0 + tt;
-    const bool in = i < CF::N * CF::T && t < L;
-    const int64_t off = (b * CF::N + n) * L + t;
+    const bool in = t_in && sl.n0 + r * RS < CF::N;
+    const int64_t off = sl.sel0 + r * sl.row + t0;
     st.b[r] = in ? ld_elem(static_cast<const E*>(a.B), off) : 0.f;
     if (with_grad) st.c[r] = in ? ld_elem(static_cast<const E*>(a.C), off) : 0.f;
   }
@@ -170,10 +203,10 @@ __device__ __forceinline__ void bwd_store(const BwdStage<CF>& st, float* sm) {
   }
 }
 
-// Per (step, channel) item: Delta (0 on padding), Delta u, softplus'(x).
-// Items are channel-fastest: item i is (t, c) = (i / CH, i % CH).
-template <class CF>
-__device__ __forceinline__ void bwd_discretise(const BwdArgs& a, float* sm, int64_t d0,
+// Per (step, channel) item: Delta (0 on padding), Delta u and (with_grad)
+// softplus'(x).  Items are channel-fastest: item i is (t, c) = (i / CH, i % CH).
+template <class CF, bool with_grad>
+__device__ __forceinline__ void bwd_discretise(const BwdArgs& a, float* sm, const BwdSlots<CF>& sl,
                                                int64_t t0) {
 #pragma unroll
   for (int it = 0; it < CF::IPT; ++it) {
@@ -181,13 +214,12 @@ __device__ __forceinline__ void bwd_discretise(const BwdArgs& a, float* sm, int6
     if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
     const int tt = i / CF::CH, c = i - tt * CF::CH;
     const int o = tt * CF::CHP + c;
-    const int64_t d = d0 + c;
-    const bool in = d < a.dim && t0 + tt < a.seqlen;
-    const float x = sm[CF::OFF_DL + o] + ((a.delta_bias && d < a.dim) ? __ldg(a.delta_bias + d) : 0.f);
+    const bool in = sl.item[it] >= 0 && t0 + tt < a.seqlen;
+    const float x = sm[CF::OFF_DL + o] + sl.bias[it];
     const float dl = in ? (a.softplus ? softplus_fast(x) : x) : 0.f;
     sm[CF::OFF_DL + o] = dl;
     sm[CF::OFF_W + o] = dl * sm[CF::OFF_U + o];
-    sm[CF::OFF_SG + o] = a.softplus ? sigmoid_fast(x) : 1.f;
+    if (with_grad) sm[CF::OFF_SG + o] = a.softplus ? sigmoid_fast(x) : 1.f;
   }
 }
 
@@ -227,6 +259,8 @@ __global__ void __launch_bounds__(CF::NT)
     A2[p] = make_float2(a0 * 1.4426950408889634f, a1 * 1.4426950408889634f);
   }
   BwdStage<CF> st;
+  BwdSlots<CF> sl;
+  bwd_slots<CF>(a, b, d0, sl);
   auto ex2_pair = [](float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); };
   auto ld_pairs = [](const float* p, float2 (&v)[2]) {
     const float4 q = *reinterpret_cast<const float4*>(p);
@@ -241,13 +275,13 @@ __global__ void __launch_bounds__(CF::NT)
 
   // ---- pass 1: forward, checkpoint the state at every chunk start ----
   float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  bwd_fetch<CF, false>(a, st, b, d0, 0);
+  bwd_fetch<CF, false>(a, st, sl, d0, 0);
   for (int64_t k = 0; k < nk; ++k) {
     st_pairs(ck_lane + k * CF::STEP_FLOATS, h);
     bwd_store<CF, false>(st, sm);
-    if (k + 1 < nk) bwd_fetch<CF, false>(a, st, b, d0, (k + 1) * T);
+    if (k + 1 < nk) bwd_fetch<CF, false>(a, st, sl, d0, (k + 1) * T);
     __syncthreads();
-    bwd_discretise<CF>(a, sm, d0, k * T);
+    bwd_discretise<CF, false>(a, sm, sl, k * T);
     __syncthreads();
 #pragma unroll 4
     for (int t = 0; t < T; ++t) {
@@ -274,7 +308,7 @@ __global__ void __launch_bounds__(CF::NT)
 #pragma unroll
   for (int it = 0; it < CF::IPT; ++it) dD_acc[it] = db_acc[it] = 0.f;
 
-  bwd_fetch<CF, true>(a, st, b, d0, (nk - 1) * T);
+  bwd_fetch<CF, true>(a, st, sl, d0, (nk - 1) * T);
   float2 ck_next[2];  // the checkpoint of the chunk to come, loaded a chunk early
   ld_pairs(ck_lane + (nk - 1) * CF::STEP_FLOATS, ck_next);
   for (int64_t k = nk - 1; k >= 0; --k) {
@@ -282,11 +316,11 @@ __global__ void __launch_bounds__(CF::NT)
     const float2 h_start[2] = {ck_next[0], ck_next[1]};
     bwd_store<CF, true>(st, sm);
     if (k > 0) {
-      bwd_fetch<CF, true>(a, st, b, d0, (k - 1) * T);
+      bwd_fetch<CF, true>(a, st, sl, d0, (k - 1) * T);
       ld_pairs(ck_lane + (k - 1) * CF::STEP_FLOATS, ck_next);
     }
     __syncthreads();
-    bwd_discretise<CF>(a, sm, d0, t0);
+    bwd_discretise<CF, true>(a, sm, sl, t0);
     __syncthreads();
     // recompute the chunk's states from its checkpoint; channel readouts
     float2 hs[2] = {h_start[0], h_start[1]};
@@ -315,18 +349,16 @@ __global__ void __launch_bounds__(CF::NT)
       if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
       const int tt = i / CF::CH, ci = i - tt * CF::CH;
       const int o = tt * CHP + ci;
-      const int64_t di = d0 + ci, t = t0 + tt;
-      const bool in = di < a.dim && t < L;
-      const float Dd = (a.D && di < a.dim) ? __ldg(a.D + di) : 0.f;
+      const bool in = sl.item[it] >= 0 && t0 + tt < L;
       const float uu = sm[CF::OFF_U + o];
-      const float q = sm[CF::OFF_P1 + o] + Dd * uu;
+      const float q = sm[CF::OFF_P1 + o] + sl.D[it] * uu;
       const float dy = sm[CF::OFF_DY + o];
       float dq = dy;
       if (a.z) {
         const float zz = sm[CF::OFF_Z + o];
         const float sg = sigmoid_fast(zz);
         dq = dy * zz * sg;
-        if (in) a.dz[(b * a.dim + di) * L + t] = dy * q * sg * (1.f + zz * (1.f - sg));
+        if (in) a.dz[sl.item[it] + t0] = dy * q * sg * (1.f + zz * (1.f - sg));
       }
       sm[CF::OFF_DY + o] = dq;
       if (in) dD_acc[it] = fmaf(dq, uu, dD_acc[it]);
@@ -398,13 +430,11 @@ __global__ void __launch_bounds__(CF::NT)
       if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
       const int tt = i / CF::CH, ci = i - tt * CF::CH;
       const int o = tt * CHP + ci;
-      const int64_t di = d0 + ci, t = t0 + tt;
-      if (di >= a.dim || t >= L) continue;
-      const float Dd = a.D ? __ldg(a.D + di) : 0.f;
+      if (sl.item[it] < 0 || t0 + tt >= L) continue;
       const float dx = sm[CF::OFF_P1 + o] * sm[CF::OFF_SG + o];
-      const int64_t off = (b * a.dim + di) * L + t;
+      const int64_t off = sl.item[it] + t0;
       a.ddelta[off] = dx;
-      a.du[off] = fmaf(sm[CF::OFF_DY + o], Dd, sm[CF::OFF_P2 + o]);
+      a.du[off] = fmaf(sm[CF::OFF_DY + o], sl.D[it], sm[CF::OFF_P2 + o]);
       db_acc[it] += dx;
     }
     __syncthreads();
