@@ -170,10 +170,10 @@ def test_device_error_word_clear():
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("L", [7, 100, 1001, 2048])
-def test_wide_shapes_warp_specialised_path(dtype, L):
+def test_wide_shapes_channel_parallel_path(dtype, L):
     """Enough channel groups (5 x ceil(1000/32) = 160) to fill the SMs, so N = 16
-    runs the warp-specialised kernel: partial last channel tile, ragged tails,
-    odd L (element-wise loads)."""
+    runs the channel-parallel kernel rather than the time split: partial last
+    channel tile, ragged tails, odd L (element-wise loads)."""
     w = I.Workload(f"wide_{dtype}_L{L}", 5, 1000, L, 16, dtype)
     rng = np.random.default_rng(L)
     channels = np.unique(np.concatenate([[0, 999, 1000, 4999], rng.choice(5000, 300, replace=False)]))
