@@ -85,6 +85,14 @@ def test_bwd_medium_workload():
     _run(w, x, _dy(w, 12))
 
 
+def test_bwd_full_workload():
+    # the bench workload, every gradient element (the oracle's reverse sweep over
+    # 12288 channels x 2048 steps takes about a minute of host time)
+    w = I.WORKLOADS["b8_l2048_d1536_n16_bf16"]
+    x = I.make_inputs(w, seed=31)
+    _run(w, x, _dy(w, 32))
+
+
 def test_bwd_workspace_too_small():
     w = I.Workload("bwdws", 1, 32, 64, 16, "f32")
     xd = to_device(I.make_inputs(w, seed=1))
