@@ -376,33 +376,53 @@ def run_step_arm(args, w: I.Workload):
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
 
-    # end to end: the token's inputs from pinned host memory, the step, y back;
-    # the carried state lives on the device between tokens
+    # end to end: each token's inputs from pinned host memory, the step, y back;
+    # the carried state lives on the device between tokens.  Uploads and
+    # downloads run on their own streams with two buffer sets, so token i+1's
+    # upload and token i-1's download overlap token i's step.
     tok_keys = ("u", "delta", "z", "B", "C")
     pinned = {k: (torch.from_numpy(host[0][k].view(np.int16)).view(torch.bfloat16)
                   if host[0][k].dtype == np.uint16 else torch.from_numpy(host[0][k])).pin_memory()
               for k in tok_keys if host[0][k] is not None}
-    y_host = torch.empty((w.batch, w.dim), dtype=torch.float32).pin_memory()
+    y_host = [torch.empty((w.batch, w.dim), dtype=torch.float32).pin_memory() for _ in range(2)]
     x0 = sets[0]
-    dbuf = {k: torch.empty_like(v, device=dev) for k, v in pinned.items()}
+    dbuf = [{k: torch.empty_like(v, device=dev) for k, v in pinned.items()} for _ in range(2)]
+    ye = [ys[0], torch.empty_like(ys[0])]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_done = [torch.cuda.Event(), torch.cuda.Event()]
+    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
+    out_done = [torch.cuda.Event(), torch.cuda.Event()]
+    for e in comp_done + out_done:
+        e.record(stream)
 
-    def e2e_step():
-        for k, v in pinned.items():
-            dbuf[k].copy_(v, non_blocking=True)
-        y = ss_scan_step(x0["state"], dbuf["u"], dbuf["delta"], x0["A"], dbuf["B"], dbuf["C"],
-                         D=x0["D"], z=dbuf.get("z"), delta_bias=x0["delta_bias"], softplus=w.softplus,
-                         y_out=ys[0], stream=stream)
-        y_host.copy_(y, non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        s_in.wait_event(comp_done[j])  # dbuf[j] was read by token i-2's step
+        with torch.cuda.stream(s_in):
+            for k, v in pinned.items():
+                dbuf[j][k].copy_(v, non_blocking=True)
+        in_done[j].record(s_in)
+        stream.wait_event(in_done[j])
+        stream.wait_event(out_done[j])  # ye[j] was read by token i-2's download
+        d = dbuf[j]
+        ss_scan_step(x0["state"], d["u"], d["delta"], x0["A"], d["B"], d["C"], D=x0["D"],
+                     z=d.get("z"), delta_bias=x0["delta_bias"], softplus=w.softplus, y_out=ye[j],
+                     stream=stream)
+        comp_done[j].record(stream)
+        s_out.wait_event(comp_done[j])
+        with torch.cuda.stream(s_out):
+            y_host[j].copy_(ye[j], non_blocking=True)
+        out_done[j].record(s_out)
 
     n_e2e = max(3, min(args.steps, 50))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
-    f1.record(stream)
+    f0.record(s_in)
+    for i in range(n_e2e):
+        e2e_step(i)
+    f1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = f0.elapsed_time(f1) / n_e2e
     chans = w.batch * w.dim
@@ -420,7 +440,7 @@ def run_step_arm(args, w: I.Workload):
                          "bytes_per_step": I.step_bytes(w), "peak_source": f"HBM copy, {p['source']}"},
             "e2e": {"value": chans / (e2e_ms * 1e-3), "unit": STEP_UNIT,
                     "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in pinned.values()),
-                    "d2h_bytes_per_step": y_host.numel() * 4},
+                    "d2h_bytes_per_step": y_host[0].numel() * 4},
             "gpu_launches": steps, "clocks": clk.summary()}
     if not args.no_cpu_baseline:
         import oracle
@@ -536,7 +556,7 @@ def run_bwd_arm(args, w: I.Workload):
     return line
 
 
-def roofline(w: I.Workload, kernel_ms: float):
+def roofline(w: I.Workload, kernel_ms: float, variant: str = ""):
     p = peaks()
     t_hbm = w.algorithmic_bytes() / (p["hbm_gbs"] * 1e9)
     sfu_rate = NUM_SMS * MUFU_EX2_PER_CLK_PER_SM * p["sm_max_mhz"] * 1e6  # ex2 per second
@@ -550,7 +570,7 @@ def roofline(w: I.Workload, kernel_ms: float):
         achieved = w.algorithmic_bytes() / s / 1e9
         r = {"bound": "hbm", "achieved": achieved, "peak": p["hbm_gbs"], "unit": "GB/s"}
     r["frac"] = r["achieved"] / r["peak"]
-    r["traffic"] = profiled_traffic(w.name)
+    r["traffic"] = profiled_traffic(w.name + variant)
     r["peak_source"] = (f"SFU: {NUM_SMS} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
                         f"{p['sm_max_mhz']:.0f} MHz" if r["bound"] == "alu"
                         else f"HBM copy, {p['source']}")
@@ -667,7 +687,7 @@ def main():
     r = run_gpu_arm(args, w)
     if r["rank"] != 0:
         return
-    roof = roofline(w, r["ms_per_step"])
+    roof = roofline(w, r["ms_per_step"], f"+conv{args.conv}" if args.conv else ("+zoh" if args.zoh else ""))
     line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": r["world"],
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
