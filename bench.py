@@ -497,10 +497,21 @@ def run_bwd_arm(args, w: I.Workload):
     ws = torch.empty(ss_scan_bwd_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate),
                      dtype=torch.uint8, device=dev)
 
+    cks = [None] * nsets
+    if args.ckpt:  # checkpoints from the training forward (not timed: the forward's work)
+        from selective_state_space_ss_b200 import ss_scan_fwd_train
+
+        for s_ in range(nsets):
+            x = sets[s_]
+            _, _, cks[s_] = ss_scan_fwd_train(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"],
+                                              z=x["z"], delta_bias=x["delta_bias"],
+                                              softplus=w.softplus, stream=stream)
+
     def step(i):
         x = sets[i % nsets]
         ss_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], dys[i % nsets], D=x["D"], z=x["z"],
-                    delta_bias=x["delta_bias"], softplus=w.softplus, workspace=ws, stream=stream)
+                    delta_bias=x["delta_bias"], softplus=w.softplus, checkpoints=cks[i % nsets],
+                    workspace=ws, stream=stream)
 
     for i in range(args.warmup):
         step(i)
@@ -520,10 +531,13 @@ def run_bwd_arm(args, w: I.Workload):
     line = {"metric": BWD_METRIC, "value": w.elements / (ms * 1e-3), "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": dict(config_of(w, 1), op="backward"),
+            "config": dict(config_of(w, 1), op="backward",
+                           checkpoints="from the training forward" if args.ckpt
+                           else "computed by the backward"),
             "roofline": {"bound": "alu", "achieved": achieved, "peak": sfu_rate / 1e9, "unit": "Gexp2/s",
                          "frac": achieved * 1e9 / sfu_rate,
-                         "traffic": profiled_traffic(w.name + "+bwd", BWD_KERNEL_SOURCES),
+                         "traffic": profiled_traffic(w.name + ("+bwdck" if args.ckpt else "+bwd"),
+                                                     BWD_KERNEL_SOURCES),
                          "exps_per_step": exps, "hbm_bytes_per_step": bwd_bytes(w),
                          "hbm_frac": bwd_bytes(w) / (ms * 1e-3) / 1e9 / p["hbm_gbs"]},
             "gpu_launches": args.steps, "clocks": clk.summary()}
@@ -655,6 +669,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--zoh", action="store_true", help="exact zero-order-hold B_bar")
+    ap.add_argument("--ckpt", action="store_true",
+                    help="--op bwd: start from checkpoints written by the training forward")
     ap.add_argument("--conv", type=int, default=0,
                     help="fuse the short causal conv1d + SiLU of this width (1-4) into the scan")
     args = ap.parse_args()

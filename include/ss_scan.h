@@ -194,6 +194,27 @@ ss_status ss_scan_step(const void* u, const void* delta, const float* A,
                        int dstate, ss_dtype in_dtype, cudaStream_t stream);
 
 /*
+ * ss_scan_fwd_train -- ss_scan_fwd that also writes the state at the start of
+ * every 16-step chunk, for ss_scan_bwd to start its recomputation from
+ * instead of running its own forward pass first (the states within a chunk
+ * are still recomputed, never stored).
+ *
+ *  checkpoints  [batch, ceil(seqlen / 16), dim, dstate] float32, 16-byte
+ *               aligned, caller-owned (required): checkpoints[b, k, d, n] = h[n]
+ *               of channel (b, d) before step 16 k (zero for k = 0).
+ *
+ * Every other argument, layout, result and error is that of ss_scan_fwd.
+ */
+ss_status ss_scan_fwd_train(const void* u, const void* delta, const float* A,
+                            const void* B, const void* C, const float* D,
+                            const void* z, const float* delta_bias,
+                            int softplus_flag, float* y_out, float* last_state_out,
+                            float* checkpoints, int64_t batch, int64_t dim,
+                            int64_t seqlen, int dstate, ss_dtype in_dtype,
+                            void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
+
+/*
  * ss_scan_bwd -- gradients of ss_scan_fwd (simplified B_bar, zero initial
  * state) for an upstream gradient dy of y (and optionally dlast_state of the
  * final state).  The forward's states are not stored anywhere: the backward
@@ -212,28 +233,33 @@ ss_status ss_scan_step(const void* u, const void* delta, const float* A,
  *   dD[d]    = sum_{b,t} dq u,   ddelta_bias[d] = sum_{b,t} ddelta
  *
  * Inputs exactly as ss_scan_fwd; dy [batch, dim, seqlen] float32 (required);
- * dlast_state [batch, dim, dstate] float32 (nullable: 0).  Outputs, all
+ * dlast_state [batch, dim, dstate] float32 (nullable: 0); checkpoints: those
+ * ss_scan_fwd_train wrote for the same inputs (nullable: the call computes
+ * them itself into the workspace, and then needs it; with checkpoints the
+ * workspace may be null).  Outputs, all
  * float32 and overwritten: du, ddelta [batch, dim, seqlen] (required); dz
  * (required when z is given, ignored otherwise); dA [dim, dstate], dB, dC
  * [batch, dstate, seqlen] (required); dD (nullable; ignored without D),
  * ddelta_bias [dim] (nullable).  dA, dB, dC, dD and ddelta_bias are summed
  * with atomic adds after the call zeroes them on `stream` (so their low bits
- * may vary from call to call).  workspace: at least
+ * may vary from call to call).  workspace (without checkpoints): at least
  * ss_scan_bwd_workspace_bytes(...) bytes, 256-byte aligned, caller-owned.
  * Any element alignment; errors as ss_scan_fwd.
  */
 ss_status ss_scan_bwd(const void* u, const void* delta, const float* A,
                       const void* B, const void* C, const float* D,
                       const void* z, const float* delta_bias, int softplus_flag,
-                      const float* dy, const float* dlast_state, float* du,
+                      const float* dy, const float* dlast_state,
+                      const float* checkpoints, float* du,
                       float* ddelta, float* dA, float* dB, float* dC, float* dD,
                       float* dz, float* ddelta_bias, int64_t batch, int64_t dim,
                       int64_t seqlen, int dstate, ss_dtype in_dtype,
                       void* workspace, size_t workspace_bytes,
                       cudaStream_t stream);
 
-/* Bytes of workspace ss_scan_bwd needs: 16 bytes x batch x dim x dstate x
- * ceil(seqlen / 16) (rounded up), or (size_t)-1 for sizes it would reject. */
+/* Bytes of workspace ss_scan_bwd needs without given checkpoints, which is
+ * also the size of the checkpoint array: 4 x batch x ceil(seqlen / 16) x dim x
+ * dstate, rounded up to 256; (size_t)-1 for sizes it would reject. */
 size_t ss_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen,
                                    int dstate);
 

@@ -31,6 +31,7 @@ from ._native import (  # noqa: F401
     ss_scan_fwd_conv,
     ss_scan_fwd_from_state,
     ss_scan_fwd_noalloc,
+    ss_scan_fwd_train,
     ss_scan_fwd_zoh,
     ss_scan_step,
     ss_scan_workspace_bytes,

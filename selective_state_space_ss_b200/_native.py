@@ -24,7 +24,7 @@ SS_F32, SS_BF16 = 0, 1
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
             "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc",
             "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv", "ss_scan_fwd_zoh",
-            "ss_scan_bwd", "ss_scan_bwd_workspace_bytes")
+            "ss_scan_bwd", "ss_scan_bwd_workspace_bytes", "ss_scan_fwd_train")
 
 # bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
 SS_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -80,7 +80,10 @@ def load_library():
         lib.ss_scan_fwd_zoh.argtypes = lib.ss_scan_fwd.argtypes
         lib.ss_scan_fwd_zoh.restype = ci
         lib.ss_scan_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp, vp, vp, vp,
-                                    vp, vp, vp, i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
+                                    vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
+        lib.ss_scan_fwd_train.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp,
+                                          i64, i64, i64, ci, ci, vp, ctypes.c_size_t, vp]
+        lib.ss_scan_fwd_train.restype = ci
         lib.ss_scan_bwd.restype = ci
         lib.ss_scan_bwd_workspace_bytes.argtypes = [i64, i64, i64, ci]
         lib.ss_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
@@ -179,6 +182,11 @@ def _fwd_call(name, initial_state, u, delta, A, B, C, D, z, delta_bias, softplus
         st = lib.ss_scan_fwd(*head, *tail)
     elif name == "ss_scan_fwd_zoh":
         st = lib.ss_scan_fwd_zoh(*head, *tail)
+    elif name == "ss_scan_fwd_train":
+        ck = initial_state
+        nk = (L + 15) // 16
+        _check_dev("checkpoints", ck, device, (torch.float32,), (batch, nk, dim, N))
+        st = lib.ss_scan_fwd_train(*head, tail[0], tail[1], _ptr(ck), *tail[2:])
     elif name == "ss_scan_fwd_conv":
         cw, cb = initial_state
         _check_dev("conv_weight", cw, device, (torch.float32,))
@@ -248,13 +256,32 @@ def ss_scan_bwd_workspace_bytes(batch: int, dim: int, seqlen: int, dstate: int) 
     return n
 
 
+def ss_scan_fwd_train(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                      y_out=None, last_state_out=None, checkpoints=None, return_last_state=True,
+                      workspace=None, stream=None):
+    """ss_scan_fwd that also writes the state at every 16-step chunk start.
+
+    Returns (y, last_state, checkpoints); checkpoints [batch, ceil(L/16), dim,
+    N] float32 (allocated with torch when not given) feed ss_scan_bwd.
+    """
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    if checkpoints is None:
+        checkpoints = torch.empty((batch, (L + 15) // 16, dim, N), dtype=torch.float32,
+                                  device=u.device)
+    y, h = _fwd_call("ss_scan_fwd_train", checkpoints, u, delta, A, B, C, D, z, delta_bias,
+                     softplus, y_out, last_state_out, return_last_state, workspace, stream)
+    return y, h, checkpoints
+
+
 def ss_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=True,
-                dlast_state=None, workspace=None, stream=None):
+                dlast_state=None, checkpoints=None, workspace=None, stream=None):
     """Gradients of ss_scan_fwd for an upstream dy [batch, dim, L] float32.
 
     Returns a dict of float32 tensors: du, ddelta, dz (None without z), dA
     [dim, N], dB, dC [batch, N, L], dD (None without D), ddelta_bias (None
-    without delta_bias).  The states are recomputed, not stored.
+    without delta_bias).  The states are recomputed, not stored; checkpoints
+    from ss_scan_fwd_train (optional) spare the call its own forward pass.
     """
     lib = load_library()
     device, batch, dim, L, N = _fwd_operands(u, delta, A, B, C, D, z, delta_bias)
@@ -267,14 +294,15 @@ def ss_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus
          "dC": torch.empty((batch, N, L), **f32),
          "dD": torch.empty((dim,), **f32) if D is not None else None,
          "ddelta_bias": torch.empty((dim,), **f32) if delta_bias is not None else None}
-    need = ss_scan_bwd_workspace_bytes(batch, dim, L, N)
-    if workspace is None:
+    _check_dev("checkpoints", checkpoints, device, (torch.float32,), (batch, (L + 15) // 16, dim, N))
+    if workspace is None and checkpoints is None:
+        need = ss_scan_bwd_workspace_bytes(batch, dim, L, N)
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
-    ws_bytes = workspace.numel() * workspace.element_size()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     dt = SS_F32 if u.dtype == torch.float32 else SS_BF16
     st = lib.ss_scan_bwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
                          _ptr(delta_bias), int(bool(softplus)), _ptr(dy), _ptr(dlast_state),
-                         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]),
+                         _ptr(checkpoints), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]),
                          _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddelta_bias"]),
                          batch, dim, L, N, dt, _ptr(workspace), ws_bytes,
                          _stream_handle(stream, device))

@@ -5,8 +5,8 @@
 // them).  One CTA owns CH channels of one batch row and the whole sequence:
 //
 //  pass 1  forward over the sequence, writing only the state at the start of
-//          every chunk of T steps to the caller's workspace (CH x N floats
-//          per chunk);
+//          every chunk of T steps to the caller's workspace (skipped when the
+//          training forward has written these checkpoints);
 //  pass 2  over the chunks in reverse: recompute the chunk's states h_t from
 //          its checkpoint into shared memory, then run the adjoint
 //          g_t = dq_t C_t + a_{t+1} g_{t+1} backwards through the chunk with
@@ -50,7 +50,8 @@ struct BwdArgs {
   float* dC;                // [batch, N, L], accumulated
   float* dD;                // [dim], accumulated, nullable
   float* dbias;             // [dim], accumulated, nullable
-  float* ckpt;              // workspace: [CTAs][chunks][CH * N]
+  float* ckpt;              // [batch][chunks][dim][N]: state at each 16-step chunk start
+  int ckpt_given;           // 1: written by the training forward (pass 1 is skipped)
   int64_t batch, dim, seqlen;
   int softplus;
 };
@@ -246,7 +247,9 @@ __global__ void __launch_bounds__(CF::NT)
   const int j = lane % K;                   // its state group
   const int64_t d = d0 + c;
   const bool chan_ok = d < a.dim;
-  float* ck = a.ckpt + (int64_t)blockIdx.x * nk * CF::STEP_FLOATS;
+  // this lane's states in checkpoint k: ckpt[b][k][d][j G ..]
+  const int64_t ck_stride = a.dim * N;
+  float* ck_lane = a.ckpt + (b * nk * a.dim + d) * N + j * G;
   float* hb = sm + CF::OFF_H;
 
   // decay constants of this lane's four states, as two packed pairs
@@ -270,14 +273,14 @@ __global__ void __launch_bounds__(CF::NT)
   auto st_pairs = [](float* p, const float2 (&v)[2]) {
     *reinterpret_cast<float4*>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
   };
-  float* ck_lane = ck + c * N + j * G;        // this lane's slot in every checkpoint
   float* hb_lane = hb + c * N + j * G;        // and in every step row of hb
 
   // ---- pass 1: forward, checkpoint the state at every chunk start ----
+  // (skipped when the training forward has written the checkpoints)
   float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  bwd_fetch<CF, false>(a, st, sl, d0, 0);
-  for (int64_t k = 0; k < nk; ++k) {
-    st_pairs(ck_lane + k * CF::STEP_FLOATS, h);
+  if (!a.ckpt_given) bwd_fetch<CF, false>(a, st, sl, d0, 0);
+  for (int64_t k = 0; k < nk && !a.ckpt_given; ++k) {
+    if (chan_ok) st_pairs(ck_lane + k * ck_stride, h);
     bwd_store<CF, false>(st, sm);
     if (k + 1 < nk) bwd_fetch<CF, false>(a, st, sl, d0, (k + 1) * T);
     __syncthreads();
@@ -309,15 +312,17 @@ __global__ void __launch_bounds__(CF::NT)
   for (int it = 0; it < CF::IPT; ++it) dD_acc[it] = db_acc[it] = 0.f;
 
   bwd_fetch<CF, true>(a, st, sl, d0, (nk - 1) * T);
-  float2 ck_next[2];  // the checkpoint of the chunk to come, loaded a chunk early
-  ld_pairs(ck_lane + (nk - 1) * CF::STEP_FLOATS, ck_next);
+  float2 ck_next[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  // the checkpoint of the chunk to come, loaded a chunk early (the same thread
+  // wrote it in pass 1, or the training forward did before this launch)
+  if (chan_ok) ld_pairs(ck_lane + (nk - 1) * ck_stride, ck_next);
   for (int64_t k = nk - 1; k >= 0; --k) {
     const int64_t t0 = k * T;
     const float2 h_start[2] = {ck_next[0], ck_next[1]};
     bwd_store<CF, true>(st, sm);
     if (k > 0) {
       bwd_fetch<CF, true>(a, st, sl, d0, (k - 1) * T);
-      ld_pairs(ck_lane + (k - 1) * CF::STEP_FLOATS, ck_next);
+      if (chan_ok) ld_pairs(ck_lane + (k - 1) * ck_stride, ck_next);
     }
     __syncthreads();
     bwd_discretise<CF, true>(a, sm, sl, t0);

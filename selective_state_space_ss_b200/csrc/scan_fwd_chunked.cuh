@@ -54,6 +54,9 @@ struct FwdArgs {
   const float* conv_w;
   const float* conv_b;  // nullable
   int conv_width;
+  // training checkpoints: the state at the start of every 16-step chunk,
+  // [batch][ceil(L / 16)][dim][N] fp32 (nullable: not written)
+  float* ckpt;
   int64_t batch, dim, seqlen;
   int softplus;
   int vec;  // 1: TMA path (16-byte aligned rows); 0: element-wise loads
@@ -68,15 +71,26 @@ struct FwdMaps {
 constexpr uint32_t kTmaSpinLimit = 1u << 24;
 constexpr int kConvTaps = 4;  // widest fused convolution
 
+// Where this lane writes training checkpoints for the current chunk: its
+// states' slot in the chunk's first 16-step checkpoint (null: none), the
+// distance to the next checkpoint, and the steps of the sequence left from
+// the chunk start.
+struct CkptCtx {
+  float* p;
+  int64_t stride;
+  int64_t left;
+};
+
 // Tin: input dtype; N: states per channel; K: lanes per channel; NWARPS: warps
 // per CTA; T: timesteps per chunk; WT: warps that split each chunk in time
 // (1: every warp walks the whole chunk for its own channels; >1: WT warps
 // share one set of channels, each scanning T/WT consecutive steps of the
 // chunk, joined with the pages' associative operator).  CONV: the u input is
 // the pre-convolution x, staged with HALO earlier steps per row, and phase 1
-// forms u = SiLU(conv(x) + bias).  ZOH: exact zero-order-hold B_bar.
+// forms u = SiLU(conv(x) + bias).  ZOH: exact zero-order-hold B_bar.  TRAIN:
+// the state at every 16-step chunk start is written out for the backward.
 template <typename Tin, int N_, int K_, int NWARPS_, int T_, int WT_ = 1, bool CONV_ = false,
-          bool ZOH_ = false>
+          bool ZOH_ = false, bool TRAIN_ = false>
 struct ChunkedCfg {
   using Elem = Tin;
   static constexpr int N = N_;            // states per channel
@@ -94,6 +108,7 @@ struct ChunkedCfg {
   static constexpr int QPR = T / 4;                  // 4-step quads per row
   static constexpr bool CONV = CONV_;
   static constexpr bool ZOH = ZOH_;
+  static constexpr bool TRAIN = TRAIN_;
   // x steps staged before the chunk: >= kConvTaps - 1, and a whole number of
   // 16-byte units so that the shifted TMA box stays aligned
   static constexpr int HALO = CONV ? 8 : 0;
@@ -150,6 +165,8 @@ struct ChunkedCfg {
                 "TMA destinations 128-byte aligned");
   static_assert(!CONV || ((HALO * ES) % 16 == 0 && HALO >= kConvTaps - 1 && XT <= 256),
                 "convolution halo");
+  static_assert(T % 16 == 0 && (WT == 1 || 16 % TW == 0),
+                "16-step checkpoints fall on quad or warp-segment starts");
   static_assert(DW_BYTES % 16 == 0 && BC_BYTES % 16 == 0, "alignment");
   static_assert(ITEMS % NT == 0 || ITEMS < NT, "whole items per thread");
   static constexpr bool ITEM_GUARD = ITEMS < NT;  // some threads have no item
@@ -427,12 +444,18 @@ template <class CF>
 __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW, const float4* dwI,
                                        const unsigned char* bc, float* sy,
                                        float2 (&h)[CF::G / 2], const float2 (&a2)[CF::G / 2],
-                                       const float2 (&ia)[CF::G / 2], int c, int j) {
+                                       const float2 (&ia)[CF::G / 2], int c, int j,
+                                       const CkptCtx& ck) {
   constexpr int G2 = CF::G / 2;  // state pairs per lane
   const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
   float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE;
 #pragma unroll kPhase2Unroll
   for (int q = 0; q < CF::QPR; ++q) {
+    if (CF::TRAIN && ck.p && (q & 3) == 0 && 4 * q < ck.left) {  // the state before step 4q
+      float2* dst = reinterpret_cast<float2*>(ck.p + (q >> 2) * ck.stride);
+#pragma unroll
+      for (int g = 0; g < CF::G / 2; ++g) dst[g] = h[g];
+    }
     const float4 D4 = dwD[q * CF::DW_STRIDE + c];
     const float4 W4 = dwW[q * CF::DW_STRIDE + c];
     const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
@@ -485,7 +508,7 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
                                              float2 (&h)[CF::G / 2],
                                              const float2 (&a2)[CF::G / 2],
                                              const float2 (&ia)[CF::G / 2], int c, int j, int wt,
-                                             int lane_g) {
+                                             int lane_g, const CkptCtx& ck) {
   constexpr int G2 = CF::G / 2;
   const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
   float2 hl[G2], P[G2];
@@ -554,6 +577,13 @@ __device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dw
     const float2* vH = reinterpret_cast<const float2*>(aggH + (v * CF::WC * 32 + lane_g) * CF::G);
 #pragma unroll
     for (int g = 0; g < G2; ++g) h[g] = __ffma2_rn(vP[g], h[g], vH[g]);
+  }
+  // hin is the state before this warp's first step: a 16-step checkpoint when
+  // the segment starts on one
+  if (CF::TRAIN && ck.p && (wt * CF::TW) % 16 == 0 && wt * CF::TW < ck.left) {
+    float2* dst = reinterpret_cast<float2*>(ck.p + (wt * CF::TW / 16) * ck.stride);
+#pragma unroll
+    for (int g = 0; g < G2; ++g) dst[g] = hin[g];
   }
   float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE + wt * CF::TW;
 #pragma unroll
@@ -794,10 +824,21 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   const int lane_g = wc * 32 + lane;             // lane within its channel set
   const bool writer = wt == 0;  // time-split warps hold the same carry: one writes it
   float4* dwI = reinterpret_cast<float4*>(smem + CF::OFF_DWI);  // ZOH only
+  const int64_t ck_nk = (a.seqlen + 15) / 16;
+  // this lane's checkpoint slot for the chunk of batch row bb starting at t0
+  auto ckpt_at = [&](int64_t bb, int64_t dd, bool ok, int64_t t0) {
+    CkptCtx ck;
+    ck.stride = a.dim * CF::N;
+    ck.left = a.seqlen - t0;
+    ck.p = (CF::TRAIN && a.ckpt && ok)
+               ? a.ckpt + ((bb * ck_nk + t0 / 16) * a.dim + dd) * CF::N + j * CF::G
+               : nullptr;
+    return ck;
+  };
   auto run_phase2 = [&](float2 (&hh)[CF::G / 2], const float2 (&aa)[CF::G / 2],
-                        const float2 (&ii)[CF::G / 2]) {
-    if constexpr (CF::WT == 1) phase2<CF>(dwD, dwW, dwI, bc, sy, hh, aa, ii, c, j);
-    else phase2_split<CF>(dwD, dwW, dwI, bc, sy, aggP, aggH, hh, aa, ii, c, j, wt, lane_g);
+                        const float2 (&ii)[CF::G / 2], const CkptCtx& ck) {
+    if constexpr (CF::WT == 1) phase2<CF>(dwD, dwW, dwI, bc, sy, hh, aa, ii, c, j, ck);
+    else phase2_split<CF>(dwD, dwW, dwI, bc, sy, aggP, aggH, hh, aa, ii, c, j, wt, lane_g, ck);
   };
 
   if (tma && tid == 0) {
@@ -861,7 +902,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     run_phase1(0);
     __syncthreads();
     for (int64_t k = 0; k < nseq; ++k) {
-      run_phase2(h, a2, ia);
+      run_phase2(h, a2, ia, ckpt_at(b, d, chan_ok, k * CF::T));
       if (k + 1 < nseq) stage_in(k + 1);
       if (!__syncthreads_and(ok)) {
         drain(k + 1, k + 1);
@@ -985,7 +1026,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
       }
       ok = ok && have;
     }
-    run_phase2(h, a2, ia);
+    run_phase2(h, a2, ia, ckpt_at(cur.b, d, chan_ok, (int64_t)cur.c * CF::T));
     const bool cout_here = cur.carry_out();
     if (cout_here && writer) {
       float* dst = sched.carries + (int64_t)w * CF::CH * CF::N + c * CF::N + j * CF::G;

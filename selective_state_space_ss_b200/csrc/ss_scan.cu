@@ -192,8 +192,8 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
 #define SS_N16_T 32
 #endif
 
-template <typename E, bool CV = false, bool Z = false>
-using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, 1, CV, Z>;
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, 1, CV, Z, TR>;
 #ifndef SS_N32_K
 #define SS_N32_K 4
 #endif
@@ -203,8 +203,8 @@ using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, 1, CV, Z>;
 #ifndef SS_N32_T
 #define SS_N32_T 32
 #endif
-template <typename E, bool CV = false, bool Z = false>
-using Cfg32 = ChunkedCfg<E, 32, SS_N32_K, SS_N32_W, SS_N32_T, 1, CV, Z>;
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Cfg32 = ChunkedCfg<E, 32, SS_N32_K, SS_N32_W, SS_N32_T, 1, CV, Z, TR>;
 #ifndef SS_N64_K
 #define SS_N64_K 4
 #endif
@@ -223,10 +223,10 @@ using Cfg32 = ChunkedCfg<E, 32, SS_N32_K, SS_N32_W, SS_N32_T, 1, CV, Z>;
 #ifndef SS_N128_T
 #define SS_N128_T 32
 #endif
-template <typename E, bool CV = false, bool Z = false>
-using Cfg64 = ChunkedCfg<E, 64, SS_N64_K, SS_N64_W, SS_N64_T, 1, CV, Z>;
-template <typename E, bool CV = false, bool Z = false>
-using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T, 1, CV, Z>;
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Cfg64 = ChunkedCfg<E, 64, SS_N64_K, SS_N64_W, SS_N64_T, 1, CV, Z, TR>;
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T, 1, CV, Z, TR>;
 
 // Time-split shapes for problems with too few channels to fill the GPU: one
 // warp's worth of channels (8) per CTA, 8 warps splitting each chunk in time.
@@ -239,10 +239,10 @@ using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T, 1, CV, Z>;
 #ifndef SS_SPLIT16_WT
 #define SS_SPLIT16_WT 8
 #endif
-template <typename E, bool CV = false, bool Z = false>
-using Split16 = ChunkedCfg<E, 16, 4, SS_SPLIT16_W, SS_SPLIT16_T, SS_SPLIT16_WT, CV, Z>;
-template <typename E, bool CV = false, bool Z = false>
-using Split32 = ChunkedCfg<E, 32, 4, 8, 32, 8, CV, Z>;
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Split16 = ChunkedCfg<E, 16, 4, SS_SPLIT16_W, SS_SPLIT16_T, SS_SPLIT16_WT, CV, Z, TR>;
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Split32 = ChunkedCfg<E, 32, 4, 8, 32, 8, CV, Z, TR>;
 
 // The time split costs ~1.5 extra instructions per (step, state); take it only
 // when the channel-parallel shape would leave SMs idle.
@@ -255,38 +255,38 @@ bool too_few_groups(int64_t batch, int64_t dim) {
   return groups < device_sms();
 }
 
-template <typename E, bool CV, bool Z>
+template <typename E, bool CV, bool Z, bool TR>
 ss_status dispatch_dtype(const FwdArgs& a, int N, void* ws, size_t wsb, cudaStream_t stream) {
   switch (N) {
     case 16:
-      if (too_few_groups<Cfg16<E, CV, Z>>(a.batch, a.dim))
-        return launch_chunked<Split16<E, CV, Z>>(a, ws, wsb, stream);
-      return launch_chunked<Cfg16<E, CV, Z>>(a, ws, wsb, stream);
+      if (too_few_groups<Cfg16<E, CV, Z, TR>>(a.batch, a.dim))
+        return launch_chunked<Split16<E, CV, Z, TR>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg16<E, CV, Z, TR>>(a, ws, wsb, stream);
     case 32:
-      if (too_few_groups<Cfg32<E, CV, Z>>(a.batch, a.dim))
-        return launch_chunked<Split32<E, CV, Z>>(a, ws, wsb, stream);
-      return launch_chunked<Cfg32<E, CV, Z>>(a, ws, wsb, stream);
-    case 64: return launch_chunked<Cfg64<E, CV, Z>>(a, ws, wsb, stream);
-    case 128: return launch_chunked<Cfg128<E, CV, Z>>(a, ws, wsb, stream);
+      if (too_few_groups<Cfg32<E, CV, Z, TR>>(a.batch, a.dim))
+        return launch_chunked<Split32<E, CV, Z, TR>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg32<E, CV, Z, TR>>(a, ws, wsb, stream);
+    case 64: return launch_chunked<Cfg64<E, CV, Z, TR>>(a, ws, wsb, stream);
+    case 128: return launch_chunked<Cfg128<E, CV, Z, TR>>(a, ws, wsb, stream);
     default: return SS_ERR_UNSUPPORTED;
   }
 }
 
-template <typename E, bool CV, bool Z>
+template <typename E, bool CV, bool Z, bool TR>
 bool plan_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N, size_t* bytes) {
   Plan p;
   bool ok = false;
   switch (N) {
     case 16:
-      ok = too_few_groups<Cfg16<E, CV, Z>>(batch, dim) ? make_plan<Split16<E, CV, Z>>(batch, dim, seqlen, &p)
-                                                    : make_plan<Cfg16<E, CV, Z>>(batch, dim, seqlen, &p);
+      ok = too_few_groups<Cfg16<E, CV, Z, TR>>(batch, dim) ? make_plan<Split16<E, CV, Z, TR>>(batch, dim, seqlen, &p)
+                                                    : make_plan<Cfg16<E, CV, Z, TR>>(batch, dim, seqlen, &p);
       break;
     case 32:
-      ok = too_few_groups<Cfg32<E, CV, Z>>(batch, dim) ? make_plan<Split32<E, CV, Z>>(batch, dim, seqlen, &p)
-                                                    : make_plan<Cfg32<E, CV, Z>>(batch, dim, seqlen, &p);
+      ok = too_few_groups<Cfg32<E, CV, Z, TR>>(batch, dim) ? make_plan<Split32<E, CV, Z, TR>>(batch, dim, seqlen, &p)
+                                                    : make_plan<Cfg32<E, CV, Z, TR>>(batch, dim, seqlen, &p);
       break;
-    case 64: ok = make_plan<Cfg64<E, CV, Z>>(batch, dim, seqlen, &p); break;
-    case 128: ok = make_plan<Cfg128<E, CV, Z>>(batch, dim, seqlen, &p); break;
+    case 64: ok = make_plan<Cfg64<E, CV, Z, TR>>(batch, dim, seqlen, &p); break;
+    case 128: ok = make_plan<Cfg128<E, CV, Z, TR>>(batch, dim, seqlen, &p); break;
   }
   *bytes = p.ws_bytes;
   return ok;
@@ -343,12 +343,12 @@ ss_status dispatch_step(const StepArgs& a, int N, bool vec, bool pipe, cudaStrea
   }
 }
 
-template <typename E, int N>
-size_t bwd_ws_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
-  using CF = BwdCfg<E, N>;
-  const int64_t ctas = batch * ((dim + CF::CH - 1) / CF::CH);
-  const int64_t nk = (seqlen + CF::T - 1) / CF::T;
-  return align256((size_t)ctas * (size_t)nk * CF::STEP_FLOATS * sizeof(float));
+// Checkpoints of the backward: the state at every 16-step chunk start,
+// [batch][ceil(L / 16)][dim][N] fp32.
+constexpr int kCkptSteps = 16;
+size_t ckpt_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N) {
+  const int64_t nk = (seqlen + kCkptSteps - 1) / kCkptSteps;
+  return align256((size_t)batch * (size_t)nk * (size_t)dim * (size_t)N * sizeof(float));
 }
 
 template <typename E, int N>
@@ -359,7 +359,8 @@ ss_status launch_bwd(const BwdArgs& a, size_t ws_bytes, cudaStream_t stream) {
     state = cudaFuncSetAttribute(scan_bwd_kernel<CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  CF::SMEM_BYTES) == cudaSuccess ? 1 : -1;
   if (state != 1) return SS_ERR_CUDA;
-  if (ws_bytes < bwd_ws_bytes<E, N>(a.batch, a.dim, a.seqlen)) return SS_ERR_INVALID_ARG;
+  static_assert(CF::T == kCkptSteps, "checkpoint spacing");
+  if (!a.ckpt_given && ws_bytes < ckpt_bytes(a.batch, a.dim, a.seqlen, N)) return SS_ERR_INVALID_ARG;
   const int64_t ctas = a.batch * ((a.dim + CF::CH - 1) / CF::CH);
   if (ctas > INT_MAX) return SS_ERR_INVALID_ARG;
   scan_bwd_kernel<CF><<<(unsigned)ctas, CF::NT, CF::SMEM_BYTES, stream>>>(a);
@@ -383,7 +384,8 @@ ss_status scan_fwd_impl(const void* u, const void* delta, const float* A, const 
                         int64_t batch, int64_t dim, int64_t seqlen, int dstate,
                         ss_dtype in_dtype, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream, const float* conv_w = nullptr,
-                        const float* conv_b = nullptr, int conv_width = 0, bool zoh = false) {
+                        const float* conv_b = nullptr, int conv_width = 0, bool zoh = false,
+                        float* ckpt = nullptr) {
   if (!u || !delta || !A || !B || !C || !y_out) return SS_ERR_INVALID_ARG;
   if (batch < 1 || dim < 1 || seqlen < 1) return SS_ERR_INVALID_ARG;
   if (in_dtype != SS_F32 && in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED;
@@ -406,6 +408,7 @@ ss_status scan_fwd_impl(const void* u, const void* delta, const float* A, const 
   a.A = A; a.D = D; a.delta_bias = delta_bias;
   a.y = y_out; a.last_state = last_state_out; a.h0 = h0;
   a.conv_w = conv_w; a.conv_b = conv_w ? conv_b : nullptr; a.conv_width = conv_w ? conv_width : 0;
+  a.ckpt = ckpt;
   a.batch = batch; a.dim = dim; a.seqlen = seqlen;
   a.softplus = softplus_flag != 0;
   bool vec = ((size_t)seqlen * es) % 16 == 0;
@@ -415,16 +418,22 @@ ss_status scan_fwd_impl(const void* u, const void* delta, const float* A, const 
   a.vec = vec ? 1 : 0;
 
   const bool f32 = in_dtype == SS_F32;
+  void* ws = workspace;
+  const size_t wsb = workspace_bytes;
   if (conv_w) {
-    if (f32) return dispatch_dtype<float, true, false>(a, dstate, workspace, workspace_bytes, stream);
-    return dispatch_dtype<__nv_bfloat16, true, false>(a, dstate, workspace, workspace_bytes, stream);
+    if (f32) return dispatch_dtype<float, true, false, false>(a, dstate, ws, wsb, stream);
+    return dispatch_dtype<__nv_bfloat16, true, false, false>(a, dstate, ws, wsb, stream);
   }
   if (zoh) {
-    if (f32) return dispatch_dtype<float, false, true>(a, dstate, workspace, workspace_bytes, stream);
-    return dispatch_dtype<__nv_bfloat16, false, true>(a, dstate, workspace, workspace_bytes, stream);
+    if (f32) return dispatch_dtype<float, false, true, false>(a, dstate, ws, wsb, stream);
+    return dispatch_dtype<__nv_bfloat16, false, true, false>(a, dstate, ws, wsb, stream);
   }
-  if (f32) return dispatch_dtype<float, false, false>(a, dstate, workspace, workspace_bytes, stream);
-  return dispatch_dtype<__nv_bfloat16, false, false>(a, dstate, workspace, workspace_bytes, stream);
+  if (ckpt) {
+    if (f32) return dispatch_dtype<float, false, false, true>(a, dstate, ws, wsb, stream);
+    return dispatch_dtype<__nv_bfloat16, false, false, true>(a, dstate, ws, wsb, stream);
+  }
+  if (f32) return dispatch_dtype<float, false, false, false>(a, dstate, ws, wsb, stream);
+  return dispatch_dtype<__nv_bfloat16, false, false, false>(a, dstate, ws, wsb, stream);
 }
 
 }  // namespace
@@ -471,17 +480,13 @@ size_t ss_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, i
   if (batch < 1 || dim < 1 || seqlen < 1 || !supported_dstate(dstate)) return (size_t)-1;
   if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
     return (size_t)-1;
-  switch (dstate) {  // the layout does not depend on the input dtype
-    case 16: return bwd_ws_bytes<float, 16>(batch, dim, seqlen);
-    case 32: return bwd_ws_bytes<float, 32>(batch, dim, seqlen);
-    case 64: return bwd_ws_bytes<float, 64>(batch, dim, seqlen);
-    default: return bwd_ws_bytes<float, 128>(batch, dim, seqlen);
-  }
+  return ckpt_bytes(batch, dim, seqlen, dstate);
 }
 
 ss_status ss_scan_bwd(const void* u, const void* delta, const float* A, const void* B,
                       const void* C, const float* D, const void* z, const float* delta_bias,
-                      int softplus_flag, const float* dy, const float* dlast_state, float* du,
+                      int softplus_flag, const float* dy, const float* dlast_state,
+                      const float* checkpoints, float* du,
                       float* ddelta, float* dA, float* dB, float* dC, float* dD, float* dz,
                       float* ddelta_bias, int64_t batch, int64_t dim, int64_t seqlen, int dstate,
                       ss_dtype in_dtype, void* workspace, size_t workspace_bytes,
@@ -503,7 +508,8 @@ ss_status ss_scan_bwd(const void* u, const void* delta, const float* A, const vo
                             ddelta_bias};
   for (const void* p : f_ptrs)
     if (p && !aligned(p, 4)) return SS_ERR_INVALID_ARG;
-  if (!workspace || !aligned(workspace, 256)) return SS_ERR_INVALID_ARG;
+  if (checkpoints ? !aligned(checkpoints, 16) : (!workspace || !aligned(workspace, 256)))
+    return SS_ERR_INVALID_ARG;
   // the sums over channels, steps and batch rows accumulate with atomics
   if (cudaMemsetAsync(dA, 0, (size_t)dim * dstate * 4, stream) != cudaSuccess ||
       cudaMemsetAsync(dB, 0, (size_t)(batch * dstate * seqlen) * 4, stream) != cudaSuccess ||
@@ -516,11 +522,24 @@ ss_status ss_scan_bwd(const void* u, const void* delta, const float* A, const vo
   a.A = A; a.D = D; a.delta_bias = delta_bias; a.dy = dy; a.dlast = dlast_state;
   a.du = du; a.ddelta = ddelta; a.dz = dz; a.dA = dA; a.dB = dB; a.dC = dC;
   a.dD = D ? dD : nullptr; a.dbias = ddelta_bias;
-  a.ckpt = static_cast<float*>(workspace);
+  a.ckpt = checkpoints ? const_cast<float*>(checkpoints) : static_cast<float*>(workspace);
+  a.ckpt_given = checkpoints != nullptr;
   a.batch = batch; a.dim = dim; a.seqlen = seqlen;
   a.softplus = softplus_flag != 0;
   if (in_dtype == SS_F32) return dispatch_bwd<float>(a, dstate, workspace_bytes, stream);
   return dispatch_bwd<__nv_bfloat16>(a, dstate, workspace_bytes, stream);
+}
+
+ss_status ss_scan_fwd_train(const void* u, const void* delta, const float* A, const void* B,
+                            const void* C, const float* D, const void* z,
+                            const float* delta_bias, int softplus_flag, float* y_out,
+                            float* last_state_out, float* checkpoints, int64_t batch, int64_t dim,
+                            int64_t seqlen, int dstate, ss_dtype in_dtype, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
+  if (!checkpoints || !aligned(checkpoints, 16)) return SS_ERR_INVALID_ARG;
+  return scan_fwd_impl(u, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, y_out,
+                       last_state_out, batch, dim, seqlen, dstate, in_dtype, workspace,
+                       workspace_bytes, stream, nullptr, nullptr, 0, false, checkpoints);
 }
 
 ss_status ss_scan_fwd_zoh(const void* u, const void* delta, const float* A, const void* B,
@@ -606,14 +625,16 @@ size_t ss_scan_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int d
   if (batch > (INT64_C(1) << 40) / dim || batch * dim > (INT64_C(1) << 62) / seqlen)
     return (size_t)-1;
   // enough for either input dtype and every kernel variant (plain, fused
-  // convolution, exact zero-order hold)
-  size_t need[6] = {0, 0, 0, 0, 0, 0};
-  if (!plan_bytes<float, false, false>(batch, dim, seqlen, dstate, &need[0]) ||
-      !plan_bytes<__nv_bfloat16, false, false>(batch, dim, seqlen, dstate, &need[1]) ||
-      !plan_bytes<float, true, false>(batch, dim, seqlen, dstate, &need[2]) ||
-      !plan_bytes<__nv_bfloat16, true, false>(batch, dim, seqlen, dstate, &need[3]) ||
-      !plan_bytes<float, false, true>(batch, dim, seqlen, dstate, &need[4]) ||
-      !plan_bytes<__nv_bfloat16, false, true>(batch, dim, seqlen, dstate, &need[5]))
+  // convolution, exact zero-order hold, training checkpoints)
+  size_t need[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (!plan_bytes<float, false, false, false>(batch, dim, seqlen, dstate, &need[0]) ||
+      !plan_bytes<__nv_bfloat16, false, false, false>(batch, dim, seqlen, dstate, &need[1]) ||
+      !plan_bytes<float, true, false, false>(batch, dim, seqlen, dstate, &need[2]) ||
+      !plan_bytes<__nv_bfloat16, true, false, false>(batch, dim, seqlen, dstate, &need[3]) ||
+      !plan_bytes<float, false, true, false>(batch, dim, seqlen, dstate, &need[4]) ||
+      !plan_bytes<__nv_bfloat16, false, true, false>(batch, dim, seqlen, dstate, &need[5]) ||
+      !plan_bytes<float, false, false, true>(batch, dim, seqlen, dstate, &need[6]) ||
+      !plan_bytes<__nv_bfloat16, false, false, true>(batch, dim, seqlen, dstate, &need[7]))
     return (size_t)-1;
   size_t m = 0;
   for (size_t v : need) m = v > m ? v : m;

@@ -163,12 +163,12 @@ def test_zoh_rejections(lib, over):
 
 def _call_bwd(lib, **over):
     a = dict(u=0x10000, delta=0x20000, A=0x30000, B=0x40000, C=0x50000, D=None, z=None,
-             bias=None, sp=1, dy=0x60000, dl=None, du=0x70000, dd=0x80000, dA=0x90000,
+             bias=None, sp=1, dy=0x60000, dl=None, ck=None, du=0x70000, dd=0x80000, dA=0x90000,
              dB=0xa0000, dC=0xb0000, dD=None, dz=None, db=None, batch=1, dim=1, L=8, N=16,
              dt=N.SS_F32, ws=0x100000, wsb=1 << 20)
     a.update(over)
     return lib.ss_scan_bwd(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
-                           a["sp"], a["dy"], a["dl"], a["du"], a["dd"], a["dA"], a["dB"], a["dC"],
+                           a["sp"], a["dy"], a["dl"], a["ck"], a["du"], a["dd"], a["dA"], a["dB"], a["dC"],
                            a["dD"], a["dz"], a["db"], a["batch"], a["dim"], a["L"], a["N"], a["dt"],
                            a["ws"], a["wsb"], None)
 
@@ -178,17 +178,26 @@ def _call_bwd(lib, **over):
     (dict(dB=None), N.SS_ERR_INVALID_ARG), (dict(z=0x110000), N.SS_ERR_INVALID_ARG),
     (dict(ws=None), N.SS_ERR_INVALID_ARG), (dict(ws=0x100010), N.SS_ERR_INVALID_ARG),
     (dict(N=12), N.SS_ERR_UNSUPPORTED), (dict(dt=3), N.SS_ERR_UNSUPPORTED),
-    (dict(L=0), N.SS_ERR_INVALID_ARG), (dict(dA=0x90002), N.SS_ERR_INVALID_ARG)])
+    (dict(L=0), N.SS_ERR_INVALID_ARG), (dict(dA=0x90002), N.SS_ERR_INVALID_ARG),
+    (dict(ck=0x120008), N.SS_ERR_INVALID_ARG)])
 def test_bwd_rejections(lib, over, status):
     assert _call_bwd(lib, **over) == status
+
+
+@pytest.mark.parametrize("ck", [None, 0x70008])
+def test_fwd_train_rejects_bad_checkpoints(lib, ck):
+    assert lib.ss_scan_fwd_train(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, None, None, 1,
+                                 0x60000, None, ck, 1, 1, 8, 16, N.SS_F32, None, 0,
+                                 None) == N.SS_ERR_INVALID_ARG
 
 
 def test_bwd_workspace_query(lib):
     assert lib.ss_scan_bwd_workspace_bytes(0, 1, 1, 16) == ctypes.c_size_t(-1).value
     assert lib.ss_scan_bwd_workspace_bytes(1, 1, 1, 24) == ctypes.c_size_t(-1).value
-    # 16 bytes per (batch, channel-tile slot, state group) per 16-step chunk, 256-aligned
+    # the checkpoint array: 4 bytes x batch x ceil(L/16) x dim x dstate, 256-aligned
     n = lib.ss_scan_bwd_workspace_bytes(8, 1536, 2048, 16)
-    assert n >= 8 * 1536 * 16 * 4 * 128 and n % 256 == 0
+    assert n == 8 * 128 * 1536 * 16 * 4
+    assert lib.ss_scan_bwd_workspace_bytes(1, 3, 17, 16) == 512  # 2 chunks x 3 x 16 x 4 = 384
 
 
 def test_workspace_query_rejects_bad_sizes(lib):

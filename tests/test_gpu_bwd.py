@@ -26,11 +26,17 @@ def _dy(w, seed):
     return I.fill(seed, 12, (w.batch, w.dim, w.seqlen))
 
 
-def _run(w, x, dy, dlast=None, softplus=True):
+def _run(w, x, dy, dlast=None, softplus=True, ckpt=False):
     xd = to_device(x)
+    checkpoints = None
+    if ckpt:  # the training forward writes the checkpoints the backward starts from
+        _, _, checkpoints = ss.ss_scan_fwd_train(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"],
+                                                 D=xd["D"], z=xd["z"], delta_bias=xd["delta_bias"],
+                                                 softplus=softplus)
     g = ss.ss_scan_bwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], torch.from_numpy(dy).cuda(),
                        D=xd["D"], z=xd["z"], delta_bias=xd["delta_bias"], softplus=softplus,
-                       dlast_state=None if dlast is None else torch.from_numpy(dlast).cuda())
+                       dlast_state=None if dlast is None else torch.from_numpy(dlast).cuda(),
+                       checkpoints=checkpoints)
     assert ss.ss_last_device_error() == ss.SS_OK
     r = oracle.scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
                         softplus=softplus, dy=dy.astype(np.float64),
@@ -47,13 +53,53 @@ def _run(w, x, dy, dlast=None, softplus=True):
     return errs
 
 
+@pytest.mark.parametrize("ckpt", [False, True])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("N", [16, 32, 64, 128])
 @pytest.mark.parametrize("L", [1, 15, 16, 17, 300])
-def test_bwd_small_shapes(dtype, N, L):
+def test_bwd_small_shapes(dtype, N, L, ckpt):
+    # 2 x 37 channels: the forward's time-split kernel writes the checkpoints
+    # for N <= 32, the channel-parallel one for N >= 64
     w = I.Workload(f"bwd_{dtype}_{N}_{L}", 2, 37, L, N, dtype)
     x = I.make_inputs(w, seed=L + N)
-    _run(w, x, _dy(w, L))
+    _run(w, x, _dy(w, L), ckpt=ckpt)
+
+
+@pytest.mark.parametrize("workers", [0, 3])
+@pytest.mark.parametrize("N", [16, 64])
+def test_bwd_checkpoints_from_wide_forward(workers, N):
+    # enough channel groups for the channel-parallel forward (and, forced, its
+    # balanced schedule) to write the checkpoints
+    w = I.Workload(f"bwdck_{N}_{workers}", 4, 1280, 200, N, "bf16")
+    x = I.make_inputs(w, seed=workers + N)
+    if workers:
+        ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, workers)
+    _run(w, x, _dy(w, 3), ckpt=True)
+
+
+@pytest.mark.parametrize("N,batch,dim", [(16, 2, 37), (16, 4, 1280), (128, 2, 40)])
+def test_fwd_train_checkpoints_are_states(N, batch, dim):
+    # checkpoint k holds the state before step 16 k: the oracle's final state of
+    # the first 16 k steps; y is that of the plain forward
+    L = 150
+    w = I.Workload("ckstates", batch, dim, L, N, "f32")
+    x = I.make_inputs(w, seed=N + dim)
+    xd = to_device(x)
+    y, h, ck = ss.ss_scan_fwd_train(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"],
+                                    z=xd["z"], delta_bias=xd["delta_bias"])
+    y0, h0 = ss.ss_scan_fwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"], z=xd["z"],
+                            delta_bias=xd["delta_bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0) and torch.equal(h, h0)
+    ck = ck.cpu().numpy()
+    assert ck.shape == (batch, 10, dim, N)
+    assert np.all(ck[:, 0] == 0.0)
+    for k in (1, 4, 9):
+        cut = {kk: (np.ascontiguousarray(v[:, :, :16 * k]) if kk in ("u", "delta", "z", "B", "C") else v)
+               for kk, v in x.items()}
+        _, hr = oracle.scan_fwd(cut["u"], cut["delta"], cut["A"], cut["B"], cut["C"], cut["D"],
+                                cut["z"], cut["delta_bias"])
+        assert rel_err(ck[:, k], hr) <= 1e-5
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -85,12 +131,12 @@ def test_bwd_medium_workload():
     _run(w, x, _dy(w, 12))
 
 
-def test_bwd_full_workload():
-    # the bench workload, every gradient element (the oracle's reverse sweep over
-    # 12288 channels x 2048 steps takes about a minute of host time)
+@pytest.mark.parametrize("ckpt", [False, True])
+def test_bwd_full_workload(ckpt):
+    # the bench workload, every gradient element
     w = I.WORKLOADS["b8_l2048_d1536_n16_bf16"]
     x = I.make_inputs(w, seed=31)
-    _run(w, x, _dy(w, 32))
+    _run(w, x, _dy(w, 32), ckpt=ckpt)
 
 
 def test_bwd_workspace_too_small():
