@@ -24,7 +24,10 @@
  *    synchronises the stream (except ss_last_device_error) and keeps no state
  *    beyond one device-side error word per device (and the static scratch
  *    array of ss_scan_fwd_noalloc, part of the loaded module).
- *  - Calls are asynchronous on `stream` (0 = the legacy default stream).
+ *  - Calls are asynchronous on `stream` (0 = the legacy default stream), and
+ *    may be captured into a CUDA graph and replayed (the captured buffers,
+ *    workspace included, are reused by every replay; replays of one graph, or
+ *    calls sharing a workspace, must not run concurrently).
  *  - Arguments are checked on the host before any launch; a rejected call
  *    launches nothing and touches no buffer.
  */

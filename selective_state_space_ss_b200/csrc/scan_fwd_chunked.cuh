@@ -735,13 +735,19 @@ struct Cursor {
   __device__ __forceinline__ bool last() const { return c == nk - 1; }
 };
 
-// Bounded wait for worker `src`'s carry of this launch (one thread).
+// Bounded wait for worker `src`'s carry of this launch (one thread).  The
+// consumer clears the flag it took: each flag has one consumer, so a replay of
+// the same launch (a captured CUDA graph keeps its epoch) never mistakes the
+// previous replay's flag for a fresh carry.
 __device__ __forceinline__ bool wait_carry(const Sched& s, int src) {
-  const unsigned long long* f = s.flags + src;
+  unsigned long long* f = s.flags + src;
   for (uint32_t i = 0; i < s.spin_limit; ++i) {
     unsigned long long v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(f) : "memory");
-    if (v == s.epoch) return true;
+    if (v == s.epoch) {
+      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(0ull) : "memory");
+      return true;
+    }
     __nanosleep(i < 64 ? 32 : 256);
   }
   atomicOr(&g_error_word, kErrLookback);

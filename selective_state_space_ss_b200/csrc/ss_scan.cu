@@ -83,10 +83,17 @@ unsigned long long next_epoch() {
   return ctr.fetch_add(0x9E3779B97F4A7C15ULL) | 1ULL;
 }
 
+// Per-device answers that never change, looked up once (every launch plans its
+// schedule, and every workspace query plans all kernel variants).
+constexpr int kDevCache = 64;
+
 int device_sms() {
+  static std::atomic<int> cache[kDevCache];
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kDevCache && (sms = cache[dev].load()) > 0) return sms;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kDevCache) cache[dev].store(sms);
   return sms;
 }
 
@@ -122,10 +129,16 @@ bool make_plan(int64_t batch, int64_t dim, int64_t seqlen, Plan* p) {
   p->tiles = (dim + CF::CH - 1) / CF::CH;
   p->groups = batch * p->tiles;
   p->nk = (seqlen + CF::T - 1) / CF::T;
-  int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_fwd_chunked_kernel<CF, true>, CF::NT,
-                                                    CF::SMEM_BYTES) != cudaSuccess || occ < 1)
-    return false;
+  static std::atomic<int> occ_cache[kDevCache];  // resident CTAs per SM, per device
+  int dev = 0, occ = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < kDevCache) occ = occ_cache[dev].load();
+  if (occ < 1) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_fwd_chunked_kernel<CF, true>, CF::NT,
+                                                      CF::SMEM_BYTES) != cudaSuccess || occ < 1)
+      return false;
+    if (dev >= 0 && dev < kDevCache) occ_cache[dev].store(occ);
+  }
   const int64_t sms = device_sms();
   if (sms < 1) return false;
   // One group per CTA (the plain loop) unless the work is between one and two

@@ -78,3 +78,42 @@ def test_debug_hooks_clear():
     ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
     w = I.Workload("clear", 1, 8, 64, 16, "f32")
     assert ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate) == 0
+
+
+@pytest.mark.parametrize("workers", [0, 3])
+def test_replay_in_a_cuda_graph(workers):
+    """The scan captured once into a CUDA graph and replayed on new inputs
+    copied into the captured buffers: the balanced schedule's carry flags are
+    consumed by each replay, so a replay never takes the previous one's carry."""
+    w = I.Workload(f"graph_{workers}", 5, 40, 1000, 16, "bf16")
+    xs = [I.make_inputs(w, seed=s) for s in (21, 22, 23)]
+    static = to_device(xs[0])
+    need = ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate) if not workers else None
+    if workers:
+        ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, workers)
+        need = ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate)
+    ws = torch.zeros(max(need, 1), dtype=torch.uint8, device="cuda")
+    y = torch.empty(w.batch, w.dim, w.seqlen, device="cuda")
+    h = torch.empty(w.batch, w.dim, w.dstate, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm up outside the capture
+        if workers:
+            ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, workers)
+        run_gpu(static, y_out=y, last_state_out=h, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    if workers:
+        ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, workers)
+    with torch.cuda.graph(graph):
+        run_gpu(static, y_out=y, last_state_out=h, workspace=ws)
+    for x in xs + [xs[0]]:
+        src = to_device(x)
+        for k, v in src.items():
+            if v is not None:
+                static[k].copy_(v)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert ss.ss_last_device_error() == ss.SS_OK
+        _check(w, x, y, h)
