@@ -125,8 +125,9 @@ struct BwdSlots {
   // (n0 + r NT/T, t_s): offsets are a base plus r times a row stride
   int64_t act0, sel0, row;  // row = (NT / T) L
   int c0, n0, t_s;
-  int64_t item[CF::IPT];    // (b dim + d) L + t of item slot it, or -1
-  float bias[CF::IPT], D[CF::IPT];
+  float act_bias[CF::ACT_PT];  // delta_bias of staging slot r's channel
+  int64_t item[CF::IPT];    // (b dim + d) L + t of item slot it, or -1 (and its D)
+  float D[CF::IPT];
 };
 
 template <class CF>
@@ -141,13 +142,18 @@ __device__ __forceinline__ void bwd_slots(const BwdArgs& a, int64_t b, int64_t d
   sl.act0 = (b * a.dim + d0 + sl.c0) * L + sl.t_s;
   sl.sel0 = (b * CF::N + sl.n0) * L + sl.t_s;
 #pragma unroll
+  for (int r = 0; r < CF::ACT_PT; ++r) {
+    const int c = sl.c0 + r * (CF::NT / CF::T);
+    const bool ok = c < CF::CH && d0 + c < a.dim;
+    sl.act_bias[r] = (ok && a.delta_bias) ? __ldg(a.delta_bias + d0 + c) : 0.f;
+  }
+#pragma unroll
   for (int it = 0; it < CF::IPT; ++it) {
     const int i = threadIdx.x + it * CF::NT;
     const int tt = i / CF::CH, c = i - tt * CF::CH;
     const int64_t d = d0 + c;
     const bool ok = (!CF::ITEM_GUARD || i < CF::ITEMS) && d < a.dim;
     sl.item[it] = ok ? (b * a.dim + d) * L + tt : -1;
-    sl.bias[it] = (ok && a.delta_bias) ? __ldg(a.delta_bias + d) : 0.f;
     sl.D[it] = (ok && a.D) ? __ldg(a.D + d) : 0.f;
   }
 }
@@ -179,17 +185,28 @@ __device__ __forceinline__ void bwd_fetch(const BwdArgs& a, BwdStage<CF>& st,
   }
 }
 
+// Store the staged chunk to shared memory, discretising on the way: the
+// thread that holds element (c, t) also forms Delta (0 on padding and beyond
+// the channels), Delta u and (with_grad) softplus'(x).
 template <class CF, bool with_grad>
-__device__ __forceinline__ void bwd_store(const BwdStage<CF>& st, float* sm) {
+__device__ __forceinline__ void bwd_store(const BwdArgs& a, const BwdStage<CF>& st,
+                                          const BwdSlots<CF>& sl, float* sm, int64_t d0,
+                                          int64_t t0) {
+  const bool t_in = t0 + sl.t_s < a.seqlen;
 #pragma unroll
   for (int r = 0; r < CF::ACT_PT; ++r) {
     const int i = threadIdx.x + r * CF::NT;
     if (i >= CF::CH * CF::T) break;
     const int c = i / CF::T, tt = i - c * CF::T;
     const int o = tt * CF::CHP + c;
+    const bool in = t_in && d0 + c < a.dim;
+    const float x = st.dl[r] + sl.act_bias[r];
+    const float dl = in ? (a.softplus ? softplus_fast(x) : x) : 0.f;
     sm[CF::OFF_U + o] = st.u[r];
-    sm[CF::OFF_DL + o] = st.dl[r];
+    sm[CF::OFF_DL + o] = dl;
+    sm[CF::OFF_W + o] = dl * st.u[r];
     if (with_grad) {
+      sm[CF::OFF_SG + o] = a.softplus ? sigmoid_fast(x) : 1.f;
       sm[CF::OFF_Z + o] = st.z[r];
       sm[CF::OFF_DY + o] = st.dy[r];
     }
@@ -201,26 +218,6 @@ __device__ __forceinline__ void bwd_store(const BwdStage<CF>& st, float* sm) {
     const int n = i / CF::T, tt = i - n * CF::T;
     sm[CF::OFF_B + tt * CF::NP + n] = st.b[r];
     if (with_grad) sm[CF::OFF_C + tt * CF::NP + n] = st.c[r];
-  }
-}
-
-// Per (step, channel) item: Delta (0 on padding), Delta u and (with_grad)
-// softplus'(x).  Items are channel-fastest: item i is (t, c) = (i / CH, i % CH).
-template <class CF, bool with_grad>
-__device__ __forceinline__ void bwd_discretise(const BwdArgs& a, float* sm, const BwdSlots<CF>& sl,
-                                               int64_t t0) {
-#pragma unroll
-  for (int it = 0; it < CF::IPT; ++it) {
-    const int i = threadIdx.x + it * CF::NT;
-    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
-    const int tt = i / CF::CH, c = i - tt * CF::CH;
-    const int o = tt * CF::CHP + c;
-    const bool in = sl.item[it] >= 0 && t0 + tt < a.seqlen;
-    const float x = sm[CF::OFF_DL + o] + sl.bias[it];
-    const float dl = in ? (a.softplus ? softplus_fast(x) : x) : 0.f;
-    sm[CF::OFF_DL + o] = dl;
-    sm[CF::OFF_W + o] = dl * sm[CF::OFF_U + o];
-    if (with_grad) sm[CF::OFF_SG + o] = a.softplus ? sigmoid_fast(x) : 1.f;
   }
 }
 
@@ -281,10 +278,8 @@ __global__ void __launch_bounds__(CF::NT)
   if (!a.ckpt_given) bwd_fetch<CF, false>(a, st, sl, d0, 0);
   for (int64_t k = 0; k < nk && !a.ckpt_given; ++k) {
     if (chan_ok) st_pairs(ck_lane + k * ck_stride, h);
-    bwd_store<CF, false>(st, sm);
+    bwd_store<CF, false>(a, st, sl, sm, d0, k * T);
     if (k + 1 < nk) bwd_fetch<CF, false>(a, st, sl, d0, (k + 1) * T);
-    __syncthreads();
-    bwd_discretise<CF, false>(a, sm, sl, k * T);
     __syncthreads();
 #pragma unroll 4
     for (int t = 0; t < T; ++t) {
@@ -319,13 +314,11 @@ __global__ void __launch_bounds__(CF::NT)
   for (int64_t k = nk - 1; k >= 0; --k) {
     const int64_t t0 = k * T;
     const float2 h_start[2] = {ck_next[0], ck_next[1]};
-    bwd_store<CF, true>(st, sm);
+    bwd_store<CF, true>(a, st, sl, sm, d0, t0);
     if (k > 0) {
       bwd_fetch<CF, true>(a, st, sl, d0, (k - 1) * T);
       if (chan_ok) ld_pairs(ck_lane + (k - 1) * ck_stride, ck_next);
     }
-    __syncthreads();
-    bwd_discretise<CF, true>(a, sm, sl, t0);
     __syncthreads();
     // recompute the chunk's states from its checkpoint; channel readouts
     float2 hs[2] = {h_start[0], h_start[1]};

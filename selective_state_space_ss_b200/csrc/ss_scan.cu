@@ -99,6 +99,24 @@ int device_sms() {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Run `setup` (attribute settings of a kernel family) once per device: the
+// dynamic shared memory limit is a per-device setting, so a process that
+// drives several GPUs needs it on each.  `Tag` keeps one cache per family.
+// Returns the cached value: 1 set up, -1 failed.
+template <class Tag, class F>
+int once_per_device(F setup) {
+  static std::atomic<int> state[kDevCache];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev < 0 || dev >= kDevCache) return setup() ? 1 : -1;  // not cached
+  int v = state[dev].load();
+  if (v == 0) {
+    v = setup() ? 1 : -1;  // idempotent: a concurrent first call may repeat it
+    state[dev].store(v);
+  }
+  return v;
+}
+
 // How the work is cut: `workers` CTAs, each an equal contiguous range of
 // (channel group, chunk) units.  workers == groups means one group per CTA and
 // no carries; fewer workers balance the load across SMs with carry handoff.
@@ -110,17 +128,14 @@ struct Plan {
 
 template <class CF>
 bool configure_kernel() {
-  static int state = 0;  // 0 unknown, 1 ok, -1 failed
-  if (state == 0)
-    state = (cudaFuncSetAttribute(scan_fwd_chunked_kernel<CF, false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) ==
-                 cudaSuccess &&
-             cudaFuncSetAttribute(scan_fwd_chunked_kernel<CF, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) ==
-                 cudaSuccess)
-                ? 1
-                : -1;
-  return state == 1;
+  return once_per_device<CF>([] {
+    return cudaFuncSetAttribute(scan_fwd_chunked_kernel<CF, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                CF::SMEM_BYTES) == cudaSuccess &&
+           cudaFuncSetAttribute(scan_fwd_chunked_kernel<CF, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                CF::SMEM_BYTES) == cudaSuccess;
+  }) == 1;
 }
 
 template <class CF>
@@ -322,19 +337,22 @@ ss_status launch_step(const StepArgs& a, bool vec, cudaStream_t stream) {
 template <typename E, int N>
 ss_status launch_step_pipe(const StepArgs& a, cudaStream_t stream) {
   using CF = StepPipeCfg<E, N>;
-  static int state = 0;  // 0 unknown, 1 ok, -1 failed
-  static int occ = 0;
-  if (state == 0) {
-    state = (cudaFuncSetAttribute(scan_step_pipe_kernel<E, N>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) ==
-                 cudaSuccess &&
-             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_step_pipe_kernel<E, N>, CF::NT,
-                                                           CF::SMEM_BYTES) == cudaSuccess &&
-             occ > 0)
-                ? 1
-                : -1;
+  if (once_per_device<CF>([] {
+        return cudaFuncSetAttribute(scan_step_pipe_kernel<E, N>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    CF::SMEM_BYTES) == cudaSuccess;
+      }) != 1)
+    return SS_ERR_CUDA;
+  static std::atomic<int> occ_cache[kDevCache];  // resident CTAs per SM, per device
+  int dev = 0, occ = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
+  if (dev >= 0 && dev < kDevCache) occ = occ_cache[dev].load();
+  if (occ < 1) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_step_pipe_kernel<E, N>, CF::NT,
+                                                      CF::SMEM_BYTES) != cudaSuccess || occ < 1)
+      return SS_ERR_CUDA;
+    if (dev >= 0 && dev < kDevCache) occ_cache[dev].store(occ);
   }
-  if (state != 1) return SS_ERR_CUDA;
   StepPipeSched sc;
   sc.tiles_per_row = (a.dim + CF::TILE_CH - 1) / CF::TILE_CH;
   sc.items = sc.tiles_per_row * a.batch;
@@ -367,11 +385,11 @@ size_t ckpt_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N) {
 template <typename E, int N>
 ss_status launch_bwd(const BwdArgs& a, size_t ws_bytes, cudaStream_t stream) {
   using CF = BwdCfg<E, N>;
-  static int state = 0;
-  if (state == 0)
-    state = cudaFuncSetAttribute(scan_bwd_kernel<CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 CF::SMEM_BYTES) == cudaSuccess ? 1 : -1;
-  if (state != 1) return SS_ERR_CUDA;
+  if (once_per_device<CF>([] {
+        return cudaFuncSetAttribute(scan_bwd_kernel<CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    CF::SMEM_BYTES) == cudaSuccess;
+      }) != 1)
+    return SS_ERR_CUDA;
   static_assert(CF::T == kCkptSteps, "checkpoint spacing");
   if (!a.ckpt_given && ws_bytes < ckpt_bytes(a.batch, a.dim, a.seqlen, N)) return SS_ERR_INVALID_ARG;
   const int64_t ctas = a.batch * ((a.dim + CF::CH - 1) / CF::CH);
