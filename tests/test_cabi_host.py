@@ -221,3 +221,12 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         N.ss_scan_step(torch.zeros(1, 2, 16), t, t, torch.zeros(2, 16), torch.zeros(1, 16),
                        torch.zeros(1, 16))
+    B = torch.zeros(1, 16, 8)
+    with pytest.raises(ValueError):
+        N.ss_scan_fwd_zoh(x, x, torch.zeros(2, 16), B, B)
+    with pytest.raises(ValueError):
+        N.ss_scan_fwd_conv(x, torch.zeros(2, 4), x, torch.zeros(2, 16), B, B)
+    with pytest.raises(ValueError):
+        N.ss_scan_fwd_train(x, x, torch.zeros(2, 16), B, B)
+    with pytest.raises(ValueError):
+        N.ss_scan_bwd(x, x, torch.zeros(2, 16), B, B, torch.zeros(1, 2, 8))
