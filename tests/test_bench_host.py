@@ -49,3 +49,23 @@ def test_cli_rejects_mixed_modes():
     assert run("--warmup", "2").returncode != 0
     assert run("--workload", "step_b128_d8192_n16_bf16").returncode != 0
     assert run("--op", "step", "--gpus", "2").returncode != 0
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one
+    JSON line with the contract's keys on the default workload."""
+    import json
+
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == bench.DEFAULT_WORKLOAD
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
