@@ -33,18 +33,23 @@ sys.path.insert(0, ROOT)
 
 from selective_state_space_ss_b200 import inputs as I  # noqa: E402
 
-DEFAULT_WORKLOAD = "b8_l2048_d1536_n16_bf16"
+# the largest single-GPU workload: the million-token sequence
+DEFAULT_WORKLOAD = "b1_l1048576_d1536_n16_bf16"
+# the backward is measured on the B8 L2048 D1536 N16 workload (its own checkpoints fit easily)
+BWD_DEFAULT_WORKLOAD = "b8_l2048_d1536_n16_bf16"
 METRIC = "selective-scan fwd (B·L·D) elements/s and % of HBM/SFU roofline"
 UNIT = "elements/s"
 L2_BYTES = 126 * 1024 * 1024
 NUM_SMS = 148
 MUFU_EX2_PER_CLK_PER_SM = 16  # ex2 results per clock per SM (special-function unit)
 _CSRC = "selective_state_space_ss_b200/csrc/"
-KERNEL_SOURCES = tuple(_CSRC + f for f in ("ss_scan.cu", "pointwise.cuh", "scan_fwd_chunked.cuh",
-                                           "scan_common.cuh"))
-BWD_KERNEL_SOURCES = tuple(_CSRC + f for f in ("pointwise.cuh", "scan_bwd.cuh", "scan_common.cuh"))
-# (the step and backward kernels' launch shapes are constants of their headers)
-STEP_KERNEL_SOURCES = tuple(_CSRC + f for f in ("pointwise.cuh", "scan_step.cuh", "scan_common.cuh"))
+# Sources each kernel's traffic record is keyed to: its device code and its own
+# host code (a change to another entry point leaves the record valid).
+_COMMON = ("pointwise.cuh", "scan_common.cuh", "host_common.cuh")
+KERNEL_SOURCES = tuple(_CSRC + f for f in _COMMON + ("scan_fwd_chunked.cuh", "scan_fix.cuh",
+                                                     "fwd_host.cuh"))
+BWD_KERNEL_SOURCES = tuple(_CSRC + f for f in _COMMON + ("scan_bwd.cuh", "bwd_host.cuh"))
+STEP_KERNEL_SOURCES = tuple(_CSRC + f for f in _COMMON + ("scan_step.cuh", "step_host.cuh"))
 
 
 def peaks():
@@ -619,33 +624,55 @@ def oracle_sample(w: I.Workload, x: dict, target_s: float):
 
 def run_reference_arm(args, w: I.Workload):
     world, rank, _ = _dist_env()
+    if world > 1:
+        # the ranks meet once (gloo, host only), then rank 0 alone times the oracle
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        print(f"reference arm: rank {rank} of {world} joined", file=sys.stderr, flush=True)
+        dist.barrier()
+        dist.destroy_process_group()
     if rank != 0:
         return None
-    x = I.make_inputs(w, seed=1000)
     import oracle
 
     cores = os.cpu_count() or 1
-    # size one step to ~2 s of oracle work so that warmup + steps stay within minutes
-    take, dt, _ = oracle_sample(w, x, target_s=2.0)
-    nch = w.batch * w.dim
     rng = np.random.default_rng(1)
-    times = []
-    for i in range(args.warmup + args.steps):
-        ch = np.sort(rng.choice(nch, take, replace=False))
+
+    def sample(k):
+        # k channels of batch row 0, full sequence each (only their rows are drawn)
+        dims = np.sort(rng.choice(w.dim, k, replace=False))
+        return I.make_row_inputs(w, 1000, 0, dims)
+
+    def oracle_time(x):
         t0 = time.perf_counter()
         oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"],
-                        softplus=w.softplus, channels=ch, nthreads=cores)
+                        softplus=w.softplus, nthreads=cores)
+        return time.perf_counter() - t0
+
+    # size one step to ~2 s of oracle work so that warmup + steps stay within minutes
+    k0 = min(w.dim, cores)
+    per_ch = oracle_time(sample(k0)) / k0
+    take = int(min(w.dim, max(k0, 2.0 / max(per_ch, 1e-9))))
+    nch = w.batch * w.dim
+    x = sample(take)  # one sample, rescanned every step
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = oracle_time(x)
         if i >= args.warmup:
-            times.append(time.perf_counter() - t0)
+            times.append(dt)
     tot = sum(times)
     value = take * w.seqlen * len(times) / tot
-    sample = f"{take} of {nch} channels x full L={w.seqlen} per step, fp64, {cores} threads"
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    desc = (f"{take} of {nch} channels (batch row 0) x full L={w.seqlen} per step, fp64, "
+            f"{cores} threads")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_of(w, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -658,11 +685,31 @@ def config_of(w: I.Workload, world: int, conv: int = 0, zoh: bool = False):
             "l2": "inputs rotated over sets totalling >= 4x L2 (126 MB); no flush"}
 
 
+def _free_port() -> int:
+    import socket
+
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def launch_ranks(n: int) -> int:
+    """Re-run this command as n ranks (one process per GPU) under
+    torch.distributed.run on this node; returns the launcher's exit code."""
+    import subprocess
+
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={_free_port()}",
+           os.path.abspath(__file__), *sys.argv[1:]]
+    env = dict(os.environ, SS_BENCH_LAUNCHED="1")
+    return subprocess.call(cmd, env=env)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--op", default="scan", choices=["scan", "step", "bwd"])
     ap.add_argument("--workload", default=None,
                     choices=sorted(I.WORKLOADS) + sorted(I.STEP_WORKLOADS))
@@ -676,6 +723,16 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # `python bench.py --gpus N` without a launcher: start the N ranks here
+        if os.environ.get("SS_BENCH_LAUNCHED"):
+            ap.error("rank launch failed: WORLD_SIZE is not set under the launcher")
+        sys.exit(launch_ranks(args.gpus))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started {world} ranks")
     if args.conv and args.zoh:
         ap.error("--conv and --zoh are separate kernel variants")
     if args.op == "step":
@@ -689,7 +746,7 @@ def main():
     if args.op == "bwd":
         if args.impl != "native" or args.gpus != 1:
             ap.error("--op bwd runs the native arm on one GPU")
-        print(json.dumps(run_bwd_arm(args, I.WORKLOADS[args.workload or DEFAULT_WORKLOAD])),
+        print(json.dumps(run_bwd_arm(args, I.WORKLOADS[args.workload or BWD_DEFAULT_WORKLOAD])),
               flush=True)
         return
     w = I.WORKLOADS[args.workload or DEFAULT_WORKLOAD]

@@ -20,6 +20,11 @@
  *   SS_DEBUG_STEP_SIMPLE    value != 0: the next ss_scan_step call takes the
  *                           plain-load kernel even where the bulk-copy
  *                           pipeline applies, so both are tested on one shape.
+ *   SS_DEBUG_FORCE_SEGMENTS value = number of segments each channel group's
+ *                           sequence is cut into (>= 1, capped at its number
+ *                           of chunks; 1: none), so the carry-in correction
+ *                           runs on problems small enough to check in full.
+ *                           Ignored by the training forward.
  *   SS_DEBUG_CLEAR          value ignored: drop every pending setting.
  *
  * Returns SS_OK, or SS_ERR_INVALID_ARG for an unknown `what`.  Host-only,
@@ -39,7 +44,8 @@ enum {
   SS_DEBUG_FORCE_WORKERS = 1,
   SS_DEBUG_SKIP_PUBLISH = 2,
   SS_DEBUG_SPIN_LIMIT = 3,
-  SS_DEBUG_STEP_SIMPLE = 4
+  SS_DEBUG_STEP_SIMPLE = 4,
+  SS_DEBUG_FORCE_SEGMENTS = 5
 };
 
 ss_status ss_debug_inject(int what, long long value);

@@ -8,6 +8,7 @@ lazily on the first call, and a missing library raises: there is no CPU path.
 from ._native import (  # noqa: F401
     EXPORTED,
     SS_DEBUG_CLEAR,
+    SS_DEBUG_FORCE_SEGMENTS,
     SS_DEBUG_FORCE_WORKERS,
     SS_DEBUG_SKIP_PUBLISH,
     SS_DEBUG_SPIN_LIMIT,

@@ -31,7 +31,7 @@ SS_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 # test hooks (include/ss_scan_debug.h)
 (SS_DEBUG_CLEAR, SS_DEBUG_FORCE_WORKERS, SS_DEBUG_SKIP_PUBLISH, SS_DEBUG_SPIN_LIMIT,
- SS_DEBUG_STEP_SIMPLE) = range(5)
+ SS_DEBUG_STEP_SIMPLE, SS_DEBUG_FORCE_SEGMENTS) = range(6)
 
 
 class SSError(RuntimeError):

@@ -57,6 +57,11 @@ struct FwdArgs {
   // training checkpoints: the state at the start of every 16-step chunk,
   // [batch][ceil(L / 16)][dim][N] fp32 (nullable: not written)
   float* ckpt;
+  // sequence segments (Sched::nseg > 1): the state each segment ends in,
+  // scanned from h = 0 (segment 0: from h0), [batch * dim][nseg][N], and the
+  // sum of Delta over each segment, [batch * dim][nseg]
+  float* seg_h;
+  float* seg_dsum;
   int64_t batch, dim, seqlen;
   int softplus;
   int vec;  // 1: TMA path (16-byte aligned rows); 0: element-wise loads
@@ -259,7 +264,8 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
                                        float4* dwD, float4* dwW, float4* dwI, float4* su,
                                        unsigned char* bc,
                                        const float (&bias_it)[CF::ITEMS_PER_THREAD],
-                                       const ConvRegs<CF>& cv, int64_t d0, int64_t t0) {
+                                       const ConvRegs<CF>& cv, int64_t d0, int64_t t0,
+                                       double (&dsum)[CF::ITEMS_PER_THREAD], bool seg) {
   using E = typename CF::Elem;
   const int tid = threadIdx.x;
   const E* rawD = raw + CF::CH * CF::XT;
@@ -306,6 +312,7 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
       for (int k = 0; k < 4; ++k)
         if (d0 + c >= a.dim || t0 + 4 * q + k >= a.seqlen) delt[k] = 0.f;
     }
+    if (seg) dsum[it] += (double)((delt[0] + delt[1]) + (delt[2] + delt[3]));
     const float2 w01 = __fmul2_rn(make_float2(delt[0], delt[1]), make_float2(uu.x, uu.y));
     const float2 w23 = __fmul2_rn(make_float2(delt[2], delt[3]), make_float2(uu.z, uu.w));
     const float w[4] = {w01.x, w01.y, w23.x, w23.y};
@@ -672,6 +679,10 @@ struct Sched {
   unsigned long long epoch;   // unique per launch, so stale flags never match
   uint32_t spin_limit;        // polls before a carry wait gives up
   int skip_publish;           // test hook: this worker never publishes (-1: none)
+  // plain schedule only: each channel group's chunks are cut into nseg
+  // segments of seg_chunks chunks (the last may be shorter), one CTA each
+  int32_t nseg;
+  int64_t seg_chunks;
 };
 
 // Walks one worker's chunk sequence without divisions: the three pieces
@@ -817,9 +828,20 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   __shared__ __align__(8) uint64_t bars[2];
 
   const int w = blockIdx.x;
-  const int64_t u0 = sched.units * w / gridDim.x;
-  const int64_t u1 = sched.units * (w + 1) / gridDim.x;
-  const int64_t nseq = u1 - u0;
+  // kMulti: worker w's range of (group, chunk) units; plain: CTA w runs
+  // segment `seg` (chunks c_begin .. c_begin + nseq - 1) of channel group `grp`
+  int64_t u0 = 0, u1 = 0, nseq = 0, c_begin = 0, grp = w;
+  int seg = 0;
+  if constexpr (kMulti) {
+    u0 = sched.units * w / gridDim.x;
+    u1 = sched.units * (w + 1) / gridDim.x;
+    nseq = u1 - u0;
+  } else {
+    grp = w / sched.nseg;
+    seg = (int)(w - grp * sched.nseg);
+    c_begin = (int64_t)seg * sched.seg_chunks;
+    nseq = sched.nk - c_begin < sched.seg_chunks ? sched.nk - c_begin : sched.seg_chunks;
+  }
   const int64_t L = a.seqlen;
   const bool has_z = a.z != nullptr;
   const bool tma = a.vec != 0;
@@ -856,40 +878,48 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   if (nseq <= 0) return;
 
   if constexpr (!kMulti) {
-    // ---- one channel group per CTA: chunk q of group w is unit q ----
-    const int64_t b = w / sched.tiles_per_b;
-    const int64_t d0 = (w - b * sched.tiles_per_b) * CF::CH;
+    // ---- one channel group (or one segment of it) per CTA: local chunk k is
+    // chunk c_begin + k of the group ----
+    const int64_t b = grp / sched.tiles_per_b;
+    const int64_t d0 = (grp - b * sched.tiles_per_b) * CF::CH;
     const int64_t d = d0 + c;
     const bool chan_ok = d < a.dim;
     const bool full_tile = d0 + CF::CH <= a.dim;
+    const bool segmented = sched.nseg > 1;
     float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
+    double dsum[CF::ITEMS_PER_THREAD];
     ConvRegs<CF> cv;
 #pragma unroll
     for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
       const int64_t di = d0 + (tid + it * CF::NT) / CF::QPR;
       bias_it[it] = (a.delta_bias && di < a.dim) ? __ldg(a.delta_bias + di) : 0.f;
       D_it[it] = (a.D && di < a.dim) ? __ldg(a.D + di) : 0.f;
+      dsum[it] = 0.0;
     }
     load_conv_regs<CF>(a, d0, cv);
     float2 h[CF::G / 2], a2[CF::G / 2], ia[CF::G / 2];
 #pragma unroll
     for (int g = 0; g < CF::G / 2; ++g) {
       const int n = j * CF::G + 2 * g;
-      // plain loads: h0 may be the last_state buffer this kernel writes
+      // plain loads: h0 may be the last_state buffer this kernel writes; only
+      // the first segment starts from it (later ones start from zero)
       const float* h0 = a.h0 + (b * a.dim + d) * CF::N + n;
-      h[g] = (a.h0 && chan_ok) ? make_float2(h0[0], h0[1]) : make_float2(0.f, 0.f);
+      h[g] = (a.h0 && chan_ok && seg == 0) ? make_float2(h0[0], h0[1]) : make_float2(0.f, 0.f);
       load_decay<CF>(a, d, n, chan_ok, a2[g], ia[g]);
     }
     bool ok = true;
-    auto full_chunk = [&](int64_t k) { return full_tile && (k + 1) * CF::T <= L; };
+    auto t_of = [&](int64_t k) { return (c_begin + k) * CF::T; };
+    auto full_chunk = [&](int64_t k) { return full_tile && t_of(k) + CF::T <= L; };
     auto stage_in = [&](int64_t k) {
       if (tma) ok = ok && mbar_wait_bounded(&bars[k & 1], (uint32_t)((k >> 1) & 1), kTmaSpinLimit);
-      else load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw(k)), b, d0, k * CF::T);
+      else load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw(k)), b, d0, t_of(k));
     };
     auto run_phase1 = [&](int64_t k) {
       const E* rp = reinterpret_cast<const E*>(raw(k));
-      if (full_chunk(k)) phase1<CF, true>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0, k * CF::T);
-      else phase1<CF, false>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0, k * CF::T);
+      if (full_chunk(k))
+        phase1<CF, true>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0, t_of(k), dsum, segmented);
+      else
+        phase1<CF, false>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0, t_of(k), dsum, segmented);
     };
     auto drain = [&](int64_t first, int64_t last) {
       if (tma)
@@ -897,8 +927,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
           mbar_wait_bounded(&bars[kk & 1], (uint32_t)((kk >> 1) & 1), kTmaSpinLimit);
     };
     if (tma && tid == 0) {
-      tma_chunk<CF>(maps, raw(0), &bars[0], (int32_t)b, (int32_t)d0, 0, has_z);
-      if (nseq > 1) tma_chunk<CF>(maps, raw(1), &bars[1], (int32_t)b, (int32_t)d0, CF::T, has_z);
+      tma_chunk<CF>(maps, raw(0), &bars[0], (int32_t)b, (int32_t)d0, (int32_t)t_of(0), has_z);
+      if (nseq > 1) tma_chunk<CF>(maps, raw(1), &bars[1], (int32_t)b, (int32_t)d0, (int32_t)t_of(1), has_z);
     }
     stage_in(0);
     if (!__syncthreads_and(ok)) {
@@ -908,22 +938,41 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     run_phase1(0);
     __syncthreads();
     for (int64_t k = 0; k < nseq; ++k) {
-      run_phase2(h, a2, ia, ckpt_at(b, d, chan_ok, k * CF::T));
+      run_phase2(h, a2, ia, ckpt_at(b, d, chan_ok, t_of(k)));
       if (k + 1 < nseq) stage_in(k + 1);
       if (!__syncthreads_and(ok)) {
         drain(k + 1, k + 1);
         return;
       }
       const E* rc = reinterpret_cast<const E*>(raw(k));
-      if (full_chunk(k)) phase3<CF, true>(a, rc, sy, su, D_it, b, d0, k * CF::T, has_z);
-      else phase3<CF, false>(a, rc, sy, su, D_it, b, d0, k * CF::T, has_z);
+      if (full_chunk(k)) phase3<CF, true>(a, rc, sy, su, D_it, b, d0, t_of(k), has_z);
+      else phase3<CF, false>(a, rc, sy, su, D_it, b, d0, t_of(k), has_z);
       if (k + 1 < nseq) run_phase1(k + 1);
       __syncthreads();
       if (tma && tid == 0 && k + 2 < nseq)
-        tma_chunk<CF>(maps, raw(k), &bars[k & 1], (int32_t)b, (int32_t)d0,
-                      (int32_t)((k + 2) * CF::T), has_z);
+        tma_chunk<CF>(maps, raw(k), &bars[k & 1], (int32_t)b, (int32_t)d0, (int32_t)t_of(k + 2), has_z);
     }
-    if (a.last_state && chan_ok && writer) {
+    if (segmented) {
+      // this segment's end state (from h = 0 unless it is the first) and its
+      // sum of Delta; the carry-in correction pass combines them
+      if (chan_ok && writer) {
+        float2* dst = reinterpret_cast<float2*>(
+            a.seg_h + (((b * a.dim + d) * sched.nseg + seg) * CF::N + j * CF::G));
+#pragma unroll
+        for (int g = 0; g < CF::G / 2; ++g) dst[g] = h[g];
+      }
+      // the QPR threads of an item's channel are consecutive lanes of a warp
+#pragma unroll
+      for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+        double v = dsum[it];
+#pragma unroll
+        for (int o = 1; o < CF::QPR; o <<= 1) v += __shfl_xor_sync(kFullMask, v, o);
+        const int i = tid + it * CF::NT;
+        const int64_t di = d0 + i / CF::QPR;
+        if ((i % CF::QPR) == 0 && i < CF::ITEMS && di < a.dim)
+          a.seg_dsum[(b * a.dim + di) * sched.nseg + seg] = (float)v;
+      }
+    } else if (a.last_state && chan_ok && writer) {
       float* dst = a.last_state + ((b * a.dim + d) * CF::N + j * CF::G);
 #pragma unroll
       for (int g = 0; g < CF::G / 2; ++g) {
@@ -944,6 +993,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   float2 h[CF::G / 2], a2[CF::G / 2], ia[CF::G / 2];
   float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
   ConvRegs<CF> cv;
+  double no_dsum[CF::ITEMS_PER_THREAD];  // (unused: the balanced schedule has no segments)
   int32_t bias_g = -1, D_g = -1;  // group whose bias (and taps) / D are cached
   bool ok = true;  // false once a bounded wait has given up (error word set)
 
@@ -977,8 +1027,10 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     }
     const E* rp = reinterpret_cast<const E*>(raw(jj));
     const int64_t t0 = (int64_t)prep.c * CF::T;
-    if (full_chunk(prep)) phase1<CF, true>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0_of(prep), t0);
-    else phase1<CF, false>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0_of(prep), t0);
+    if (full_chunk(prep))
+      phase1<CF, true>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0_of(prep), t0, no_dsum, false);
+    else
+      phase1<CF, false>(a, rp, dwD, dwW, dwI, su, bc, bias_it, cv, d0_of(prep), t0, no_dsum, false);
   };
   // On a timed-out wait: wait (bounded) for every copy this CTA still has in
   // flight, so that none lands in shared memory after the CTA has left.

@@ -177,6 +177,38 @@ def make_inputs(w: Workload, seed: int = 1234, nthreads: int | None = None) -> d
     return x
 
 
+def make_row_inputs(w: Workload, seed: int, b: int, dims, nthreads: int | None = None) -> dict:
+    """Channels `dims` of batch row b of make_inputs(w, seed), and nothing else.
+
+    Returns the inputs of a workload with batch 1 and dim len(dims): every
+    tensor holds exactly the values make_inputs draws for those channels (the
+    streams are counter-based, so each row is drawn at its own offset), which
+    lets a timing sample of a very long sequence skip the other channels."""
+    dims = np.asarray(dims, dtype=np.int64)
+    out = "f32" if w.dtype == "f32" else "bf16"
+    D_, L_, N_ = w.dim, w.seqlen, w.dstate
+    k = len(dims)
+
+    def rows(name, scale=1.0):
+        dt = _OUT[out][1]
+        arr = np.empty((1, k, L_), dtype=dt)
+        for i, d in enumerate(dims):
+            arr[0, i] = fill(seed, STREAM[name], (L_,), scale=scale, out=out,
+                             offset=int((b * D_ + d) * L_), nthreads=nthreads)
+        return arr
+
+    x = {"u": rows("u"), "delta": rows("delta", 0.5), "z": rows("z") if w.with_z else None}
+    for name in ("B", "C"):
+        x[name] = fill(seed, STREAM[name], (1, N_, L_), out=out, offset=b * N_ * L_,
+                       nthreads=nthreads)
+    full = make_inputs(dataclasses.replace(w, batch=1, seqlen=1), seed=seed, nthreads=nthreads)
+    x["A"] = np.ascontiguousarray(full["A"][dims])
+    x["D"] = None if full["D"] is None else np.ascontiguousarray(full["D"][dims])
+    x["delta_bias"] = (None if full["delta_bias"] is None
+                       else np.ascontiguousarray(full["delta_bias"][dims]))
+    return x
+
+
 def make_state(batch: int, dim: int, dstate: int, seed: int = 1234, scale: float = 1.0,
                nthreads: int | None = None) -> np.ndarray:
     """A carried state [batch, dim, dstate] float32, N(0, scale^2)."""

@@ -87,6 +87,9 @@ def test_fwd_train_checkpoints_are_states(N, batch, dim):
     xd = to_device(x)
     y, h, ck = ss.ss_scan_fwd_train(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"],
                                     z=xd["z"], delta_bias=xd["delta_bias"])
+    # the training forward never cuts the sequence into segments: it matches
+    # the plain forward run unsegmented bit for bit
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_SEGMENTS, 1)
     y0, h0 = ss.ss_scan_fwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"], z=xd["z"],
                             delta_bias=xd["delta_bias"])
     torch.cuda.synchronize()

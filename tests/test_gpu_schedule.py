@@ -74,10 +74,18 @@ def test_carry_wait_times_out_cleanly():
 
 
 def test_debug_hooks_clear():
-    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, 2)
-    ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
-    w = I.Workload("clear", 1, 8, 64, 16, "f32")
+    # one channel group of 8 channels x 2 chunks: a single segment of one chunk
+    # needs no scratch, so any bytes here would come from a pending setting
+    w = I.Workload("clear", 1, 8, 32, 16, "f32")
     assert ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate) == 0
+    for hook in (ss.SS_DEBUG_FORCE_WORKERS, ss.SS_DEBUG_FORCE_SEGMENTS):
+        ss.ss_debug_inject(hook, 2)
+        ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
+        assert ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate) == 0
+    w2 = I.Workload("clear2", 1, 8, 64, 16, "f32")  # two chunks: segments when asked
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_SEGMENTS, 2)
+    assert ss.ss_scan_workspace_bytes(w2.batch, w2.dim, w2.seqlen, w2.dstate) > 0
+    ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
 
 
 @pytest.mark.parametrize("workers", [0, 3])

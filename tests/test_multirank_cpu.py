@@ -43,18 +43,27 @@ def test_job_throughput_is_weak_scaling():
     assert bench.rank_seed(0, 0) != bench.rank_seed(1, 0)
 
 
-@pytest.mark.parametrize("rank", [0, 1])
-def test_reference_arm_prints_on_rank_zero_only(rank):
-    env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+def test_gpus_two_launches_two_ranks():
+    """`bench.py --gpus 2` with no launcher starts two ranks itself; both join
+    (gloo), rank 0 alone times the oracle and prints one line with n_gpus 2."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--workload", "b2_l1024_d512_n16_f32", "--steps", "3", "--warmup", "3",
+                        "--workload", "b2_l1024_d512_n16_f32", "--steps", "1", "--warmup", "3",
                         "--gpus", "2"], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
-    if rank == 0:
-        assert len(lines) == 1
-        rec = json.loads(lines[0])
-        assert rec["impl"] == "reference" and rec["cpu_baseline"]["kind"] == "oracle"
-        assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["value"] > 0
-    else:
-        assert lines == []
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["value"] > 0
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0
+    joined = sorted(ln for ln in r.stderr.splitlines() if "joined" in ln)
+    assert joined == ["reference arm: rank 0 of 2 joined", "reference arm: rank 1 of 2 joined"]
+
+
+def test_gpus_mismatch_with_launcher_is_refused():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "b2_l1024_d512_n16_f32", "--gpus", "2"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "launcher started 1" in r.stderr

@@ -2,9 +2,9 @@
 where they call it (for example inside a framework that owns every device
 allocation).  Its scratch is the library's static device array, so the test
 checks it through the C ABI against ss_scan_fwd, whose workspace the caller
-allocates: same inputs, results within the parity tolerance, on two calls in a
-row (the array keeps the previous call's contents).  This file is collected
-last on purpose.
+allocates, and against the fp64 oracle: same inputs, results within the
+parity tolerance, on two calls in a row (the array keeps the previous call's
+contents).  This file is collected last on purpose.
 """
 import ctypes
 
@@ -14,6 +14,7 @@ import pytest
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
+import oracle  # noqa: E402
 import selective_state_space_ss_b200 as ss  # noqa: E402
 from selective_state_space_ss_b200 import _native as N  # noqa: E402
 from selective_state_space_ss_b200 import inputs as I  # noqa: E402
@@ -41,19 +42,23 @@ def _reference(xd):
     ((4, 5120, 256, 16), "bf16", 0),   # 640 channel groups: the balanced schedule, scratch in use
     ((3, 200, 777, 32), "bf16", 5),    # forced split of 7 groups: carries on a small problem
     ((2, 64, 301, 16), "f32", 3),      # element-wise load path (1204-byte rows) with a split
-    ((2, 96, 200, 64), "bf16", 0),     # plain schedule: no scratch needed at all
+    ((2, 96, 200, 64), "bf16", 0),     # few channel groups: sequence segments, scratch in use
+    ((1, 64, 5000, 16), "f32", 0),     # long segments with the carry-in correction
 ])
 def test_noalloc_matches_workspace_entry_point(shape, dtype, workers):
     ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
     b, d, L, n = shape
     w = I.Workload("noalloc", b, d, L, n, dtype)
-    xd = to_device(I.make_inputs(w, seed=77))
+    x = I.make_inputs(w, seed=77)
+    xd = to_device(x)
+    yo, ho = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                             x["delta_bias"])
     if workers:
         ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, workers)
     need = ss.ss_scan_workspace_bytes(b, d, L, n)
     assert need <= N.SS_NOALLOC_SCRATCH_BYTES
-    if shape[1] == 5120:
-        assert need > 0  # this case really runs the kernel that uses scratch
+    if shape[1] == 5120 or shape[2] >= 200:
+        assert need > 0  # this case really runs a kernel that uses scratch
     y_ref, h_ref = _reference(xd)
     torch.cuda.synchronize()
     assert ss.ss_last_device_error() == ss.SS_OK
@@ -66,6 +71,8 @@ def test_noalloc_matches_workspace_entry_point(shape, dtype, workers):
         assert ss.ss_last_device_error() == ss.SS_OK
         assert rel_err(y.cpu().numpy(), y_ref.cpu().numpy()) <= TOL[dtype], f"call {call}"
         assert rel_err(h.cpu().numpy(), h_ref.cpu().numpy()) <= TOL[dtype], f"call {call}"
+        assert rel_err(y.cpu().numpy(), yo) <= TOL[dtype], f"call {call} vs oracle"
+        assert rel_err(h.cpu().numpy(), ho) <= TOL[dtype], f"call {call} vs oracle"
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
