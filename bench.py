@@ -713,6 +713,9 @@ def main():
     ap.add_argument("--op", default="scan", choices=["scan", "step", "bwd"])
     ap.add_argument("--workload", default=None,
                     choices=sorted(I.WORKLOADS) + sorted(I.STEP_WORKLOADS))
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="override the workload's sequence length (a shorter proxy of the same "
+                         "batch, width and distributions, for profiling captures)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--zoh", action="store_true", help="exact zero-order-hold B_bar")
@@ -750,6 +753,11 @@ def main():
               flush=True)
         return
     w = I.WORKLOADS[args.workload or DEFAULT_WORKLOAD]
+    if args.seqlen:
+        import dataclasses
+
+        w = dataclasses.replace(w, name=w.name.replace(f"_l{w.seqlen}_", f"_l{args.seqlen}_"),
+                                seqlen=args.seqlen)
 
     if args.impl == "reference":
         line = run_reference_arm(args, w)

@@ -50,6 +50,35 @@ enum {
 
 ss_status ss_debug_inject(int what, long long value);
 
+/*
+ * ss_debug_pointwise -- evaluate one of the scan kernels' pointwise functions
+ * element by element on the device, so that a test can compare it with
+ * float64 over its input range: y[i] = f(x[i]) for i < n.
+ *
+ *   fn  SS_PW_SOFTPLUS, SS_PW_SILU: softplus(x) = log(1 + e^x) and
+ *       SiLU(x) = x sigmoid(x) as the forward kernel evaluates them (one
+ *       special-function op for softplus, two for SiLU);
+ *       SS_PW_SOFTPLUS2, SS_PW_SILU2: the packed forms, on pairs (x[2i], x[2i+1]);
+ *       SS_PW_EXP2_NEG_FMA: 2^x for x <= 0 by polynomial on the FMA pipe
+ *       (x is clamped at -126);
+ *       SS_PW_RCP_1_2: 1/x for x in [1, 2] by Newton-Raphson on the FMA pipe;
+ *       SS_PW_EX2: the special-function unit's 2^x (ex2.approx.ftz).
+ *   x, y  device float arrays of n elements (4-byte aligned; may not overlap).
+ *
+ * Asynchronous on `stream`.  SS_ERR_INVALID_ARG for an unknown fn, n < 0 or
+ * null or misaligned pointers with n > 0; SS_ERR_CUDA if the launch fails.
+ */
+enum {
+  SS_PW_SOFTPLUS = 0,
+  SS_PW_SILU = 1,
+  SS_PW_SOFTPLUS2 = 2,
+  SS_PW_SILU2 = 3,
+  SS_PW_EXP2_NEG_FMA = 4,
+  SS_PW_RCP_1_2 = 5,
+  SS_PW_EX2 = 6
+};
+ss_status ss_debug_pointwise(int fn, const float* x, float* y, int64_t n, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

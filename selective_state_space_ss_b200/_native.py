@@ -24,7 +24,8 @@ SS_F32, SS_BF16 = 0, 1
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
             "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc",
             "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv", "ss_scan_fwd_zoh",
-            "ss_scan_bwd", "ss_scan_bwd_workspace_bytes", "ss_scan_fwd_train")
+            "ss_scan_bwd", "ss_scan_bwd_workspace_bytes", "ss_scan_fwd_train",
+            "ss_debug_pointwise")
 
 # bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
 SS_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -32,6 +33,9 @@ SS_NOALLOC_SCRATCH_BYTES = 4 << 20
 # test hooks (include/ss_scan_debug.h)
 (SS_DEBUG_CLEAR, SS_DEBUG_FORCE_WORKERS, SS_DEBUG_SKIP_PUBLISH, SS_DEBUG_SPIN_LIMIT,
  SS_DEBUG_STEP_SIMPLE, SS_DEBUG_FORCE_SEGMENTS) = range(6)
+# pointwise functions ss_debug_pointwise evaluates (include/ss_scan_debug.h)
+(SS_PW_SOFTPLUS, SS_PW_SILU, SS_PW_SOFTPLUS2, SS_PW_SILU2, SS_PW_EXP2_NEG_FMA, SS_PW_RCP_1_2,
+ SS_PW_EX2) = range(7)
 
 
 class SSError(RuntimeError):
@@ -88,6 +92,8 @@ def load_library():
         lib.ss_scan_bwd_workspace_bytes.argtypes = [i64, i64, i64, ci]
         lib.ss_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.ss_scan_step.restype = ci
+        lib.ss_debug_pointwise.argtypes = [ci, vp, vp, i64, vp]
+        lib.ss_debug_pointwise.restype = ci
         _lib = lib
         return lib
 
@@ -119,6 +125,20 @@ def ss_debug_inject(what: int, value: int = 0) -> None:
     st = load_library().ss_debug_inject(int(what), int(value))
     if st != SS_OK:
         raise SSError(st, "ss_debug_inject")
+
+
+def ss_debug_pointwise(fn: int, x, stream=None):
+    """Evaluate one of the kernels' pointwise functions on a CUDA float32 tensor
+    (test hook, include/ss_scan_debug.h); returns a new tensor."""
+    if x.device.type != "cuda" or x.dtype != torch.float32:
+        raise ValueError("x must be a float32 CUDA tensor")
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    st = load_library().ss_debug_pointwise(int(fn), x.data_ptr(), y.data_ptr(), x.numel(),
+                                           _stream_handle(stream, x.device))
+    if st != SS_OK:
+        raise SSError(st, "ss_debug_pointwise")
+    return y
 
 
 def _ptr(t):

@@ -6,7 +6,8 @@ Prints C initialisers.  Each fit is a weighted least-squares polynomial on a
 dense grid (Chebyshev-distributed nodes), solved in float64, then the
 coefficients are rounded to float32 and the worst error of the float32 Horner
 evaluation is reported.  The constants in pointwise.cuh are this script's
-output; tests/test_pointwise_fits.py re-runs the fits and checks them.
+output; tests/test_pointwise_fits.py re-runs the fits, checks them against the header
+and evaluates every function on the device against float64.
 
 Fits
   log1p_over:  log1p(e) / e  on e in [0, 1]        (softplus = max(x,0) + log1p(e^-|x|))

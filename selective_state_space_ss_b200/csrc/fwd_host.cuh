@@ -164,6 +164,9 @@ bool make_plan(int64_t batch, int64_t dim, int64_t seqlen, Plan* p) {
   return true;
 }
 
+template <typename E, int N>
+struct FixTag {};  // one once-per-device cache per correction kernel
+
 template <class CF>
 ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
                          cudaStream_t stream) {
@@ -210,11 +213,26 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
   f.seg_len = p.seg_chunks * CF::T;
   f.nseg = p.nseg;
   f.softplus = a.softplus;
-  f.vec = a.vec;  // 16-byte aligned rows: L a multiple of 4 (fp32) or 8 (bf16)
+  using E = typename CF::Elem;
+  using FS = FixStage<E, CF::N>;
+  const bool bf16 = sizeof(E) == 2;
+  FixMaps fm;
+  memset(&fm, 0, sizeof fm);
+  // TMA blocks need the forward's 16-byte aligned rows (a.vec)
+  f.tma = a.vec && encode_3d(&fm.delta, a.delta, bf16, a.seqlen, a.dim, a.batch, kFixBlock, 1) &&
+          encode_3d(&fm.z, a.z ? a.z : a.delta, bf16, a.seqlen, a.dim, a.batch, kFixBlock, 1) &&
+          encode_3d(&fm.y, a.y, false, a.seqlen, a.dim, a.batch, kFixBlock, 1) &&
+          (!FS::STAGE_C || encode_3d(&fm.C, a.C, bf16, a.seqlen, CF::N, a.batch, kFixBlock, CF::N));
   const int64_t tasks = a.batch * a.dim * (p.nseg - 1);
   const int64_t blocks = (tasks + kFixWarps - 1) / kFixWarps;
   if (blocks > INT_MAX) return SS_ERR_INVALID_ARG;
-  scan_fix_kernel<typename CF::Elem, CF::N><<<(unsigned)blocks, kFixWarps * 32, 0, stream>>>(f);
+  if (once_per_device<FixTag<E, CF::N>>([] {
+        return cudaFuncSetAttribute(scan_fix_kernel<E, CF::N>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    FS::SMEM) == cudaSuccess;
+      }) != 1)
+    return SS_ERR_CUDA;
+  scan_fix_kernel<E, CF::N><<<(unsigned)blocks, kFixWarps * 32, FS::SMEM, stream>>>(f, fm);
   return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
@@ -230,8 +248,13 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
 #define SS_N16_T 32
 #endif
 
+// Channels per lane of the plain forward at N = 16 (the variants use one).
+#ifndef SS_N16_CPL
+#define SS_N16_CPL 1
+#endif
 template <typename E, bool CV = false, bool Z = false, bool TR = false>
-using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, 1, CV, Z, TR>;
+using Cfg16 = ChunkedCfg<E, 16, SS_N16_K, SS_N16_W, SS_N16_T, (CV || Z || TR) ? 1 : SS_N16_CPL,
+                         CV, Z, TR>;
 #ifndef SS_N32_K
 #define SS_N32_K 4
 #endif

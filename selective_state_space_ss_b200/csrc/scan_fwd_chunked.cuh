@@ -25,6 +25,12 @@
 // associative operator of "Mamba 选择性机制", sec. 3.1, is not needed here
 // because no thread ever holds a time range whose carry-in is unknown.
 //
+// With two channels per lane (CPL = 2) a lane keeps the same G states of two
+// channels and packs its fp32x2 arithmetic over the channel pair: the pair's
+// Delta and w arrive together from shared memory, and every B_t[n], C_t[n] a
+// lane widens serves both channels (half the shared-memory traffic and
+// conversions per state of the one-channel layout).
+//
 // Shared-memory layouts are chosen so that each quarter-warp (the unit a
 // 16-byte access is serviced in) touches distinct banks.  Rows whose start
 // is not 16-byte aligned (odd L, offset views) take an element-wise load
@@ -86,28 +92,27 @@ struct CkptCtx {
   int64_t left;
 };
 
-// Tin: input dtype; N: states per channel; K: lanes per channel; NWARPS: warps
-// per CTA; T: timesteps per chunk; WT: warps that split each chunk in time
-// (1: every warp walks the whole chunk for its own channels; >1: WT warps
-// share one set of channels, each scanning T/WT consecutive steps of the
-// chunk, joined with the pages' associative operator).  CONV: the u input is
-// the pre-convolution x, staged with HALO earlier steps per row, and phase 1
-// forms u = SiLU(conv(x) + bias).  ZOH: exact zero-order-hold B_bar.  TRAIN:
-// the state at every 16-step chunk start is written out for the backward.
-template <typename Tin, int N_, int K_, int NWARPS_, int T_, int WT_ = 1, bool CONV_ = false,
+// Tin: input dtype; N: states per channel; K: lanes per channel (per channel
+// pair with CPL = 2); NWARPS: warps per CTA; T: timesteps per chunk; CPL:
+// channels per lane (1 or 2).  CONV: the u input is the pre-convolution x,
+// staged with HALO earlier steps per row, and phase 1 forms
+// u = SiLU(conv(x) + bias).  ZOH: exact zero-order-hold B_bar.  TRAIN: the
+// state at every 16-step chunk start is written out for the backward.  The
+// variants (CONV, ZOH, TRAIN) use one channel per lane.
+template <typename Tin, int N_, int K_, int NWARPS_, int T_, int CPL_ = 1, bool CONV_ = false,
           bool ZOH_ = false, bool TRAIN_ = false>
 struct ChunkedCfg {
   using Elem = Tin;
   static constexpr int N = N_;            // states per channel
-  static constexpr int K = K_;            // lanes per channel
-  static constexpr int G = N / K;         // states per lane
+  static constexpr int K = K_;            // lanes per channel (or channel pair)
+  static constexpr int G = N / K;         // states per lane and channel
+  static constexpr int CPL = CPL_;        // channels per lane
+  static constexpr int HP = CPL == 1 ? G / 2 : G;  // float2 registers per lane state
   static constexpr int NWARPS = NWARPS_;
   static constexpr int T = T_;            // timesteps per chunk
-  static constexpr int WT = WT_;          // time-split warps per channel set
-  static constexpr int WC = NWARPS / WT;  // warps across channels
-  static constexpr int TW = T / WT;       // steps per warp per chunk
-  static constexpr int CPW = 32 / K;      // channels per warp
-  static constexpr int CH = WC * CPW;     // channels per CTA
+  static constexpr int LGW = 32 / K;      // lane groups per warp
+  static constexpr int LG = NWARPS * LGW; // lane groups per CTA
+  static constexpr int CH = LG * CPL;     // channels per CTA
   static constexpr int NT = NWARPS * 32;
   static constexpr int ES = (int)sizeof(Tin);
   static constexpr int QPR = T / 4;                  // 4-step quads per row
@@ -127,7 +132,11 @@ struct ChunkedCfg {
   static constexpr int OFF_B_T = X_TILE + 2 * ACT_TILE;
   static constexpr int OFF_C_T = OFF_B_T + SEL_TILE;
   static constexpr int RAW_BYTES = OFF_C_T + SEL_TILE;
-  static constexpr int DW_STRIDE = CH + 1;           // float4 per quad row (odd: conflict-free)
+  // Delta and w per (quad, channel) as float4 of four steps; with CPL = 2 a
+  // lane group's two float4 hold its channel pair interleaved by step:
+  // {c0 t0, c1 t0, c0 t1, c1 t1}, {c0 t2, c1 t2, c0 t3, c1 t3}.  The row pitch
+  // (float4 units) is odd, so a quarter-warp's writes hit distinct banks.
+  static constexpr int DW_STRIDE = CH + 1;
   static constexpr int DW_BYTES = QPR * DW_STRIDE * 16;
   static constexpr int PAIR_BYTES = 4 * ES;          // one state pair: B_lo, B_hi, C_lo, C_hi
   static constexpr int BC_BLOCK = 2 * PAIR_BYTES;    // two pairs: four states
@@ -143,12 +152,9 @@ struct ChunkedCfg {
   static constexpr int OFF_DWW = OFF_DWD + DW_BYTES;
   static constexpr int OFF_BC = OFF_DWW + DW_BYTES;
   static constexpr int OFF_SY = OFF_BC + BC_BYTES;
-  // time-split aggregates: (prod A_bar, local end state) per warp and lane state
-  static constexpr int AGG_FLOATS = WT > 1 ? WT * WC * 32 * G : 0;
-  static constexpr int OFF_AGG = OFF_SY + SY_BYTES;
   // CONV: u = SiLU(conv) per (quad, channel), for phase 3's D u
   static constexpr int SU_BYTES = CONV ? DW_BYTES : 0;
-  static constexpr int OFF_SU = OFF_AGG + 2 * AGG_FLOATS * 4;
+  static constexpr int OFF_SU = OFF_SY + SY_BYTES;
   // ZOH: 1 / Delta per (quad, channel)
   static constexpr int DWI_BYTES = ZOH ? DW_BYTES : 0;
   static constexpr int OFF_DWI = OFF_SU + SU_BYTES;
@@ -159,22 +165,30 @@ struct ChunkedCfg {
   static constexpr int SMEM_CTAS = 227 * 1024 / (SMEM_USED + 128 + 1024);
   static constexpr int THREAD_CTAS = 512 / NT > 0 ? 512 / NT : 1;
   static constexpr int MIN_CTAS = SMEM_CTAS < THREAD_CTAS ? SMEM_CTAS : THREAD_CTAS;
-  static constexpr int ITEMS = CH * QPR;             // (channel, quad) items per chunk
+  // phase 1 works on (lane group, quad) items (CPL channels x 4 steps each),
+  // phase 3 on (channel, quad) items
+  static constexpr int ITEMS1 = LG * QPR;
+  static constexpr int ITEMS1_PER_THREAD = (ITEMS1 + NT - 1) / NT;
+  static constexpr int ITEMS = CH * QPR;
   static constexpr int ITEMS_PER_THREAD = (ITEMS + NT - 1) / NT;
 
   static_assert(N % K == 0 && 32 % K == 0, "lane split");
-  static_assert(NWARPS % WT == 0 && T % (4 * WT) == 0, "time split");
-  static_assert(G % 2 == 0, "a lane holds whole state pairs");
+  static_assert(CPL == 1 || CPL == 2, "channels per lane");
+  static_assert(CPL == 1 || (!CONV && !ZOH && !TRAIN), "the variants use one channel per lane");
+  static_assert(CPL == 2 || G % 2 == 0, "a lane holds whole state pairs");
+  static_assert(G % 4 == 0 || (CPL == 1 && G % 2 == 0), "B, C loads of whole state pairs");
   static_assert(T % 8 == 0 && (T * ES) % 16 == 0 && T <= 256 && CH <= 256, "TMA box");
   static_assert(ACT_TILE % 128 == 0 && SEL_TILE % 128 == 0 && X_TILE % 128 == 0,
                 "TMA destinations 128-byte aligned");
   static_assert(!CONV || ((HALO * ES) % 16 == 0 && HALO >= kConvTaps - 1 && XT <= 256),
                 "convolution halo");
-  static_assert(T % 16 == 0 && (WT == 1 || 16 % TW == 0),
-                "16-step checkpoints fall on quad or warp-segment starts");
+  static_assert(T % 16 == 0, "16-step checkpoints fall on quad starts");
   static_assert(DW_BYTES % 16 == 0 && BC_BYTES % 16 == 0, "alignment");
-  static_assert(ITEMS % NT == 0 || ITEMS < NT, "whole items per thread");
-  static constexpr bool ITEM_GUARD = ITEMS < NT;  // some threads have no item
+  static_assert((ITEMS % NT == 0 || ITEMS < NT) && (ITEMS1 % NT == 0 || ITEMS1 < NT),
+                "whole items per thread");
+  static_assert(QPR <= 32 && (NT % QPR) == 0, "an item's quads are lanes of one warp");
+  static constexpr bool ITEM_GUARD = ITEMS < NT;    // some threads have no phase-3 item
+  static constexpr bool ITEM1_GUARD = ITEMS1 < NT;  // some threads have no phase-1 item
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -255,72 +269,91 @@ __device__ __forceinline__ void load_chunk_scalar(const FwdArgs& a, typename CF:
 // (bias, convolution taps, D) stay in its registers.
 template <class CF>
 struct ConvRegs {  // per-item convolution taps, right-aligned: tap kConvTaps-1 meets step t
-  float w[CF::CONV ? CF::ITEMS_PER_THREAD : 1][kConvTaps];
-  float b[CF::CONV ? CF::ITEMS_PER_THREAD : 1];
+  float w[CF::CONV ? CF::ITEMS1_PER_THREAD : 1][kConvTaps];
+  float b[CF::CONV ? CF::ITEMS1_PER_THREAD : 1];
 };
 
 template <class CF, bool kFull>
 __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem* raw,
                                        float4* dwD, float4* dwW, float4* dwI, float4* su,
                                        unsigned char* bc,
-                                       const float (&bias_it)[CF::ITEMS_PER_THREAD],
+                                       const float (&bias_it)[CF::ITEMS1_PER_THREAD][CF::CPL],
                                        const ConvRegs<CF>& cv, int64_t d0, int64_t t0,
-                                       double (&dsum)[CF::ITEMS_PER_THREAD], bool seg) {
+                                       double (&dsum)[CF::ITEMS1_PER_THREAD][CF::CPL], bool seg) {
   using E = typename CF::Elem;
   const int tid = threadIdx.x;
   const E* rawD = raw + CF::CH * CF::XT;
 #pragma unroll
-  for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+  for (int it = 0; it < CF::ITEMS1_PER_THREAD; ++it) {
     const int i = tid + it * CF::NT;
-    if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
-    const int c = i / CF::QPR, q = i - c * CF::QPR;
-    const float4 dl = load4_f32(rawD + c * CF::T + 4 * q);
-    float4 uu;
-    if constexpr (CF::CONV) {
-      // u = SiLU(b + sum_k w[k] x[t - (kConvTaps-1) + k]); the row holds x from
-      // step t0 - HALO, so steps t0+4q-4 .. t0+4q+3 are elements 4q+HALO-4 ..
-      const E* xr = raw + c * CF::XT + 4 * q + CF::HALO - 4;
-      const float4 xa = load4_f32(xr), xb = load4_f32(xr + 4);
-      const float win[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-      float o[4];
+    if (CF::ITEM1_GUARD && i >= CF::ITEMS1) break;
+    const int lg = i / CF::QPR, q = i - lg * CF::QPR;
+    float delt[CF::CPL][4], w[CF::CPL][4];
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        float acc = cv.b[it];
+    for (int cc = 0; cc < CF::CPL; ++cc) {
+      const int c = lg * CF::CPL + cc;
+      const float4 dl = load4_f32(rawD + c * CF::T + 4 * q);
+      float4 uu;
+      if constexpr (CF::CONV) {
+        // u = SiLU(b + sum_k w[k] x[t - (kConvTaps-1) + k]); the row holds x from
+        // step t0 - HALO, so steps t0+4q-4 .. t0+4q+3 are elements 4q+HALO-4 ..
+        const E* xr = raw + c * CF::XT + 4 * q + CF::HALO - 4;
+        const float4 xa = load4_f32(xr), xb = load4_f32(xr + 4);
+        const float win[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        float o[4];
 #pragma unroll
-        for (int k = 0; k < kConvTaps; ++k) acc = fmaf(cv.w[it][k], win[k4 + 5 - kConvTaps + k], acc);
-        o[k4] = acc;
+        for (int k4 = 0; k4 < 4; ++k4) {
+          float acc = cv.b[it];
+#pragma unroll
+          for (int k = 0; k < kConvTaps; ++k) acc = fmaf(cv.w[it][k], win[k4 + 5 - kConvTaps + k], acc);
+          o[k4] = acc;
+        }
+        const float2 u01 = silu_fast2(make_float2(o[0], o[1]));
+        const float2 u23 = silu_fast2(make_float2(o[2], o[3]));
+        uu = make_float4(u01.x, u01.y, u23.x, u23.y);
+        su[q * CF::DW_STRIDE + c] = uu;
+      } else {
+        uu = load4_f32(raw + c * CF::XT + 4 * q);
       }
-      const float2 u01 = silu_fast2(make_float2(o[0], o[1]));
-      const float2 u23 = silu_fast2(make_float2(o[2], o[3]));
-      uu = make_float4(u01.x, u01.y, u23.x, u23.y);
-      su[q * CF::DW_STRIDE + c] = uu;
-    } else {
-      uu = load4_f32(raw + c * CF::XT + 4 * q);
-    }
-    const float bias = bias_it[it];
-    const float2 b2 = make_float2(bias, bias);
-    float2 x01 = __fadd2_rn(make_float2(dl.x, dl.y), b2);
-    float2 x23 = __fadd2_rn(make_float2(dl.z, dl.w), b2);
-    if (a.softplus) {
-      x01 = softplus_fast2(x01);
-      x23 = softplus_fast2(x23);
-    }
-    float delt[4] = {x01.x, x01.y, x23.x, x23.y};
-    if constexpr (!kFull) {
-      // padding steps and channels: A_bar = 1, B_bar u = 0 (state unchanged)
+      const float bias = bias_it[it][cc];
+      const float2 b2 = make_float2(bias, bias);
+      float2 x01 = __fadd2_rn(make_float2(dl.x, dl.y), b2);
+      float2 x23 = __fadd2_rn(make_float2(dl.z, dl.w), b2);
+      if (a.softplus) {
+        x01 = softplus_fast2(x01);
+        x23 = softplus_fast2(x23);
+      }
+      delt[cc][0] = x01.x;
+      delt[cc][1] = x01.y;
+      delt[cc][2] = x23.x;
+      delt[cc][3] = x23.y;
+      if constexpr (!kFull) {
+        // padding steps and channels: A_bar = 1, B_bar u = 0 (state unchanged)
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (d0 + c >= a.dim || t0 + 4 * q + k >= a.seqlen) delt[k] = 0.f;
+        for (int k = 0; k < 4; ++k)
+          if (d0 + c >= a.dim || t0 + 4 * q + k >= a.seqlen) delt[cc][k] = 0.f;
+      }
+      if (seg) dsum[it][cc] += (double)((delt[cc][0] + delt[cc][1]) + (delt[cc][2] + delt[cc][3]));
+      const float2 w01 = __fmul2_rn(make_float2(delt[cc][0], delt[cc][1]), make_float2(uu.x, uu.y));
+      const float2 w23 = __fmul2_rn(make_float2(delt[cc][2], delt[cc][3]), make_float2(uu.z, uu.w));
+      w[cc][0] = w01.x;
+      w[cc][1] = w01.y;
+      w[cc][2] = w23.x;
+      w[cc][3] = w23.y;
     }
-    if (seg) dsum[it] += (double)((delt[0] + delt[1]) + (delt[2] + delt[3]));
-    const float2 w01 = __fmul2_rn(make_float2(delt[0], delt[1]), make_float2(uu.x, uu.y));
-    const float2 w23 = __fmul2_rn(make_float2(delt[2], delt[3]), make_float2(uu.z, uu.w));
-    const float w[4] = {w01.x, w01.y, w23.x, w23.y};
-    dwD[q * CF::DW_STRIDE + c] = make_float4(delt[0], delt[1], delt[2], delt[3]);
-    dwW[q * CF::DW_STRIDE + c] = make_float4(w[0], w[1], w[2], w[3]);
-    if constexpr (CF::ZOH)  // 1/0 = inf on padding steps: the series branch of phi takes them
-      dwI[q * CF::DW_STRIDE + c] = make_float4(rcp_approx(delt[0]), rcp_approx(delt[1]),
-                                               rcp_approx(delt[2]), rcp_approx(delt[3]));
+    const int row = q * CF::DW_STRIDE + lg * CF::CPL;
+    if constexpr (CF::CPL == 1) {
+      dwD[row] = make_float4(delt[0][0], delt[0][1], delt[0][2], delt[0][3]);
+      dwW[row] = make_float4(w[0][0], w[0][1], w[0][2], w[0][3]);
+      if constexpr (CF::ZOH)  // 1/0 = inf on padding steps: the series branch of phi takes them
+        dwI[row] = make_float4(rcp_approx(delt[0][0]), rcp_approx(delt[0][1]),
+                               rcp_approx(delt[0][2]), rcp_approx(delt[0][3]));
+    } else {  // the channel pair interleaved by step
+      dwD[row] = make_float4(delt[0][0], delt[1][0], delt[0][1], delt[1][1]);
+      dwD[row + 1] = make_float4(delt[0][2], delt[1][2], delt[0][3], delt[1][3]);
+      dwW[row] = make_float4(w[0][0], w[1][0], w[0][1], w[1][1]);
+      dwW[row + 1] = make_float4(w[0][2], w[1][2], w[0][3], w[1][3]);
+    }
   }
   // B and C rows [n][t] -> [t][n/2 pairs][B_2p, B_2p+1, C_2p, C_2p+1]
   const E* rawB = raw + CF::OFF_B_T / CF::ES;
@@ -450,8 +483,8 @@ __device__ __forceinline__ float2 zoh_phi2(float2 x2, float2 e, float2 inv_a, fl
 template <class CF>
 __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW, const float4* dwI,
                                        const unsigned char* bc, float* sy,
-                                       float2 (&h)[CF::G / 2], const float2 (&a2)[CF::G / 2],
-                                       const float2 (&ia)[CF::G / 2], int c, int j,
+                                       float2 (&h)[CF::HP], const float2 (&a2)[CF::HP],
+                                       const float2 (&ia)[CF::HP], int c, int j,
                                        const CkptCtx& ck) {
   constexpr int G2 = CF::G / 2;  // state pairs per lane
   const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
@@ -498,113 +531,52 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW, con
   }
 }
 
-// The time-split recurrence (WT > 1).  Warp wt scans steps
-// [wt TW, (wt+1) TW) of the chunk from h = 0 while tracking the product of
-// its decays P_t = prod A_bar and the fix-up coefficients Q_t = C_t P_t; the
-// WT warps then swap their aggregates (P_end, h_end) through shared memory and
-// each folds the chunk's carry-in through the aggregates before it with the
-// operator (a1,b1) then (a2,b2) = (a2 a1, a2 b1 + b2) ("Mamba 选择性机制",
-// sec. 3.1), which gives its own carry-in h_in exactly: h_t = local h_t +
-// P_t h_in, so the readout is corrected by sum_n Q_t[n] h_in[n].  Every warp
-// folds all WT aggregates, so all of them leave with the chunk's carry-out in
-// h.  No ex2 is evaluated twice.
+// The recurrence with two channels per lane (CPL = 2): the lane's G states n
+// of channels c0 = 2 lg and c1 = 2 lg + 1 sit in G float2 registers
+// {h_c0[n], h_c1[n]}, and each fp32x2 operation advances one state of both
+// channels: A_bar = 2^({Delta_c0, Delta_c1} A log2 e), h = A_bar h + {w_c0, w_c1}
+// B_t[n].  B_t[n] and C_t[n] are widened once and used for both channels; the
+// partial readouts of the two channels go to their own rows of sy.
 template <class CF>
-__device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dwW,
-                                             const float4* dwI, const unsigned char* bc,
-                                             float* sy, float* aggP, float* aggH,
-                                             float2 (&h)[CF::G / 2],
-                                             const float2 (&a2)[CF::G / 2],
-                                             const float2 (&ia)[CF::G / 2], int c, int j, int wt,
-                                             int lane_g, const CkptCtx& ck) {
-  constexpr int G2 = CF::G / 2;
-  const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
-  float2 hl[G2], P[G2];
-#pragma unroll
-  for (int g = 0; g < G2; ++g) {
-    hl[g] = make_float2(0.f, 0.f);
-    P[g] = make_float2(1.f, 1.f);
-  }
-  float2 Q[CF::TW][G2];
-  float s[CF::TW];
-#pragma unroll
-  for (int q = 0; q < CF::TW / 4; ++q) {
-    const int qq = wt * (CF::TW / 4) + q;
-    const float4 D4 = dwD[qq * CF::DW_STRIDE + c];
-    const float4 W4 = dwW[qq * CF::DW_STRIDE + c];
-    const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
-    const float ws[4] = {W4.x, W4.y, W4.z, W4.w};
-    float idl[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (CF::ZOH) {
-      const float4 I4 = dwI[qq * CF::DW_STRIDE + c];
-      idl[0] = I4.x; idl[1] = I4.y; idl[2] = I4.z; idl[3] = I4.w;
-    }
+__device__ __forceinline__ void phase2_cpl2(const float4* dwD, const float4* dwW,
+                                            const unsigned char* bc, float* sy,
+                                            float2 (&h)[CF::HP], const float2 (&a2)[CF::HP],
+                                            int lg, int j) {
+  constexpr int G = CF::G;
+  const unsigned char* bcj = bc + j * (G / 2) * CF::PAIR_BYTES;
+  float* sy0 = sy + (2 * lg * CF::K + j) * CF::SY_STRIDE;
+  float* sy1 = sy0 + CF::K * CF::SY_STRIDE;
+#pragma unroll kPhase2Unroll
+  for (int q = 0; q < CF::QPR; ++q) {
+    const int row = q * CF::DW_STRIDE + 2 * lg;
+    const float4 D01 = dwD[row], D23 = dwD[row + 1];
+    const float4 W01 = dwW[row], W23 = dwW[row + 1];
+    const float2 dls[4] = {make_float2(D01.x, D01.y), make_float2(D01.z, D01.w),
+                           make_float2(D23.x, D23.y), make_float2(D23.z, D23.w)};
+    const float2 ws[4] = {make_float2(W01.x, W01.y), make_float2(W01.z, W01.w),
+                          make_float2(W23.x, W23.y), make_float2(W23.z, W23.w)};
+    float s0[4], s1[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int t = 4 * q + k;
-      const unsigned char* row = bcj + (4 * qq + k) * CF::BC_ROW;
-      const float2 dl2 = make_float2(dls[k], dls[k]);
-      const float2 w2 = make_float2(ws[k], ws[k]);
-      float2 acc = make_float2(0.f, 0.f);
-      float2 bb[G2], cc[G2];
-      bc_pairs<CF, G2>(row, bb, cc);
+      float2 bb[G / 2], cc[G / 2];
+      bc_pairs<CF, G / 2>(bcj + (4 * q + k) * CF::BC_ROW, bb, cc);
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int g = 0; g < G2; ++g) {
-        const float2 x = __fmul2_rn(dl2, a2[g]);
+      for (int n = 0; n < G; ++n) {
+        const float bn = (n & 1) ? bb[n >> 1].y : bb[n >> 1].x;
+        const float cn = (n & 1) ? cc[n >> 1].y : cc[n >> 1].x;
+        const float2 x = __fmul2_rn(dls[k], a2[n]);
         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        float2 wb;
-        if constexpr (CF::ZOH)
-          wb = __fmul2_rn(__fmul2_rn(zoh_phi2(x, e, ia[g], make_float2(idl[k], idl[k])), w2), bb[g]);
-        else
-          wb = __fmul2_rn(w2, bb[g]);
-        hl[g] = __ffma2_rn(e, hl[g], wb);
-        P[g] = __fmul2_rn(e, P[g]);
-        acc = __ffma2_rn(cc[g], hl[g], acc);
-        Q[t][g] = __fmul2_rn(cc[g], P[g]);
+        const float2 wb = make_float2(ws[k].x * bn, ws[k].y * bn);
+        h[n] = __ffma2_rn(e, h[n], wb);
+        acc0 = fmaf(cn, h[n].x, acc0);
+        acc1 = fmaf(cn, h[n].y, acc1);
       }
-      s[t] = acc.x + acc.y;
+      s0[k] = acc0;
+      s1[k] = acc1;
     }
-  }
-  // publish this warp's aggregate: [wt][lane in channel set][state]
-  float2* myP = reinterpret_cast<float2*>(aggP + (wt * CF::WC * 32 + lane_g) * CF::G);
-  float2* myH = reinterpret_cast<float2*>(aggH + (wt * CF::WC * 32 + lane_g) * CF::G);
-#pragma unroll
-  for (int g = 0; g < G2; ++g) {
-    myP[g] = P[g];
-    myH[g] = hl[g];
-  }
-  __syncthreads();
-  float2 hin[G2];
-#pragma unroll
-  for (int v = 0; v < CF::WT; ++v) {
-    if (v == wt) {
-#pragma unroll
-      for (int g = 0; g < G2; ++g) hin[g] = h[g];
-    }
-    const float2* vP = reinterpret_cast<const float2*>(aggP + (v * CF::WC * 32 + lane_g) * CF::G);
-    const float2* vH = reinterpret_cast<const float2*>(aggH + (v * CF::WC * 32 + lane_g) * CF::G);
-#pragma unroll
-    for (int g = 0; g < G2; ++g) h[g] = __ffma2_rn(vP[g], h[g], vH[g]);
-  }
-  // hin is the state before this warp's first step: a 16-step checkpoint when
-  // the segment starts on one
-  if (CF::TRAIN && ck.p && (wt * CF::TW) % 16 == 0 && wt * CF::TW < ck.left) {
-    float2* dst = reinterpret_cast<float2*>(ck.p + (wt * CF::TW / 16) * ck.stride);
-#pragma unroll
-    for (int g = 0; g < G2; ++g) dst[g] = hin[g];
-  }
-  float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE + wt * CF::TW;
-#pragma unroll
-  for (int q = 0; q < CF::TW / 4; ++q) {
-    float out[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int t = 4 * q + k;
-      float2 fix = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int g = 0; g < G2; ++g) fix = __ffma2_rn(Q[t][g], hin[g], fix);
-      out[k] = s[t] + (fix.x + fix.y);
-    }
-    *reinterpret_cast<float4*>(syr + 4 * q) = make_float4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<float4*>(sy0 + 4 * q) = make_float4(s0[0], s0[1], s0[2], s0[3]);
+    *reinterpret_cast<float4*>(sy1 + 4 * q) = make_float4(s1[0], s1[1], s1[2], s1[3]);
   }
 }
 
@@ -790,7 +762,7 @@ __device__ __forceinline__ void load_conv_regs(const FwdArgs& a, int64_t d0, Con
   if constexpr (CF::CONV) {
     const int W = a.conv_width;
 #pragma unroll
-    for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+    for (int it = 0; it < CF::ITEMS1_PER_THREAD; ++it) {
       const int64_t d = d0 + (threadIdx.x + it * CF::NT) / CF::QPR;
       const bool ok = d < a.dim;
 #pragma unroll
@@ -803,15 +775,86 @@ __device__ __forceinline__ void load_conv_regs(const FwdArgs& a, int64_t d0, Con
   }
 }
 
+// A lane's states of its CPL channels as HP float2 registers (see phase2 and
+// phase2_cpl2 for the packing), read from or written to [channel][N] fp32
+// rows; row(cc) gives the row of the lane's channel cc, or null (zeros; not
+// written).
+template <class CF, class RowFn>
+__device__ __forceinline__ void lane_load_state(float2 (&h)[CF::HP], RowFn row, int j) {
+  if constexpr (CF::CPL == 1) {
+    const float* r = row(0);
+#pragma unroll
+    for (int g = 0; g < CF::HP; ++g) {
+      const int n = j * CF::G + 2 * g;
+      h[g] = r ? make_float2(r[n], r[n + 1]) : make_float2(0.f, 0.f);
+    }
+  } else {
+    const float* r0 = row(0);
+    const float* r1 = row(1);
+#pragma unroll
+    for (int g = 0; g < CF::HP; ++g) {
+      const int n = j * CF::G + g;
+      h[g] = make_float2(r0 ? r0[n] : 0.f, r1 ? r1[n] : 0.f);
+    }
+  }
+}
+
+template <class CF, class RowFn>
+__device__ __forceinline__ void lane_store_state(const float2 (&h)[CF::HP], RowFn row, int j) {
+  if constexpr (CF::CPL == 1) {
+    float* r = row(0);
+    if (r)
+#pragma unroll
+      for (int g = 0; g < CF::HP; ++g) {
+        const int n = j * CF::G + 2 * g;
+        r[n] = h[g].x;
+        r[n + 1] = h[g].y;
+      }
+  } else {
+    float* r0 = row(0);
+    float* r1 = row(1);
+#pragma unroll
+    for (int g = 0; g < CF::HP; ++g) {
+      const int n = j * CF::G + g;
+      if (r0) r0[n] = h[g].x;
+      if (r1) r1[n] = h[g].y;
+    }
+  }
+}
+
+// The lane's decay constants A log2 e (and 1/A for the exact zero-order hold)
+// for channels d0 + lg CPL + cc, packed like its states (zeros past dim).
+template <class CF>
+__device__ __forceinline__ void lane_load_decay(const FwdArgs& a, int64_t d0, int lg, int j,
+                                                float2 (&a2)[CF::HP], float2 (&ia)[CF::HP]) {
+  if constexpr (CF::CPL == 1) {
+    const int64_t d = d0 + lg;
+#pragma unroll
+    for (int g = 0; g < CF::HP; ++g) load_decay<CF>(a, d, j * CF::G + 2 * g, d < a.dim, a2[g], ia[g]);
+  } else {
+    const int64_t e0 = d0 + 2 * lg, e1 = e0 + 1;
+#pragma unroll
+    for (int g = 0; g < CF::HP; ++g) {
+      const int n = j * CF::G + g;
+      const float A0 = e0 < a.dim ? __ldg(a.A + e0 * CF::N + n) : 0.f;
+      const float A1 = e1 < a.dim ? __ldg(a.A + e1 * CF::N + n) : 0.f;
+      a2[g] = make_float2(A0 * 1.4426950408889634f, A1 * 1.4426950408889634f);
+      ia[g] = make_float2(0.f, 0.f);
+    }
+  }
+}
+
 // -------------------------------------------------------------- kernel ---
 
-// kMulti = false: one channel group per CTA (gridDim = groups), a plain loop
-// over its chunks.  kMulti = true: balanced ranges with carry handoff.
+// kMulti = false: one channel group (or one segment of its sequence) per CTA,
+// a plain loop over its chunks.  kMulti = true: balanced ranges with carry
+// handoff.
 template <class CF, bool kMulti>
 __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     scan_fwd_chunked_kernel(const FwdArgs a, const __grid_constant__ FwdMaps maps,
                             const Sched sched) {
   using E = typename CF::Elem;
+  constexpr int HP = CF::HP, CPL = CF::CPL;
   extern __shared__ __align__(128) unsigned char smem_dyn[];
   // TMA destinations want 128-byte alignment; the dynamic window follows the
   // static arrays, so align its base explicitly (SMEM_BYTES has the slack).
@@ -822,9 +865,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   float4* dwW = reinterpret_cast<float4*>(smem + CF::OFF_DWW);
   unsigned char* bc = smem + CF::OFF_BC;
   float* sy = reinterpret_cast<float*>(smem + CF::OFF_SY);
-  float* aggP = reinterpret_cast<float*>(smem + CF::OFF_AGG);
-  float* aggH = aggP + CF::AGG_FLOATS;
-  float4* su = reinterpret_cast<float4*>(smem + CF::OFF_SU);  // CONV only
+  float4* su = reinterpret_cast<float4*>(smem + CF::OFF_SU);    // CONV only
+  float4* dwI = reinterpret_cast<float4*>(smem + CF::OFF_DWI);  // ZOH only
   __shared__ __align__(8) uint64_t bars[2];
 
   const int w = blockIdx.x;
@@ -846,14 +888,11 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   const bool has_z = a.z != nullptr;
   const bool tma = a.vec != 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wc = warp % CF::WC, wt = warp / CF::WC;  // channel warp, time-split slot
-  const int c = wc * CF::CPW + lane / CF::K;     // this lane's channel within the CTA
+  const int lg = warp * CF::LGW + lane / CF::K;  // this lane's group: channels lg CPL + cc
   const int j = lane % CF::K;                    // this lane's state group
-  const int lane_g = wc * 32 + lane;             // lane within its channel set
-  const bool writer = wt == 0;  // time-split warps hold the same carry: one writes it
-  float4* dwI = reinterpret_cast<float4*>(smem + CF::OFF_DWI);  // ZOH only
   const int64_t ck_nk = (a.seqlen + 15) / 16;
   // this lane's checkpoint slot for the chunk of batch row bb starting at t0
+  // (training variant, one channel per lane)
   auto ckpt_at = [&](int64_t bb, int64_t dd, bool ok, int64_t t0) {
     CkptCtx ck;
     ck.stride = a.dim * CF::N;
@@ -863,10 +902,35 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
                : nullptr;
     return ck;
   };
-  auto run_phase2 = [&](float2 (&hh)[CF::G / 2], const float2 (&aa)[CF::G / 2],
-                        const float2 (&ii)[CF::G / 2], const CkptCtx& ck) {
-    if constexpr (CF::WT == 1) phase2<CF>(dwD, dwW, dwI, bc, sy, hh, aa, ii, c, j, ck);
-    else phase2_split<CF>(dwD, dwW, dwI, bc, sy, aggP, aggH, hh, aa, ii, c, j, wt, lane_g, ck);
+  auto run_phase2 = [&](float2 (&hh)[HP], const float2 (&aa)[HP], const float2 (&ii)[HP],
+                        const CkptCtx& ck) {
+    if constexpr (CPL == 1) phase2<CF>(dwD, dwW, dwI, bc, sy, hh, aa, ii, lg, j, ck);
+    else phase2_cpl2<CF>(dwD, dwW, bc, sy, hh, aa, lg, j);
+  };
+  // [channel][N] rows of this lane's channels in a per-(b, d) array, for batch
+  // row bb of channel tile d0 (null past dim)
+  auto rows_in = [&](float* base, int64_t bb, int64_t d0) {
+    return [=](int cc) -> float* {
+      const int64_t d = d0 + lg * CPL + cc;
+      return (base && d < a.dim) ? base + (bb * a.dim + d) * CF::N : nullptr;
+    };
+  };
+  // per-item constants: bias per (phase-1 item, channel), D per phase-3 item
+  auto load_bias = [&](int64_t d0, float (&dst)[CF::ITEMS1_PER_THREAD][CPL]) {
+#pragma unroll
+    for (int it = 0; it < CF::ITEMS1_PER_THREAD; ++it)
+#pragma unroll
+      for (int cc = 0; cc < CPL; ++cc) {
+        const int64_t d = d0 + ((tid + it * CF::NT) / CF::QPR) * CPL + cc;
+        dst[it][cc] = (a.delta_bias && d < a.dim) ? __ldg(a.delta_bias + d) : 0.f;
+      }
+  };
+  auto load_D = [&](int64_t d0, float (&dst)[CF::ITEMS_PER_THREAD]) {
+#pragma unroll
+    for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
+      const int64_t d = d0 + (tid + it * CF::NT) / CF::QPR;
+      dst[it] = (a.D && d < a.dim) ? __ldg(a.D + d) : 0.f;
+    }
   };
 
   if (tma && tid == 0) {
@@ -882,31 +946,24 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     // chunk c_begin + k of the group ----
     const int64_t b = grp / sched.tiles_per_b;
     const int64_t d0 = (grp - b * sched.tiles_per_b) * CF::CH;
-    const int64_t d = d0 + c;
-    const bool chan_ok = d < a.dim;
     const bool full_tile = d0 + CF::CH <= a.dim;
     const bool segmented = sched.nseg > 1;
-    float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
-    double dsum[CF::ITEMS_PER_THREAD];
+    float bias_it[CF::ITEMS1_PER_THREAD][CPL], D_it[CF::ITEMS_PER_THREAD];
+    double dsum[CF::ITEMS1_PER_THREAD][CPL];
     ConvRegs<CF> cv;
+    load_bias(d0, bias_it);
+    load_D(d0, D_it);
 #pragma unroll
-    for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
-      const int64_t di = d0 + (tid + it * CF::NT) / CF::QPR;
-      bias_it[it] = (a.delta_bias && di < a.dim) ? __ldg(a.delta_bias + di) : 0.f;
-      D_it[it] = (a.D && di < a.dim) ? __ldg(a.D + di) : 0.f;
-      dsum[it] = 0.0;
-    }
+    for (int it = 0; it < CF::ITEMS1_PER_THREAD; ++it)
+#pragma unroll
+      for (int cc = 0; cc < CPL; ++cc) dsum[it][cc] = 0.0;
     load_conv_regs<CF>(a, d0, cv);
-    float2 h[CF::G / 2], a2[CF::G / 2], ia[CF::G / 2];
-#pragma unroll
-    for (int g = 0; g < CF::G / 2; ++g) {
-      const int n = j * CF::G + 2 * g;
-      // plain loads: h0 may be the last_state buffer this kernel writes; only
-      // the first segment starts from it (later ones start from zero)
-      const float* h0 = a.h0 + (b * a.dim + d) * CF::N + n;
-      h[g] = (a.h0 && chan_ok && seg == 0) ? make_float2(h0[0], h0[1]) : make_float2(0.f, 0.f);
-      load_decay<CF>(a, d, n, chan_ok, a2[g], ia[g]);
-    }
+    float2 h[HP], a2[HP], ia[HP];
+    // plain loads: h0 may be the last_state buffer this kernel writes; only
+    // the first segment starts from it (later ones start from zero)
+    lane_load_state<CF>(h, rows_in(seg == 0 ? const_cast<float*>(a.h0) : nullptr, b, d0), j);
+    lane_load_decay<CF>(a, d0, lg, j, a2, ia);
+    const int64_t d_ck = d0 + lg;  // training variant: the lane's channel
     bool ok = true;
     auto t_of = [&](int64_t k) { return (c_begin + k) * CF::T; };
     auto full_chunk = [&](int64_t k) { return full_tile && t_of(k) + CF::T <= L; };
@@ -938,7 +995,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     run_phase1(0);
     __syncthreads();
     for (int64_t k = 0; k < nseq; ++k) {
-      run_phase2(h, a2, ia, ckpt_at(b, d, chan_ok, t_of(k)));
+      run_phase2(h, a2, ia, ckpt_at(b, d_ck, d_ck < a.dim, t_of(k)));
       if (k + 1 < nseq) stage_in(k + 1);
       if (!__syncthreads_and(ok)) {
         drain(k + 1, k + 1);
@@ -955,30 +1012,25 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     if (segmented) {
       // this segment's end state (from h = 0 unless it is the first) and its
       // sum of Delta; the carry-in correction pass combines them
-      if (chan_ok && writer) {
-        float2* dst = reinterpret_cast<float2*>(
-            a.seg_h + (((b * a.dim + d) * sched.nseg + seg) * CF::N + j * CF::G));
+      lane_store_state<CF>(h, [&](int cc) -> float* {
+        const int64_t d = d0 + lg * CPL + cc;
+        return d < a.dim ? a.seg_h + ((b * a.dim + d) * sched.nseg + seg) * CF::N : nullptr;
+      }, j);
+      // the QPR threads of a phase-1 item are consecutive lanes of one warp
 #pragma unroll
-        for (int g = 0; g < CF::G / 2; ++g) dst[g] = h[g];
-      }
-      // the QPR threads of an item's channel are consecutive lanes of a warp
+      for (int it = 0; it < CF::ITEMS1_PER_THREAD; ++it)
 #pragma unroll
-      for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
-        double v = dsum[it];
+        for (int cc = 0; cc < CPL; ++cc) {
+          double v = dsum[it][cc];
 #pragma unroll
-        for (int o = 1; o < CF::QPR; o <<= 1) v += __shfl_xor_sync(kFullMask, v, o);
-        const int i = tid + it * CF::NT;
-        const int64_t di = d0 + i / CF::QPR;
-        if ((i % CF::QPR) == 0 && i < CF::ITEMS && di < a.dim)
-          a.seg_dsum[(b * a.dim + di) * sched.nseg + seg] = (float)v;
-      }
-    } else if (a.last_state && chan_ok && writer) {
-      float* dst = a.last_state + ((b * a.dim + d) * CF::N + j * CF::G);
-#pragma unroll
-      for (int g = 0; g < CF::G / 2; ++g) {
-        dst[2 * g] = h[g].x;
-        dst[2 * g + 1] = h[g].y;
-      }
+          for (int o = 1; o < CF::QPR; o <<= 1) v += __shfl_xor_sync(kFullMask, v, o);
+          const int i = tid + it * CF::NT;
+          const int64_t di = d0 + (i / CF::QPR) * CPL + cc;
+          if ((i % CF::QPR) == 0 && i < CF::ITEMS1 && di < a.dim)
+            a.seg_dsum[(b * a.dim + di) * sched.nseg + seg] = (float)v;
+        }
+    } else {
+      lane_store_state<CF>(h, rows_in(a.last_state, b, d0), j);
     }
     return;
   }
@@ -990,10 +1042,10 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   prep = cur;
   fetch = cur;
 
-  float2 h[CF::G / 2], a2[CF::G / 2], ia[CF::G / 2];
-  float bias_it[CF::ITEMS_PER_THREAD], D_it[CF::ITEMS_PER_THREAD];
+  float2 h[HP], a2[HP], ia[HP];
+  float bias_it[CF::ITEMS1_PER_THREAD][CPL], D_it[CF::ITEMS_PER_THREAD];
+  double no_dsum[CF::ITEMS1_PER_THREAD][CPL];  // (unused: the balanced schedule has no segments)
   ConvRegs<CF> cv;
-  double no_dsum[CF::ITEMS_PER_THREAD];  // (unused: the balanced schedule has no segments)
   int32_t bias_g = -1, D_g = -1;  // group whose bias (and taps) / D are cached
   bool ok = true;  // false once a bounded wait has given up (error word set)
 
@@ -1012,16 +1064,9 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
       load_chunk_scalar<CF>(a, reinterpret_cast<E*>(raw(jj)), r.b, d0_of(r), (int64_t)r.c * CF::T);
     }
   };
-  auto load_items = [&](const float* src, const Cursor& r, float (&dst)[CF::ITEMS_PER_THREAD]) {
-#pragma unroll
-    for (int it = 0; it < CF::ITEMS_PER_THREAD; ++it) {
-      const int64_t d = d0_of(r) + (tid + it * CF::NT) / CF::QPR;
-      dst[it] = (src && d < a.dim) ? __ldg(src + d) : 0.f;
-    }
-  };
   auto run_phase1 = [&](int64_t jj) {  // jj = prep's chunk
     if (prep.g != bias_g) {
-      load_items(a.delta_bias, prep, bias_it);
+      load_bias(d0_of(prep), bias_it);
       load_conv_regs<CF>(a, d0_of(prep), cv);
       bias_g = prep.g;
     }
@@ -1058,8 +1103,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   __syncthreads();
 
   for (int64_t q = 0; q < nseq; ++q) {
-    const int64_t d0 = d0_of(cur), d = d0 + c;
-    const bool chan_ok = d < a.dim;
+    const int64_t d0 = d0_of(cur);
+    const int64_t d_ck = d0 + lg;  // training variant: the lane's channel
     if (cur.first()) {
       // a new piece: this lane's A values, and h from 0 or the predecessor's carry
       bool have = true;
@@ -1068,38 +1113,26 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
         if (tid == 0) have = wait_carry(sched, w - 1);
         have = __syncthreads_and(have);  // also orders the carry reads after the wait
       }
-      const float* cin = have && cin_here ? sched.carries + (int64_t)(w - 1) * CF::CH * CF::N : nullptr;
-#pragma unroll
-      for (int g = 0; g < CF::G / 2; ++g) {
-        const int n = j * CF::G + 2 * g;
-        load_decay<CF>(a, d, n, chan_ok, a2[g], ia[g]);
-        if (cin)
-          h[g] = make_float2(__ldcg(cin + c * CF::N + n), __ldcg(cin + c * CF::N + n + 1));
-        else if (a.h0 && chan_ok) {  // a piece that starts the group (chunk 0)
-          const float* h0 = a.h0 + ((int64_t)cur.b * a.dim + d) * CF::N + n;
-          h[g] = make_float2(h0[0], h0[1]);
-        }
-        else
-          h[g] = make_float2(0.f, 0.f);
+      lane_load_decay<CF>(a, d0, lg, j, a2, ia);
+      if (have && cin_here) {
+        const float* cin = sched.carries + (int64_t)(w - 1) * CF::CH * CF::N;
+        lane_load_state<CF>(h, [&](int cc) -> const float* {
+          return cin + (lg * CPL + cc) * CF::N;
+        }, j);
+      } else {
+        // a piece that starts the group (chunk 0) reads h0, if given
+        lane_load_state<CF>(h, rows_in(const_cast<float*>(a.h0), cur.b, d0), j);
       }
       ok = ok && have;
     }
-    run_phase2(h, a2, ia, ckpt_at(cur.b, d, chan_ok, (int64_t)cur.c * CF::T));
+    run_phase2(h, a2, ia, ckpt_at(cur.b, d_ck, d_ck < a.dim, (int64_t)cur.c * CF::T));
     const bool cout_here = cur.carry_out();
-    if (cout_here && writer) {
-      float* dst = sched.carries + (int64_t)w * CF::CH * CF::N + c * CF::N + j * CF::G;
-#pragma unroll
-      for (int g = 0; g < CF::G / 2; ++g) __stcg(reinterpret_cast<float2*>(dst) + g, h[g]);
+    if (cout_here) {
+      float* cdst = sched.carries + (int64_t)w * CF::CH * CF::N;
+      lane_store_state<CF>(h, [&](int cc) -> float* { return cdst + (lg * CPL + cc) * CF::N; }, j);
       __threadfence();
     }
-    if (cur.last() && a.last_state && chan_ok && writer) {
-      float* dst = a.last_state + (((int64_t)cur.b * a.dim + d) * CF::N + j * CF::G);
-#pragma unroll
-      for (int g = 0; g < CF::G / 2; ++g) {
-        dst[2 * g] = h[g].x;
-        dst[2 * g + 1] = h[g].y;
-      }
-    }
+    if (cur.last()) lane_store_state<CF>(h, rows_in(a.last_state, cur.b, d0), j);
     if (q + 1 < nseq) stage_in(q + 1, prep);
     if (!__syncthreads_and(ok)) {
       drain(q + 1, q + 1);
@@ -1107,7 +1140,7 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     }
     if (cout_here && tid == 0 && w != sched.skip_publish) publish_carry(sched, w);
     if (cur.g != D_g) {
-      load_items(a.D, cur, D_it);
+      load_D(d0, D_it);
       D_g = cur.g;
     }
     const E* rc = reinterpret_cast<const E*>(raw(q));

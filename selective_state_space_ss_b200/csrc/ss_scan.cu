@@ -13,6 +13,7 @@
 #include "fwd_host.cuh"
 #include "step_host.cuh"
 #include "bwd_host.cuh"
+#include "debug_pointwise.cuh"
 
 using namespace ssscan;
 
@@ -232,6 +233,16 @@ ss_status ss_debug_inject(int what, long long value) {
       return SS_OK;
   }
   return SS_ERR_INVALID_ARG;
+}
+
+ss_status ss_debug_pointwise(int fn, const float* x, float* y, int64_t n, cudaStream_t stream) {
+  if (fn < kPwSoftplus || fn > kPwEx2 || n < 0 || (n > 0 && (!x || !y))) return SS_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(y, 4)) return SS_ERR_INVALID_ARG;
+  if (n == 0) return SS_OK;
+  const int64_t pairs = (n + 1) / 2;
+  const int64_t blocks = (pairs + 255) / 256 < 4096 ? (pairs + 255) / 256 : 4096;
+  pointwise_kernel<<<(unsigned)blocks, 256, 0, stream>>>(fn, x, y, n);
+  return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
 const char* ss_status_string(ss_status s) {
