@@ -49,7 +49,9 @@ typedef enum {
   SS_ERR_UNSUPPORTED = 2, /* dstate not in {16, 32, 64, 128}, unknown dtype, or more
                              scratch than ss_scan_fwd_noalloc holds */
   SS_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
-  SS_ERR_TIMEOUT = 4      /* a bounded inter-block wait gave up (see ss_last_device_error) */
+  SS_ERR_TIMEOUT = 4,     /* a bounded inter-block wait gave up (see ss_last_device_error) */
+  SS_ERR_BOUNDS = 5       /* checked builds only: a kernel formed an index outside its
+                             tensor and skipped the access (see ss_last_device_error) */
 } ss_status;
 
 typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
@@ -314,8 +316,11 @@ size_t ss_scan_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen,
 const char* ss_status_string(ss_status status);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
- * current device: SS_OK, or SS_ERR_TIMEOUT when a bounded wait inside a
- * kernel gave up since the last query.  SS_ERR_CUDA if the synchronisation
+ * current device: SS_OK, SS_ERR_BOUNDS when a kernel of a checked build
+ * (compiled with SS_BOUNDS_CHECK: every global index compared with its
+ * tensor's extent, a miss skipped and recorded instead of trapping) met an
+ * index outside its tensor, or SS_ERR_TIMEOUT when a bounded wait inside a
+ * kernel gave up, since the last query.  SS_ERR_CUDA if the synchronisation
  * itself failed. */
 ss_status ss_last_device_error(cudaStream_t stream);
 

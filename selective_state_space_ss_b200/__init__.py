@@ -14,6 +14,7 @@ from ._native import (  # noqa: F401
     SS_DEBUG_SPIN_LIMIT,
     SS_DEBUG_STEP_SIMPLE,
     SS_BF16,
+    SS_ERR_BOUNDS,
     SS_ERR_CUDA,
     SS_ERR_INVALID_ARG,
     SS_ERR_TIMEOUT,

@@ -18,7 +18,7 @@ _LIB_PATH = os.environ.get("SSSCAN_LIBRARY") or os.path.join(
 _lock = threading.Lock()
 _lib = None
 
-SS_OK, SS_ERR_INVALID_ARG, SS_ERR_UNSUPPORTED, SS_ERR_CUDA, SS_ERR_TIMEOUT = range(5)
+SS_OK, SS_ERR_INVALID_ARG, SS_ERR_UNSUPPORTED, SS_ERR_CUDA, SS_ERR_TIMEOUT, SS_ERR_BOUNDS = range(6)
 SS_F32, SS_BF16 = 0, 1
 
 EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",

@@ -50,6 +50,19 @@ def build(force: bool = False, ptxas_verbose: bool = False, out: str | None = No
     return target
 
 
+CHECKED_LIB = os.path.join(PKG, "libssscan_checked.so")
+
+
+def build_checked(force: bool = False) -> str:
+    """Compile the checked build (SS_BOUNDS_CHECK: every global index the kernels
+    form is compared with its tensor's extent; a miss is skipped and reported by
+    ss_last_device_error as SS_ERR_BOUNDS).  Same C ABI; for tests."""
+    if not force and os.path.exists(CHECKED_LIB) and not any(
+            os.path.getmtime(p) > os.path.getmtime(CHECKED_LIB) for p in deps()):
+        return CHECKED_LIB
+    return build(out=CHECKED_LIB, defines=["SS_BOUNDS_CHECK"])
+
+
 def build_probe() -> str:
     """Compile the standalone issue-rate probe (probe_rates.cu) next to the library."""
     out = os.path.join(PKG, "probe_rates")
@@ -62,4 +75,6 @@ def build_probe() -> str:
 if __name__ == "__main__":
     build_probe()
     build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv)
+    if "--checked" in sys.argv:
+        build_checked(force=True)
     print(LIB)

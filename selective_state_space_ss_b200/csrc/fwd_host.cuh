@@ -143,9 +143,10 @@ bool make_plan(int64_t batch, int64_t dim, int64_t seqlen, Plan* p) {
   // Segments: fill the resident slots once (groups x nseg CTAs).  Not for the
   // training variant, whose checkpoints must hold true states.
   int64_t nseg = 1;
-  if (!CF::TRAIN && forced <= 0 && p->groups < slots) nseg = slots / p->groups;
+  const bool can_segment = !CF::TRAIN && CF::WT == 1;
+  if (can_segment && forced <= 0 && p->groups < slots) nseg = slots / p->groups;
   const long long fseg = g_dbg_segments.load();
-  if (fseg > 0 && !CF::TRAIN) nseg = fseg;
+  if (fseg > 0 && can_segment) nseg = fseg;
   if (nseg > p->nk) nseg = p->nk;
   if (nseg > 1) {
     p->seg_chunks = (p->nk + nseg - 1) / nseg;
@@ -289,11 +290,36 @@ using Cfg64 = ChunkedCfg<E, 64, SS_N64_K, SS_N64_W, SS_N64_T, 1, CV, Z, TR>;
 template <typename E, bool CV = false, bool Z = false, bool TR = false>
 using Cfg128 = ChunkedCfg<E, 128, SS_N128_K, SS_N128_W, SS_N128_T, 1, CV, Z, TR>;
 
+// Time-split shapes for short sequences over too few channels to fill the GPU:
+// one warp's worth of channels (8) per CTA, 8 warps splitting each chunk in
+// time, joined inside the CTA.  (Long sequences are cut into segments instead,
+// whose carry-in correction is a second pass; over a short sequence that pass
+// would cost about as much as the scan.)
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Split16 = ChunkedCfg<E, 16, 4, 8, 128, 1, CV, Z, TR, 8>;
+template <typename E, bool CV = false, bool Z = false, bool TR = false>
+using Split32 = ChunkedCfg<E, 32, 4, 8, 32, 1, CV, Z, TR, 8>;
+constexpr int64_t kSplitMaxSeq = 65536;  // longer sequences take segments
+
+// The time split for this shape (not when a test forces segments).
+template <class CF>
+bool use_time_split(int64_t batch, int64_t dim, int64_t seqlen) {
+  if (g_dbg_segments.load() > 0 || seqlen >= kSplitMaxSeq) return false;
+  const int64_t groups = batch * ((dim + CF::CH - 1) / CF::CH);
+  return groups < device_sms();
+}
+
 template <typename E, bool CV, bool Z, bool TR>
 ss_status dispatch_dtype(const FwdArgs& a, int N, void* ws, size_t wsb, cudaStream_t stream) {
   switch (N) {
-    case 16: return launch_chunked<Cfg16<E, CV, Z, TR>>(a, ws, wsb, stream);
-    case 32: return launch_chunked<Cfg32<E, CV, Z, TR>>(a, ws, wsb, stream);
+    case 16:
+      if (use_time_split<Cfg16<E, CV, Z, TR>>(a.batch, a.dim, a.seqlen))
+        return launch_chunked<Split16<E, CV, Z, TR>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg16<E, CV, Z, TR>>(a, ws, wsb, stream);
+    case 32:
+      if (use_time_split<Cfg32<E, CV, Z, TR>>(a.batch, a.dim, a.seqlen))
+        return launch_chunked<Split32<E, CV, Z, TR>>(a, ws, wsb, stream);
+      return launch_chunked<Cfg32<E, CV, Z, TR>>(a, ws, wsb, stream);
     case 64: return launch_chunked<Cfg64<E, CV, Z, TR>>(a, ws, wsb, stream);
     case 128: return launch_chunked<Cfg128<E, CV, Z, TR>>(a, ws, wsb, stream);
     default: return SS_ERR_UNSUPPORTED;
@@ -305,8 +331,16 @@ bool plan_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N, size_t* bytes
   Plan p;
   bool ok = false;
   switch (N) {
-    case 16: ok = make_plan<Cfg16<E, CV, Z, TR>>(batch, dim, seqlen, &p); break;
-    case 32: ok = make_plan<Cfg32<E, CV, Z, TR>>(batch, dim, seqlen, &p); break;
+    case 16:
+      ok = use_time_split<Cfg16<E, CV, Z, TR>>(batch, dim, seqlen)
+               ? make_plan<Split16<E, CV, Z, TR>>(batch, dim, seqlen, &p)
+               : make_plan<Cfg16<E, CV, Z, TR>>(batch, dim, seqlen, &p);
+      break;
+    case 32:
+      ok = use_time_split<Cfg32<E, CV, Z, TR>>(batch, dim, seqlen)
+               ? make_plan<Split32<E, CV, Z, TR>>(batch, dim, seqlen, &p)
+               : make_plan<Cfg32<E, CV, Z, TR>>(batch, dim, seqlen, &p);
+      break;
     case 64: ok = make_plan<Cfg64<E, CV, Z, TR>>(batch, dim, seqlen, &p); break;
     case 128: ok = make_plan<Cfg128<E, CV, Z, TR>>(batch, dim, seqlen, &p); break;
   }

@@ -50,6 +50,26 @@ namespace ssscan {
 __device__ unsigned int g_error_word = 0;
 constexpr unsigned kErrTmaWait = 1u;     // a TMA completion wait timed out
 constexpr unsigned kErrLookback = 2u;    // an inter-CTA carry wait timed out
+constexpr unsigned kErrBounds = 4u;      // (checked builds) an index outside its tensor
+
+// Checked builds (-DSS_BOUNDS_CHECK): every global index the kernels form is
+// compared with its tensor's extent before the access; a miss records
+// kErrBounds in the device error word and the access is skipped (no trap, so
+// the context stays usable and the host reads the status).  In the product
+// build the check is compiled out.
+#ifdef SS_BOUNDS_CHECK
+__device__ __forceinline__ bool in_range(int64_t i, int64_t n) {
+  if (i >= 0 && i < n) return true;
+  atomicOr(&g_error_word, kErrBounds);
+  return false;
+}
+#else
+__device__ __forceinline__ bool in_range(int64_t, int64_t) { return true; }
+#endif
+// [i, i + len) inside [0, n)
+__device__ __forceinline__ bool in_range(int64_t i, int64_t len, int64_t n) {
+  return in_range(i, n) && in_range(i + len - 1, n);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

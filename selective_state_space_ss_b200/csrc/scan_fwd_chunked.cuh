@@ -98,9 +98,13 @@ struct CkptCtx {
 // staged with HALO earlier steps per row, and phase 1 forms
 // u = SiLU(conv(x) + bias).  ZOH: exact zero-order-hold B_bar.  TRAIN: the
 // state at every 16-step chunk start is written out for the backward.  The
-// variants (CONV, ZOH, TRAIN) use one channel per lane.
+// variants (CONV, ZOH, TRAIN) use one channel per lane.  WT: warps that split
+// each chunk in time (1: every warp walks the whole chunk for its own
+// channels; > 1, one channel per lane only: WT warps share one set of
+// channels, each scanning T/WT consecutive steps of the chunk, joined with the
+// associative operator; for short sequences over few channels).
 template <typename Tin, int N_, int K_, int NWARPS_, int T_, int CPL_ = 1, bool CONV_ = false,
-          bool ZOH_ = false, bool TRAIN_ = false>
+          bool ZOH_ = false, bool TRAIN_ = false, int WT_ = 1>
 struct ChunkedCfg {
   using Elem = Tin;
   static constexpr int N = N_;            // states per channel
@@ -110,8 +114,11 @@ struct ChunkedCfg {
   static constexpr int HP = CPL == 1 ? G / 2 : G;  // float2 registers per lane state
   static constexpr int NWARPS = NWARPS_;
   static constexpr int T = T_;            // timesteps per chunk
+  static constexpr int WT = WT_;          // time-split warps per channel set
+  static constexpr int WC = NWARPS / WT;  // warps across channels
+  static constexpr int TW = T / WT;       // steps per warp per chunk
   static constexpr int LGW = 32 / K;      // lane groups per warp
-  static constexpr int LG = NWARPS * LGW; // lane groups per CTA
+  static constexpr int LG = WC * LGW;     // lane groups per CTA
   static constexpr int CH = LG * CPL;     // channels per CTA
   static constexpr int NT = NWARPS * 32;
   static constexpr int ES = (int)sizeof(Tin);
@@ -141,9 +148,26 @@ struct ChunkedCfg {
   static constexpr int PAIR_BYTES = 4 * ES;          // one state pair: B_lo, B_hi, C_lo, C_hi
   static constexpr int BC_BLOCK = 2 * PAIR_BYTES;    // two pairs: four states
   static constexpr int BC_DATA = (N / 4) * BC_BLOCK; // bytes of one timestep
-  // Row pitch: a quarter-warp of the transpose writes rows 2tp and 2tp+2;
-  // a pitch of 32 mod 64 bytes puts them on opposite halves of the banks.
-  static constexpr int BC_ROW = (BC_DATA % 128 == 64) ? BC_DATA + 32 : BC_DATA;
+  // A timestep's B, C are 16-byte units (four bf16 states or two fp32
+  // states); lane j of a channel owns UPL units.  With more than one unit per
+  // lane they are stored unit-major, unit h of lane j at position h K + j, so
+  // that the lanes of a quarter-warp load 16 consecutive bytes each (one
+  // 128-byte wavefront) rather than every other 16 (two).
+  static constexpr int UNIT_STATES = 16 / (2 * ES);
+  static constexpr int UPL = G / UNIT_STATES;         // units per lane (0: half a unit)
+  static constexpr bool BC_PERMUTE = UPL >= 2;
+  static constexpr int UNIT_STRIDE = BC_PERMUTE ? K * 16 : 16;  // between a lane's units
+  __host__ __device__ static constexpr int bc_pos(int u) {  // byte offset of unit u
+    return (BC_PERMUTE ? (u % UPL) * K + u / UPL : u) * 16;
+  }
+  // The bf16 transpose of phase 1 (T = 32) runs its items step-fastest: a
+  // quarter-warp writes the same unit of rows 2 tp, tp = 8 consecutive values,
+  // so a row pitch of 16 mod 64 bytes spreads those writes over four bank
+  // quarters (two-way at most).  The fp32 transpose runs blocks-fastest, and a
+  // pitch of 32 mod 64 puts its rows 2tp and 2tp+2 on opposite bank halves.
+  static constexpr bool TP_FAST = ES == 2 && T == 32;
+  static constexpr int BC_ROW = TP_FAST ? (BC_DATA % 64 == 0 ? BC_DATA + 16 : BC_DATA)
+                                        : ((BC_DATA % 128 == 64) ? BC_DATA + 32 : BC_DATA);
   static constexpr int BC_BYTES = T * BC_ROW;
   static constexpr int SY_STRIDE = T + 4;            // floats per (channel, lane) row
   static constexpr int SY_BYTES = CH * K * SY_STRIDE * 4;
@@ -152,9 +176,12 @@ struct ChunkedCfg {
   static constexpr int OFF_DWW = OFF_DWD + DW_BYTES;
   static constexpr int OFF_BC = OFF_DWW + DW_BYTES;
   static constexpr int OFF_SY = OFF_BC + BC_BYTES;
+  // time-split aggregates: (prod A_bar, local end state) per warp and lane state
+  static constexpr int AGG_FLOATS = WT > 1 ? WT * WC * 32 * G : 0;
+  static constexpr int OFF_AGG = OFF_SY + SY_BYTES;
   // CONV: u = SiLU(conv) per (quad, channel), for phase 3's D u
   static constexpr int SU_BYTES = CONV ? DW_BYTES : 0;
-  static constexpr int OFF_SU = OFF_SY + SY_BYTES;
+  static constexpr int OFF_SU = OFF_AGG + 2 * AGG_FLOATS * 4;
   // ZOH: 1 / Delta per (quad, channel)
   static constexpr int DWI_BYTES = ZOH ? DW_BYTES : 0;
   static constexpr int OFF_DWI = OFF_SU + SU_BYTES;
@@ -175,6 +202,7 @@ struct ChunkedCfg {
   static_assert(N % K == 0 && 32 % K == 0, "lane split");
   static_assert(CPL == 1 || CPL == 2, "channels per lane");
   static_assert(CPL == 1 || (!CONV && !ZOH && !TRAIN), "the variants use one channel per lane");
+  static_assert(NWARPS % WT == 0 && T % (4 * WT) == 0 && (WT == 1 || CPL == 1), "time split");
   static_assert(CPL == 2 || G % 2 == 0, "a lane holds whole state pairs");
   static_assert(G % 4 == 0 || (CPL == 1 && G % 2 == 0), "B, C loads of whole state pairs");
   static_assert(T % 8 == 0 && (T * ES) % 16 == 0 && T <= 256 && CH <= 256, "TMA box");
@@ -182,7 +210,8 @@ struct ChunkedCfg {
                 "TMA destinations 128-byte aligned");
   static_assert(!CONV || ((HALO * ES) % 16 == 0 && HALO >= kConvTaps - 1 && XT <= 256),
                 "convolution halo");
-  static_assert(T % 16 == 0, "16-step checkpoints fall on quad starts");
+  static_assert(T % 16 == 0 && (WT == 1 || 16 % TW == 0),
+                "16-step checkpoints fall on quad or warp-segment starts");
   static_assert(DW_BYTES % 16 == 0 && BC_BYTES % 16 == 0, "alignment");
   static_assert((ITEMS % NT == 0 || ITEMS < NT) && (ITEMS1 % NT == 0 || ITEMS1 < NT),
                 "whole items per thread");
@@ -238,7 +267,10 @@ __device__ __forceinline__ void load_chunk_scalar(const FwdArgs& a, typename CF:
     const int c = i / CF::XT, tt = i - c * CF::XT;
     const int64_t t = t0 - CF::HALO + tt, d = d0 + c;
     E val = zero_elem<E>();
-    if (t >= 0 && t < L && d < a.dim) val = static_cast<const E*>(a.u)[(b * a.dim + d) * L + t];
+    if (t >= 0 && t < L && d < a.dim) {
+      const int64_t ix = (b * a.dim + d) * L + t;
+      if (in_range(ix, a.batch * a.dim * L)) val = static_cast<const E*>(a.u)[ix];
+    }
     raw[i] = val;
   }
   // delta, z, B, C: [2 CH + 2 N] rows of T steps
@@ -252,10 +284,13 @@ __device__ __forceinline__ void load_chunk_scalar(const FwdArgs& a, typename CF:
         const int which = r / CF::CH, c = r - which * CF::CH;
         const int64_t d = d0 + c;
         const void* base = which == 0 ? a.delta : a.z;
-        if (d < a.dim && base) val = static_cast<const E*>(base)[(b * a.dim + d) * L + t];
+        const int64_t ix = (b * a.dim + d) * L + t;
+        if (d < a.dim && base && in_range(ix, a.batch * a.dim * L))
+          val = static_cast<const E*>(base)[ix];
       } else {
         const int rr = r - 2 * CF::CH, which = rr / CF::N, n = rr - which * CF::N;
-        val = static_cast<const E*>(which == 0 ? a.B : a.C)[(b * CF::N + n) * L + t];
+        const int64_t ix = (b * CF::N + n) * L + t;
+        if (in_range(ix, a.batch * CF::N * L)) val = static_cast<const E*>(which == 0 ? a.B : a.C)[ix];
       }
     }
     rest[i] = val;
@@ -363,16 +398,32 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     const uint32_t* B32 = reinterpret_cast<const uint32_t*>(rawB);
     const uint32_t* C32 = reinterpret_cast<const uint32_t*>(rawC);
     constexpr int NB4 = CF::N / 4;
+    // Item (tp, nb) reads rows 4 nb .. 4 nb + 3 at word tp.  The steps vary
+    // fastest over the lanes, so a half-warp reads 16 consecutive words of a
+    // row (with blocks fastest, every lane of a warp would read the same bank),
+    // and the odd blocks take their rows in rotated order so that the two
+    // half-warps read rows of opposite parity, i.e. opposite halves of the
+    // banks.
+    constexpr bool TP_FAST = CF::TP_FAST && TP == 16;
     for (int i = tid; i < NB4 * TP; i += CF::NT) {
-      const int tp = i / NB4, nb = i - tp * NB4;
-      uint32_t bw[4], cw[4];
+      const int tp = TP_FAST ? i % TP : i / NB4;
+      const int nb = TP_FAST ? i / TP : i - tp * NB4;
+      const int rot = TP_FAST ? (nb & 1) : 0;
+      uint32_t bv[4], cv4[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        bw[r] = B32[(4 * nb + r) * TP + tp];
-        cw[r] = C32[(4 * nb + r) * TP + tp];
+        const int row = 4 * nb + ((r + rot) & 3);
+        bv[r] = B32[row * TP + tp];
+        cv4[r] = C32[row * TP + tp];
       }
-      uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + nb * CF::BC_BLOCK);
-      uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + nb * CF::BC_BLOCK);
+      uint32_t bw[4], cw[4];  // bw[k]: row 4 nb + k
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        bw[k] = rot ? bv[(k + 3) & 3] : bv[k];
+        cw[k] = rot ? cv4[(k + 3) & 3] : cv4[k];
+      }
+      uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + CF::bc_pos(nb));
+      uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + CF::bc_pos(nb));
       *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(cw[0], cw[1], 0x5410),
                          __byte_perm(bw[2], bw[3], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
       *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(cw[0], cw[1], 0x7632),
@@ -383,11 +434,13 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
     const float* fc = reinterpret_cast<const float*>(rawC);
     for (int i = tid; i < (CF::N / 4) * CF::T; i += CF::NT) {
       const int nb = i / CF::T, t = i - nb * CF::T;
-      float4* dst = reinterpret_cast<float4*>(bc + t * CF::BC_ROW + nb * CF::BC_BLOCK);
-      dst[0] = make_float4(fb[(4 * nb) * CF::T + t], fb[(4 * nb + 1) * CF::T + t],
-                           fc[(4 * nb) * CF::T + t], fc[(4 * nb + 1) * CF::T + t]);
-      dst[1] = make_float4(fb[(4 * nb + 2) * CF::T + t], fb[(4 * nb + 3) * CF::T + t],
-                           fc[(4 * nb + 2) * CF::T + t], fc[(4 * nb + 3) * CF::T + t]);
+      unsigned char* row = bc + t * CF::BC_ROW;  // fp32: units 2 nb and 2 nb + 1
+      *reinterpret_cast<float4*>(row + CF::bc_pos(2 * nb)) =
+          make_float4(fb[(4 * nb) * CF::T + t], fb[(4 * nb + 1) * CF::T + t],
+                      fc[(4 * nb) * CF::T + t], fc[(4 * nb + 1) * CF::T + t]);
+      *reinterpret_cast<float4*>(row + CF::bc_pos(2 * nb + 1)) =
+          make_float4(fb[(4 * nb + 2) * CF::T + t], fb[(4 * nb + 3) * CF::T + t],
+                      fc[(4 * nb + 2) * CF::T + t], fc[(4 * nb + 3) * CF::T + t]);
     }
   }
 }
@@ -395,7 +448,8 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
 // ------------------------------------------------------------- phase 2 ---
 
 // B and C of NP consecutive state pairs at one timestep, as fp32 pairs; p
-// points at the first pair (16-byte loads where the pairs allow).
+// points at the lane's first unit (16-byte loads where the pairs allow; the
+// lane's next unit is UNIT_STRIDE bytes on).
 template <class CF, int NP>
 __device__ __forceinline__ void bc_pairs(const unsigned char* p, float2 (&b)[NP],
                                          float2 (&c)[NP]) {
@@ -403,7 +457,7 @@ __device__ __forceinline__ void bc_pairs(const unsigned char* p, float2 (&b)[NP]
     if constexpr (NP % 2 == 0) {
 #pragma unroll
       for (int i = 0; i < NP / 2; ++i) {
-        const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+        const uint4 v = *reinterpret_cast<const uint4*>(p + i * CF::UNIT_STRIDE);
         b[2 * i] = bf16x2_to_float2(v.x);
         c[2 * i] = bf16x2_to_float2(v.y);
         b[2 * i + 1] = bf16x2_to_float2(v.z);
@@ -420,7 +474,7 @@ __device__ __forceinline__ void bc_pairs(const unsigned char* p, float2 (&b)[NP]
   } else {
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
-      const float4 v = reinterpret_cast<const float4*>(p)[i];
+      const float4 v = *reinterpret_cast<const float4*>(p + i * CF::UNIT_STRIDE);
       b[i] = make_float2(v.x, v.y);
       c[i] = make_float2(v.z, v.w);
     }
@@ -487,7 +541,8 @@ __device__ __forceinline__ void phase2(const float4* dwD, const float4* dwW, con
                                        const float2 (&ia)[CF::HP], int c, int j,
                                        const CkptCtx& ck) {
   constexpr int G2 = CF::G / 2;  // state pairs per lane
-  const unsigned char* bcj = bc + j * G2 * CF::PAIR_BYTES;
+  // the lane's first unit (half units: G = 2 bf16 states, 8 bytes a lane)
+  const unsigned char* bcj = bc + (CF::UPL >= 1 ? CF::bc_pos(j * CF::UPL) : j * G2 * CF::PAIR_BYTES);
   float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE;
 #pragma unroll kPhase2Unroll
   for (int q = 0; q < CF::QPR; ++q) {
@@ -543,7 +598,7 @@ __device__ __forceinline__ void phase2_cpl2(const float4* dwD, const float4* dwW
                                             float2 (&h)[CF::HP], const float2 (&a2)[CF::HP],
                                             int lg, int j) {
   constexpr int G = CF::G;
-  const unsigned char* bcj = bc + j * (G / 2) * CF::PAIR_BYTES;
+  const unsigned char* bcj = bc + CF::bc_pos(j * CF::UPL);
   float* sy0 = sy + (2 * lg * CF::K + j) * CF::SY_STRIDE;
   float* sy1 = sy0 + CF::K * CF::SY_STRIDE;
 #pragma unroll kPhase2Unroll
@@ -577,6 +632,115 @@ __device__ __forceinline__ void phase2_cpl2(const float4* dwD, const float4* dwW
     }
     *reinterpret_cast<float4*>(sy0 + 4 * q) = make_float4(s0[0], s0[1], s0[2], s0[3]);
     *reinterpret_cast<float4*>(sy1 + 4 * q) = make_float4(s1[0], s1[1], s1[2], s1[3]);
+  }
+}
+
+// The time-split recurrence (WT > 1).  Warp wt scans steps
+// [wt TW, (wt+1) TW) of the chunk from h = 0 while tracking the product of
+// its decays P_t = prod A_bar and the fix-up coefficients Q_t = C_t P_t; the
+// WT warps then swap their aggregates (P_end, h_end) through shared memory and
+// each folds the chunk's carry-in through the aggregates before it with the
+// operator (a1,b1) then (a2,b2) = (a2 a1, a2 b1 + b2) ("Mamba 选择性机制",
+// sec. 3.1), which gives its own carry-in h_in exactly: h_t = local h_t +
+// P_t h_in, so the readout is corrected by sum_n Q_t[n] h_in[n].  Every warp
+// folds all WT aggregates, so all of them leave with the chunk's carry-out in
+// h.  No ex2 is evaluated twice.
+template <class CF>
+__device__ __forceinline__ void phase2_split(const float4* dwD, const float4* dwW,
+                                             const float4* dwI, const unsigned char* bc,
+                                             float* sy, float* aggP, float* aggH,
+                                             float2 (&h)[CF::HP], const float2 (&a2)[CF::HP],
+                                             const float2 (&ia)[CF::HP], int c, int j, int wt,
+                                             int lane_g, const CkptCtx& ck) {
+  constexpr int G2 = CF::G / 2;
+  const unsigned char* bcj = bc + (CF::UPL >= 1 ? CF::bc_pos(j * CF::UPL) : j * G2 * CF::PAIR_BYTES);
+  float2 hl[G2], P[G2];
+#pragma unroll
+  for (int g = 0; g < G2; ++g) {
+    hl[g] = make_float2(0.f, 0.f);
+    P[g] = make_float2(1.f, 1.f);
+  }
+  float2 Q[CF::TW][G2];
+  float s[CF::TW];
+#pragma unroll
+  for (int q = 0; q < CF::TW / 4; ++q) {
+    const int qq = wt * (CF::TW / 4) + q;
+    const float4 D4 = dwD[qq * CF::DW_STRIDE + c];
+    const float4 W4 = dwW[qq * CF::DW_STRIDE + c];
+    const float dls[4] = {D4.x, D4.y, D4.z, D4.w};
+    const float ws[4] = {W4.x, W4.y, W4.z, W4.w};
+    float idl[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (CF::ZOH) {
+      const float4 I4 = dwI[qq * CF::DW_STRIDE + c];
+      idl[0] = I4.x; idl[1] = I4.y; idl[2] = I4.z; idl[3] = I4.w;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = 4 * q + k;
+      const unsigned char* row = bcj + (4 * qq + k) * CF::BC_ROW;
+      const float2 dl2 = make_float2(dls[k], dls[k]);
+      const float2 w2 = make_float2(ws[k], ws[k]);
+      float2 acc = make_float2(0.f, 0.f);
+      float2 bb[G2], cc[G2];
+      bc_pairs<CF, G2>(row, bb, cc);
+#pragma unroll
+      for (int g = 0; g < G2; ++g) {
+        const float2 x = __fmul2_rn(dl2, a2[g]);
+        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        float2 wb;
+        if constexpr (CF::ZOH)
+          wb = __fmul2_rn(__fmul2_rn(zoh_phi2(x, e, ia[g], make_float2(idl[k], idl[k])), w2), bb[g]);
+        else
+          wb = __fmul2_rn(w2, bb[g]);
+        hl[g] = __ffma2_rn(e, hl[g], wb);
+        P[g] = __fmul2_rn(e, P[g]);
+        acc = __ffma2_rn(cc[g], hl[g], acc);
+        Q[t][g] = __fmul2_rn(cc[g], P[g]);
+      }
+      s[t] = acc.x + acc.y;
+    }
+  }
+  // publish this warp's aggregate: [wt][lane in channel set][state]
+  float2* myP = reinterpret_cast<float2*>(aggP + (wt * CF::WC * 32 + lane_g) * CF::G);
+  float2* myH = reinterpret_cast<float2*>(aggH + (wt * CF::WC * 32 + lane_g) * CF::G);
+#pragma unroll
+  for (int g = 0; g < G2; ++g) {
+    myP[g] = P[g];
+    myH[g] = hl[g];
+  }
+  __syncthreads();
+  float2 hin[G2];
+#pragma unroll
+  for (int v = 0; v < CF::WT; ++v) {
+    if (v == wt) {
+#pragma unroll
+      for (int g = 0; g < G2; ++g) hin[g] = h[g];
+    }
+    const float2* vP = reinterpret_cast<const float2*>(aggP + (v * CF::WC * 32 + lane_g) * CF::G);
+    const float2* vH = reinterpret_cast<const float2*>(aggH + (v * CF::WC * 32 + lane_g) * CF::G);
+#pragma unroll
+    for (int g = 0; g < G2; ++g) h[g] = __ffma2_rn(vP[g], h[g], vH[g]);
+  }
+  // hin is the state before this warp's first step: a 16-step checkpoint when
+  // the segment starts on one
+  if (CF::TRAIN && ck.p && (wt * CF::TW) % 16 == 0 && wt * CF::TW < ck.left) {
+    float2* dst = reinterpret_cast<float2*>(ck.p + (wt * CF::TW / 16) * ck.stride);
+#pragma unroll
+    for (int g = 0; g < G2; ++g) dst[g] = hin[g];
+  }
+  float* syr = sy + (c * CF::K + j) * CF::SY_STRIDE + wt * CF::TW;
+#pragma unroll
+  for (int q = 0; q < CF::TW / 4; ++q) {
+    float out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = 4 * q + k;
+      float2 fix = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int g = 0; g < G2; ++g) fix = __ffma2_rn(Q[t][g], hin[g], fix);
+      out[k] = s[t] + (fix.x + fix.y);
+    }
+    *reinterpret_cast<float4*>(syr + 4 * q) = make_float4(out[0], out[1], out[2], out[3]);
   }
 }
 
@@ -620,13 +784,15 @@ __device__ __forceinline__ void phase3(const FwdArgs& a, const typename CF::Elem
       y23 = __fmul2_rn(y23, silu_fast2(make_float2(zz.z, zz.w)));
     }
     const float y[4] = {y01.x, y01.y, y23.x, y23.y};
-    float* dst = a.y + (b * D + d) * L + t;
+    const int64_t iy = (b * D + d) * L + t;
+    float* dst = a.y + iy;
     if (a.vec && (kFull || t + 3 < L)) {  // 16-byte stores only on aligned rows
-      *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
+      if (in_range(iy, 4, a.batch * D * L))
+        *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
     } else {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        if (t + k < L) dst[k] = y[k];
+        if (t + k < L && in_range(iy + k, a.batch * D * L)) dst[k] = y[k];
     }
   }
 }
@@ -723,6 +889,7 @@ struct Cursor {
 // the same launch (a captured CUDA graph keeps its epoch) never mistakes the
 // previous replay's flag for a fresh carry.
 __device__ __forceinline__ bool wait_carry(const Sched& s, int src) {
+  if (!in_range(src, gridDim.x)) return false;
   unsigned long long* f = s.flags + src;
   for (uint32_t i = 0; i < s.spin_limit; ++i) {
     unsigned long long v;
@@ -738,6 +905,7 @@ __device__ __forceinline__ bool wait_carry(const Sched& s, int src) {
 }
 
 __device__ __forceinline__ void publish_carry(const Sched& s, int w) {
+  if (!in_range(w, gridDim.x)) return;
   unsigned long long* f = s.flags + w;
   asm volatile("st.release.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(s.epoch) : "memory");
 }
@@ -748,8 +916,9 @@ __device__ __forceinline__ void publish_carry(const Sched& s, int w) {
 template <class CF>
 __device__ __forceinline__ void load_decay(const FwdArgs& a, int64_t d, int n, bool chan_ok,
                                            float2& a2, float2& ia) {
-  const float A0 = chan_ok ? __ldg(a.A + d * CF::N + n) : 0.f;
-  const float A1 = chan_ok ? __ldg(a.A + d * CF::N + n + 1) : 0.f;
+  const bool in = chan_ok && in_range(d * CF::N + n, 2, a.dim * CF::N);
+  const float A0 = in ? __ldg(a.A + d * CF::N + n) : 0.f;
+  const float A1 = in ? __ldg(a.A + d * CF::N + n + 1) : 0.f;
   a2 = make_float2(A0 * 1.4426950408889634f, A1 * 1.4426950408889634f);
   ia = CF::ZOH ? make_float2(A0 != 0.f ? 1.f / A0 : 0.f, A1 != 0.f ? 1.f / A1 : 0.f)
                : make_float2(0.f, 0.f);
@@ -768,7 +937,7 @@ __device__ __forceinline__ void load_conv_regs(const FwdArgs& a, int64_t d0, Con
 #pragma unroll
       for (int k = 0; k < kConvTaps; ++k) {
         const int src = k - (kConvTaps - W);
-        cv.w[it][k] = (ok && src >= 0) ? __ldg(a.conv_w + d * W + src) : 0.f;
+        cv.w[it][k] = (ok && src >= 0 && in_range(d * W + src, a.dim * W)) ? __ldg(a.conv_w + d * W + src) : 0.f;
       }
       cv.b[it] = (ok && a.conv_b) ? __ldg(a.conv_b + d) : 0.f;
     }
@@ -836,8 +1005,8 @@ __device__ __forceinline__ void lane_load_decay(const FwdArgs& a, int64_t d0, in
 #pragma unroll
     for (int g = 0; g < CF::HP; ++g) {
       const int n = j * CF::G + g;
-      const float A0 = e0 < a.dim ? __ldg(a.A + e0 * CF::N + n) : 0.f;
-      const float A1 = e1 < a.dim ? __ldg(a.A + e1 * CF::N + n) : 0.f;
+      const float A0 = (e0 < a.dim && in_range(e0 * CF::N + n, a.dim * CF::N)) ? __ldg(a.A + e0 * CF::N + n) : 0.f;
+      const float A1 = (e1 < a.dim && in_range(e1 * CF::N + n, a.dim * CF::N)) ? __ldg(a.A + e1 * CF::N + n) : 0.f;
       a2[g] = make_float2(A0 * 1.4426950408889634f, A1 * 1.4426950408889634f);
       ia[g] = make_float2(0.f, 0.f);
     }
@@ -867,6 +1036,8 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   float* sy = reinterpret_cast<float*>(smem + CF::OFF_SY);
   float4* su = reinterpret_cast<float4*>(smem + CF::OFF_SU);    // CONV only
   float4* dwI = reinterpret_cast<float4*>(smem + CF::OFF_DWI);  // ZOH only
+  float* aggP = reinterpret_cast<float*>(smem + CF::OFF_AGG);     // time split only
+  float* aggH = aggP + CF::AGG_FLOATS;
   __shared__ __align__(8) uint64_t bars[2];
 
   const int w = blockIdx.x;
@@ -888,8 +1059,11 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   const bool has_z = a.z != nullptr;
   const bool tma = a.vec != 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int lg = warp * CF::LGW + lane / CF::K;  // this lane's group: channels lg CPL + cc
-  const int j = lane % CF::K;                    // this lane's state group
+  const int wc = warp % CF::WC, wt = warp / CF::WC;  // channel warp, time-split slot
+  const int lg = wc * CF::LGW + lane / CF::K;  // this lane's group: channels lg CPL + cc
+  const int j = lane % CF::K;                  // this lane's state group
+  const int lane_g = wc * 32 + lane;           // lane within its channel set (time split)
+  const bool writer = wt == 0;  // time-split warps hold the same carry: one writes it
   const int64_t ck_nk = (a.seqlen + 15) / 16;
   // this lane's checkpoint slot for the chunk of batch row bb starting at t0
   // (training variant, one channel per lane)
@@ -897,22 +1071,32 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     CkptCtx ck;
     ck.stride = a.dim * CF::N;
     ck.left = a.seqlen - t0;
-    ck.p = (CF::TRAIN && a.ckpt && ok)
-               ? a.ckpt + ((bb * ck_nk + t0 / 16) * a.dim + dd) * CF::N + j * CF::G
+    // this chunk's checkpoints: every 16th step while steps remain
+    const int64_t i0 = ((bb * ck_nk + t0 / 16) * a.dim + dd) * CF::N + j * CF::G;
+    const int64_t nck = (ck.left + 15) / 16 < CF::T / 16 ? (ck.left + 15) / 16 : CF::T / 16;
+    ck.p = (CF::TRAIN && a.ckpt && ok &&
+            in_range(i0 + (nck - 1) * ck.stride, CF::G, a.batch * ck_nk * a.dim * CF::N))
+               ? a.ckpt + i0
                : nullptr;
     return ck;
   };
   auto run_phase2 = [&](float2 (&hh)[HP], const float2 (&aa)[HP], const float2 (&ii)[HP],
                         const CkptCtx& ck) {
-    if constexpr (CPL == 1) phase2<CF>(dwD, dwW, dwI, bc, sy, hh, aa, ii, lg, j, ck);
-    else phase2_cpl2<CF>(dwD, dwW, bc, sy, hh, aa, lg, j);
+    if constexpr (CF::WT > 1)
+      phase2_split<CF>(dwD, dwW, dwI, bc, sy, aggP, aggH, hh, aa, ii, lg, j, wt, lane_g, ck);
+    else if constexpr (CPL == 1)
+      phase2<CF>(dwD, dwW, dwI, bc, sy, hh, aa, ii, lg, j, ck);
+    else
+      phase2_cpl2<CF>(dwD, dwW, bc, sy, hh, aa, lg, j);
   };
   // [channel][N] rows of this lane's channels in a per-(b, d) array, for batch
   // row bb of channel tile d0 (null past dim)
   auto rows_in = [&](float* base, int64_t bb, int64_t d0) {
     return [=](int cc) -> float* {
       const int64_t d = d0 + lg * CPL + cc;
-      return (base && d < a.dim) ? base + (bb * a.dim + d) * CF::N : nullptr;
+      return (base && d < a.dim && in_range((bb * a.dim + d) * CF::N, CF::N, a.batch * a.dim * CF::N))
+                 ? base + (bb * a.dim + d) * CF::N
+                 : nullptr;
     };
   };
   // per-item constants: bias per (phase-1 item, channel), D per phase-3 item
@@ -1012,9 +1196,12 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     if (segmented) {
       // this segment's end state (from h = 0 unless it is the first) and its
       // sum of Delta; the carry-in correction pass combines them
-      lane_store_state<CF>(h, [&](int cc) -> float* {
+      if (writer) lane_store_state<CF>(h, [&](int cc) -> float* {
         const int64_t d = d0 + lg * CPL + cc;
-        return d < a.dim ? a.seg_h + ((b * a.dim + d) * sched.nseg + seg) * CF::N : nullptr;
+        const int64_t i0 = ((b * a.dim + d) * sched.nseg + seg) * CF::N;
+        return (d < a.dim && in_range(i0, CF::N, a.batch * a.dim * sched.nseg * CF::N))
+                   ? a.seg_h + i0
+                   : nullptr;
       }, j);
       // the QPR threads of a phase-1 item are consecutive lanes of one warp
 #pragma unroll
@@ -1026,10 +1213,12 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
           for (int o = 1; o < CF::QPR; o <<= 1) v += __shfl_xor_sync(kFullMask, v, o);
           const int i = tid + it * CF::NT;
           const int64_t di = d0 + (i / CF::QPR) * CPL + cc;
-          if ((i % CF::QPR) == 0 && i < CF::ITEMS1 && di < a.dim)
-            a.seg_dsum[(b * a.dim + di) * sched.nseg + seg] = (float)v;
+          const int64_t is = (b * a.dim + di) * sched.nseg + seg;
+          if ((i % CF::QPR) == 0 && i < CF::ITEMS1 && di < a.dim &&
+              in_range(is, a.batch * a.dim * sched.nseg))
+            a.seg_dsum[is] = (float)v;
         }
-    } else {
+    } else if (writer) {
       lane_store_state<CF>(h, rows_in(a.last_state, b, d0), j);
     }
     return;
@@ -1117,7 +1306,9 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
       if (have && cin_here) {
         const float* cin = sched.carries + (int64_t)(w - 1) * CF::CH * CF::N;
         lane_load_state<CF>(h, [&](int cc) -> const float* {
-          return cin + (lg * CPL + cc) * CF::N;
+          const int64_t i0 = ((int64_t)(w - 1) * CF::CH + lg * CPL + cc) * CF::N;
+          return in_range(i0, CF::N, (int64_t)gridDim.x * CF::CH * CF::N) ? cin + (lg * CPL + cc) * CF::N
+                                                                          : nullptr;
         }, j);
       } else {
         // a piece that starts the group (chunk 0) reads h0, if given
@@ -1127,12 +1318,16 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
     }
     run_phase2(h, a2, ia, ckpt_at(cur.b, d_ck, d_ck < a.dim, (int64_t)cur.c * CF::T));
     const bool cout_here = cur.carry_out();
-    if (cout_here) {
+    if (cout_here && writer) {
       float* cdst = sched.carries + (int64_t)w * CF::CH * CF::N;
-      lane_store_state<CF>(h, [&](int cc) -> float* { return cdst + (lg * CPL + cc) * CF::N; }, j);
+      lane_store_state<CF>(h, [&](int cc) -> float* {
+        const int64_t i0 = ((int64_t)w * CF::CH + lg * CPL + cc) * CF::N;
+        return in_range(i0, CF::N, (int64_t)gridDim.x * CF::CH * CF::N) ? cdst + (lg * CPL + cc) * CF::N
+                                                                       : nullptr;
+      }, j);
       __threadfence();
     }
-    if (cur.last()) lane_store_state<CF>(h, rows_in(a.last_state, cur.b, d0), j);
+    if (cur.last() && writer) lane_store_state<CF>(h, rows_in(a.last_state, cur.b, d0), j);
     if (q + 1 < nseq) stage_in(q + 1, prep);
     if (!__syncthreads_and(ok)) {
       drain(q + 1, q + 1);

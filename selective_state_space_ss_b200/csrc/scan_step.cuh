@@ -116,8 +116,9 @@ __global__ void __launch_bounds__(kStepThreads, SS_STEP_MIN_BLOCKS)
 #pragma unroll
     for (int k = 0; k < kStepUnits; ++k) {
       const int r = base + k * kStepThreads;
-      const bool in = r < row_units;
       const int d = r / LPC;
+      const bool in = r < row_units && in_range((int64_t)b * row_units + r, a.batch * row_units) &&
+                      in_range(crow + d, a.batch * a.dim);
       h[k] = in ? ld_state<kVec>(srow + r * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
       av[k] = in ? ld4<kVec>(a.A + r * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
       uu[k] = in ? to_f32(u[crow + d]) : 0.f;
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kStepThreads, SS_STEP_MIN_BLOCKS)
       part = fmaf(cv.w, h[k].w, part);
 #pragma unroll
       for (int off = LPC / 2; off > 0; off >>= 1) part += __shfl_xor_sync(kFullMask, part, off);
-      if (r < row_units) {
+      if (r < row_units && in_range((int64_t)b * row_units + r, a.batch * row_units)) {
         st_state<kVec>(srow + r * 4, h[k]);
         if (j == 0) {
           float y = part + Dd[k] * uu[k];
@@ -234,6 +235,10 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
     const uint32_t sb = (uint32_t)(nch * N * 4), ab = (uint32_t)(nch * CF::ES);
     const uint32_t tx = sb + (has_z ? 3u : 2u) * ab + 2u * N * CF::ES;
     const int64_t ch0 = b * a.dim + d0;
+    // (checked builds: the copied ranges lie inside their tensors, else nothing is copied)
+    if (!in_range(ch0 * N, nch * N, a.batch * a.dim * N) || !in_range(ch0, nch, a.batch * a.dim) ||
+        !in_range(b * N, N, a.batch * N))
+      return;
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&full[k % S], tx);
     bulk_load(st, a.state + ch0 * N, sb, &full[k % S]);
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
       for (int q = 0; q < UPT; ++q) {
         const int unit = tid + q * CF::NT;
         const int64_t d = c * CF::TILE_CH + unit / LPC;
-        const bool in = d < a.dim;
+        const bool in = d < a.dim && in_range(d * N + 4 * j, 4, a.dim * N);
         const float4 A4 = in ? __ldg(reinterpret_cast<const float4*>(a.A + d * N + 4 * j))
                              : make_float4(0.f, 0.f, 0.f, 0.f);
         av[q] = make_float4(A4.x * 1.4426950408889634f, A4.y * 1.4426950408889634f,
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
       part = fmaf(cv.w, h.w, part);
 #pragma unroll
       for (int off = LPC / 2; off > 0; off >>= 1) part += __shfl_xor_sync(kFullMask, part, off);
-      if (c * CF::TILE_CH + cl < a.dim) {
+      if (c * CF::TILE_CH + cl < a.dim && in_range((ch0 + cl) * N + 4 * j, 4, a.batch * a.dim * N)) {
         *reinterpret_cast<float4*>(a.state + (ch0 + cl) * N + 4 * j) = h;
         if (j == 0) {
           float y = part + Dd[q] * uu;

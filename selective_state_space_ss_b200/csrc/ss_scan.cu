@@ -252,6 +252,7 @@ const char* ss_status_string(ss_status s) {
     case SS_ERR_UNSUPPORTED: return "SS_ERR_UNSUPPORTED: dstate must be 16, 32, 64 or 128 and dtype f32 or bf16";
     case SS_ERR_CUDA: return "SS_ERR_CUDA: a CUDA runtime call or launch failed";
     case SS_ERR_TIMEOUT: return "SS_ERR_TIMEOUT: a bounded wait inside a kernel gave up";
+    case SS_ERR_BOUNDS: return "SS_ERR_BOUNDS: a checked build met an index outside its tensor";
   }
   return "unknown ss_status";
 }
@@ -263,7 +264,7 @@ ss_status ss_last_device_error(cudaStream_t stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero) != cudaSuccess) return SS_ERR_CUDA;
-    return SS_ERR_TIMEOUT;
+    return (word & kErrBounds) ? SS_ERR_BOUNDS : SS_ERR_TIMEOUT;
   }
   return SS_OK;
 }

@@ -46,7 +46,7 @@ def test_debug_inject_rejects_unknown_code(lib):
 
 
 def test_status_strings(lib):
-    for s in range(5):
+    for s in range(6):
         assert N.ss_status_string(s).startswith("SS_")
     assert "unknown" in N.ss_status_string(99)
 

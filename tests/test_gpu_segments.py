@@ -167,8 +167,9 @@ def test_training_forward_is_never_segmented():
 
 
 def test_auto_segments_on_few_channels():
-    # one batch row of 64 channels: the default plan segments the sequence
-    w = I.Workload("segauto", 1, 64, 20000, 16, "bf16", dt_min=1e-4, dt_max=1e-2)
+    # one batch row of 64 channels over 70000 steps: the default plan segments
+    # the sequence (shorter ones take the time split)
+    w = I.Workload("segauto", 1, 64, 70000, 16, "bf16", dt_min=1e-4, dt_max=1e-2)
     x = I.make_inputs(w, seed=17)
     y, h = _fwd(to_device(x), 0)
     _check(w, y, h, *_ref(x))

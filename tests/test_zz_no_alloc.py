@@ -43,7 +43,7 @@ def _reference(xd):
     ((3, 200, 777, 32), "bf16", 5),    # forced split of 7 groups: carries on a small problem
     ((2, 64, 301, 16), "f32", 3),      # element-wise load path (1204-byte rows) with a split
     ((2, 96, 200, 64), "bf16", 0),     # few channel groups: sequence segments, scratch in use
-    ((1, 64, 5000, 16), "f32", 0),     # long segments with the carry-in correction
+    ((1, 64, 70000, 16), "f32", 0),    # long segments with the carry-in correction
 ])
 def test_noalloc_matches_workspace_entry_point(shape, dtype, workers):
     ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
