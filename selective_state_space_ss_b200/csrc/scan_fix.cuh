@@ -17,13 +17,14 @@
 // segment come from a per-lane sum and a warp scan (the running total in
 // double).  The term of state n is evaluated as sign(h_in[n]) 2^(a_n S_t +
 // log2|h_in[n]|) C_t[n] (one fused multiply-add for the exponent).  A state's
-// term is dropped once its weight P is below 2^-40 for the rest of the
-// segment: with softplus on (Delta >= 0) and A[d,n] < 0 the weight only falls,
-// and 2^-40 |h_in| lies 16 binary orders below the fp32 resolution of the
-// state it would be added to.  Otherwise (A >= 0, or Delta of either sign) the
-// term is kept for the whole segment.  The states are visited slowest decay
-// first, so the live ones are always a prefix of that order, and the walk ends
-// at the first block where none is live.
+// term is dropped once |h_in[n]| P_t[n] < 2^-36 max_m |h_in[m]| for the rest of
+// the segment: with softplus on (Delta >= 0) and A[d,n] < 0 the weight only
+// falls, and a term 2^-36 below the largest state lies 12 binary orders below
+// the fp32 resolution of the readout it would be added to.  Otherwise
+// (A >= 0, or Delta of either sign) the term is kept for the whole segment.
+// The states are visited in the order they are dropped, latest first, so the
+// live ones are always a prefix of that order, and the walk ends at the first
+// block where none is live.
 //
 // With 16-byte aligned rows, one lane of the warp brings each block's delta,
 // z, y (and, for N = 16, the block's C tile) into shared memory with TMA, two
@@ -60,7 +61,8 @@ struct FixMaps {
 
 constexpr int kFixWarps = 4;
 constexpr int kFixBlock = 128;         // steps per block (4 per lane)
-constexpr float kFixDropLog2 = -40.f;  // log2 of the weight below which a term is dropped
+constexpr float kFixDropLog2 = -36.f;  // log2 of a term's weight, relative to the largest
+                                       // state, below which it is dropped
 
 // Per-warp staging of one block (byte offsets, each a multiple of 128).
 template <typename Tin, int N>
@@ -78,11 +80,14 @@ struct FixStage {
 };
 
 // Four consecutive elements from t (zeros past `end`), widened to float.
+// (row_ix: the row's first element index in its tensor of `total` elements)
 template <typename T>
-__device__ __forceinline__ float4 fix_load4(const T* row, int64_t t, int64_t end) {
+__device__ __forceinline__ float4 fix_load4(const T* row, int64_t t, int64_t end, int64_t row_ix,
+                                            int64_t total) {
   float e[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) e[k] = t + k < end ? to_f32(row[t + k]) : 0.f;
+  for (int k = 0; k < 4; ++k)
+    e[k] = (t + k < end && in_range(row_ix + t + k, total)) ? to_f32(row[t + k]) : 0.f;
   return make_float4(e[0], e[1], e[2], e[3]);
 }
 
@@ -104,6 +109,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
   __shared__ __align__(16) float4 sh_p[kFixWarps][N];  // {a, a, log2|h_in|, log2|h_in|}
   __shared__ int sh_n[kFixWarps][N];    // state index at each position (slowest decay first)
   __shared__ int sh_neg[kFixWarps][N];  // sign of h_in at each position
+  __shared__ float sh_sd[kFixWarps][N];  // the largest sum of Delta at which it is kept
   __shared__ __align__(8) uint64_t fbar[kFixWarps][2];
   extern __shared__ __align__(128) unsigned char fix_dyn[];
   unsigned char* fix_smem = fix_dyn + ((128u - (smem_u32(fix_dyn) & 127u)) & 127u);
@@ -115,31 +121,73 @@ __global__ void __launch_bounds__(kFixWarps * 32)
   const int s = (int)(task - bd * per_ch) + 1;
   const int64_t b = bd / a.dim, d = bd - b * a.dim;
   const int64_t L = a.seqlen;
+  const int64_t n_act = a.batch * a.dim * L;  // elements of delta, z and y
   const bool tma = a.tma != 0;
 
   // h_in of segment s: fold the (prod A_bar, end state) pairs of segments
   // 0 .. s-1 in order; the last segment's task also writes the final state.
-  // Position of state n: its rank by A log2 e, largest (slowest decay) first.
   const float* hs = a.seg_h + bd * a.nseg * N;
   const float* ds = a.seg_dsum + bd * a.nseg;
   const float* Ad = a.A + d * N;
+  const int64_t n_seg = a.batch * a.dim * a.nseg;  // extents of the segment arrays
+  if (!in_range(bd * a.nseg, a.nseg, n_seg) || !in_range(d * N, N, a.dim * N)) return;
+  float lh_max = -INFINITY;  // log2 max_n |h_in[n]|
   for (int n = lane; n < N; n += 32) {
     const float an = __ldg(Ad + n) * 1.4426950408889634f;
     float h = hs[n];
     for (int q = 1; q < s; ++q) h = fmaf(ex2_approx(an * ds[q]), h, hs[(int64_t)q * N + n]);
-    if (s == a.nseg - 1 && a.last_state)
+    if (s == a.nseg - 1 && a.last_state && in_range(bd * N + n, a.batch * a.dim * N))
       a.last_state[bd * N + n] = fmaf(ex2_approx(an * ds[s]), h, hs[(int64_t)s * N + n]);
-    int rank = 0;
-    for (int m = 0; m < N; ++m) {
-      const float am = __ldg(Ad + m) * 1.4426950408889634f;
-      rank += (am > an || (am == an && m < n)) ? 1 : 0;
-    }
     float lh;  // log2|h_in|: -inf for 0, so that its terms vanish
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lh) : "f"(fabsf(h)));
-    sh_p[warp][rank] = make_float4(an, an, lh, lh);
-    sh_n[warp][rank] = n;
-    sh_neg[warp][rank] = h < 0.f;
+    sh_p[warp][n] = make_float4(an, an, lh, lh);  // by state for now
+    sh_neg[warp][n] = h < 0.f;
+    lh_max = fmaxf(lh_max, lh);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lh_max = fmaxf(lh_max, __shfl_xor_sync(kFullMask, lh_max, o));
+  // The largest S = sum Delta at which state n's term is kept:
+  // a_n S + log2|h_in[n]| >= log2 max|h_in| + kFixDropLog2.  It falls with S
+  // only for a_n < 0 with Delta >= 0 (softplus); otherwise it is kept.
+  for (int n = lane; n < N; n += 32) {
+    const float4 p = sh_p[warp][n];
+    const bool decays = a.softplus && p.x < 0.f;
+    sh_sd[warp][n] = decays ? (lh_max + kFixDropLog2 - p.z) / p.x : INFINITY;
+  }
+  __syncwarp();
+  // positions: states by that limit, latest first, so that the live states
+  // are always a prefix of the positions
+  float4 pp[(N + 31) / 32];
+  float sdv[(N + 31) / 32];
+  int ng[(N + 31) / 32], rk[(N + 31) / 32];
+#pragma unroll
+  for (int q = 0; q < (N + 31) / 32; ++q) {
+    const int n = lane + 32 * q;
+    if (n < N) {
+      const float sd = sh_sd[warp][n];
+      int rank = 0;
+      for (int m = 0; m < N; ++m) {
+        const float sm = sh_sd[warp][m];
+        rank += (sm > sd || (sm == sd && m < n)) ? 1 : 0;
+      }
+      pp[q] = sh_p[warp][n];
+      sdv[q] = sd;
+      ng[q] = sh_neg[warp][n];
+      rk[q] = rank;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < (N + 31) / 32; ++q) {
+    const int n = lane + 32 * q;
+    if (n < N) {
+      sh_p[warp][rk[q]] = pp[q];
+      sh_sd[warp][rk[q]] = sdv[q];
+      sh_neg[warp][rk[q]] = ng[q];
+      sh_n[warp][rk[q]] = n;
+    }
+  }
+  __syncwarp();
   const Tin* drow = static_cast<const Tin*>(a.delta) + bd * L;
   const Tin* zrow = a.z ? static_cast<const Tin*>(a.z) + bd * L : nullptr;
   const Tin* Cb = static_cast<const Tin*>(a.C) + b * (int64_t)N * L;
@@ -183,7 +231,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
       if (!ok) break;
     }
     const float4 dl4 = tma ? fix_lds4<Tin>(cur + FS::D_OFF + 4 * lane * FS::ES)
-                           : fix_load4(drow, t, t_end);
+                           : fix_load4(drow, t, t_end, bd * L, n_act);
     const float2 b2 = make_float2(bias, bias);
     float2 x01 = __fadd2_rn(make_float2(dl4.x, dl4.y), b2);
     float2 x23 = __fadd2_rn(make_float2(dl4.z, dl4.w), b2);
@@ -213,10 +261,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
     const float S_first = __shfl_sync(kFullMask, S[0], 0);
     carry += (double)__shfl_sync(kFullMask, incl, 31);
     // S_first is the block's smallest sum: a position dead now stays dead
-    if (a.softplus)
-      while (live > 0 && sh_p[warp][live - 1].x < 0.f &&
-             sh_p[warp][live - 1].x * S_first < kFixDropLog2)
-        --live;
+    while (live > 0 && S_first > sh_sd[warp][live - 1]) --live;
     if (live == 0) break;
     const float2 S01 = make_float2(S[0], S[1]), S23 = make_float2(S[2], S[3]);
     float2 pos01 = make_float2(0.f, 0.f), pos23 = pos01, neg01 = pos01, neg23 = pos01;
@@ -225,7 +270,8 @@ __global__ void __launch_bounds__(kFixWarps * 32)
       const float4 pr = sh_p[warp][i];
       const float4 c4 = (tma && FS::STAGE_C)
                             ? fix_lds4<Tin>(cur + sh_n[warp][i] * FS::ROW + 4 * lane * FS::ES)
-                            : fix_load4(Cb + (int64_t)sh_n[warp][i] * L, t, t_end);
+                            : fix_load4(Cb + (int64_t)sh_n[warp][i] * L, t, t_end,
+                                        (b * N + sh_n[warp][i]) * L, a.batch * N * L);
       const float2 x01e = __ffma2_rn(S01, make_float2(pr.x, pr.y), make_float2(pr.z, pr.w));
       const float2 x23e = __ffma2_rn(S23, make_float2(pr.x, pr.y), make_float2(pr.z, pr.w));
       const float2 e01 = make_float2(ex2_approx(x01e.x), ex2_approx(x01e.y));
@@ -240,23 +286,25 @@ __global__ void __launch_bounds__(kFixWarps * 32)
     }
     const float2 c01 = __fadd2_rn(pos01, make_float2(-neg01.x, -neg01.y));
     const float2 c23 = __fadd2_rn(pos23, make_float2(-neg23.x, -neg23.y));
-    const float4 y4 = tma ? fix_lds4<float>(cur + FS::Y_OFF + 16 * lane) : fix_load4(yrow, t, t_end);
+    const float4 y4 = tma ? fix_lds4<float>(cur + FS::Y_OFF + 16 * lane)
+                          : fix_load4(yrow, t, t_end, bd * L, n_act);
     float2 g01 = make_float2(1.f, 1.f), g23 = g01;
     if (zrow) {
       const float4 z4 = tma ? fix_lds4<Tin>(cur + FS::Z_OFF + 4 * lane * FS::ES)
-                            : fix_load4(zrow, t, t_end);
+                            : fix_load4(zrow, t, t_end, bd * L, n_act);
       g01 = silu_fast2(make_float2(z4.x, z4.y));
       g23 = silu_fast2(make_float2(z4.z, z4.w));
     }
     const float2 o01 = __ffma2_rn(c01, g01, make_float2(y4.x, y4.y));
     const float2 o23 = __ffma2_rn(c23, g23, make_float2(y4.z, y4.w));
     if (tma && t + 3 < t_end) {
-      *reinterpret_cast<float4*>(yrow + t) = make_float4(o01.x, o01.y, o23.x, o23.y);
+      if (in_range(bd * L + t, 4, n_act))
+        *reinterpret_cast<float4*>(yrow + t) = make_float4(o01.x, o01.y, o23.x, o23.y);
     } else {
       const float out[4] = {o01.x, o01.y, o23.x, o23.y};
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        if (t + kk < t_end) yrow[t + kk] = out[kk];
+        if (t + kk < t_end && in_range(bd * L + t + kk, n_act)) yrow[t + kk] = out[kk];
     }
     __syncwarp();  // every lane is done with this stage before TMA refills it
     if (tma && lane == 0 && k + 2 < nblk) issue(k + 2);

@@ -41,6 +41,10 @@
 
 #include "pointwise.cuh"
 
+#ifndef SS_BC_F32
+#define SS_BC_F32 0  // 1: bf16 B, C widened to fp32 once, in the transpose
+#endif
+
 namespace ssscan {
 
 struct FwdArgs {
@@ -145,7 +149,11 @@ struct ChunkedCfg {
   // (float4 units) is odd, so a quarter-warp's writes hit distinct banks.
   static constexpr int DW_STRIDE = CH + 1;
   static constexpr int DW_BYTES = QPR * DW_STRIDE * 16;
-  static constexpr int PAIR_BYTES = 4 * ES;          // one state pair: B_lo, B_hi, C_lo, C_hi
+  // bytes of one B or C value in the transposed tile: the input's, or fp32
+  // when bf16 inputs are widened once in the transpose (SS_BC_F32) instead of
+  // by every lane in the recurrence
+  static constexpr int BCES = (ES == 2 && SS_BC_F32) ? 4 : ES;
+  static constexpr int PAIR_BYTES = 4 * BCES;        // one state pair: B_lo, B_hi, C_lo, C_hi
   static constexpr int BC_BLOCK = 2 * PAIR_BYTES;    // two pairs: four states
   static constexpr int BC_DATA = (N / 4) * BC_BLOCK; // bytes of one timestep
   // A timestep's B, C are 16-byte units (four bf16 states or two fp32
@@ -153,7 +161,7 @@ struct ChunkedCfg {
   // lane they are stored unit-major, unit h of lane j at position h K + j, so
   // that the lanes of a quarter-warp load 16 consecutive bytes each (one
   // 128-byte wavefront) rather than every other 16 (two).
-  static constexpr int UNIT_STATES = 16 / (2 * ES);
+  static constexpr int UNIT_STATES = 16 / (2 * BCES);
   static constexpr int UPL = G / UNIT_STATES;         // units per lane (0: half a unit)
   static constexpr bool BC_PERMUTE = UPL >= 2;
   static constexpr int UNIT_STRIDE = BC_PERMUTE ? K * 16 : 16;  // between a lane's units
@@ -422,12 +430,27 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
         bw[k] = rot ? bv[(k + 3) & 3] : bv[k];
         cw[k] = rot ? cv4[(k + 3) & 3] : cv4[k];
       }
-      uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + CF::bc_pos(nb));
-      uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + CF::bc_pos(nb));
-      *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(cw[0], cw[1], 0x5410),
-                         __byte_perm(bw[2], bw[3], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
-      *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(cw[0], cw[1], 0x7632),
-                         __byte_perm(bw[2], bw[3], 0x7632), __byte_perm(cw[2], cw[3], 0x7632));
+      if constexpr (CF::BCES == 2) {
+        uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + CF::bc_pos(nb));
+        uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + CF::bc_pos(nb));
+        *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(cw[0], cw[1], 0x5410),
+                           __byte_perm(bw[2], bw[3], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
+        *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(cw[0], cw[1], 0x7632),
+                           __byte_perm(bw[2], bw[3], 0x7632), __byte_perm(cw[2], cw[3], 0x7632));
+      } else {  // widened: units 2 nb, 2 nb + 1 of rows 2 tp (low halves) and 2 tp + 1
+        auto lo = [](uint32_t v) { return __uint_as_float(v << 16); };
+        auto hi = [](uint32_t v) { return __uint_as_float(v & 0xffff0000u); };
+        unsigned char* r0 = bc + (2 * tp) * CF::BC_ROW;
+        unsigned char* r1 = r0 + CF::BC_ROW;
+        *reinterpret_cast<float4*>(r0 + CF::bc_pos(2 * nb)) =
+            make_float4(lo(bw[0]), lo(bw[1]), lo(cw[0]), lo(cw[1]));
+        *reinterpret_cast<float4*>(r0 + CF::bc_pos(2 * nb + 1)) =
+            make_float4(lo(bw[2]), lo(bw[3]), lo(cw[2]), lo(cw[3]));
+        *reinterpret_cast<float4*>(r1 + CF::bc_pos(2 * nb)) =
+            make_float4(hi(bw[0]), hi(bw[1]), hi(cw[0]), hi(cw[1]));
+        *reinterpret_cast<float4*>(r1 + CF::bc_pos(2 * nb + 1)) =
+            make_float4(hi(bw[2]), hi(bw[3]), hi(cw[2]), hi(cw[3]));
+      }
     }
   } else {
     const float* fb = reinterpret_cast<const float*>(rawB);
@@ -453,7 +476,7 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
 template <class CF, int NP>
 __device__ __forceinline__ void bc_pairs(const unsigned char* p, float2 (&b)[NP],
                                          float2 (&c)[NP]) {
-  if constexpr (CF::ES == 2) {
+  if constexpr (CF::BCES == 2) {
     if constexpr (NP % 2 == 0) {
 #pragma unroll
       for (int i = 0; i < NP / 2; ++i) {
