@@ -72,6 +72,13 @@ typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
  *                caller-owned, 256-byte aligned (nullable when that is 0).
  *                Its contents on entry do not matter; the call may overwrite it.
  *                Two calls in flight at once must not share one workspace.
+ *                It holds what the chosen schedule hands between CTAs: the
+ *                carries of the load-balanced schedule, or, when the sequence
+ *                is cut into segments scanned at once (few channels, long L),
+ *                each segment's end state and sum of Delta, from which a
+ *                second kernel adds every segment's carry-in to y and forms
+ *                last_state (the associative operator of "Mamba 选择性机制",
+ *                sec. 3.1).
  *
  * Alignment: every tensor pointer must be aligned to its element size.  When
  * seqlen*sizeof(in_dtype) is a multiple of 16 and u, delta, z, B, C, y_out are
@@ -279,7 +286,8 @@ size_t ss_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen,
  *
  * Arguments, layouts, results and errors are those of ss_scan_fwd, minus the
  * workspace.  The scratch the scan may need (the carries handed between CTAs
- * of the load-balanced schedule) lives in one static device array of
+ * of the load-balanced schedule, or the segment states and sums of a long
+ * sequence cut into segments) lives in one static device array of
  * SS_NOALLOC_SCRATCH_BYTES that the library owns; every GPU that loads the
  * library holds it until the process exits.  This entry point calls no
  * cudaMalloc, cudaFree or allocating library routine.

@@ -41,10 +41,6 @@
 
 #include "pointwise.cuh"
 
-#ifndef SS_BC_F32
-#define SS_BC_F32 0  // 1: bf16 B, C widened to fp32 once, in the transpose
-#endif
-
 namespace ssscan {
 
 struct FwdArgs {
@@ -149,10 +145,7 @@ struct ChunkedCfg {
   // (float4 units) is odd, so a quarter-warp's writes hit distinct banks.
   static constexpr int DW_STRIDE = CH + 1;
   static constexpr int DW_BYTES = QPR * DW_STRIDE * 16;
-  // bytes of one B or C value in the transposed tile: the input's, or fp32
-  // when bf16 inputs are widened once in the transpose (SS_BC_F32) instead of
-  // by every lane in the recurrence
-  static constexpr int BCES = (ES == 2 && SS_BC_F32) ? 4 : ES;
+  static constexpr int BCES = ES;  // bytes of one B or C value in the transposed tile
   static constexpr int PAIR_BYTES = 4 * BCES;        // one state pair: B_lo, B_hi, C_lo, C_hi
   static constexpr int BC_BLOCK = 2 * PAIR_BYTES;    // two pairs: four states
   static constexpr int BC_DATA = (N / 4) * BC_BLOCK; // bytes of one timestep
@@ -430,27 +423,12 @@ __device__ __forceinline__ void phase1(const FwdArgs& a, const typename CF::Elem
         bw[k] = rot ? bv[(k + 3) & 3] : bv[k];
         cw[k] = rot ? cv4[(k + 3) & 3] : cv4[k];
       }
-      if constexpr (CF::BCES == 2) {
-        uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + CF::bc_pos(nb));
-        uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + CF::bc_pos(nb));
-        *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(cw[0], cw[1], 0x5410),
-                           __byte_perm(bw[2], bw[3], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
-        *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(cw[0], cw[1], 0x7632),
-                           __byte_perm(bw[2], bw[3], 0x7632), __byte_perm(cw[2], cw[3], 0x7632));
-      } else {  // widened: units 2 nb, 2 nb + 1 of rows 2 tp (low halves) and 2 tp + 1
-        auto lo = [](uint32_t v) { return __uint_as_float(v << 16); };
-        auto hi = [](uint32_t v) { return __uint_as_float(v & 0xffff0000u); };
-        unsigned char* r0 = bc + (2 * tp) * CF::BC_ROW;
-        unsigned char* r1 = r0 + CF::BC_ROW;
-        *reinterpret_cast<float4*>(r0 + CF::bc_pos(2 * nb)) =
-            make_float4(lo(bw[0]), lo(bw[1]), lo(cw[0]), lo(cw[1]));
-        *reinterpret_cast<float4*>(r0 + CF::bc_pos(2 * nb + 1)) =
-            make_float4(lo(bw[2]), lo(bw[3]), lo(cw[2]), lo(cw[3]));
-        *reinterpret_cast<float4*>(r1 + CF::bc_pos(2 * nb)) =
-            make_float4(hi(bw[0]), hi(bw[1]), hi(cw[0]), hi(cw[1]));
-        *reinterpret_cast<float4*>(r1 + CF::bc_pos(2 * nb + 1)) =
-            make_float4(hi(bw[2]), hi(bw[3]), hi(cw[2]), hi(cw[3]));
-      }
+      uint4* dst0 = reinterpret_cast<uint4*>(bc + (2 * tp) * CF::BC_ROW + CF::bc_pos(nb));
+      uint4* dst1 = reinterpret_cast<uint4*>(bc + (2 * tp + 1) * CF::BC_ROW + CF::bc_pos(nb));
+      *dst0 = make_uint4(__byte_perm(bw[0], bw[1], 0x5410), __byte_perm(cw[0], cw[1], 0x5410),
+                         __byte_perm(bw[2], bw[3], 0x5410), __byte_perm(cw[2], cw[3], 0x5410));
+      *dst1 = make_uint4(__byte_perm(bw[0], bw[1], 0x7632), __byte_perm(cw[0], cw[1], 0x7632),
+                         __byte_perm(bw[2], bw[3], 0x7632), __byte_perm(cw[2], cw[3], 0x7632));
     }
   } else {
     const float* fb = reinterpret_cast<const float*>(rawB);
