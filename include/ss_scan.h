@@ -73,7 +73,9 @@ typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
  *                Its contents on entry do not matter; the call may overwrite it.
  *                Two calls in flight at once must not share one workspace.
  *                It holds what the chosen schedule hands between CTAs: the
- *                carries of the load-balanced schedule, or, when the sequence
+ *                carries of the load-balanced schedule and the counter from
+ *                which its CTAs take their worker ids (the call zeroes it on
+ *                the stream before its kernel), or, when the sequence
  *                is cut into segments scanned at once (few channels, long L),
  *                each segment's end state and sum of Delta, from which a
  *                second kernel adds every segment's carry-in to y and forms

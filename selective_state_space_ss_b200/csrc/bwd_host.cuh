@@ -23,9 +23,13 @@ size_t ckpt_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N) {
   return align256((size_t)batch * (size_t)nk * (size_t)dim * (size_t)N * sizeof(float));
 }
 
+#ifndef SS_BWD_G
+#define SS_BWD_G 4
+#endif
+
 template <typename E, int N>
 ss_status launch_bwd(const BwdArgs& a, size_t ws_bytes, cudaStream_t stream) {
-  using CF = BwdCfg<E, N>;
+  using CF = BwdCfg<E, N, (N == 16 ? SS_BWD_G : 4)>;
   if (once_per_device<CF>([] {
         return cudaFuncSetAttribute(scan_bwd_kernel<CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     CF::SMEM_BYTES) == cudaSuccess;

@@ -88,7 +88,7 @@ struct Plan {
   int64_t groups = 0, nk = 0, tiles = 0;
   int nseg = 1;
   int64_t seg_chunks = 0;
-  size_t carry_bytes = 0, seg_h_bytes = 0, ws_bytes = 0;
+  size_t carry_bytes = 0, flag_bytes = 0, seg_h_bytes = 0, ws_bytes = 0;
 };
 
 template <class CF>
@@ -137,7 +137,8 @@ bool make_plan(int64_t batch, int64_t dim, int64_t seqlen, Plan* p) {
   p->workers = (int)w;
   if (p->workers < p->groups) {
     p->carry_bytes = align256((size_t)p->workers * CF::CH * CF::N * sizeof(float));
-    p->ws_bytes = p->carry_bytes + align256((size_t)p->workers * sizeof(unsigned long long));
+    p->flag_bytes = align256((size_t)p->workers * sizeof(unsigned long long));
+    p->ws_bytes = p->carry_bytes + p->flag_bytes + 256;  // + the worker ticket counter
     return true;
   }
   // Segments: fill the resident slots once (groups x nseg CTAs).  Not for the
@@ -188,6 +189,7 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
                                                                  p.carry_bytes)
                         : nullptr;
   sc.epoch = next_epoch();
+  sc.ticket = nullptr;
   const long long spin = g_dbg_spin_limit.exchange(0);
   sc.spin_limit = spin > 0 ? (uint32_t)spin : kCarrySpinLimit;
   sc.skip_publish = (int)g_dbg_skip_publish.exchange(-1);
@@ -196,6 +198,12 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
   g_dbg_workers.store(0);
   g_dbg_segments.store(0);
   if (p.workers < p.groups) {
+    // worker ids come from a counter taken at CTA start, so a worker's
+    // predecessor is always already resident; the counter starts at 0 per launch
+    sc.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + p.carry_bytes +
+                                                p.flag_bytes);
+    if (cudaMemsetAsync(sc.ticket, 0, sizeof(unsigned int), stream) != cudaSuccess)
+      return SS_ERR_CUDA;
     scan_fwd_chunked_kernel<CF, true><<<(unsigned)p.workers, CF::NT, CF::SMEM_BYTES, stream>>>(a, maps, sc);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
   }
@@ -220,20 +228,26 @@ ss_status launch_chunked(FwdArgs a, void* workspace, size_t workspace_bytes,
   FixMaps fm;
   memset(&fm, 0, sizeof fm);
   // TMA blocks need the forward's 16-byte aligned rows (a.vec)
-  f.tma = a.vec && encode_3d(&fm.delta, a.delta, bf16, a.seqlen, a.dim, a.batch, kFixBlock, 1) &&
-          encode_3d(&fm.z, a.z ? a.z : a.delta, bf16, a.seqlen, a.dim, a.batch, kFixBlock, 1) &&
-          encode_3d(&fm.y, a.y, false, a.seqlen, a.dim, a.batch, kFixBlock, 1) &&
-          (!FS::STAGE_C || encode_3d(&fm.C, a.C, bf16, a.seqlen, CF::N, a.batch, kFixBlock, CF::N));
+  f.tma = a.vec && encode_3d(&fm.delta, a.delta, bf16, a.seqlen, a.dim, a.batch, FS::BLOCK, 1) &&
+          encode_3d(&fm.z, a.z ? a.z : a.delta, bf16, a.seqlen, a.dim, a.batch, FS::BLOCK, 1) &&
+          encode_3d(&fm.y, a.y, false, a.seqlen, a.dim, a.batch, FS::BLOCK, 1) &&
+          (!FS::STAGE_C || encode_3d(&fm.C, a.C, bf16, a.seqlen, CF::N, a.batch, FS::BLOCK, CF::N));
   const int64_t tasks = a.batch * a.dim * (p.nseg - 1);
   const int64_t blocks = (tasks + kFixWarps - 1) / kFixWarps;
   if (blocks > INT_MAX) return SS_ERR_INVALID_ARG;
   if (once_per_device<FixTag<E, CF::N>>([] {
-        return cudaFuncSetAttribute(scan_fix_kernel<E, CF::N>,
+        return cudaFuncSetAttribute(scan_fix_kernel<E, CF::N, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    FS::SMEM) == cudaSuccess &&
+               cudaFuncSetAttribute(scan_fix_kernel<E, CF::N, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     FS::SMEM) == cudaSuccess;
       }) != 1)
     return SS_ERR_CUDA;
-  scan_fix_kernel<E, CF::N><<<(unsigned)blocks, kFixWarps * 32, FS::SMEM, stream>>>(f, fm);
+  if (f.tma)
+    scan_fix_kernel<E, CF::N, true><<<(unsigned)blocks, kFixWarps * 32, FS::SMEM, stream>>>(f, fm);
+  else
+    scan_fix_kernel<E, CF::N, false><<<(unsigned)blocks, kFixWarps * 32, 0, stream>>>(f, fm);
   return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 

@@ -56,11 +56,12 @@ struct BwdArgs {
   int softplus;
 };
 
-template <typename Tin, int N_>
+template <typename Tin, int N_, int G_ = 4>
 struct BwdCfg {
   using Elem = Tin;
   static constexpr int N = N_;
-  static constexpr int G = 4;             // states per lane
+  static constexpr int G = G_;            // states per lane (2 or 4)
+  static constexpr int HP = G / 2;        // packed pairs per lane
   static constexpr int K = N / G;         // lanes per channel
   static constexpr int CPW = 32 / K;      // channels per warp
   static constexpr int NWARPS = 4;
@@ -71,6 +72,10 @@ struct BwdCfg {
   static constexpr int ITEMS = CH * T;    // (step, channel) items per chunk
   static constexpr int IPT = (ITEMS + NT - 1) / NT;
   static constexpr int STEP_FLOATS = CH * N;  // one step's states of the CTA
+  // row pitch of the per-step states: 64 bytes of padding, so that the
+  // 16-byte reads of two consecutive steps by a quarter-warp in the channel
+  // reductions fall on opposite halves of the banks
+  static constexpr int HB_STRIDE = STEP_FLOATS + 16;
   // staged inputs per thread (register prefetch of the next chunk)
   static constexpr int ACT_PT = (CH * T + NT - 1) / NT;
   static constexpr int SEL_PT = (N * T + NT - 1) / NT;
@@ -88,9 +93,9 @@ struct BwdCfg {
   static constexpr int OFF_B = (OFF_P2 + T * CHP + 3) / 4 * 4;  // [T][NP]
   static constexpr int OFF_C = OFF_B + T * NP;
   static constexpr int OFF_H = OFF_C + T * NP;          // [T][CH*N] states, then g Delta u
-  static constexpr int SMEM_FLOATS = OFF_H + T * STEP_FLOATS;
+  static constexpr int SMEM_FLOATS = OFF_H + T * HB_STRIDE;
   static constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
-  static_assert(N % G == 0 && 32 % K == 0, "lane split");
+  static_assert(N % G == 0 && 32 % K == 0 && (G == 2 || G == 4), "lane split");
   static_assert(ITEMS % NT == 0 || ITEMS < NT, "whole items per thread");
   static constexpr bool ITEM_GUARD = ITEMS < NT;  // some threads have no item
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -249,10 +254,11 @@ __global__ void __launch_bounds__(CF::NT)
   float* ck_lane = a.ckpt + (b * nk * a.dim + d) * N + j * G;
   float* hb = sm + CF::OFF_H;
 
-  // decay constants of this lane's four states, as two packed pairs
-  float2 A2[2], An[2];
+  constexpr int HP = CF::HP;
+  // decay constants of this lane's G states, as HP packed pairs
+  float2 A2[HP], An[HP];
 #pragma unroll
-  for (int p = 0; p < 2; ++p) {
+  for (int p = 0; p < HP; ++p) {
     const float a0 = chan_ok ? __ldg(a.A + d * N + j * G + 2 * p) : 0.f;
     const float a1 = chan_ok ? __ldg(a.A + d * N + j * G + 2 * p + 1) : 0.f;
     An[p] = make_float2(a0, a1);
@@ -262,19 +268,31 @@ __global__ void __launch_bounds__(CF::NT)
   BwdSlots<CF> sl;
   bwd_slots<CF>(a, b, d0, sl);
   auto ex2_pair = [](float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); };
-  auto ld_pairs = [](const float* p, float2 (&v)[2]) {
-    const float4 q = *reinterpret_cast<const float4*>(p);
-    v[0] = make_float2(q.x, q.y);
-    v[1] = make_float2(q.z, q.w);
+  auto ld_pairs = [](const float* p, float2 (&v)[HP]) {  // one 16- or 8-byte load
+    if constexpr (HP == 2) {
+      const float4 q = *reinterpret_cast<const float4*>(p);
+      v[0] = make_float2(q.x, q.y);
+      v[HP - 1] = make_float2(q.z, q.w);
+    } else {
+      v[0] = *reinterpret_cast<const float2*>(p);
+    }
   };
-  auto st_pairs = [](float* p, const float2 (&v)[2]) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+  auto st_pairs = [](float* p, const float2 (&v)[HP]) {
+    if constexpr (HP == 2)
+      *reinterpret_cast<float4*>(p) = make_float4(v[0].x, v[0].y, v[HP - 1].x, v[HP - 1].y);
+    else
+      *reinterpret_cast<float2*>(p) = v[0];
+  };
+  auto zero_pairs = [](float2 (&v)[HP]) {
+#pragma unroll
+    for (int p = 0; p < HP; ++p) v[p] = make_float2(0.f, 0.f);
   };
   float* hb_lane = hb + c * N + j * G;        // and in every step row of hb
 
   // ---- pass 1: forward, checkpoint the state at every chunk start ----
   // (skipped when the training forward has written the checkpoints)
-  float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 h[HP];
+  zero_pairs(h);
   if (!a.ckpt_given) bwd_fetch<CF, false>(a, st, sl, d0, 0);
   for (int64_t k = 0; k < nk && !a.ckpt_given; ++k) {
     if (chan_ok) st_pairs(ck_lane + k * ck_stride, h);
@@ -285,35 +303,39 @@ __global__ void __launch_bounds__(CF::NT)
     for (int t = 0; t < T; ++t) {
       const float dl = sm[CF::OFF_DL + t * CHP + c], w = sm[CF::OFF_W + t * CHP + c];
       const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w);
-      float2 bb[2];
+      float2 bb[HP];
       ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
 #pragma unroll
-      for (int p = 0; p < 2; ++p)
+      for (int p = 0; p < HP; ++p)
         h[p] = __ffma2_rn(ex2_pair(__fmul2_rn(dl2, A2[p])), h[p], __fmul2_rn(w2, bb[p]));
     }
     __syncthreads();
   }
 
   // ---- pass 2: chunks in reverse ----
-  float2 carry[2];
+  float2 carry[HP];
 #pragma unroll
-  for (int p = 0; p < 2; ++p) {
+  for (int p = 0; p < HP; ++p) {
     const float* dl_ = a.dlast + (b * a.dim + d) * N + j * G + 2 * p;
     carry[p] = (a.dlast && chan_ok) ? make_float2(dl_[0], dl_[1]) : make_float2(0.f, 0.f);
   }
-  float2 dA_acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 dA_acc[HP];
+  zero_pairs(dA_acc);
   float dD_acc[CF::IPT], db_acc[CF::IPT];
 #pragma unroll
   for (int it = 0; it < CF::IPT; ++it) dD_acc[it] = db_acc[it] = 0.f;
 
   bwd_fetch<CF, true>(a, st, sl, d0, (nk - 1) * T);
-  float2 ck_next[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 ck_next[HP];
+  zero_pairs(ck_next);
   // the checkpoint of the chunk to come, loaded a chunk early (the same thread
   // wrote it in pass 1, or the training forward did before this launch)
   if (chan_ok) ld_pairs(ck_lane + (nk - 1) * ck_stride, ck_next);
   for (int64_t k = nk - 1; k >= 0; --k) {
     const int64_t t0 = k * T;
-    const float2 h_start[2] = {ck_next[0], ck_next[1]};
+    float2 h_start[HP];
+#pragma unroll
+    for (int p = 0; p < HP; ++p) h_start[p] = ck_next[p];
     bwd_store<CF, true>(a, st, sl, sm, d0, t0);
     if (k > 0) {
       bwd_fetch<CF, true>(a, st, sl, d0, (k - 1) * T);
@@ -321,21 +343,23 @@ __global__ void __launch_bounds__(CF::NT)
     }
     __syncthreads();
     // recompute the chunk's states from its checkpoint; channel readouts
-    float2 hs[2] = {h_start[0], h_start[1]};
+    float2 hs[HP];
+#pragma unroll
+    for (int p = 0; p < HP; ++p) hs[p] = h_start[p];
 #pragma unroll 4
     for (int t = 0; t < T; ++t) {
       const float dl = sm[CF::OFF_DL + t * CHP + c], w = sm[CF::OFF_W + t * CHP + c];
       const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w);
-      float2 bb[2], cc[2];
+      float2 bb[HP], cc[HP];
       ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
       ld_pairs(sm + CF::OFF_C + t * CF::NP + j * G, cc);
       float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
+      for (int p = 0; p < HP; ++p) {
         hs[p] = __ffma2_rn(ex2_pair(__fmul2_rn(dl2, A2[p])), hs[p], __fmul2_rn(w2, bb[p]));
         acc = __ffma2_rn(cc[p], hs[p], acc);
       }
-      st_pairs(hb_lane + t * CF::STEP_FLOATS, hs);
+      st_pairs(hb_lane + t * CF::HB_STRIDE, hs);
       const float part = lane_sum<K>(acc.x + acc.y);
       if (j == 0) sm[CF::OFF_P1 + t * CHP + c] = part;
     }
@@ -362,15 +386,24 @@ __global__ void __launch_bounds__(CF::NT)
       if (in) dD_acc[it] = fmaf(dq, uu, dD_acc[it]);
     }
     __syncthreads();
-    // dC[b, n, t] += sum_c dq[t, c] h_t[c, n]
-    for (int i = tid; i < N * T; i += CF::NT) {
-      const int tt = i / N, n = i - tt * N;
+    // dC[b, n, t] += sum_c dq[t, c] h_t[c, n], four consecutive states per item
+    for (int i = tid; i < (N / 4) * T; i += CF::NT) {
+      const int tt = i / (N / 4), n = 4 * (i - tt * (N / 4));
       if (t0 + tt >= L) continue;
-      float acc = 0.f;
+      float2 s01 = make_float2(0.f, 0.f), s23 = s01;
+      const float* hr = hb + tt * CF::HB_STRIDE + n;
 #pragma unroll 8
-      for (int cc = 0; cc < CF::CH; ++cc)
-        acc = fmaf(sm[CF::OFF_DY + tt * CHP + cc], hb[tt * CF::STEP_FLOATS + cc * N + n], acc);
-      atomicAdd(a.dC + (b * N + n) * L + t0 + tt, acc);
+      for (int cc = 0; cc < CF::CH; ++cc) {
+        const float dq = sm[CF::OFF_DY + tt * CHP + cc];
+        const float4 h4 = *reinterpret_cast<const float4*>(hr + cc * N);
+        s01 = __ffma2_rn(make_float2(dq, dq), make_float2(h4.x, h4.y), s01);
+        s23 = __ffma2_rn(make_float2(dq, dq), make_float2(h4.z, h4.w), s23);
+      }
+      float* dst = a.dC + (b * N + n) * L + t0 + tt;
+      atomicAdd(dst, s01.x);
+      atomicAdd(dst + L, s01.y);
+      atomicAdd(dst + 2 * L, s23.x);
+      atomicAdd(dst + 3 * L, s23.y);
     }
     __syncthreads();
     // the adjoint, backwards through the chunk
@@ -379,47 +412,59 @@ __global__ void __launch_bounds__(CF::NT)
       const float dl = sm[CF::OFF_DL + t * CHP + c];
       const float uu = sm[CF::OFF_U + t * CHP + c];
       const float dq = sm[CF::OFF_DY + t * CHP + c];
-      const float2 dl2 = make_float2(dl, dl), uu2 = make_float2(uu, uu), dq2 = make_float2(dq, dq);
-      float2 bb[2], cc[2], prev[2];
+      const float w = sm[CF::OFF_W + t * CHP + c];
+      const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w), dq2 = make_float2(dq, dq);
+      float2 bb[HP], cc[HP], prev[HP];
       ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
       ld_pairs(sm + CF::OFF_C + t * CF::NP + j * G, cc);
       if (t > 0) {
-        ld_pairs(hb_lane + (t - 1) * CF::STEP_FLOATS, prev);
+        ld_pairs(hb_lane + (t - 1) * CF::HB_STRIDE, prev);
       } else {
-        prev[0] = h_start[0];
-        prev[1] = h_start[1];
-      }
-      float2 ddl = make_float2(0.f, 0.f), dup = make_float2(0.f, 0.f), gdu[2];
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
+        for (int p = 0; p < HP; ++p) prev[p] = h_start[p];
+      }
+      // per state: g_t, and with a_t h_{t-1} (eprev) the terms of
+      //   dDelta_t = u_t sum_n g B + sum_n g A a h_{t-1},  du_t - dq D = Delta_t sum_n g B,
+      //   dA += Delta_t g a h_{t-1},  dB_t += g Delta_t u_t
+      float2 gB = make_float2(0.f, 0.f), gAe = make_float2(0.f, 0.f), gdu[HP];
+#pragma unroll
+      for (int p = 0; p < HP; ++p) {
         const float2 e = ex2_pair(__fmul2_rn(dl2, A2[p]));
         const float2 gt = __ffma2_rn(dq2, cc[p], carry[p]);
-        const float2 eprev = __fmul2_rn(e, prev[p]);
-        ddl = __ffma2_rn(gt, __ffma2_rn(bb[p], uu2, __fmul2_rn(An[p], eprev)), ddl);
-        const float2 gdl = __fmul2_rn(gt, dl2);
-        dup = __ffma2_rn(gdl, bb[p], dup);
-        dA_acc[p] = __ffma2_rn(gdl, eprev, dA_acc[p]);
-        gdu[p] = __fmul2_rn(gdl, uu2);
+        const float2 ge = __fmul2_rn(gt, __fmul2_rn(e, prev[p]));
+        gB = __ffma2_rn(gt, bb[p], gB);
+        gAe = __ffma2_rn(An[p], ge, gAe);
+        dA_acc[p] = __ffma2_rn(dl2, ge, dA_acc[p]);
+        gdu[p] = __fmul2_rn(gt, w2);
         carry[p] = __fmul2_rn(e, gt);
       }
       // h_t is no longer needed (its dC and its step's prev are done): reuse the slot
-      st_pairs(hb_lane + t * CF::STEP_FLOATS, gdu);
-      const float ddl_c = lane_sum<K>(ddl.x + ddl.y);
-      const float dup_c = lane_sum<K>(dup.x + dup.y);
+      st_pairs(hb_lane + t * CF::HB_STRIDE, gdu);
+      const float gB_c = lane_sum<K>(gB.x + gB.y);
+      const float gAe_c = lane_sum<K>(gAe.x + gAe.y);
       if (j == 0) {
-        sm[CF::OFF_P1 + t * CHP + c] = ddl_c;
-        sm[CF::OFF_P2 + t * CHP + c] = dup_c;
+        sm[CF::OFF_P1 + t * CHP + c] = fmaf(uu, gB_c, gAe_c);
+        sm[CF::OFF_P2 + t * CHP + c] = dl * gB_c;
       }
     }
     __syncthreads();
-    // dB[b, n, t] += sum_c g Delta u
-    for (int i = tid; i < N * T; i += CF::NT) {
-      const int tt = i / N, n = i - tt * N;
+    // dB[b, n, t] += sum_c g Delta u, four consecutive states per item
+    for (int i = tid; i < (N / 4) * T; i += CF::NT) {
+      const int tt = i / (N / 4), n = 4 * (i - tt * (N / 4));
       if (t0 + tt >= L) continue;
-      float acc = 0.f;
+      float2 s01 = make_float2(0.f, 0.f), s23 = s01;
+      const float* hr = hb + tt * CF::HB_STRIDE + n;
 #pragma unroll 8
-      for (int cc = 0; cc < CF::CH; ++cc) acc += hb[tt * CF::STEP_FLOATS + cc * N + n];
-      atomicAdd(a.dB + (b * N + n) * L + t0 + tt, acc);
+      for (int cc = 0; cc < CF::CH; ++cc) {
+        const float4 g4 = *reinterpret_cast<const float4*>(hr + cc * N);
+        s01 = __fadd2_rn(s01, make_float2(g4.x, g4.y));
+        s23 = __fadd2_rn(s23, make_float2(g4.z, g4.w));
+      }
+      float* dst = a.dB + (b * N + n) * L + t0 + tt;
+      atomicAdd(dst, s01.x);
+      atomicAdd(dst + L, s01.y);
+      atomicAdd(dst + 2 * L, s23.x);
+      atomicAdd(dst + 3 * L, s23.y);
     }
     // per item: du, ddelta, the bias gradient
 #pragma unroll
@@ -441,7 +486,7 @@ __global__ void __launch_bounds__(CF::NT)
   // per-channel sums over this CTA's part of the batch
   if (chan_ok) {
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
+    for (int p = 0; p < HP; ++p) {
       atomicAdd(a.dA + d * N + j * G + 2 * p, dA_acc[p].x);
       atomicAdd(a.dA + d * N + j * G + 2 * p + 1, dA_acc[p].y);
     }

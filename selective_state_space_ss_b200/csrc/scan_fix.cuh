@@ -12,10 +12,11 @@
 // readout therefore misses sum_n C_t[n] P_t[n] h_in[n], gated by SiLU(z_t);
 // this kernel adds it to y and writes the final state.
 //
-// One warp per (batch row, channel, segment >= 1).  Each lane takes four
-// consecutive steps of every 128-step block; the prefix sums of Delta over the
-// segment come from a per-lane sum and a warp scan (the running total in
-// double).  The term of state n is evaluated as sign(h_in[n]) 2^(a_n S_t +
+// One warp per (batch row, channel, segment >= 1).  Each lane takes SPL
+// consecutive steps of every block of 32 SPL steps; the prefix sums of Delta
+// over the segment come from a per-lane sum and a warp scan, the running
+// total kept as an unevaluated sum of two floats (Knuth's two-sum), so that
+// it does not drift over a long segment.  The term of state n is evaluated as sign(h_in[n]) 2^(a_n S_t +
 // log2|h_in[n]|) C_t[n] (one fused multiply-add for the exponent).  A state's
 // term is dropped once |h_in[n]| P_t[n] < 2^-36 max_m |h_in[m]| for the rest of
 // the segment: with softplus on (Delta >= 0) and A[d,n] < 0 the weight only
@@ -26,10 +27,11 @@
 // live ones are always a prefix of that order, and the walk ends at the first
 // block where none is live.
 //
-// With 16-byte aligned rows, one lane of the warp brings each block's delta,
+// With 16-byte aligned rows, four lanes of the warp bring each block's delta,
 // z, y (and, for N = 16, the block's C tile) into shared memory with TMA, two
 // blocks deep, completing on a per-warp mbarrier; otherwise the lanes load
-// element-wise.
+// element-wise.  A staged C value takes the sign of h_in[n] by an xor of its
+// sign bit as it is read, so that each term is one fused multiply-add.
 #pragma once
 
 #include "pointwise.cuh"
@@ -59,22 +61,30 @@ struct FixMaps {
   CUtensorMap delta, z, y, C;
 };
 
-constexpr int kFixWarps = 4;
-constexpr int kFixBlock = 128;         // steps per block (4 per lane)
+// One warp (one task) per CTA: tasks differ in length by orders of magnitude
+// (a state's term lives for ~1/(Delta |A|) steps), and a CTA holds its
+// resources until its longest warp is done.  Measured on B1 L1048576 D1536
+// N16: 1, 2 and 4 warps per CTA take 2.87, 2.97 and 3.01 ms.
+constexpr int kFixWarps = 1;
 constexpr float kFixDropLog2 = -36.f;  // log2 of a term's weight, relative to the largest
                                        // state, below which it is dropped
 
 // Per-warp staging of one block (byte offsets, each a multiple of 128).
+// SPL consecutive steps per lane: 8 for bf16 (the per-position loads and
+// the block's fixed work are spread over more steps: 2.68 against 2.87 ms
+// with 4 on the workload above), 4 for fp32 (half the staging per step).
 template <typename Tin, int N>
 struct FixStage {
   static constexpr int ES = (int)sizeof(Tin);
+  static constexpr int SPL = ES == 2 ? 8 : 4;
+  static constexpr int BLOCK = 32 * SPL;  // steps per block
   static constexpr bool STAGE_C = N == 16;
-  static constexpr int ROW = kFixBlock * ES;  // one 128-step row of an input
+  static constexpr int ROW = BLOCK * ES;  // one block-long row of an input
   static constexpr int C_BYTES = STAGE_C ? N * ROW : 0;
   static constexpr int D_OFF = C_BYTES;
   static constexpr int Z_OFF = D_OFF + ROW;
   static constexpr int Y_OFF = Z_OFF + ROW;
-  static constexpr int BYTES = Y_OFF + kFixBlock * 4;  // one stage
+  static constexpr int BYTES = Y_OFF + BLOCK * 4;  // one stage
   static constexpr int SMEM = kFixWarps * 2 * BYTES + 128;  // + slack to align the base
   static_assert(ROW % 128 == 0 && BYTES % 128 == 0, "TMA destinations 128-byte aligned");
 };
@@ -91,6 +101,23 @@ __device__ __forceinline__ float4 fix_load4(const T* row, int64_t t, int64_t end
   return make_float4(e[0], e[1], e[2], e[3]);
 }
 
+// Four staged elements widened to float, their sign bits flipped by `flip`
+// (0, or the sign bits of every element of a 32-bit word).
+template <typename T>
+__device__ __forceinline__ float4 fix_lds4x(const unsigned char* p, uint32_t flip) {
+  if constexpr (sizeof(T) == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    return make_float4(__uint_as_float(v.x ^ flip), __uint_as_float(v.y ^ flip),
+                       __uint_as_float(v.z ^ flip), __uint_as_float(v.w ^ flip));
+  } else {
+    uint2 v = *reinterpret_cast<const uint2*>(p);
+    v.x ^= flip;
+    v.y ^= flip;
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                       __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ float4 fix_lds4(const unsigned char* p) {
   if constexpr (sizeof(T) == 4) {
@@ -102,13 +129,17 @@ __device__ __forceinline__ float4 fix_lds4(const unsigned char* p) {
   }
 }
 
-template <typename Tin, int N>
+// TMA: the blocks come in by TMA (a.tma set); otherwise the lanes load them
+// element-wise.  A template parameter, so that neither path's code sits,
+// predicated off, in the other's loops.
+template <typename Tin, int N, bool TMA>
 __global__ void __launch_bounds__(kFixWarps * 32)
     scan_fix_kernel(const FixArgs a, const __grid_constant__ FixMaps maps) {
   using FS = FixStage<Tin, N>;
   __shared__ __align__(16) float4 sh_p[kFixWarps][N];  // {a, a, log2|h_in|, log2|h_in|}
-  __shared__ int sh_n[kFixWarps][N];    // state index at each position (slowest decay first)
-  __shared__ int sh_neg[kFixWarps][N];  // sign of h_in at each position
+  // {state index, sign bits of h_in < 0 for a 32-bit word of C} at each position
+  __shared__ int2 sh_nq[kFixWarps][N];
+  constexpr int kFlip = sizeof(Tin) == 2 ? (int)0x80008000u : (int)0x80000000u;
   __shared__ float sh_sd[kFixWarps][N];  // the largest sum of Delta at which it is kept
   __shared__ __align__(8) uint64_t fbar[kFixWarps][2];
   extern __shared__ __align__(128) unsigned char fix_dyn[];
@@ -122,7 +153,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
   const int64_t b = bd / a.dim, d = bd - b * a.dim;
   const int64_t L = a.seqlen;
   const int64_t n_act = a.batch * a.dim * L;  // elements of delta, z and y
-  const bool tma = a.tma != 0;
+  constexpr bool tma = TMA;
 
   // h_in of segment s: fold the (prod A_bar, end state) pairs of segments
   // 0 .. s-1 in order; the last segment's task also writes the final state.
@@ -141,7 +172,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
     float lh;  // log2|h_in|: -inf for 0, so that its terms vanish
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lh) : "f"(fabsf(h)));
     sh_p[warp][n] = make_float4(an, an, lh, lh);  // by state for now
-    sh_neg[warp][n] = h < 0.f;
+    sh_nq[warp][n] = make_int2(n, h < 0.f ? kFlip : 0);
     lh_max = fmaxf(lh_max, lh);
   }
 #pragma unroll
@@ -172,7 +203,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
       }
       pp[q] = sh_p[warp][n];
       sdv[q] = sd;
-      ng[q] = sh_neg[warp][n];
+      ng[q] = sh_nq[warp][n].y;
       rk[q] = rank;
     }
   }
@@ -183,8 +214,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
     if (n < N) {
       sh_p[warp][rk[q]] = pp[q];
       sh_sd[warp][rk[q]] = sdv[q];
-      sh_neg[warp][rk[q]] = ng[q];
-      sh_n[warp][rk[q]] = n;
+      sh_nq[warp][rk[q]] = make_int2(n, ng[q]);
     }
   }
   __syncwarp();
@@ -195,119 +225,166 @@ __global__ void __launch_bounds__(kFixWarps * 32)
   const float bias = a.delta_bias ? __ldg(a.delta_bias + d) : 0.f;
   const int64_t t_begin = (int64_t)s * a.seg_len;
   const int64_t t_end = t_begin + a.seg_len < L ? t_begin + a.seg_len : L;
-  const int64_t nblk = (t_end - t_begin + kFixBlock - 1) / kFixBlock;
+  const int64_t nblk = (t_end - t_begin + FS::BLOCK - 1) / FS::BLOCK;
   unsigned char* stage = fix_smem + warp * 2 * FS::BYTES;
   uint64_t* bar = fbar[warp];
-  const uint32_t tx = FS::C_BYTES + FS::ROW * (zrow ? 2 : 1) + kFixBlock * 4;
-  auto issue = [&](int64_t k) {  // lane 0: the TMA loads of block k into stage k & 1
+  int live = N;  // positions [0, live) may still carry weight
+  const uint32_t tx = FS::C_BYTES + FS::ROW * (zrow ? 2 : 1) + FS::BLOCK * 4;
+  // The TMA loads of block k into stage k & 1, after lane 0 has armed the
+  // barrier with their bytes: lanes 28..31 the [N][block] tile of C (N = 16),
+  // delta, z and y.  Called by the whole warp.
+  auto issue = [&](int64_t k) {
     unsigned char* st = stage + (k & 1) * FS::BYTES;
-    const int32_t t0 = (int32_t)(t_begin + k * kFixBlock);
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&bar[k & 1], tx);
-    if constexpr (FS::STAGE_C) tma_load_3d(st, &maps.C, &bar[k & 1], t0, 0, (int32_t)b);
-    tma_load_3d(st + FS::D_OFF, &maps.delta, &bar[k & 1], t0, (int32_t)d, (int32_t)b);
-    if (zrow) tma_load_3d(st + FS::Z_OFF, &maps.z, &bar[k & 1], t0, (int32_t)d, (int32_t)b);
-    tma_load_3d(st + FS::Y_OFF, &maps.y, &bar[k & 1], t0, (int32_t)d, (int32_t)b);
+    const int32_t t0 = (int32_t)(t_begin + k * FS::BLOCK);
+    if (lane == 0) mbar_arrive_expect_tx(&bar[k & 1], tx);
+    __syncwarp();
+    if (lane >= 28) {
+      fence_proxy_async_smem();
+      if (FS::STAGE_C && lane == 28) tma_load_3d(st, &maps.C, &bar[k & 1], t0, 0, (int32_t)b);
+      if (lane == 29) tma_load_3d(st + FS::D_OFF, &maps.delta, &bar[k & 1], t0, (int32_t)d, (int32_t)b);
+      if (lane == 30 && zrow) tma_load_3d(st + FS::Z_OFF, &maps.z, &bar[k & 1], t0, (int32_t)d, (int32_t)b);
+      if (lane == 31) tma_load_3d(st + FS::Y_OFF, &maps.y, &bar[k & 1], t0, (int32_t)d, (int32_t)b);
+    }
   };
-  if (tma && lane == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    fence_mbar_init();
+  if (tma) {
+    if (lane == 0) {
+      mbar_init(&bar[0], 1);
+      mbar_init(&bar[1], 1);
+      fence_mbar_init();
+    }
+    __syncwarp();
     issue(0);
     if (nblk > 1) issue(1);
   }
   __syncwarp();
 
-  int live = N;        // positions [0, live) may still carry weight
-  double carry = 0.0;  // sum of Delta over the blocks before this one
+  // sum of Delta over the blocks before this one: c_hi + c_lo
+  float c_hi = 0.f, c_lo = 0.f;
   int64_t k = 0;
   bool ok = true;  // false once a bounded wait has given up (error word set)
+  constexpr int SP = FS::SPL, SP2 = SP / 2, SP4 = SP / 4;
+  static_assert(SP % 4 == 0, "whole quads per lane");
   for (; k < nblk; ++k) {
-    const int64_t t = t_begin + k * kFixBlock + 4 * lane;
+    const int64_t t = t_begin + k * FS::BLOCK + SP * lane;
     const unsigned char* cur = stage + (k & 1) * FS::BYTES;
     if (tma) {
       ok = __all_sync(kFullMask, mbar_wait_bounded(&bar[k & 1], (uint32_t)((k >> 1) & 1),
                                                    kTmaSpinLimit));
       if (!ok) break;
     }
-    const float4 dl4 = tma ? fix_lds4<Tin>(cur + FS::D_OFF + 4 * lane * FS::ES)
-                           : fix_load4(drow, t, t_end, bd * L, n_act);
+    float dl[SP];
     const float2 b2 = make_float2(bias, bias);
-    float2 x01 = __fadd2_rn(make_float2(dl4.x, dl4.y), b2);
-    float2 x23 = __fadd2_rn(make_float2(dl4.z, dl4.w), b2);
-    if (a.softplus) {
-      x01 = softplus_fast2(x01);
-      x23 = softplus_fast2(x23);
-    }
-    float dl[4] = {x01.x, x01.y, x23.x, x23.y};
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
+    for (int q = 0; q < SP4; ++q) {
+      const float4 dl4 = tma ? fix_lds4<Tin>(cur + FS::D_OFF + (SP * lane + 4 * q) * FS::ES)
+                             : fix_load4(drow, t + 4 * q, t_end, bd * L, n_act);
+      float2 x01 = __fadd2_rn(make_float2(dl4.x, dl4.y), b2);
+      float2 x23 = __fadd2_rn(make_float2(dl4.z, dl4.w), b2);
+      if (a.softplus) {
+        x01 = softplus_fast2(x01);
+        x23 = softplus_fast2(x23);
+      }
+      dl[4 * q] = x01.x;
+      dl[4 * q + 1] = x01.y;
+      dl[4 * q + 2] = x23.x;
+      dl[4 * q + 3] = x23.y;
+    }
+#pragma unroll
+    for (int kk = 0; kk < SP; ++kk)
       if (t + kk >= t_end) dl[kk] = 0.f;
-    float p[4];
+    float p[SP];
     p[0] = dl[0];
-    p[1] = p[0] + dl[1];
-    p[2] = p[1] + dl[2];
-    p[3] = p[2] + dl[3];
-    float incl = p[3];  // inclusive scan of the lane totals
+#pragma unroll
+    for (int kk = 1; kk < SP; ++kk) p[kk] = p[kk - 1] + dl[kk];
+    float incl = p[SP - 1];  // inclusive scan of the lane totals
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float v = __shfl_up_sync(kFullMask, incl, o);
       if (lane >= o) incl += v;
     }
-    const float excl = incl - p[3];
-    float S[4];
+    const float excl = incl - p[SP - 1];
+    float2 S2[SP2];
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) S[kk] = (float)(carry + (double)(excl + p[kk]));
-    const float S_first = __shfl_sync(kFullMask, S[0], 0);
-    carry += (double)__shfl_sync(kFullMask, incl, 31);
+    for (int q = 0; q < SP2; ++q)
+      S2[q] = make_float2(c_hi + (c_lo + (excl + p[2 * q])), c_hi + (c_lo + (excl + p[2 * q + 1])));
+    const float S_first = __shfl_sync(kFullMask, S2[0].x, 0);
+    {  // two-sum: c_hi + tot = hi + err exactly
+      const float tot = __shfl_sync(kFullMask, incl, 31);
+      const float hi = c_hi + tot;
+      const float bt = hi - c_hi;
+      const float err = (c_hi - (hi - bt)) + (tot - bt);
+      c_hi = hi;
+      c_lo += err;
+    }
     // S_first is the block's smallest sum: a position dead now stays dead
     while (live > 0 && S_first > sh_sd[warp][live - 1]) --live;
     if (live == 0) break;
-    const float2 S01 = make_float2(S[0], S[1]), S23 = make_float2(S[2], S[3]);
-    float2 pos01 = make_float2(0.f, 0.f), pos23 = pos01, neg01 = pos01, neg23 = pos01;
+    float2 pos[SP2], neg[SP2];
+#pragma unroll
+    for (int q = 0; q < SP2; ++q) pos[q] = neg[q] = make_float2(0.f, 0.f);
+    // staged C: the sign of h_in is flipped into C's bits as it is loaded
+    constexpr bool XOR = tma && FS::STAGE_C;
 #pragma unroll 4
     for (int i = 0; i < live; ++i) {
       const float4 pr = sh_p[warp][i];
-      const float4 c4 = (tma && FS::STAGE_C)
-                            ? fix_lds4<Tin>(cur + sh_n[warp][i] * FS::ROW + 4 * lane * FS::ES)
-                            : fix_load4(Cb + (int64_t)sh_n[warp][i] * L, t, t_end,
-                                        (b * N + sh_n[warp][i]) * L, a.batch * N * L);
-      const float2 x01e = __ffma2_rn(S01, make_float2(pr.x, pr.y), make_float2(pr.z, pr.w));
-      const float2 x23e = __ffma2_rn(S23, make_float2(pr.x, pr.y), make_float2(pr.z, pr.w));
-      const float2 e01 = make_float2(ex2_approx(x01e.x), ex2_approx(x01e.y));
-      const float2 e23 = make_float2(ex2_approx(x23e.x), ex2_approx(x23e.y));
-      if (sh_neg[warp][i]) {  // warp-uniform
-        neg01 = __ffma2_rn(make_float2(c4.x, c4.y), e01, neg01);
-        neg23 = __ffma2_rn(make_float2(c4.z, c4.w), e23, neg23);
+      const int2 nq = sh_nq[warp][i];
+      float2 cv[SP2];
+#pragma unroll
+      for (int q = 0; q < SP4; ++q) {
+        float4 c4;
+        if constexpr (tma && FS::STAGE_C) {
+          c4 = fix_lds4x<Tin>(cur + nq.x * FS::ROW + (SP * lane + 4 * q) * FS::ES, (uint32_t)nq.y);
+        } else {
+          c4 = fix_load4(Cb + (int64_t)nq.x * L, t + 4 * q, t_end, (b * N + nq.x) * L, a.batch * N * L);
+        }
+        cv[2 * q] = make_float2(c4.x, c4.y);
+        cv[2 * q + 1] = make_float2(c4.z, c4.w);
+      }
+      float2 e[SP2];
+#pragma unroll
+      for (int q = 0; q < SP2; ++q) {
+        const float2 x = __ffma2_rn(S2[q], make_float2(pr.x, pr.y), make_float2(pr.z, pr.w));
+        e[q] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
+      if (XOR) {  // the sign is in cv
+#pragma unroll
+        for (int q = 0; q < SP2; ++q) pos[q] = __ffma2_rn(cv[q], e[q], pos[q]);
+      } else if (nq.y) {  // warp-uniform
+#pragma unroll
+        for (int q = 0; q < SP2; ++q) neg[q] = __ffma2_rn(cv[q], e[q], neg[q]);
       } else {
-        pos01 = __ffma2_rn(make_float2(c4.x, c4.y), e01, pos01);
-        pos23 = __ffma2_rn(make_float2(c4.z, c4.w), e23, pos23);
+#pragma unroll
+        for (int q = 0; q < SP2; ++q) pos[q] = __ffma2_rn(cv[q], e[q], pos[q]);
       }
     }
-    const float2 c01 = __fadd2_rn(pos01, make_float2(-neg01.x, -neg01.y));
-    const float2 c23 = __fadd2_rn(pos23, make_float2(-neg23.x, -neg23.y));
-    const float4 y4 = tma ? fix_lds4<float>(cur + FS::Y_OFF + 16 * lane)
-                          : fix_load4(yrow, t, t_end, bd * L, n_act);
-    float2 g01 = make_float2(1.f, 1.f), g23 = g01;
-    if (zrow) {
-      const float4 z4 = tma ? fix_lds4<Tin>(cur + FS::Z_OFF + 4 * lane * FS::ES)
-                            : fix_load4(zrow, t, t_end, bd * L, n_act);
-      g01 = silu_fast2(make_float2(z4.x, z4.y));
-      g23 = silu_fast2(make_float2(z4.z, z4.w));
-    }
-    const float2 o01 = __ffma2_rn(c01, g01, make_float2(y4.x, y4.y));
-    const float2 o23 = __ffma2_rn(c23, g23, make_float2(y4.z, y4.w));
-    if (tma && t + 3 < t_end) {
-      if (in_range(bd * L + t, 4, n_act))
-        *reinterpret_cast<float4*>(yrow + t) = make_float4(o01.x, o01.y, o23.x, o23.y);
-    } else {
-      const float out[4] = {o01.x, o01.y, o23.x, o23.y};
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        if (t + kk < t_end && in_range(bd * L + t + kk, n_act)) yrow[t + kk] = out[kk];
+    for (int q = 0; q < SP4; ++q) {
+      const int64_t tq = t + 4 * q;
+      const float2 c01 = __fadd2_rn(pos[2 * q], make_float2(-neg[2 * q].x, -neg[2 * q].y));
+      const float2 c23 = __fadd2_rn(pos[2 * q + 1], make_float2(-neg[2 * q + 1].x, -neg[2 * q + 1].y));
+      const float4 y4 = tma ? fix_lds4<float>(cur + FS::Y_OFF + 4 * (SP * lane + 4 * q))
+                            : fix_load4(yrow, tq, t_end, bd * L, n_act);
+      float2 g01 = make_float2(1.f, 1.f), g23 = g01;
+      if (zrow) {
+        const float4 z4 = tma ? fix_lds4<Tin>(cur + FS::Z_OFF + (SP * lane + 4 * q) * FS::ES)
+                              : fix_load4(zrow, tq, t_end, bd * L, n_act);
+        g01 = silu_fast2(make_float2(z4.x, z4.y));
+        g23 = silu_fast2(make_float2(z4.z, z4.w));
+      }
+      const float2 o01 = __ffma2_rn(c01, g01, make_float2(y4.x, y4.y));
+      const float2 o23 = __ffma2_rn(c23, g23, make_float2(y4.z, y4.w));
+      if (tma && tq + 3 < t_end) {
+        if (in_range(bd * L + tq, 4, n_act))
+          *reinterpret_cast<float4*>(yrow + tq) = make_float4(o01.x, o01.y, o23.x, o23.y);
+      } else {
+        const float out[4] = {o01.x, o01.y, o23.x, o23.y};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          if (tq + kk < t_end && in_range(bd * L + tq + kk, n_act)) yrow[tq + kk] = out[kk];
+      }
     }
     __syncwarp();  // every lane is done with this stage before TMA refills it
-    if (tma && lane == 0 && k + 2 < nblk) issue(k + 2);
+    if (tma && k + 2 < nblk) issue(k + 2);
   }
   // No copy may land after the warp has left.  Issued: blocks up to k + 1
   // (the loop issues k + 2 only at the end of iteration k).  Waited: up to

@@ -816,6 +816,7 @@ struct Sched {
   float* carries;       // [workers][CH * N] published prefix states (nullable)
   unsigned long long* flags;  // [workers] epoch of the published carry
   unsigned long long epoch;   // unique per launch, so stale flags never match
+  unsigned int* ticket;       // balanced schedule: worker-id counter, 0 at launch
   uint32_t spin_limit;        // polls before a carry wait gives up
   int skip_publish;           // test hook: this worker never publishes (-1: none)
   // plain schedule only: each channel group's chunks are cut into nseg
@@ -1041,7 +1042,17 @@ __global__ void __launch_bounds__(CF::NT, CF::MIN_CTAS)
   float* aggH = aggP + CF::AGG_FLOATS;
   __shared__ __align__(8) uint64_t bars[2];
 
-  const int w = blockIdx.x;
+  // kMulti: the worker id is the CTA's place in the order in which CTAs
+  // started (an atomic ticket), not blockIdx.x: worker w - 1, whose carry
+  // worker w waits for, then always runs already, whatever else holds SM slots.
+  int w = blockIdx.x;
+  if constexpr (kMulti) {
+    __shared__ int sh_ticket;
+    if (threadIdx.x == 0) sh_ticket = (int)atomicAdd(sched.ticket, 1u);
+    __syncthreads();
+    w = sh_ticket;
+    if (!in_range(w, gridDim.x)) return;
+  }
   // kMulti: worker w's range of (group, chunk) units; plain: CTA w runs
   // segment `seg` (chunks c_begin .. c_begin + nseq - 1) of channel group `grp`
   int64_t u0 = 0, u1 = 0, nseq = 0, c_begin = 0, grp = w;

@@ -17,14 +17,15 @@
 // shuffles inside the warp):
 //
 //  scan_step_pipe_kernel (16-byte aligned rows, the normal case): persistent
-//    CTAs walk tiles of (batch row b, TILE_CH consecutive channels); one thread
-//    streams each tile's 16 KB of state, its u/delta/z runs and the row's B, C
-//    into a ring of shared-memory stages with bulk asynchronous copies
-//    completing on mbarriers, several tiles ahead, so the bytes in flight do
-//    not cost registers.  The other threads compute from shared memory and
-//    store the new state and y straight to HBM.  Tiles are ordered
-//    channel-tile-major, so a CTA's consecutive tiles share A, D and the bias,
-//    which stay in registers.
+//    CTAs walk tiles of (batch row b, TILE_CH consecutive channels); a
+//    producer warp streams each tile's 16 KB of state, its u/delta/z runs and
+//    the row's B, C into a ring of shared-memory stages with bulk asynchronous
+//    copies completing on "full" mbarriers, several tiles ahead, so the bytes
+//    in flight do not cost registers.  The eight compute warps read a stage,
+//    store the new state and y straight to HBM and release the stage on its
+//    "empty" mbarrier, each warp on its own, so that no CTA-wide barrier holds
+//    the fast warps back.  Tiles are ordered channel-tile-major, so a CTA's
+//    consecutive tiles share A, D and the bias, which stay in registers.
 //  scan_step_kernel (any alignment): one batch row per grid row, plain loads.
 #pragma once
 
@@ -173,7 +174,9 @@ struct StepPipeSched {
 
 template <typename E, int N>
 struct StepPipeCfg {
-  static constexpr int NT = 256;                  // threads per CTA
+  static constexpr int NT = 256;                  // compute threads per CTA
+  static constexpr int CWARPS = NT / 32;          // compute warps (arrivals on an empty barrier)
+  static constexpr int THREADS = NT + 32;         // + the producer warp
   static constexpr int UPT = SS_STEP_PIPE_UPT;    // 4-state vectors per thread per tile
   static constexpr int LPC = N / 4;               // lanes per channel
   static constexpr int UNITS = NT * UPT;          // 4-state vectors per tile
@@ -195,13 +198,14 @@ struct StepPipeCfg {
 };
 
 template <typename E, int N>
-__global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
+__global__ void __launch_bounds__(StepPipeCfg<E, N>::THREADS, SS_STEP_PIPE_CTAS)
     scan_step_pipe_kernel(const StepArgs a, const StepPipeSched sc) {
   using CF = StepPipeCfg<E, N>;
   constexpr int LPC = CF::LPC, UPT = CF::UPT, S = CF::STAGES;
   extern __shared__ __align__(128) unsigned char smem_dyn[];
   unsigned char* smem = smem_dyn + ((128u - (smem_u32(smem_dyn) & 127u)) & 127u);
-  __shared__ __align__(8) uint64_t full[S];
+  __shared__ __align__(8) uint64_t full[S];   // stage holds its tile (1 arrival + bytes)
+  __shared__ __align__(8) uint64_t empty[S];  // every compute warp is done with the stage
 
   const int w = blockIdx.x;
   const int64_t i0 = sc.items * w / gridDim.x, i1 = sc.items * (w + 1) / gridDim.x;
@@ -216,14 +220,17 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
   const E* Cp = static_cast<const E*>(a.C);
 
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], CF::CWARPS);
+    }
     fence_mbar_init();
   }
   __syncthreads();
   if (n <= 0) return;
 
-  // item i -> (channel tile c, batch row b), c-major; the issuing thread walks
-  // its own copy of the cursor S items ahead of the consumers
+  // item i -> (channel tile c, batch row b), c-major; the producer walks its
+  // own copy of the cursor up to S items ahead of the compute warps
   auto seat = [&](int64_t i, int64_t& c, int64_t& b) {
     c = i / a.batch;
     b = i - c * a.batch;
@@ -249,13 +256,25 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
     bulk_load(st + CF::OFF_C, Cp + b * N, N * CF::ES, &full[k % S]);
   };
 
-  int64_t pc = 0, pb = 0;  // issuing cursor (thread 0 only)
-  if (tid == 0) {
-    seat(i0, pc, pb);
-    for (int64_t k = 0; k < S && k < n; ++k) {
-      issue(k, pc, pb);
-      if (++pb == a.batch) { pb = 0; ++pc; }
+  if (tid >= CF::NT) {  // the producer warp: one lane issues, the rest leave
+    if (tid == CF::NT) {
+      int64_t pc, pb;
+      seat(i0, pc, pb);
+      int64_t k = 0;
+      for (; k < n; ++k) {
+        // stage k % S is free once every compute warp has released item k - S
+        if (k >= S &&
+            !mbar_wait_bounded(&empty[k % S], (uint32_t)((k / S - 1) & 1), kTmaSpinLimit))
+          break;
+        issue(k, pc, pb);
+        if (++pb == a.batch) { pb = 0; ++pc; }
+      }
+      // no copy may land after the CTA has left: wait (bounded) for the last
+      // S items issued (the earlier ones were released, so they have landed)
+      for (int64_t kk = k > S ? k - S : 0; kk < k; ++kk)
+        mbar_wait_bounded(&full[kk % S], (uint32_t)((kk / S) & 1), kTmaSpinLimit);
     }
+    return;
   }
 
   int64_t c, b;
@@ -263,7 +282,6 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
   int64_t c_regs = -1;  // channel tile whose A, D, bias sit in registers
   float4 av[UPT];
   float Dd[UPT], bias[UPT];
-  bool ok = true;
   for (int64_t k = 0; k < n; ++k) {
     if (c != c_regs) {
 #pragma unroll
@@ -280,14 +298,11 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
       }
       c_regs = c;
     }
-    ok = ok && mbar_wait_bounded(&full[k % S], (uint32_t)((k / S) & 1), kTmaSpinLimit);
-    if (!__syncthreads_and(ok)) {
-      // a copy never completed: wait (bounded) for the others in flight, then leave
-      if (tid == 0)
-        for (int64_t kk = k + 1; kk < n && kk < k + S; ++kk)
-          mbar_wait_bounded(&full[kk % S], (uint32_t)((kk / S) & 1), kTmaSpinLimit);
+    // a copy that never completes ends this warp; the producer then stops at
+    // its next bounded wait for this warp's release and drains its copies
+    if (!__all_sync(kFullMask, mbar_wait_bounded(&full[k % S], (uint32_t)((k / S) & 1),
+                                                 kTmaSpinLimit)))
       return;
-    }
     const unsigned char* st = smem + (k % S) * CF::STAGE;
     const E* su = reinterpret_cast<const E*>(st + CF::OFF_U);
     const E* sd = reinterpret_cast<const E*>(st + CF::OFF_DELTA);
@@ -323,11 +338,8 @@ __global__ void __launch_bounds__(256, SS_STEP_PIPE_CTAS)
         }
       }
     }
-    __syncthreads();  // stage k % S is free again
-    if (tid == 0 && k + S < n) {
-      issue(k + S, pc, pb);
-      if (++pb == a.batch) { pb = 0; ++pc; }
-    }
+    __syncwarp();  // the warp's lanes are done with stage k % S
+    if ((tid & 31) == 0) mbar_arrive(&empty[k % S]);
     if (++b == a.batch) { b = 0; ++c; }
   }
 }

@@ -42,8 +42,9 @@ ss_status launch_step_pipe(const StepArgs& a, cudaStream_t stream) {
   if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
   if (dev >= 0 && dev < kDevCache) occ = occ_cache[dev].load();
   if (occ < 1) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_step_pipe_kernel<E, N>, CF::NT,
-                                                      CF::SMEM_BYTES) != cudaSuccess || occ < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, scan_step_pipe_kernel<E, N>,
+                                                      CF::THREADS, CF::SMEM_BYTES) != cudaSuccess ||
+        occ < 1)
       return SS_ERR_CUDA;
     if (dev >= 0 && dev < kDevCache) occ_cache[dev].store(occ);
   }
@@ -53,7 +54,7 @@ ss_status launch_step_pipe(const StepArgs& a, cudaStream_t stream) {
   const int64_t slots = (int64_t)device_sms() * occ;
   if (slots < 1) return SS_ERR_CUDA;
   const int64_t grid = sc.items < slots ? sc.items : slots;
-  scan_step_pipe_kernel<E, N><<<(unsigned)grid, CF::NT, CF::SMEM_BYTES, stream>>>(a, sc);
+  scan_step_pipe_kernel<E, N><<<(unsigned)grid, CF::THREADS, CF::SMEM_BYTES, stream>>>(a, sc);
   return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
