@@ -72,10 +72,10 @@ struct BwdCfg {
   static constexpr int ITEMS = CH * T;    // (step, channel) items per chunk
   static constexpr int IPT = (ITEMS + NT - 1) / NT;
   static constexpr int STEP_FLOATS = CH * N;  // one step's states of the CTA
-  // row pitch of the per-step states: 64 bytes of padding, so that the
-  // 16-byte reads of two consecutive steps by a quarter-warp in the channel
-  // reductions fall on opposite halves of the banks
-  static constexpr int HB_STRIDE = STEP_FLOATS + 16;
+  // row pitch of the per-step states: 16 bytes of padding, so that the
+  // 16-byte reads of eight consecutive steps by a quarter-warp in the channel
+  // reductions fall on distinct banks
+  static constexpr int HB_STRIDE = STEP_FLOATS + 4;
   // staged inputs per thread (register prefetch of the next chunk)
   static constexpr int ACT_PT = (CH * T + NT - 1) / NT;
   static constexpr int SEL_PT = (N * T + NT - 1) / NT;
@@ -122,8 +122,9 @@ struct BwdStage {
 
 // A thread's fixed element slots: staging slot r is activation element
 // (c, t) = (i / T, i % T) and B/C element (n, t) of every chunk, i = tid + r NT;
-// item slot it is (t, c) = (i / CH, i % CH).  Their row offsets, validity and
-// per-channel constants are computed once, so a chunk only adds t0.
+// item slot it is (c, t) = (i / T, i % T), steps fastest, so that a warp's
+// stores of du, ddelta and dz are runs along t.  Their row offsets, validity
+// and per-channel constants are computed once, so a chunk only adds t0.
 template <class CF>
 struct BwdSlots {
   // staging slot r covers element (c, t) = (c0 + r NT/T, t_s) and B/C element
@@ -155,7 +156,7 @@ __device__ __forceinline__ void bwd_slots(const BwdArgs& a, int64_t b, int64_t d
 #pragma unroll
   for (int it = 0; it < CF::IPT; ++it) {
     const int i = threadIdx.x + it * CF::NT;
-    const int tt = i / CF::CH, c = i - tt * CF::CH;
+    const int c = i / CF::T, tt = i - c * CF::T;
     const int64_t d = d0 + c;
     const bool ok = (!CF::ITEM_GUARD || i < CF::ITEMS) && d < a.dim;
     sl.item[it] = ok ? (b * a.dim + d) * L + tt : -1;
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(CF::NT)
     for (int it = 0; it < CF::IPT; ++it) {
       const int i = tid + it * CF::NT;
       if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
-      const int tt = i / CF::CH, ci = i - tt * CF::CH;
+      const int ci = i / CF::T, tt = i - ci * CF::T;
       const int o = tt * CHP + ci;
       const bool in = sl.item[it] >= 0 && t0 + tt < L;
       const float uu = sm[CF::OFF_U + o];
@@ -386,9 +387,10 @@ __global__ void __launch_bounds__(CF::NT)
       if (in) dD_acc[it] = fmaf(dq, uu, dD_acc[it]);
     }
     __syncthreads();
-    // dC[b, n, t] += sum_c dq[t, c] h_t[c, n], four consecutive states per item
+    // dC[b, n, t] += sum_c dq[t, c] h_t[c, n], four consecutive states per
+    // item, steps fastest (a warp's atomics are runs along t)
     for (int i = tid; i < (N / 4) * T; i += CF::NT) {
-      const int tt = i / (N / 4), n = 4 * (i - tt * (N / 4));
+      const int n = 4 * (i / T), tt = i - (n / 4) * T;
       if (t0 + tt >= L) continue;
       float2 s01 = make_float2(0.f, 0.f), s23 = s01;
       const float* hr = hb + tt * CF::HB_STRIDE + n;
@@ -448,9 +450,9 @@ __global__ void __launch_bounds__(CF::NT)
       }
     }
     __syncthreads();
-    // dB[b, n, t] += sum_c g Delta u, four consecutive states per item
+    // dB[b, n, t] += sum_c g Delta u, four consecutive states per item, steps fastest
     for (int i = tid; i < (N / 4) * T; i += CF::NT) {
-      const int tt = i / (N / 4), n = 4 * (i - tt * (N / 4));
+      const int n = 4 * (i / T), tt = i - (n / 4) * T;
       if (t0 + tt >= L) continue;
       float2 s01 = make_float2(0.f, 0.f), s23 = s01;
       const float* hr = hb + tt * CF::HB_STRIDE + n;
@@ -471,7 +473,7 @@ __global__ void __launch_bounds__(CF::NT)
     for (int it = 0; it < CF::IPT; ++it) {
       const int i = tid + it * CF::NT;
       if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
-      const int tt = i / CF::CH, ci = i - tt * CF::CH;
+      const int ci = i / CF::T, tt = i - ci * CF::T;
       const int o = tt * CHP + ci;
       if (sl.item[it] < 0 || t0 + tt >= L) continue;
       const float dx = sm[CF::OFF_P1 + o] * sm[CF::OFF_SG + o];
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(CF::NT)
   for (int it = 0; it < CF::IPT; ++it) {
     const int i = tid + it * CF::NT;
     if (CF::ITEM_GUARD && i >= CF::ITEMS) break;
-    const int64_t di = d0 + (i - (i / CF::CH) * CF::CH);
+    const int64_t di = d0 + i / CF::T;
     if (di >= a.dim) continue;
     if (a.dD) atomicAdd(a.dD + di, dD_acc[it]);
     if (a.dbias) atomicAdd(a.dbias + di, db_acc[it]);
