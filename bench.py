@@ -631,7 +631,10 @@ def run_reference_arm(args, w: I.Workload):
         import torch.distributed as dist
 
         dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
-        print(f"reference arm: rank {rank} of {world} joined", file=sys.stderr, flush=True)
+        # one write per message (text and newline together), so that the
+        # ranks' lines do not interleave on the shared stream
+        sys.stderr.write(f"reference arm: rank {rank} of {world} joined\n")
+        sys.stderr.flush()
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:

@@ -4,6 +4,7 @@ on rank 0 only.  No GPU and no data-path collective (the scan shards with no
 exchange)."""
 import json
 import os
+import re
 import subprocess
 import sys
 
@@ -30,7 +31,7 @@ def _worker(rank, world, port, out):
 
 
 def test_max_over_ranks_gloo():
-    port = 29500 + os.getpid() % 1000
+    port = bench._free_port()
     with mp.Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
@@ -57,7 +58,7 @@ def test_gpus_two_launches_two_ranks():
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
-    joined = sorted(ln for ln in r.stderr.splitlines() if "joined" in ln)
+    joined = sorted(re.findall(r"reference arm: rank \d of \d joined", r.stderr))
     assert joined == ["reference arm: rank 0 of 2 joined", "reference arm: rank 1 of 2 joined"]
 
 
