@@ -26,6 +26,12 @@
 //    "empty" mbarrier, each warp on its own, so that no CTA-wide barrier holds
 //    the fast warps back.  Tiles are ordered channel-tile-major, so a CTA's
 //    consecutive tiles share A, D and the bias, which stay in registers.
+//    The kernel is launched as a programmatic dependent of the previous
+//    kernel in the stream: its CTAs may start and set up their barriers while
+//    that kernel drains; every thread then waits for the previous grid to
+//    complete (griddepcontrol.wait, which also makes its writes visible)
+//    before it reads anything from global memory.  Each CTA in turn lets the
+//    next step's grid launch as soon as it starts.
 //  scan_step_kernel (any alignment): one batch row per grid row, plain loads.
 #pragma once
 
@@ -225,6 +231,9 @@ __global__ void __launch_bounds__(StepPipeCfg<E, N>::THREADS, SS_STEP_PIPE_CTAS)
       mbar_init(&empty[s], CF::CWARPS);
     }
     fence_mbar_init();
+    // the next kernel in the stream may be scheduled once every CTA of this
+    // grid has started (it waits for this grid's completion before its reads)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
   __syncthreads();
   if (n <= 0) return;
@@ -258,6 +267,8 @@ __global__ void __launch_bounds__(StepPipeCfg<E, N>::THREADS, SS_STEP_PIPE_CTAS)
 
   if (tid >= CF::NT) {  // the producer warp: one lane issues, the rest leave
     if (tid == CF::NT) {
+      // every read below may see writes of the previous kernel in the stream
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       int64_t pc, pb;
       seat(i0, pc, pb);
       int64_t k = 0;
@@ -277,6 +288,7 @@ __global__ void __launch_bounds__(StepPipeCfg<E, N>::THREADS, SS_STEP_PIPE_CTAS)
     return;
   }
 
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // as the producer's
   int64_t c, b;
   seat(i0, c, b);
   int64_t c_regs = -1;  // channel tile whose A, D, bias sit in registers

@@ -54,7 +54,19 @@ ss_status launch_step_pipe(const StepArgs& a, cudaStream_t stream) {
   const int64_t slots = (int64_t)device_sms() * occ;
   if (slots < 1) return SS_ERR_CUDA;
   const int64_t grid = sc.items < slots ? sc.items : slots;
-  scan_step_pipe_kernel<E, N><<<(unsigned)grid, CF::THREADS, CF::SMEM_BYTES, stream>>>(a, sc);
+  // a programmatic dependent launch: the grid may start while the previous
+  // kernel in the stream drains; the kernel waits for it before any read
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(CF::THREADS);
+  cfg.dynamicSmemBytes = CF::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, scan_step_pipe_kernel<E, N>, a, sc) != cudaSuccess) return SS_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
