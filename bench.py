@@ -321,8 +321,14 @@ def run_gpu_arm(args, w: I.Workload):
 
     if world > 1:
         dist.destroy_process_group()
+    from selective_state_space_ss_b200 import SS_BF16, SS_F32, ss_debug_fwd_kernels
+
+    # kernels one forward call launches for this shape: the scan, and the
+    # carry-in correction when the sequence is cut into segments
+    kernels = ss_debug_fwd_kernels(w.batch, w.dim, w.seqlen, w.dstate,
+                                   SS_BF16 if w.dtype == "bf16" else SS_F32)
     return dict(ms_per_step=ms_per_step, value=value, world=world, rank=rank,
-                clocks=clk.summary(), e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=h2d,
+                kernels_per_step=kernels, clocks=clk.summary(), e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=h2d,
                                                 d2h_bytes_per_step=d2h, steps=e2e_steps),
                 nsets=nsets, host=host[0])
 
@@ -777,7 +783,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": config_of(w, r["world"], args.conv, args.zoh),
             "roofline": roof,
-            "e2e": r["e2e"], "gpu_launches": args.steps, "clocks": r["clocks"]}
+            "e2e": r["e2e"], "gpu_launches": args.steps * r["kernels_per_step"],
+            "clocks": r["clocks"]}
     if r["world"] == 1 and not args.no_cpu_baseline:
         take, dt, cores = oracle_sample(w, r["host"], target_s=10.0)
         line["cpu_baseline"] = {"value": take * w.seqlen / dt, "unit": UNIT, "cores": cores,

@@ -51,6 +51,16 @@ enum {
 ss_status ss_debug_inject(int what, long long value);
 
 /*
+ * ss_debug_fwd_kernels -- how many kernels one ss_scan_fwd call launches for
+ * this shape and input dtype on the current device: 1, or 2 when the
+ * sequence is cut into segments scanned at once (the scan, then the carry-in
+ * correction).  Pending debug settings are honoured, not cleared.  -1 for
+ * unsupported arguments or when the device cannot be queried.  Host-only,
+ * launches nothing.  (For benchmarks that count their launches.)
+ */
+int ss_debug_fwd_kernels(int64_t batch, int64_t dim, int64_t seqlen, int dstate, ss_dtype in_dtype);
+
+/*
  * ss_debug_pointwise -- evaluate one of the scan kernels' pointwise functions
  * element by element on the device, so that a test can compare it with
  * float64 over its input range: y[i] = f(x[i]) for i < n.

@@ -25,6 +25,7 @@ from ._native import (  # noqa: F401
     SSError,
     library_path,
     load_library,
+    ss_debug_fwd_kernels,
     ss_debug_inject,
     ss_last_device_error,
     ss_scan_bwd,

@@ -25,7 +25,7 @@ EXPORTED = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_status_string",
             "ss_last_device_error", "ss_debug_inject", "ss_scan_fwd_noalloc",
             "ss_scan_fwd_from_state", "ss_scan_step", "ss_scan_fwd_conv", "ss_scan_fwd_zoh",
             "ss_scan_bwd", "ss_scan_bwd_workspace_bytes", "ss_scan_fwd_train",
-            "ss_debug_pointwise")
+            "ss_debug_pointwise", "ss_debug_fwd_kernels")
 
 # bytes of the library's static scratch array (SS_NOALLOC_SCRATCH_BYTES)
 SS_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -94,6 +94,8 @@ def load_library():
         lib.ss_scan_step.restype = ci
         lib.ss_debug_pointwise.argtypes = [ci, vp, vp, i64, vp]
         lib.ss_debug_pointwise.restype = ci
+        lib.ss_debug_fwd_kernels.argtypes = [i64, i64, i64, ci, ci]
+        lib.ss_debug_fwd_kernels.restype = ci
         _lib = lib
         return lib
 
@@ -125,6 +127,14 @@ def ss_debug_inject(what: int, value: int = 0) -> None:
     st = load_library().ss_debug_inject(int(what), int(value))
     if st != SS_OK:
         raise SSError(st, "ss_debug_inject")
+
+
+def ss_debug_fwd_kernels(batch: int, dim: int, seqlen: int, dstate: int, in_dtype: int) -> int:
+    """Kernels one ss_scan_fwd call launches for this shape (include/ss_scan_debug.h)."""
+    n = load_library().ss_debug_fwd_kernels(batch, dim, seqlen, dstate, int(in_dtype))
+    if n < 1:
+        raise SSError(SS_ERR_INVALID_ARG, "ss_debug_fwd_kernels")
+    return n
 
 
 def ss_debug_pointwise(fn: int, x, stream=None):

@@ -217,6 +217,36 @@ size_t ss_scan_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int d
   return m;
 }
 
+extern "C++" {
+namespace {
+// The plain forward's plan for this shape (the kernel choice of dispatch_dtype).
+template <typename E>
+bool fwd_plan(int64_t batch, int64_t dim, int64_t seqlen, int N, ssscan::Plan* p) {
+  using namespace ssscan;
+  switch (N) {
+    case 16:
+      return use_time_split<Cfg16<E>>(batch, dim, seqlen) ? make_plan<Split16<E>>(batch, dim, seqlen, p)
+                                                          : make_plan<Cfg16<E>>(batch, dim, seqlen, p);
+    case 32:
+      return use_time_split<Cfg32<E>>(batch, dim, seqlen) ? make_plan<Split32<E>>(batch, dim, seqlen, p)
+                                                          : make_plan<Cfg32<E>>(batch, dim, seqlen, p);
+    case 64: return make_plan<Cfg64<E>>(batch, dim, seqlen, p);
+    case 128: return make_plan<Cfg128<E>>(batch, dim, seqlen, p);
+  }
+  return false;
+}
+}  // namespace
+}  // extern "C++"
+
+int ss_debug_fwd_kernels(int64_t batch, int64_t dim, int64_t seqlen, int dstate, ss_dtype in_dtype) {
+  if (batch < 1 || dim < 1 || seqlen < 1 || !supported_dstate(dstate)) return -1;
+  ssscan::Plan p;
+  const bool ok = in_dtype == SS_BF16 ? fwd_plan<__nv_bfloat16>(batch, dim, seqlen, dstate, &p)
+                                      : fwd_plan<float>(batch, dim, seqlen, dstate, &p);
+  if (!ok) return -1;
+  return p.nseg > 1 ? 2 : 1;
+}
+
 ss_status ss_debug_inject(int what, long long value) {
   switch (what) {
     case SS_DEBUG_FORCE_WORKERS: g_dbg_workers.store(value); return SS_OK;

@@ -173,3 +173,15 @@ def test_auto_segments_on_few_channels():
     x = I.make_inputs(w, seed=17)
     y, h = _fwd(to_device(x), 0)
     _check(w, y, h, *_ref(x))
+
+
+def test_kernels_per_call():
+    # the million-token shape is cut into segments (scan + correction); the
+    # B8 L2048 D1536 shape fills the GPU with channel groups (one kernel)
+    assert ss.ss_debug_fwd_kernels(1, 1536, 1 << 20, 16, ss.SS_BF16) == 2
+    assert ss.ss_debug_fwd_kernels(8, 1536, 2048, 16, ss.SS_BF16) == 1
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_SEGMENTS, 4)
+    assert ss.ss_debug_fwd_kernels(1, 64, 4096, 16, ss.SS_F32) == 2
+    ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
+    with pytest.raises(ss.SSError):
+        ss.ss_debug_fwd_kernels(1, 64, 4096, 24, ss.SS_F32)
