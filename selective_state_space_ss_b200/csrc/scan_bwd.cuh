@@ -90,9 +90,13 @@ struct BwdCfg {
   static constexpr int OFF_P1 = OFF_SG + T * CHP;       // per-channel sums (readout, dDelta)
   static constexpr int OFF_P2 = OFF_P1 + T * CHP;       // per-channel sums (du)
   static constexpr int NP = N + 4;                      // B, C row pitch (16-byte aligned)
-  static constexpr int OFF_B = (OFF_P2 + T * CHP + 3) / 4 * 4;  // [T][NP]
-  static constexpr int OFF_C = OFF_B + T * NP;
-  static constexpr int OFF_H = OFF_C + T * NP;          // [T][CH*N] states, then g Delta u
+  // bf16 inputs with four states per lane: B and C stay bf16, a step's row
+  // holding 16-byte units [B_4j, B_4j+1, C_4j, C_4j+1, B_4j+2, B_4j+3, C_4j+2,
+  // C_4j+3], so that a lane reads its states' B and C in one 16-byte load
+  static constexpr bool BC16 = sizeof(Tin) == 2 && G == 4;
+  static constexpr int OFF_B = (OFF_P2 + T * CHP + 3) / 4 * 4;  // [T][NP] (BC16: the units)
+  static constexpr int OFF_C = OFF_B + T * NP;                  // [T][NP] (not with BC16)
+  static constexpr int OFF_H = OFF_C + (BC16 ? 0 : T * NP);     // [T][CH*N] states, then g Delta u
   static constexpr int SMEM_FLOATS = OFF_H + T * HB_STRIDE;
   static constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
   static_assert(N % G == 0 && 32 % K == 0 && (G == 2 || G == 4), "lane split");
@@ -222,8 +226,15 @@ __device__ __forceinline__ void bwd_store(const BwdArgs& a, const BwdStage<CF>& 
     const int i = threadIdx.x + r * CF::NT;
     if (i >= CF::N * CF::T) break;
     const int n = i / CF::T, tt = i - n * CF::T;
-    sm[CF::OFF_B + tt * CF::NP + n] = st.b[r];
-    if (with_grad) sm[CF::OFF_C + tt * CF::NP + n] = st.c[r];
+    if constexpr (CF::BC16) {  // the values are bf16, so their fp32 high halves are exact
+      uint16_t* row = reinterpret_cast<uint16_t*>(sm + CF::OFF_B + tt * CF::NP);
+      const int e = 8 * (n >> 2) + 4 * ((n >> 1) & 1) + (n & 1);  // B's place in its unit
+      row[e] = (uint16_t)(__float_as_uint(st.b[r]) >> 16);
+      if (with_grad) row[e + 2] = (uint16_t)(__float_as_uint(st.c[r]) >> 16);
+    } else {
+      sm[CF::OFF_B + tt * CF::NP + n] = st.b[r];
+      if (with_grad) sm[CF::OFF_C + tt * CF::NP + n] = st.c[r];
+    }
   }
 }
 
@@ -284,6 +295,29 @@ __global__ void __launch_bounds__(CF::NT)
     else
       *reinterpret_cast<float2*>(p) = v[0];
   };
+  // B (and C) of this lane's states at step t of the staged chunk
+  auto ld_bc = [&](int t, float2 (&bb)[HP], float2 (&cc)[HP]) {
+    if constexpr (CF::BC16) {
+      const uint4 v = *reinterpret_cast<const uint4*>(sm + CF::OFF_B + t * CF::NP + j * G);
+      auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
+      auto hi = [](uint32_t x) { return __uint_as_float(x & 0xffff0000u); };
+      bb[0] = make_float2(lo(v.x), hi(v.x));
+      cc[0] = make_float2(lo(v.y), hi(v.y));
+      bb[HP - 1] = make_float2(lo(v.z), hi(v.z));
+      cc[HP - 1] = make_float2(lo(v.w), hi(v.w));
+    } else {
+      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
+      ld_pairs(sm + CF::OFF_C + t * CF::NP + j * G, cc);
+    }
+  };
+  auto ld_b = [&](int t, float2 (&bb)[HP]) {
+    if constexpr (CF::BC16) {
+      float2 cc[HP];
+      ld_bc(t, bb, cc);
+    } else {
+      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
+    }
+  };
   auto zero_pairs = [](float2 (&v)[HP]) {
 #pragma unroll
     for (int p = 0; p < HP; ++p) v[p] = make_float2(0.f, 0.f);
@@ -305,7 +339,7 @@ __global__ void __launch_bounds__(CF::NT)
       const float dl = sm[CF::OFF_DL + t * CHP + c], w = sm[CF::OFF_W + t * CHP + c];
       const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w);
       float2 bb[HP];
-      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
+      ld_b(t, bb);
 #pragma unroll
       for (int p = 0; p < HP; ++p)
         h[p] = __ffma2_rn(ex2_pair(__fmul2_rn(dl2, A2[p])), h[p], __fmul2_rn(w2, bb[p]));
@@ -352,8 +386,7 @@ __global__ void __launch_bounds__(CF::NT)
       const float dl = sm[CF::OFF_DL + t * CHP + c], w = sm[CF::OFF_W + t * CHP + c];
       const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w);
       float2 bb[HP], cc[HP];
-      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
-      ld_pairs(sm + CF::OFF_C + t * CF::NP + j * G, cc);
+      ld_bc(t, bb, cc);
       float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
       for (int p = 0; p < HP; ++p) {
@@ -417,8 +450,7 @@ __global__ void __launch_bounds__(CF::NT)
       const float w = sm[CF::OFF_W + t * CHP + c];
       const float2 dl2 = make_float2(dl, dl), w2 = make_float2(w, w), dq2 = make_float2(dq, dq);
       float2 bb[HP], cc[HP], prev[HP];
-      ld_pairs(sm + CF::OFF_B + t * CF::NP + j * G, bb);
-      ld_pairs(sm + CF::OFF_C + t * CF::NP + j * G, cc);
+      ld_bc(t, bb, cc);
       if (t > 0) {
         ld_pairs(hb_lane + (t - 1) * CF::HB_STRIDE, prev);
       } else {

@@ -251,3 +251,42 @@ def test_step_full_workloads(name):
     y = _step_gpu(xd, xd["state"])
     yr, hr = _step_oracle(x)
     _check(w, y, xd["state"], yr, hr)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_chain_in_a_cuda_graph(dtype):
+    # eight consecutive decode steps captured in one CUDA graph: each step is a
+    # programmatic dependent of the one before (it may start while that one
+    # drains and waits for it before reading the state it wrote)
+    S = 8
+    w = I.Workload(f"stepgraph_{dtype}", 3, 1000, S, 16, dtype)
+    x = I.make_inputs(w, seed=71)
+    h0 = I.make_state(w.batch, w.dim, w.dstate, seed=72)
+    xd = to_device(x)
+    toks = [{k: xd[k][:, :, t].contiguous() for k in ("u", "delta", "z", "B", "C")} for t in range(S)]
+    state = torch.from_numpy(h0).cuda()
+    ys = [torch.empty(w.batch, w.dim, device="cuda") for _ in range(S)]
+
+    def chain():
+        for t in range(S):
+            tk = toks[t]
+            ss.ss_scan_step(state, tk["u"], tk["delta"], xd["A"], tk["B"], tk["C"], D=xd["D"],
+                            z=tk["z"], delta_bias=xd["delta_bias"], y_out=ys[t])
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm up outside the capture
+        chain()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        chain()
+    state.copy_(torch.from_numpy(h0))
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert ss.ss_last_device_error() == ss.SS_OK
+    yr, hr = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                             x["delta_bias"], h0=h0)
+    _check(w, torch.stack(ys, dim=2), state, yr, hr)
