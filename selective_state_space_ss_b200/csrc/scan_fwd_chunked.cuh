@@ -11,9 +11,10 @@
 // buffered on mbarriers, so the next chunk's copy overlaps this chunk's math):
 //   phase 1  per element: Delta = softplus(delta + bias), w = Delta * u, kept
 //            as float4 of four timesteps; B_t and C_t transposed from their
-//            [n][t] rows into [t][state pair][B_lo, B_hi, C_lo, C_hi] in the
-//            input dtype, so a lane's states' B and C are one contiguous run
-//            (one 16-byte load for four bf16 states);
+//            [n][t] rows into 16-byte units per step [B_2p, B_2p+1, C_2p,
+//            C_2p+1, ...] in the input dtype (four bf16 or two fp32 states a
+//            unit), a lane's units interleaved with its neighbours' so that a
+//            quarter-warp reads 128 contiguous bytes;
 //   phase 2  per (channel, state): A_bar = 2^(Delta * A * log2 e),
 //            h = A_bar * h + w * B_t[n], and the lane's partial readout
 //            sum_n C_t[n] h[n], in packed fp32x2 arithmetic; B_t and C_t are
@@ -21,9 +22,13 @@
 //            sharing of "从Transformer的痛点 ... Mamba", sec. 4.2);
 //   phase 3  per element: s = sum of the K lane partials,
 //            y = (s + D u) * SiLU(z), coalesced fp32 stores.
-// The serial time loop inside a thread is the recurrence itself; the
-// associative operator of "Mamba 选择性机制", sec. 3.1, is not needed here
-// because no thread ever holds a time range whose carry-in is unknown.
+// The serial time loop inside a thread is the recurrence itself.  Where a
+// time range starts with its carry-in unknown, the associative operator of
+// "Mamba 选择性机制", sec. 3.1, joins it to what came before: the time-split
+// warps of a CTA (phase2_split, short sequences over few channels), the
+// balanced schedule's carries between CTAs, and the segments of a long
+// sequence scanned at once from h = 0, whose end states and sums of Delta the
+// correction kernel (scan_fix.cuh) folds into each segment's carry-in.
 //
 // With two channels per lane (CPL = 2) a lane keeps the same G states of two
 // channels and packs its fp32x2 arithmetic over the channel pair: the pair's
