@@ -23,6 +23,9 @@ size_t ckpt_bytes(int64_t batch, int64_t dim, int64_t seqlen, int N) {
   return align256((size_t)batch * (size_t)nk * (size_t)dim * (size_t)N * sizeof(float));
 }
 
+// States per lane of the N = 16 backward (tuning builds may set 2: twice the
+// warps; measured faster on B4 L8192 D5120, slower on B8 L2048 D1536 and
+// B16 L4096 D2048, so 4 stays the default).
 #ifndef SS_BWD_G
 #define SS_BWD_G 4
 #endif
