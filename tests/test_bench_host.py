@@ -69,3 +69,25 @@ def test_reference_arm_prints_the_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["config"]["workload"] == bench.DEFAULT_WORKLOAD
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_traffic_records_key_the_code_not_the_comments():
+    # a comment or blank-line edit keeps a kernel's traffic record valid; any
+    # code edit voids it
+    src = "// header\nint f(int x) {  // trailing\n  /* block\n  comment */ return x + 1;\n\n}\n"
+    assert bench._code_only(src) == bench._code_only(src.replace("trailing", "other") + "\n// more\n")
+    assert bench._code_only(src) != bench._code_only(src.replace("x + 1", "x + 2"))
+    assert "header" not in bench._code_only(src) and "block" not in bench._code_only(src)
+
+
+def test_traffic_records_match_the_current_sources():
+    # every record the bench reports on the committed sources was taken on them
+    import json
+
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)
+    fwd = bench.kernel_hash()
+    keys = {bench.kernel_hash(), bench.kernel_hash(bench.BWD_KERNEL_SOURCES),
+            bench.kernel_hash(bench.STEP_KERNEL_SOURCES)}
+    assert recs["b1_l1048576_d1536_n16_bf16"]["kernel_hash"] == fwd
+    assert all(r["kernel_hash"] in keys for r in recs.values())
