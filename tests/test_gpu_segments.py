@@ -185,3 +185,21 @@ def test_kernels_per_call():
     ss.ss_debug_inject(ss.SS_DEBUG_CLEAR)
     with pytest.raises(ss.SSError):
         ss.ss_debug_fwd_kernels(1, 64, 4096, 24, ss.SS_F32)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("drop", ["z", "D", "bias"])
+def test_segments_optional_inputs(dtype, drop):
+    # the correction gates by SiLU(z) only when z is given, and reads no D or bias
+    w = I.Workload(f"segopt_{dtype}_{drop}", 1, 70, 3000, 16, dtype)
+    x = I.make_inputs(w, seed=31)
+    key = {"z": "z", "D": "D", "bias": "delta_bias"}[drop]
+    x[key] = None
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_SEGMENTS, 5)
+    xd = to_device(x)
+    y, h = ss.ss_scan_fwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"], z=xd["z"],
+                          delta_bias=xd["delta_bias"])
+    torch.cuda.synchronize()
+    assert ss.ss_last_device_error() == ss.SS_OK
+    yr, hr = _ref(x)
+    _check(w, y.cpu().numpy(), h.cpu().numpy(), yr, hr)
