@@ -5,6 +5,7 @@
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -26,11 +27,27 @@ def deps():
             + [os.path.join(ROOT, "include", "ss_scan.h"), os.path.abspath(__file__)])
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def source_hash(defines=()) -> str:
+    """Hash of every source the library is built from, and the -D flags."""
+    h = hashlib.sha256(" ".join(defines).encode())
+    for p in sorted(deps()):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def _stale(target: str, defines=()) -> bool:
+    # by content, not by time stamps (a copied tree may carry any mtimes): the
+    # hash of the sources a library was built from sits beside it in <lib>.src
+    try:
+        with open(target + ".src") as f:
+            return not os.path.exists(target) or f.read().strip() != source_hash(defines)
+    except OSError:
         return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(p) > t for p in deps())
+
+
+def stale() -> bool:
+    return _stale(LIB)
 
 
 def build(force: bool = False, ptxas_verbose: bool = False, out: str | None = None,
@@ -47,6 +64,8 @@ def build(force: bool = False, ptxas_verbose: bool = False, out: str | None = No
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
     os.replace(tmp, target)
+    with open(target + ".src", "w") as f:
+        f.write(source_hash(defines))
     return target
 
 
@@ -57,8 +76,7 @@ def build_checked(force: bool = False) -> str:
     """Compile the checked build (SS_BOUNDS_CHECK: every global index the kernels
     form is compared with its tensor's extent; a miss is skipped and reported by
     ss_last_device_error as SS_ERR_BOUNDS).  Same C ABI; for tests."""
-    if not force and os.path.exists(CHECKED_LIB) and not any(
-            os.path.getmtime(p) > os.path.getmtime(CHECKED_LIB) for p in deps()):
+    if not force and not _stale(CHECKED_LIB, ["SS_BOUNDS_CHECK"]):
         return CHECKED_LIB
     return build(out=CHECKED_LIB, defines=["SS_BOUNDS_CHECK"])
 
@@ -67,8 +85,17 @@ def build_probe() -> str:
     """Compile the standalone issue-rate probe (probe_rates.cu) next to the library."""
     out = os.path.join(PKG, "probe_rates")
     src = os.path.join(CSRC, "probe_rates.cu")
-    if not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    try:
+        with open(out + ".src") as f:
+            fresh = os.path.exists(out) and f.read().strip() == h
+    except OSError:
+        fresh = False
+    if not fresh:
         subprocess.check_call([NVCC, *ARCH, "-O3", "-o", out, src])
+        with open(out + ".src", "w") as f:
+            f.write(h)
     return out
 
 
