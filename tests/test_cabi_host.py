@@ -230,3 +230,13 @@ def test_binding_refuses_cpu_tensors():
         N.ss_scan_fwd_train(x, x, torch.zeros(2, 16), B, B)
     with pytest.raises(ValueError):
         N.ss_scan_bwd(x, x, torch.zeros(2, 16), B, B, torch.zeros(1, 2, 8))
+
+
+def test_built_libraries_match_their_sources():
+    # each library records the hash of the sources (and -D flags) it was built
+    # from; a build is redone exactly when that hash changes
+    assert B.source_hash() == B.source_hash()
+    assert B.source_hash() != B.source_hash(["SS_BOUNDS_CHECK"])
+    assert not B.stale(), "libssscan.so is older than its sources"
+    with open(B.LIB + ".src") as f:
+        assert f.read().strip() == B.source_hash()
