@@ -232,7 +232,7 @@ def test_binding_refuses_cpu_tensors():
         N.ss_scan_bwd(x, x, torch.zeros(2, 16), B, B, torch.zeros(1, 2, 8))
 
 
-def test_built_libraries_match_their_sources():
+def test_built_libraries_match_their_sources(lib):
     # each library records the hash of the sources (and -D flags) it was built
     # from; a build is redone exactly when that hash changes
     assert B.source_hash() == B.source_hash()
