@@ -16,8 +16,9 @@
 // consecutive steps of every block of 32 SPL steps; the prefix sums of Delta
 // over the segment come from a per-lane sum and a warp scan, the running
 // total kept as an unevaluated sum of two floats (Knuth's two-sum), so that
-// it does not drift over a long segment.  The term of state n is evaluated as sign(h_in[n]) 2^(a_n S_t +
-// log2|h_in[n]|) C_t[n] (one fused multiply-add for the exponent).  A state's
+// it does not drift over a long segment.  The term of state n is evaluated
+// as sign(h_in[n]) 2^(a_n S_t + log2|h_in[n]|) C_t[n] (one fused
+// multiply-add for the exponent).  A state's
 // term is dropped once |h_in[n]| P_t[n] < 2^-36 max_m |h_in[m]| for the rest of
 // the segment: with softplus on (Delta >= 0) and A[d,n] < 0 the weight only
 // falls, and a term 2^-36 below the largest state lies 12 binary orders below
@@ -56,7 +57,8 @@ struct FixArgs {
 };
 
 // TMA descriptors of the correction: delta, z and y as [batch][dim][L] with a
-// [1][1][128] box, C as [batch][N][L] with a [1][N][128] box (N = 16 only).
+// [1][1][block] box, C as [batch][N][L] with a [1][N][block] box (N = 16
+// only); a block is 32 SPL steps (FixStage).
 struct FixMaps {
   CUtensorMap delta, z, y, C;
 };
