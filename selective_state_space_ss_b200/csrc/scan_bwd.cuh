@@ -19,9 +19,10 @@
 //          with dq_t = dy_t SiLU(z_t), dz_t = dy_t q_t SiLU'(z_t),
 //          q_t = C_t . h_t + D u_t, ddelta = dDelta softplus'(x).
 //
-// Lane layout: four states of one channel per lane (N/4 lanes per channel).
-// Per-channel sums over a lane's states go through shared memory; sums over
-// the CTA's channels (dB, dC) are reduced in shared memory and added to HBM
+// Lane layout: G states of one channel per lane (N/G lanes per channel; G = 4
+// unless a tuning build sets 2).  Per-channel sums over the states meet by
+// xor shuffles among a channel's lanes; sums over the CTA's channels (dB, dC)
+// are reduced in shared memory (four states per 16-byte load) and added to HBM
 // with one atomic per (state, step) per CTA; dA, dD and the bias gradient
 // with one atomic per channel state per CTA.  Those outputs are zeroed by
 // the host before the launch.
