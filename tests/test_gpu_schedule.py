@@ -125,3 +125,29 @@ def test_replay_in_a_cuda_graph(workers):
         torch.cuda.synchronize()
         assert ss.ss_last_device_error() == ss.SS_OK
         _check(w, x, y, h)
+
+
+def test_balanced_schedule_beside_other_work():
+    # The balanced schedule's workers take their ids from a counter as they
+    # start, so a worker only ever waits for one that is already running.  A
+    # matmul on another stream holds SM slots while the scan launches more
+    # workers than channel groups fit at once; the scan must finish without a
+    # carry wait giving up.
+    w = I.Workload("split_busy", 64, 512, 2048, 16, "bf16")
+    x = I.make_inputs(w, seed=41)
+    xd = to_device(x)
+    groups = w.batch * (w.dim // 32)
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, groups - 1)
+    need = ss.ss_scan_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    a = torch.randn(8192, 8192, device="cuda")
+    side = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        for _ in range(4):
+            a = a @ a.T * 1e-4
+    ss.ss_debug_inject(ss.SS_DEBUG_FORCE_WORKERS, groups - 1)
+    y, h = run_gpu(xd, workspace=ws)
+    torch.cuda.synchronize()
+    assert ss.ss_last_device_error() == ss.SS_OK
+    _check(w, x, y, h)
