@@ -726,17 +726,21 @@ def launch_ranks(n: int) -> int:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--op", default="scan", choices=["scan", "step", "bwd"])
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="ranks on this node, one per GPU (started here unless a launcher did)")
+    ap.add_argument("--steps", type=int, default=50, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed steps before them")
+    ap.add_argument("--op", default="scan", choices=["scan", "step", "bwd"],
+                    help="the forward scan, the recurrent decode step, or the backward")
     ap.add_argument("--workload", default=None,
                     choices=sorted(I.WORKLOADS) + sorted(I.STEP_WORKLOADS))
     ap.add_argument("--seqlen", type=int, default=None,
                     help="override the workload's sequence length (a shorter proxy of the same "
                          "batch, width and distributions, for profiling captures)")
-    ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"],
+                    help="reference: time the fp64 CPU oracle on a bounded sample instead")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip timing the fp64 oracle beside the GPU line")
     ap.add_argument("--zoh", action="store_true", help="exact zero-order-hold B_bar")
     ap.add_argument("--ckpt", action="store_true",
                     help="--op bwd: start from checkpoints written by the training forward")
